@@ -1,0 +1,23 @@
+"""fp64 CPU oracle for the spacetime-attention hot path.
+
+TEST INFRASTRUCTURE ONLY: imported by the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline legs of ``bench.py``.  The CUDA library neither imports nor calls it.
+"""
+
+from .spacetime_oracle import (  # noqa: F401
+    SKIP_GROUP,
+    SKIP_SINGLE,
+    attention_head_ref,
+    attn_ref,
+    default_scale,
+    rope3d_positions_ref,
+    rope3d_ref,
+    rope_frequencies,
+    skiparse_attn_ref,
+    skiparse_gather_ref,
+    skiparse_index_map,
+    skiparse_scatter_ref,
+    skiparse_sets,
+    softmax_rows,
+    video_positions,
+)

@@ -1,0 +1,294 @@
+"""Plain fp64 CPU oracle for spacetime attention (3D RoPE, 3D full attention, Skiparse).
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this module.  It shares
+no code with the CUDA library and never calls it; the library never calls this module.
+
+Everything here is the written-out definition of what the method computes, in float64,
+starting from the exact values of the (bf16) inputs.  Library primitives (a matmul, exp) are
+used as single steps; there is no blocking, fusion or reordering beyond splitting query rows
+into chunks to bound memory, which does not change any value.
+
+Sources (page title, section):
+  * "CogVideoX: Text-to-Video Diffusion Models with an Expert Transformer", section 2
+    (latents are patchified and unfolded into one sequence; text embeddings are concatenated
+    with it along the sequence axis), section 2.2 "Patchify" (sequence length), "3D-RoPE"
+    (independent 1D RoPE per coordinate axis over channel shares, concatenated along the
+    channel axis), "3D Full Attention"; section 3.1 and the appendix on RoPE interpolation
+    (positions are raw indices, extrapolated, never rescaled).
+  * "Open Video Models", The Breakthrough (HunyuanVideo's 3D RoPE: separate rotation
+    frequencies along time, height and width).
+  * RoFormer (reference [14] of the CogVideoX paper): rotation of channel pairs by
+    position times a geometric frequency series with base 10000.
+  * "Open-Sora Plan: Open-Source Large Video Generation Model", section 2.2.2 "Skiparse
+    Attention" (sequence cut to 1/k with the batch grown k-fold; Single Skip; Group Skip
+    groups adjacent tokens and connects groups that are k-1 groups apart; THW mod k = 0).
+  * "Attention is all you need" (reference [1]): softmax(q k^T / sqrt(d)) v.
+
+Readings where the pages are silent (each also listed in the design notes):
+  * flattening order of the (t, h, w) grid is row-major, w fastest; text tokens come first;
+  * channel chunks are ordered t, h, w; pairs inside a chunk are interleaved (2j, 2j+1);
+    the frequency of pair j in a chunk of size d_a is theta^(-2j/d_a);
+  * text tokens are not rotated;
+  * Single Skip set g = tokens {s*k + g}; Group Skip uses groups of k adjacent tokens and
+    set g = groups whose index is congruent to g mod k, i.e. slot s = o*k + r maps to token
+    o*k*k + g*k + r; each set lists its tokens in ascending order;
+  * the k-fold batch produced by the gather is ordered b*k + g (b outer);
+  * softmax scale 1/sqrt(head_dim) unless given.
+
+Parity is pinned for every function here by ``tests/test_oracle_pins.py``.  Match to any
+trained checkpoint is "parity unpinned": no weights or code exist to compare against, and the
+pages do not fix the pairing convention of RoPE channels.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Sequence
+
+import numpy as np
+
+SKIP_SINGLE = 0
+SKIP_GROUP = 1
+
+
+# ----------------------------------------------------------------------------------------------
+# Token positions
+# ----------------------------------------------------------------------------------------------
+
+def video_positions(T: int, H: int, W: int):
+    """(t, h, w) integer coordinates of every video token, in sequence order.
+
+    The latent grid T x H x W is unfolded into one sequence (CogVideoX section 2 and 2.2
+    "Patchify"); reading: row-major, w fastest.  Token v has t = v div (H W),
+    h = (v div W) mod H, w = v mod W.  Positions start at 0 and are not rescaled
+    (CogVideoX section 3.1: extrapolation, not interpolation).
+    """
+    n = T * H * W
+    v = np.arange(n, dtype=np.int64)
+    t = v // (H * W)
+    h = (v // W) % H
+    w = v % W
+    return t, h, w
+
+
+# ----------------------------------------------------------------------------------------------
+# 3D RoPE
+# ----------------------------------------------------------------------------------------------
+
+def rope_frequencies(d_axis: int, theta: float = 10000.0) -> np.ndarray:
+    """Frequencies of one axis's 1D RoPE: omega_j = theta^(-2j/d_axis), j < d_axis/2.
+
+    RoFormer's geometric series, applied per axis with the axis's own channel count
+    ("Open Video Models": separate rotation frequencies along time, height and width).
+    """
+    if d_axis % 2:
+        raise ValueError("each RoPE channel chunk must be even")
+    j = np.arange(d_axis // 2, dtype=np.float64)
+    return np.power(float(theta), -2.0 * j / float(d_axis))
+
+
+def rope_rotate_chunk(x: np.ndarray, pos: np.ndarray, d_axis: int, theta: float) -> np.ndarray:
+    """1D RoPE on one channel chunk.
+
+    x: [..., n_tok, n_heads, d_axis] float64, pos: [n_tok] integer positions.
+    Pair j = channels (2j, 2j+1) is rotated by angle pos * omega_j:
+        x' = x cos(a) - y sin(a),  y' = x sin(a) + y cos(a).
+    """
+    omega = rope_frequencies(d_axis, theta)                      # [d_axis/2]
+    ang = pos.astype(np.float64)[:, None] * omega[None, :]       # [n_tok, d_axis/2]
+    c = np.cos(ang)[:, None, :]                                  # broadcast over heads
+    s = np.sin(ang)[:, None, :]
+    xe = x[..., 0::2]
+    xo = x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = xe * c - xo * s
+    out[..., 1::2] = xe * s + xo * c
+    return out
+
+
+def rope3d_positions_ref(x: np.ndarray, pos_t, pos_h, pos_w, split: Sequence[int],
+                         theta: float = 10000.0) -> np.ndarray:
+    """3D RoPE of video tokens with explicit positions.
+
+    x: [B, n_tok, n_heads, d] (values of the bf16 inputs); pos_*: [n_tok] integers.
+    CogVideoX section 2.2 "3D-RoPE": an independent 1D RoPE per coordinate axis, each on its
+    own share of the channels, the results concatenated along the channel axis.  Reading:
+    chunk order t, h, w with sizes split = (d_t, d_h, d_w).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d_t, d_h, d_w = (int(a) for a in split)
+    if d_t + d_h + d_w != x.shape[-1]:
+        raise ValueError("RoPE split must sum to head_dim")
+    out = np.empty_like(x)
+    out[..., 0:d_t] = rope_rotate_chunk(x[..., 0:d_t], np.asarray(pos_t), d_t, theta)
+    out[..., d_t:d_t + d_h] = rope_rotate_chunk(x[..., d_t:d_t + d_h], np.asarray(pos_h), d_h, theta)
+    out[..., d_t + d_h:] = rope_rotate_chunk(x[..., d_t + d_h:], np.asarray(pos_w), d_w, theta)
+    return out
+
+
+def rope3d_ref(x: np.ndarray, grid: Sequence[int], text_len: int, split: Sequence[int],
+               theta: float = 10000.0) -> np.ndarray:
+    """3D RoPE over a [B, text_len + T*H*W, n_heads, d] sequence.
+
+    Text tokens (the first text_len; CogVideoX section 2 concatenates text before video) are
+    left unrotated (reading: the pages give text no spatio-temporal position); video tokens
+    are rotated by their (t, h, w) grid coordinates.
+    """
+    T, H, W = (int(a) for a in grid)
+    x = np.asarray(x, dtype=np.float64)
+    if x.shape[1] != text_len + T * H * W:
+        raise ValueError("sequence length does not match text_len + T*H*W")
+    out = x.copy()
+    t, h, w = video_positions(T, H, W)
+    out[:, text_len:] = rope3d_positions_ref(x[:, text_len:], t, h, w, split, theta)
+    return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Skiparse index maps
+# ----------------------------------------------------------------------------------------------
+
+def skiparse_sets(n_video: int, k: int, mode: int) -> list[list[int]]:
+    """The k token sets of Skiparse attention, each as an explicit ascending list.
+
+    Open-Sora Plan section 2.2.2: the sequence is cut to 1/k of its length and the batch
+    grown k-fold.  Single Skip: set g holds every k-th token starting at g.  Group Skip:
+    adjacent tokens form groups (of k tokens, reading) and a set joins groups that are
+    k-1 groups apart, i.e. the groups whose index is congruent to g mod k.
+    """
+    if k < 1:
+        raise ValueError("k must be >= 1")
+    if mode == SKIP_SINGLE:
+        if n_video % k:
+            raise ValueError("Single Skip needs n_video mod k == 0")
+        return [[s * k + g for s in range(n_video // k)] for g in range(k)]
+    if mode == SKIP_GROUP:
+        if n_video % (k * k):
+            raise ValueError("Group Skip needs n_video mod k^2 == 0")
+        n_groups = n_video // k
+        sets = []
+        for g in range(k):
+            members = []
+            for group in range(n_groups):
+                if group % k == g:
+                    members.extend(range(group * k, group * k + k))
+            sets.append(members)
+        return sets
+    raise ValueError("mode must be SKIP_SINGLE or SKIP_GROUP")
+
+
+def skiparse_index_map(n_video: int, k: int, mode: int) -> np.ndarray:
+    """Concatenation of the k sets: entry g*(n_video/k) + s is the token at slot s of set g."""
+    return np.asarray([tok for st in skiparse_sets(n_video, k, mode) for tok in st], dtype=np.int32)
+
+
+# ----------------------------------------------------------------------------------------------
+# Gather / scatter (the k-fold batch)
+# ----------------------------------------------------------------------------------------------
+
+def skiparse_gather_ref(x: np.ndarray, k: int, mode: int) -> np.ndarray:
+    """[B, N, n_h, d] -> [B*k, N/k, n_h, d]: out[b*k + g, s] = x[b, set_g[s]]."""
+    B, N = x.shape[0], x.shape[1]
+    sets = skiparse_sets(N, k, mode)
+    out = np.empty((B * k, N // k) + tuple(x.shape[2:]), dtype=x.dtype)
+    for b in range(B):
+        for g in range(k):
+            out[b * k + g] = x[b, sets[g]]
+    return out
+
+
+def skiparse_scatter_ref(y: np.ndarray, k: int, mode: int) -> np.ndarray:
+    """Inverse of the gather: out[b, set_g[s]] = y[b*k + g, s]."""
+    Bk, n_set = y.shape[0], y.shape[1]
+    B, N = Bk // k, n_set * k
+    sets = skiparse_sets(N, k, mode)
+    out = np.empty((B, N) + tuple(y.shape[2:]), dtype=y.dtype)
+    for b in range(B):
+        for g in range(k):
+            out[b, sets[g]] = y[b * k + g]
+    return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Attention
+# ----------------------------------------------------------------------------------------------
+
+def softmax_rows(s: np.ndarray) -> np.ndarray:
+    """Row softmax p_ij = exp(s_ij - max_j s_ij) / sum_j exp(s_ij - max_j s_ij)."""
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def attention_head_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                       rows=None, chunk: int = 1024) -> np.ndarray:
+    """Exact attention for one head: o_i = sum_j softmax_j(q_i . k_j * scale) v_j.
+
+    q: [n_q, d], k: [n_kv, d], v: [n_kv, d] float64.  ``rows`` optionally selects query rows
+    (the result then has len(rows) rows).  Query rows are processed ``chunk`` at a time.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if rows is not None:
+        q = q[np.asarray(rows)]
+    out = np.empty((q.shape[0], v.shape[1]), dtype=np.float64)
+    for r0 in range(0, q.shape[0], chunk):
+        s = (q[r0:r0 + chunk] @ k.T) * scale
+        out[r0:r0 + chunk] = softmax_rows(s) @ v
+    return out
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
+
+
+def attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float | None = None,
+             rows=None, heads=None) -> np.ndarray:
+    """3D full attention (CogVideoX "3D Full Attention"): every token of a sample attends to
+    every token of the same sample (text and video), bidirectionally, per head.
+
+    q, k, v: [B, N, n_h, d].  Returns [B, N, n_h, d] float64, or, with ``rows`` (query token
+    indices) and/or ``heads``, only those rows/heads: [B, len(rows), len(heads), d].
+    """
+    B, N, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    rows_ = np.arange(N) if rows is None else np.asarray(rows)
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    out = np.empty((B, len(rows_), len(heads_), d), dtype=np.float64)
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            out[b, :, hi] = attention_head_ref(q[b, :, h], k[b, :, h], v[b, :, h], scale, rows_)
+    return out
+
+
+def skiparse_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, k_ratio: int, mode: int,
+                      scale: float | None = None, rows=None, heads=None) -> np.ndarray:
+    """Skiparse attention: each token attends only to the tokens of its own set
+    (Open-Sora Plan section 2.2.2), output in natural token order.
+
+    q, k, v: [B, N, n_h, d] with no text tokens.  ``rows`` optionally restricts the query
+    tokens computed (natural indices); the result is then [B, len(rows), len(heads), d].
+    """
+    B, N, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    sets = skiparse_sets(N, k_ratio, mode)
+    set_of = np.empty(N, dtype=np.int64)
+    slot_of = np.empty(N, dtype=np.int64)
+    for g, st in enumerate(sets):
+        set_of[st] = g
+        slot_of[st] = np.arange(len(st))
+    rows_ = np.arange(N) if rows is None else np.asarray(rows)
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    out = np.empty((B, len(rows_), len(heads_), d), dtype=np.float64)
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            for g, st in enumerate(sets):
+                sel = np.nonzero(set_of[rows_] == g)[0]
+                if sel.size == 0:
+                    continue
+                idx = np.asarray(st)
+                out[b, sel, hi] = attention_head_ref(q[b, idx, h], k[b, idx, h], v[b, idx, h],
+                                                     scale, slot_of[rows_[sel]])
+    return out

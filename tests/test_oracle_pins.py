@@ -1,0 +1,325 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself: every expected value is a hand-written fixture
+(tests/golden/, each with its source), a closed form, an invariant, or a brute-force pure-Python
+evaluation of the definition on tiny inputs.  Each group is chosen so that a plausible slip in
+the oracle (a dropped term, a wrong sign or index, a transposed operand, a wrong frequency or
+pairing convention) fails at least one test.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+
+# ----------------------------------------------------------------------------------------------
+# fixtures
+# ----------------------------------------------------------------------------------------------
+
+def _read_sets(golden_dir):
+    cases = []
+    with open(os.path.join(golden_dir, "skiparse_sets.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, body = line.split(":")
+            mode, n, k = head.split()
+            sets = [[int(t) for t in part.split()] for part in body.split("|")]
+            cases.append((O.SKIP_SINGLE if mode == "single" else O.SKIP_GROUP, int(n), int(k), sets))
+    return cases
+
+
+def _read_rope(golden_dir):
+    rows = []
+    with open(os.path.join(golden_dir, "rope_unit_rotations.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            p = line.split()
+            rows.append((int(p[0]), int(p[1]), int(p[2]), int(p[3]), int(p[4]), float(p[5]),
+                         int(p[6]), float(p[7])))
+    return rows
+
+
+# ----------------------------------------------------------------------------------------------
+# index maps
+# ----------------------------------------------------------------------------------------------
+
+def test_sets_match_hand_written_golden(golden_dir):
+    cases = _read_sets(golden_dir)
+    assert len(cases) >= 8
+    for mode, n, k, sets in cases:
+        assert O.skiparse_sets(n, k, mode) == sets, (mode, n, k)
+
+
+@pytest.mark.parametrize("mode", [O.SKIP_SINGLE, O.SKIP_GROUP])
+def test_sets_are_partitions_exhaustive(mode):
+    for k in range(1, 7):
+        step = k if mode == O.SKIP_SINGLE else k * k
+        for n in range(step, 73, step):
+            sets = O.skiparse_sets(n, k, mode)
+            assert len(sets) == k
+            assert all(len(s) == n // k for s in sets)
+            assert sorted(t for s in sets for t in s) == list(range(n))
+            assert all(s == sorted(s) for s in sets)
+            m = O.skiparse_index_map(n, k, mode)
+            assert m.dtype == np.int32 and sorted(m.tolist()) == list(range(n))
+
+
+def test_single_skip_membership_is_residue_class():
+    for k in range(1, 6):
+        n = 12 * k
+        for g, s in enumerate(O.skiparse_sets(n, k, O.SKIP_SINGLE)):
+            assert all(t % k == g for t in s)
+
+
+def test_group_skip_connects_groups_k_minus_1_apart():
+    # tokens i, j in one set: their groups floor(i/k), floor(j/k) differ by a multiple of k,
+    # i.e. k-1 groups lie between consecutive groups of a set; and each group is whole.
+    for k in range(2, 6):
+        n = 3 * k * k
+        for s in O.skiparse_sets(n, k, O.SKIP_GROUP):
+            groups = sorted({t // k for t in s})
+            for a, b in zip(groups, groups[1:]):
+                assert b - a == k
+            for gr in groups:
+                assert all(gr * k + r in s for r in range(k))
+
+
+def test_k1_is_identity_and_divisibility_errors():
+    for mode in (O.SKIP_SINGLE, O.SKIP_GROUP):
+        assert O.skiparse_index_map(10, 1, mode).tolist() == list(range(10))
+    with pytest.raises(ValueError):
+        O.skiparse_sets(10, 4, O.SKIP_SINGLE)
+    with pytest.raises(ValueError):
+        O.skiparse_sets(8, 4, O.SKIP_GROUP)
+
+
+def test_config_sizes_divide():
+    # 4x8x8 with k=2; 24x30x40 and 16x36x64 with k=4 (single needs k | N, group k^2 | N)
+    for n, k in [(256, 2), (28800, 4), (36864, 4)]:
+        for mode in (O.SKIP_SINGLE, O.SKIP_GROUP):
+            m = O.skiparse_index_map(n, k, mode)
+            assert np.array_equal(np.sort(m), np.arange(n))
+
+
+# ----------------------------------------------------------------------------------------------
+# gather / scatter
+# ----------------------------------------------------------------------------------------------
+
+def test_gather_layout_and_inverse(golden_dir):
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((2, 8, 3, 4))
+    y = O.skiparse_gather_ref(x, 2, O.SKIP_GROUP)
+    assert y.shape == (4, 4, 3, 4)
+    # group, n=8, k=2: set0 = 0 1 4 5, set1 = 2 3 6 7 (golden); batch order b*k + g
+    assert np.array_equal(y[0], x[0, [0, 1, 4, 5]])
+    assert np.array_equal(y[1], x[0, [2, 3, 6, 7]])
+    assert np.array_equal(y[3], x[1, [2, 3, 6, 7]])
+    for mode in (O.SKIP_SINGLE, O.SKIP_GROUP):
+        assert np.array_equal(O.skiparse_scatter_ref(O.skiparse_gather_ref(x, 2, mode), 2, mode), x)
+
+
+# ----------------------------------------------------------------------------------------------
+# 3D RoPE
+# ----------------------------------------------------------------------------------------------
+
+def test_rope_unit_vectors_match_closed_forms(golden_dir):
+    rows = _read_rope(golden_dir)
+    assert len(rows) >= 6
+    for t, h, w, cin, ca, va, cb, vb in rows:
+        x = np.zeros((1, 1, 1, 24))
+        x[0, 0, 0, cin] = 1.0
+        y = O.rope3d_positions_ref(x, [t], [h], [w], (8, 8, 8), 10000.0)[0, 0, 0]
+        expect = np.zeros(24)
+        expect[ca] = va
+        expect[cb] = vb
+        np.testing.assert_allclose(y, expect, rtol=0, atol=1e-14)
+
+
+def test_rope_identity_at_origin_and_on_text_tokens():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((2, 5 + 2 * 3 * 4, 3, 64))
+    y = O.rope3d_ref(x, (2, 3, 4), 5, (16, 24, 24))
+    assert np.array_equal(y[:, :5], x[:, :5])          # text tokens untouched
+    assert np.array_equal(y[:, 5], x[:, 5])            # video token 0 is at (0,0,0)
+    assert not np.allclose(y[:, 6], x[:, 6])           # token 1 is at (0,0,1)
+
+
+def test_rope_token_positions_follow_raster_order():
+    # token v of a 2x3x4 grid: t = v // 12, h = (v // 4) % 3, w = v % 4
+    t, h, w = O.video_positions(2, 3, 4)
+    assert (t[13], h[13], w[13]) == (1, 0, 1)
+    assert (t[11], h[11], w[11]) == (0, 2, 3)
+    # and rope3d_ref uses them: only the w chunk of token 1 rotates, only h of token 4, t of 12
+    x = np.ones((1, 24, 1, 24))
+    y = O.rope3d_ref(x, (2, 3, 4), 0, (8, 8, 8))[0, :, 0]
+    changed = lambda v: np.nonzero(~np.isclose(y[v], 1.0))[0]
+    assert set(changed(1)) <= set(range(16, 24)) and len(changed(1)) > 0
+    assert set(changed(4)) <= set(range(8, 16)) and len(changed(4)) > 0
+    assert set(changed(12)) <= set(range(0, 8)) and len(changed(12)) > 0
+
+
+def test_rope_preserves_pair_norms():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((1, 3 * 4 * 5, 2, 96))
+    y = O.rope3d_ref(x, (3, 4, 5), 0, (32, 32, 32))
+    nx = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    ny = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    np.testing.assert_allclose(ny, nx, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("split", [(16, 24, 24), (32, 32, 32), (32, 48, 48)])
+def test_rope_score_depends_only_on_offset(split):
+    d = sum(split)
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, 6, 1, d))
+    k = rng.standard_normal((1, 6, 1, d))
+    pt, ph, pw = rng.integers(0, 40, 6), rng.integers(0, 40, 6), rng.integers(0, 40, 6)
+    rq = O.rope3d_positions_ref(q, pt, ph, pw, split)[0, :, 0]
+    rk = O.rope3d_positions_ref(k, pt, ph, pw, split)[0, :, 0]
+    s0 = rq @ rk.T
+    for shift in [(1, 0, 0), (0, 5, 0), (0, 0, 7), (3, 11, 29)]:
+        sq = O.rope3d_positions_ref(q, pt + shift[0], ph + shift[1], pw + shift[2], split)[0, :, 0]
+        sk = O.rope3d_positions_ref(k, pt + shift[0], ph + shift[1], pw + shift[2], split)[0, :, 0]
+        np.testing.assert_allclose(sq @ sk.T, s0, rtol=0, atol=1e-11)
+    # and it does depend on the offset
+    sq = O.rope3d_positions_ref(q, pt + np.arange(6), ph, pw, split)[0, :, 0]
+    assert not np.allclose(sq @ rk.T, s0)
+
+
+def test_rope_one_axis_grid_is_textbook_1d_rope():
+    # H = W = 1: the h and w chunks sit at position 0 (identity) and the t chunk is RoFormer's
+    # 1D RoPE, written here as complex multiplication z * exp(i * pos * omega).
+    T, d_t, d_h, d_w = 9, 16, 8, 8
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((1, T, 1, d_t + d_h + d_w))
+    y = O.rope3d_ref(x, (T, 1, 1), 0, (d_t, d_h, d_w))
+    np.testing.assert_array_equal(y[..., d_t:], x[..., d_t:])
+    for pos in range(T):
+        for j in range(d_t // 2):
+            z = complex(x[0, pos, 0, 2 * j], x[0, pos, 0, 2 * j + 1])
+            zr = z * complex(math.cos(pos * 10000.0 ** (-j / 8.0)), math.sin(pos * 10000.0 ** (-j / 8.0)))
+            assert abs(y[0, pos, 0, 2 * j] - zr.real) < 1e-12
+            assert abs(y[0, pos, 0, 2 * j + 1] - zr.imag) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------------------------
+
+def _brute_masked_attention(q, k, v, allowed, scale):
+    """Pure-Python loops: o_i = sum_j e^{s_ij - m_i} v_j / sum_j e^{s_ij - m_i} over allowed j."""
+    n, d = len(q), len(q[0])
+    out = []
+    for i in range(n):
+        js = [j for j in range(len(k)) if allowed(i, j)]
+        s = [sum(q[i][c] * k[j][c] for c in range(d)) * scale for j in js]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = sum(e)
+        out.append([sum(e[t] * v[js[t]][c] for t in range(len(js))) / z for c in range(d)])
+    return np.asarray(out)
+
+
+def test_attention_matches_brute_force():
+    rng = np.random.default_rng(5)
+    B, N, nh, d = 2, 7, 2, 5
+    q, k, v = (rng.standard_normal((B, N, nh, d)) for _ in range(3))
+    got = O.attn_ref(q, k, v)
+    for b in range(B):
+        for h in range(nh):
+            ref = _brute_masked_attention(q[b, :, h].tolist(), k[b, :, h].tolist(), v[b, :, h].tolist(),
+                                          lambda i, j: True, 1 / math.sqrt(d))
+            np.testing.assert_allclose(got[b, :, h], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_two_key_closed_form():
+    # q.k0 - q.k1 = ln 3 (scale 1) -> weights 3/4, 1/4
+    q = np.zeros((1, 1, 1, 2)); q[0, 0, 0, 0] = 1.0
+    k = np.zeros((1, 2, 1, 2)); k[0, 0, 0, 0] = math.log(3.0)
+    v = np.zeros((1, 2, 1, 2)); v[0, 0, 0] = [4.0, 0.0]; v[0, 1, 0] = [0.0, 8.0]
+    kk = np.concatenate([k, k], axis=1)[:, :2]
+    o = O.attn_ref(np.concatenate([q, q], axis=1), kk, v, scale=1.0)
+    np.testing.assert_allclose(o[0, 0, 0], [3.0, 2.0], rtol=1e-14)
+    # the softmax scale multiplies the scores: scale 2 -> weights 9/10, 1/10
+    o2 = O.attn_ref(np.concatenate([q, q], axis=1), kk, v, scale=2.0)
+    np.testing.assert_allclose(o2[0, 0, 0], [3.6, 0.8], rtol=1e-14)
+
+
+def test_softmax_rows_sum_to_one():
+    rng = np.random.default_rng(6)
+    s = rng.standard_normal((9, 31)) * 30
+    p = O.softmax_rows(s)
+    assert (p >= 0).all()
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-14)
+    assert np.argmax(p, -1).tolist() == np.argmax(s, -1).tolist()
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(7)
+    k, v = rng.standard_normal((1, 11, 2, 8)), rng.standard_normal((1, 11, 2, 8))
+    o = O.attn_ref(np.zeros((1, 11, 2, 8)), k, v)            # q = 0 -> mean of v
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(1, keepdims=True), o.shape), atol=1e-14)
+    q1, k1, v1 = (rng.standard_normal((1, 1, 3, 8)) for _ in range(3))
+    np.testing.assert_allclose(O.attn_ref(q1, k1, v1), v1, atol=1e-15)   # one token -> v
+    # huge scores do not overflow (max subtraction)
+    o = O.attn_ref(q1 * 1e3, k1 * 1e3, v1)
+    assert np.isfinite(o).all()
+
+
+def test_attention_rows_heads_subset():
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((2, 40, 3, 8)) for _ in range(3))
+    full = O.attn_ref(q, k, v)
+    rows, heads = [0, 7, 39], [2, 0]
+    np.testing.assert_allclose(O.attn_ref(q, k, v, rows=rows, heads=heads),
+                               full[:, rows][:, :, heads], rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("mode,k", [(O.SKIP_SINGLE, 2), (O.SKIP_GROUP, 2), (O.SKIP_SINGLE, 3),
+                                    (O.SKIP_GROUP, 3), (O.SKIP_SINGLE, 4)])
+def test_skiparse_is_masked_full_attention_brute_force(mode, k):
+    # membership written independently of the oracle's set lists:
+    # single: same residue mod k; group: same group index mod k.
+    N = 36 if k == 3 else 16 if k == 4 else 24
+    rng = np.random.default_rng(9 + k)
+    q, kk, v = (rng.standard_normal((1, N, 1, 4)) for _ in range(3))
+    if mode == O.SKIP_SINGLE:
+        allowed = lambda i, j: i % k == j % k
+    else:
+        allowed = lambda i, j: (i // k) % k == (j // k) % k
+    ref = _brute_masked_attention(q[0, :, 0].tolist(), kk[0, :, 0].tolist(), v[0, :, 0].tolist(),
+                                  allowed, 0.5)
+    got = O.skiparse_attn_ref(q, kk, v, k, mode)[0, :, 0]
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+    # and the sparse result differs from dense attention
+    assert not np.allclose(got, O.attn_ref(q, kk, v)[0, :, 0])
+
+
+def test_skiparse_k1_is_dense_and_rows_subset():
+    rng = np.random.default_rng(10)
+    q, k, v = (rng.standard_normal((2, 32, 2, 8)) for _ in range(3))
+    for mode in (O.SKIP_SINGLE, O.SKIP_GROUP):
+        np.testing.assert_allclose(O.skiparse_attn_ref(q, k, v, 1, mode), O.attn_ref(q, k, v),
+                                   rtol=0, atol=1e-13)
+        full = O.skiparse_attn_ref(q, k, v, 2, mode)
+        rows = [1, 5, 30]
+        np.testing.assert_allclose(O.skiparse_attn_ref(q, k, v, 2, mode, rows=rows, heads=[1]),
+                                   full[:, rows][:, :, [1]], rtol=0, atol=1e-14)
+
+
+def test_skiparse_equals_gather_dense_scatter():
+    # the k-fold batch formulation of the page: gather -> dense attention -> scatter
+    rng = np.random.default_rng(11)
+    q, k, v = (rng.standard_normal((2, 32, 2, 8)) for _ in range(3))
+    for mode in (O.SKIP_SINGLE, O.SKIP_GROUP):
+        g = [O.skiparse_gather_ref(t, 2, mode) for t in (q, k, v)]
+        o = O.skiparse_scatter_ref(O.attn_ref(*g), 2, mode)
+        np.testing.assert_allclose(o, O.skiparse_attn_ref(q, k, v, 2, mode), rtol=0, atol=1e-13)
