@@ -1,0 +1,145 @@
+/*
+ * osp.h — C ABI of libosp.so: spacetime attention for video diffusion transformers on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library computes, on one GPU, the attention hot path that the Open-Sora Plan and
+ * CogVideoX pages describe:
+ *   - 3D RoPE over the (t, h, w) latent token grid ("CogVideoX: Text-to-Video Diffusion
+ *     Models with an Expert Transformer", section 2.2 "3D-RoPE"; "Open Video Models",
+ *     The Breakthrough: separate rotation frequencies per axis);
+ *   - dense 3D full attention over text + video tokens (CogVideoX section 2 and section 2.2
+ *     "3D Full Attention");
+ *   - Skiparse sparse attention, Single Skip and Group Skip with sparse ratio k
+ *     ("Open-Sora Plan: Open-Source Large Video Generation Model", section 2.2.2).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Layout. Every q/k/v/o tensor is contiguous BSHD bf16: [B][N][heads][head_dim], where
+ *    N = text_len + T*H*W. Text tokens come first; video token v = text_len + (t*H + h)*W + w
+ *    (row-major over the grid, w fastest).
+ *  Pointers. All tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *    The library never frees or retains them beyond the call's stream work.
+ *  Streams. `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *    enqueues work on that stream and returns; results are ready when the stream is.
+ *  Errors. Every entry point returns an osp_status. On a non-zero return nothing has been
+ *    enqueued and osp_get_last_error() describes the problem. Device-side faults of the
+ *    bounded-wait kind (OSP_ERR_TIMEOUT) are reported later by osp_check_status().
+ *  Scratch. On first use per device the library allocates (cudaMalloc) one small status
+ *    word and caches it until process exit. No other allocation happens in any call.
+ *  Threads. Entry points may be called from several host threads; the last-error message is
+ *    per thread.
+ */
+#ifndef OSP_H_
+#define OSP_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  OSP_OK = 0,
+  OSP_ERR_INVALID_ARG = 1,  /* null pointer, bad dimension, RoPE split not summing to head_dim */
+  OSP_ERR_UNSUPPORTED = 2,  /* head_dim not in {64, 96, 128}; text tokens with Skiparse; ... */
+  OSP_ERR_DIVISIBILITY = 3, /* T*H*W mod k != 0 (Single Skip) or mod k*k != 0 (Group Skip) */
+  OSP_ERR_CUDA = 4,         /* a CUDA runtime/driver call or a kernel launch failed */
+  OSP_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see osp_check_status) */
+  OSP_ERR_BOUNDS = 6        /* a device-side index check failed (see osp_check_status) */
+} osp_status;
+
+/* Skiparse modes ("Open-Sora Plan", section 2.2.2).
+ *  OSP_SKIP_SINGLE: set g = video tokens {s*k + g : 0 <= s < T*H*W/k}.
+ *  OSP_SKIP_GROUP:  groups of k adjacent tokens; set g = groups whose index is g mod k,
+ *                   i.e. slot s = o*k + r of set g is token o*k*k + g*k + r.
+ * Each set lists its tokens in ascending order ("slot" = position within the set). */
+enum { OSP_SKIP_SINGLE = 0, OSP_SKIP_GROUP = 1 };
+
+/* Problem shape. N = text_len + T*H*W tokens per sample. */
+typedef struct {
+  int32_t B;         /* batch size, >= 1 */
+  int32_t text_len;  /* text tokens before the video tokens, >= 0 */
+  int32_t T, H, W;   /* latent token grid, each >= 1 */
+  int32_t heads;     /* attention heads, >= 1 */
+  int32_t head_dim;  /* channels per head; RoPE needs it even, attention needs 64, 96 or 128 */
+} osp_shape;
+
+/* 3D RoPE parameters ("CogVideoX" section 2.2 "3D-RoPE"): channels [0, d_t) rotate with t,
+ * [d_t, d_t+d_h) with h, [d_t+d_h, head_dim) with w. Inside a chunk of size d_a, channel pair
+ * (2j, 2j+1) rotates by angle pos * theta^(-2j/d_a) (RoFormer). Positions are raw integer grid
+ * indices (extrapolation, CogVideoX section 3.1). Text tokens are not rotated. */
+typedef struct {
+  int32_t d_t, d_h, d_w;  /* each even and > 0... or 0; d_t + d_h + d_w == head_dim */
+  double theta;           /* frequency base, > 0 (10000 on the pages) */
+} osp_rope;
+
+/* 3D RoPE of q and k.
+ *  q, k:          [B][N][heads][head_dim] bf16, device.
+ *  q_out, k_out:  same shape; may equal q / k (in place) but must not overlap them otherwise.
+ *  Text tokens are copied unchanged (nothing is written for them when out == in).
+ *  Arithmetic: fp32 rotation of the bf16 inputs, rounded to bf16 (RNE).
+ *  Errors: OSP_ERR_INVALID_ARG (null, bad shape or split), OSP_ERR_CUDA (launch failed). */
+int osp_rope3d(const void* q, const void* k, void* q_out, void* k_out, const osp_shape* shape,
+               const osp_rope* rope, void* stream);
+
+/* Dense 3D full attention ("CogVideoX" section 2.2 "3D Full Attention"): for every sample b
+ * and head h, O = softmax(Q K^T * scale) V over all N tokens (text and video), bidirectional.
+ *  q, k, v: [B][N][heads][head_dim] bf16, device (apply osp_rope3d first for 3D RoPE).
+ *  o:       same shape, bf16, device; must not overlap q, k or v.
+ *  softmax_scale: <= 0 selects 1/sqrt(head_dim).
+ *  Arithmetic: bf16 operands on tcgen05 tensor cores, fp32 accumulation in tensor memory,
+ *    fp32 online softmax, probabilities rounded to bf16 for the PV product, O rounded to bf16.
+ *  Errors: OSP_ERR_INVALID_ARG, OSP_ERR_UNSUPPORTED (head_dim not 64/96/128), OSP_ERR_CUDA. */
+int osp_attn_full(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                  float softmax_scale, void* stream);
+
+/* Skiparse gather ("Open-Sora Plan" section 2.2.2: sequence cut to 1/k, batch grown k-fold):
+ *   x_out[b*k + g][s] = RoPE(x[b][token(g, s)])   for q and k (RoPE skipped if rope == NULL),
+ *   v_out[b*k + g][s] = v[b][token(g, s)]         (exact copy).
+ *  q, k, v:     [B][T*H*W][heads][head_dim] bf16, device; shape->text_len must be 0.
+ *               k/k_out and v/v_out may be NULL together (that tensor is skipped).
+ *  *_out:       [B*k][T*H*W/k][heads][head_dim] bf16, device, not overlapping the inputs.
+ *  Errors: OSP_ERR_INVALID_ARG (k < 1, bad mode, null q/q_out), OSP_ERR_UNSUPPORTED
+ *  (text_len != 0), OSP_ERR_DIVISIBILITY, OSP_ERR_CUDA. */
+int osp_skiparse_gather(const void* q, const void* k, const void* v, void* q_out, void* k_out,
+                        void* v_out, const osp_shape* shape, int32_t sparse_k, int32_t mode,
+                        const osp_rope* rope, void* stream);
+
+/* Inverse of the gather for one tensor: o[b][token(g, s)] = o_perm[b*k + g][s] (exact copy).
+ *  o_perm: [B*k][T*H*W/k][heads][head_dim] bf16, device; o: [B][T*H*W][heads][head_dim].
+ *  Errors as for osp_skiparse_gather. */
+int osp_skiparse_scatter(const void* o_perm, void* o, const osp_shape* shape, int32_t sparse_k,
+                         int32_t mode, void* stream);
+
+/* Fused Skiparse attention: every video token attends only to the tokens of its own set
+ * ("Open-Sora Plan" section 2.2.2). The set structure is folded into the kernel's tile
+ * address map, so no permuted copy of q/k/v/o is ever written.
+ *  q, k, v, o: [B][T*H*W][heads][head_dim] bf16, device, natural token order; text_len == 0.
+ *  Group Skip additionally needs k to divide 128 (a power of two up to 128).
+ *  Same arithmetic and scale convention as osp_attn_full. k == 1 is dense attention.
+ *  Errors: OSP_ERR_INVALID_ARG, OSP_ERR_UNSUPPORTED, OSP_ERR_DIVISIBILITY, OSP_ERR_CUDA. */
+int osp_skiparse_attn(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                      int32_t sparse_k, int32_t mode, float softmax_scale, void* stream);
+
+/* Skiparse index map: dev_out[g*(n_video/k) + s] = token(g, s), int32, device, n_video entries.
+ *  Errors: OSP_ERR_INVALID_ARG, OSP_ERR_DIVISIBILITY, OSP_ERR_CUDA. */
+int osp_skiparse_index_map(int32_t n_video, int32_t sparse_k, int32_t mode, int32_t* dev_out,
+                           void* stream);
+
+/* Synchronises `stream`, then reads and clears this device's status word.
+ * Returns OSP_OK, OSP_ERR_TIMEOUT (a kernel's bounded wait gave up; its output is invalid),
+ * OSP_ERR_BOUNDS, or OSP_ERR_CUDA (the synchronisation itself failed). */
+int osp_check_status(void* stream);
+
+/* Message for the last non-zero return on the calling thread ("" if none). The pointer stays
+ * valid until the next call on the same thread. */
+const char* osp_get_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int osp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OSP_H_ */

@@ -1,0 +1,465 @@
+// Flash-style attention forward for sm_100a on tcgen05 tensor cores.
+//
+// Computes, per (sample b, head h, token set g), O = softmax(Q K^T * scale) V over the set's n
+// tokens: the whole sequence for 3D full attention ("CogVideoX" section 2.2 "3D Full
+// Attention"), or one Skiparse set ("Open-Sora Plan" section 2.2.2).  The Skiparse sets are
+// folded into the TMA tensor maps: a Single Skip set is a strided view of the token axis and a
+// Group Skip set a 2-level view, so the k-fold permuted tensor never exists in memory.
+//
+// CTA = 2 query tiles of 128 rows sharing one K/V stream (320 threads):
+//   warps 0-3  softmax for query tile 0 (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax for query tile 1
+//   warp 8     TMA producer: Q once, then K/V tiles into a ring of shared-memory stages
+//   warp 9     tensor-memory allocator and MMA issuer (one elected thread)
+// Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1 [128,256) fp32 scores,
+// O0 [256, 256+D), O1 [384, 384+D) fp32 output accumulators.  The softmax overwrites the first
+// 64 columns of S_i with P_i in bf16 pairs, and the PV product reads P_i from tensor memory as
+// its A operand, so probabilities never touch shared memory.
+// MMA issue order per KV tile j: PV0(j), S0(j+1), PV1(j), S1(j+1): while one softmax group
+// works on its scores the tensor core runs the other group's two products.
+// Online softmax keeps a per-row running max m and sum l in registers; O is rescaled only when
+// the max grows by more than 2^8 (the final O/l uses the same stale max on both sides, so the
+// result is exact), which removes most TMEM round trips of O.
+// Every mbarrier wait is bounded: on timeout the CTA raises a shared abort flag, records
+// kDevTimeout in the device status word, drains its in-flight TMA loads and MMAs, frees its
+// tensor memory and exits.
+
+#include <cuda.h>
+
+#include "osp_internal.h"
+
+namespace osp {
+namespace {
+
+constexpr int kBM = 128;               // query rows per tile
+constexpr int kBN = 128;               // keys per KV tile
+constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 channels (one 128-byte swizzle atom wide)
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = (D + 63) / 64;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
+  // o_full[2], mma_done
+  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+};
+
+struct AttnParams {
+  int n;          // tokens per set (query rows = key rows)
+  int N;          // tokens per sample in the natural-order tensors
+  int heads;
+  int G;          // sets per sample
+  int k;          // sparse ratio (1 for dense)
+  int layout;     // 0 dense, 1 Single Skip, 2 Group Skip
+  float scale_log2;
+  __nv_bfloat16* o;
+  unsigned* status;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
+                                          int chan, int row0, int g, int b, int k) {
+  if (layout == 0) tma_load_3d(dst, tm, bar, chan, row0, b);
+  else if (layout == 1) tma_load_4d(dst, tm, bar, chan, g, row0, b);
+  else tma_load_5d(dst, tm, bar, chan, 0, g, row0 / k, b);
+}
+
+// Natural token index of slot s of set g.
+__device__ __forceinline__ int slot_token(int layout, int s, int g, int k) {
+  if (layout == 0) return s;
+  if (layout == 1) return s * k + g;
+  const int o = s / k;
+  return (o * k + g) * k + (s - o * k);
+}
+
+// Warp-uniform bounded wait (tcgen05.ld/st that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  const bool ok = mbar_wait(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = Cfg<D>;
+  constexpr int S = C::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + S, B_VFULL = 1 + 2 * S, B_VEMPTY = 1 + 3 * S;
+  const int B_SFULL = 1 + 4 * S, B_PREADY = B_SFULL + 2, B_OFULL = B_PREADY + 2, B_MMADONE = B_OFULL + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z / p.G, g = blockIdx.z % p.G;
+  const int q0 = blockIdx.x * (2 * kBM);
+  const int n_kv = (p.n + kBN - 1) / kBN;
+  const int chan0 = h * D;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_QFULL), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_SFULL + i), 1);
+      mbar_init(bar(B_PREADY + i), 128);
+      mbar_init(bar(B_OFULL + i), 1);
+    }
+    mbar_init(bar(B_MMADONE), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+
+  auto sQ = [&](int i) { return sbase + C::kQOff + (uint32_t)(i * C::kTileBytes); };
+  auto sK = [&](int s) { return sbase + C::kKOff + (uint32_t)(s * C::kTileBytes); };
+  auto sV = [&](int s) { return sbase + C::kVOff + (uint32_t)(s * C::kTileBytes); };
+  auto colS = [](int i) { return i ? 128u : 0u; };
+  auto colO = [](int i) { return i ? 384u : 256u; };
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
+      mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
+      for (int i = 0; i < 2; ++i)
+        for (int c = 0; c < C::kChunks; ++c)
+          load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, q0 + i * kBM, g, b,
+                    p.k);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % S, u = j / S;
+        if (j >= S && !mbar_wait(bar(B_KEMPTY + s), (u - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
+                    p.k);
+        k_issued = j + 1;
+        if (j >= S && !mbar_wait(bar(B_VEMPTY + s), (u - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
+                    p.k);
+        v_issued = j + 1;
+      }
+      // Drain: every load this thread issued has landed before the CTA may exit.  Only the
+      // last S tiles of each ring can still be in flight.
+      mbar_drain(bar(B_QFULL), 0, p.timeout_ns);
+      for (int t = (k_issued > S ? k_issued - S : 0); t < k_issued; ++t)
+        mbar_drain(bar(B_KFULL + t % S), (t / S) & 1, p.timeout_ns);
+      for (int t = (v_issued > S ? v_issued - S : 0); t < v_issued; ++t)
+        mbar_drain(bar(B_VFULL + t % S), (t / S) & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      // S_i = Q_i K^T: both operands K-major (channels contiguous), 16 channels per MMA.
+      auto issue_s = [&](int i, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * kChunkBytes + (kk & 3) * 32);
+          mma_ss(tmem + colS(i), sdesc_sw128(sQ(i) + off, 16, 1024), sdesc_sw128(sK(s) + off, 16, 1024),
+                 idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_i += P_i V: P_i from tensor memory (bf16 pairs in S_i's first 64 columns), V MN-major
+      // (channels contiguous), 16 keys per MMA.
+      auto issue_pv = [&](int i, int s, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tmem + colO(i), tmem + colS(i) + 8u * kk, sdesc_sw128(sV(s) + 2048u * kk, kChunkBytes, 1024),
+                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(B_QFULL), 0, wc) && mbar_wait(bar(B_KFULL), 0, wc);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        tc_commit(bar(B_SFULL + 0));
+        issue_s(1, 0);
+        tc_commit(bar(B_SFULL + 1));
+        tc_commit(bar(B_KEMPTY + 0));
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j % S, u = j / S;
+          const bool more = j + 1 < n_kv;
+          const int s1 = (j + 1) % S, u1 = (j + 1) / S;
+          if (!mbar_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          if (more && !mbar_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
+          if (!mbar_wait(bar(B_PREADY + 0), j & 1, wc)) break;
+          tc_fence_after();
+          issue_pv(0, s, j > 0);
+          if (more) {
+            issue_s(0, s1);
+            tc_commit(bar(B_SFULL + 0));
+          } else {
+            tc_commit(bar(B_OFULL + 0));
+          }
+          if (!mbar_wait(bar(B_PREADY + 1), j & 1, wc)) break;
+          tc_fence_after();
+          issue_pv(1, s, j > 0);
+          tc_commit(bar(B_VEMPTY + s));
+          if (more) {
+            issue_s(1, s1);
+            tc_commit(bar(B_SFULL + 1));
+            tc_commit(bar(B_KEMPTY + s1));
+          } else {
+            tc_commit(bar(B_OFULL + 1));
+          }
+        }
+      }
+      // Drain: all issued MMAs complete before tensor memory is freed.
+      tc_commit(bar(B_MMADONE));
+      mbar_drain(bar(B_MMADONE), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int i = warp >> 2;                       // query tile
+    const int quarter = warp & 3;                  // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;           // row within the tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + colS(i);
+    const uint32_t tO = tmem + lane_base + colO(i);
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!warp_wait(bar(B_SFULL + i), j & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      float sv[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
+      const int valid = p.n - j * kBN;
+      if (valid < kBN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) sv[c] = -INFINITY;
+      }
+      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, sv[c]);
+        mx1 = fmaxf(mx1, sv[c + 1]);
+        mx2 = fmaxf(mx2, sv[c + 2]);
+        mx3 = fmaxf(mx3, sv[c + 3]);
+      }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_cand = fmaxf(m, mx);
+      const bool rescale = m_cand > m + kRescaleThreshold;
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx(m - m_cand);
+        m = m_cand;
+      }
+      const float neg_m = -m;
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float e0 = ex2_approx(fmaf(sv[64 * half + 2 * c], sl2, neg_m));
+          const float e1 = ex2_approx(fmaf(sv[64 * half + 2 * c + 1], sl2, neg_m));
+          rs0 += e0;
+          rs1 += e1;
+          pk[c] = pack_bf16x2(e0, e1);
+        }
+        tmem_st32(tS + 32 * half, pk);
+      }
+      l = l * alpha + (rs0 + rs1);
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * cc, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PREADY + i));
+    }
+    if (ok && warp_wait(bar(B_OFULL + i), 0, wc)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const int slot = q0 + i * kBM + row;
+      const bool live = slot < p.n;
+      const int token = slot_token(p.layout, live ? slot : 0, g, p.k);
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N + token) * p.heads + h) * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * cc, o);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        if (live) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[4 * cc + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map over a BSHD [B][N][heads][D] bf16 tensor, viewed per `layout`:
+//   dense:  (heads*D, N, B)                    box (64, 128, 1)
+//   single: (heads*D, k, N/k, B)               box (64, 1, 128, 1)   token = s*k + g
+//   group:  (heads*D, k, k, N/(k*k), B)         box (64, k, 1, 128/k, 1)  token = (o*k + g)*k + r
+// The channel axis merges heads and head_dim; a box starts at channel h*D + 64c.
+int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return set_error(OSP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t HD = (cuuint64_t)s.heads * s.head_dim;
+  const cuuint64_t row = HD * 2;  // bytes per token
+  cuuint64_t dims[5], strides[4];
+  cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
+  cuuint32_t rank;
+  if (layout == 0) {
+    rank = 3;
+    dims[0] = HD; dims[1] = (cuuint64_t)N; dims[2] = (cuuint64_t)s.B;
+    strides[0] = row; strides[1] = row * N;
+    box[0] = 64; box[1] = kBM; box[2] = 1;
+  } else if (layout == 1) {
+    rank = 4;
+    dims[0] = HD; dims[1] = (cuuint64_t)k; dims[2] = (cuuint64_t)(N / k); dims[3] = (cuuint64_t)s.B;
+    strides[0] = row; strides[1] = row * k; strides[2] = row * N;
+    box[0] = 64; box[1] = 1; box[2] = kBM; box[3] = 1;
+  } else {
+    rank = 5;
+    dims[0] = HD; dims[1] = (cuuint64_t)k; dims[2] = (cuuint64_t)k; dims[3] = (cuuint64_t)(N / (k * k));
+    dims[4] = (cuuint64_t)s.B;
+    strides[0] = row; strides[1] = row * k; strides[2] = row * k * k; strides[3] = row * N;
+    box[0] = 64; box[1] = (cuuint32_t)k; box[2] = 1; box[3] = (cuuint32_t)(kBM / k); box[4] = 1;
+  }
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(OSP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return OSP_OK;
+}
+
+template <int D>
+int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+             dim3 grid, cudaStream_t stream) {
+  constexpr int smem = Cfg<D>::kSmemBytes;
+  static bool attr_done = false;  // per process; the attribute is per function, not per device
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_fwd_kernel<%d>) failed", D);
+    attr_done = true;
+  }
+  attn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  return check_launch("attn_fwd_kernel");
+}
+
+}  // namespace
+
+int attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
+                     int sparse_k, float scale, cudaStream_t stream) {
+  const int N = s.text_len + s.T * s.H * s.W;
+  const int G = (layout == 0) ? 1 : sparse_k;
+  const int n = N / G;
+  AttnParams p{};
+  p.n = n;
+  p.N = N;
+  p.heads = s.heads;
+  p.G = G;
+  p.k = (layout == 0) ? 1 : sparse_k;
+  p.layout = layout;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.status = device_status_word();
+  if (!p.status) return OSP_ERR_CUDA;
+  p.timeout_ns = wait_timeout_ns();
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap(&tq, q, s, N, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tk, k, s, N, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tv, v, s, N, layout, p.k)) != OSP_OK) return rc;
+  const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
+  if ((long long)s.B * G > 65535 || s.heads > 65535)
+    return set_error(OSP_ERR_UNSUPPORTED, "B*sets (%lld) or heads (%d) exceeds the grid limit 65535",
+                     (long long)s.B * G, s.heads);
+  dim3 grid((unsigned)qblocks, (unsigned)s.heads, (unsigned)(s.B * G));
+  switch (s.head_dim) {
+    case 64: return launch_d<64>(tq, tk, tv, p, grid, stream);
+    case 96: return launch_d<96>(tq, tk, tv, p, grid, stream);
+    case 128: return launch_d<128>(tq, tk, tv, p, grid, stream);
+    default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  }
+}
+
+}  // namespace osp

@@ -1,0 +1,240 @@
+// C entry points of libosp.so: argument validation, error reporting and dispatch to the
+// kernels.  Every check here runs on the host before anything is enqueued.
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "osp_internal.h"
+
+namespace osp {
+
+namespace {
+thread_local char g_last_error[512] = "";
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned* g_status[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int check_shape(const osp_shape* s, bool attention) {
+  if (!s) return set_error(OSP_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 1 || s->text_len < 0 || s->T < 1 || s->H < 1 || s->W < 1 || s->heads < 1 || s->head_dim < 2)
+    return set_error(OSP_ERR_INVALID_ARG, "bad shape: B=%d text_len=%d T=%d H=%d W=%d heads=%d head_dim=%d", s->B,
+                     s->text_len, s->T, s->H, s->W, s->heads, s->head_dim);
+  if (s->head_dim % 8)
+    return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d is not a multiple of 8", s->head_dim);
+  const long long n = (long long)s->text_len + (long long)s->T * s->H * s->W;
+  if (n > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "sequence length %lld too large", n);
+  if (attention && s->head_dim != 64 && s->head_dim != 96 && s->head_dim != 128)
+    return set_error(OSP_ERR_UNSUPPORTED, "attention head_dim %d not in {64, 96, 128}", s->head_dim);
+  return OSP_OK;
+}
+
+int check_rope(const osp_rope* r, int head_dim) {
+  if (!r) return set_error(OSP_ERR_INVALID_ARG, "rope is NULL");
+  if (r->d_t < 0 || r->d_h < 0 || r->d_w < 0 || (r->d_t | r->d_h | r->d_w) & 1)
+    return set_error(OSP_ERR_INVALID_ARG, "RoPE chunks must be even and >= 0 (got %d/%d/%d)", r->d_t, r->d_h,
+                     r->d_w);
+  if (r->d_t + r->d_h + r->d_w != head_dim)
+    return set_error(OSP_ERR_INVALID_ARG, "RoPE split %d/%d/%d does not sum to head_dim %d", r->d_t, r->d_h,
+                     r->d_w, head_dim);
+  if (!(r->theta > 0.0) || !std::isfinite(r->theta))
+    return set_error(OSP_ERR_INVALID_ARG, "RoPE theta must be finite and > 0");
+  if (head_dim > 256) return set_error(OSP_ERR_UNSUPPORTED, "RoPE head_dim %d > 256", head_dim);
+  return OSP_OK;
+}
+
+int check_skiparse(const osp_shape* s, int k, int mode) {
+  if (k < 1) return set_error(OSP_ERR_INVALID_ARG, "sparse ratio k=%d < 1", k);
+  if (mode != OSP_SKIP_SINGLE && mode != OSP_SKIP_GROUP)
+    return set_error(OSP_ERR_INVALID_ARG, "mode %d is neither OSP_SKIP_SINGLE nor OSP_SKIP_GROUP", mode);
+  if (s->text_len != 0)
+    return set_error(OSP_ERR_UNSUPPORTED, "Skiparse with text tokens (text_len=%d) is not supported", s->text_len);
+  const long long nv = (long long)s->T * s->H * s->W;
+  const long long step = (mode == OSP_SKIP_SINGLE) ? k : (long long)k * k;
+  if (nv % step)
+    return set_error(OSP_ERR_DIVISIBILITY, "T*H*W=%lld is not a multiple of %lld", nv, step);
+  return OSP_OK;
+}
+}  // namespace
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(OSP_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return OSP_OK;
+}
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_sms[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sms[dev] = n > 0 ? n : 148;
+  }
+  return g_sms[dev];
+}
+
+unsigned* device_status_word() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_error(OSP_ERR_CUDA, "no current CUDA device");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status[dev]) {
+    void* p = nullptr;
+    if (cudaMalloc(&p, 256) != cudaSuccess || cudaMemset(p, 0, 256) != cudaSuccess) {
+      set_error(OSP_ERR_CUDA, "status word allocation failed");
+      return nullptr;
+    }
+    g_status[dev] = static_cast<unsigned*>(p);
+  }
+  return g_status[dev];
+}
+
+uint64_t wait_timeout_ns() {
+  static const uint64_t ns = [] {
+    const char* e = getenv("OSP_WAIT_TIMEOUT_MS");
+    const long long ms = e ? atoll(e) : 2000;
+    return (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
+  }();
+  return ns;
+}
+
+}  // namespace osp
+
+using namespace osp;
+
+extern "C" {
+
+const char* osp_get_last_error(void) { return g_last_error; }
+
+int osp_version(void) { return 100; }
+
+int osp_rope3d(const void* q, const void* k, void* q_out, void* k_out, const osp_shape* shape, const osp_rope* rope,
+               void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, false);
+  if (rc) return rc;
+  if ((rc = check_rope(rope, shape->head_dim))) return rc;
+  if (!q || !k || !q_out || !k_out) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return rope3d_launch(q, k, q_out, k_out, *shape, *rope, static_cast<cudaStream_t>(stream));
+}
+
+int osp_attn_full(const void* q, const void* k, const void* v, void* o, const osp_shape* shape, float softmax_scale,
+                  void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_launch(q, k, v, o, *shape, 0, 1, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+int osp_skiparse_gather(const void* q, const void* k, const void* v, void* q_out, void* k_out, void* v_out,
+                        const osp_shape* shape, int32_t sparse_k, int32_t mode, const osp_rope* rope, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, false);
+  if (rc) return rc;
+  if ((rc = check_skiparse(shape, sparse_k, mode))) return rc;
+  if (rope && (rc = check_rope(rope, shape->head_dim))) return rc;
+  if (!q || !q_out) return set_error(OSP_ERR_INVALID_ARG, "q and q_out must not be NULL");
+  if ((!k) != (!k_out) || (!v) != (!v_out))
+    return set_error(OSP_ERR_INVALID_ARG, "k/k_out and v/v_out must be both set or both NULL");
+  const void* src[3];
+  void* dst[3];
+  int n = 0;
+  src[n] = q; dst[n++] = q_out;
+  if (k) { src[n] = k; dst[n++] = k_out; }
+  if (v) { src[n] = v; dst[n++] = v_out; }
+  for (int i = 0; i < n; ++i)
+    if (!aligned16(src[i]) || !aligned16(dst[i]))
+      return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  // RoPE applies to q and k only; with k omitted, v (if given) must not be rotated.
+  if (rope && !k && v) {
+    rc = skiparse_gather_launch(src, dst, 1, *shape, sparse_k, mode, rope, static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+    const void* s2[3] = {v, nullptr, nullptr};
+    void* d2[3] = {v_out, nullptr, nullptr};
+    return skiparse_gather_launch(s2, d2, 1, *shape, sparse_k, mode, nullptr, static_cast<cudaStream_t>(stream));
+  }
+  return skiparse_gather_launch(src, dst, n, *shape, sparse_k, mode, rope, static_cast<cudaStream_t>(stream));
+}
+
+int osp_skiparse_scatter(const void* o_perm, void* o, const osp_shape* shape, int32_t sparse_k, int32_t mode,
+                         void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, false);
+  if (rc) return rc;
+  if ((rc = check_skiparse(shape, sparse_k, mode))) return rc;
+  if (!o_perm || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(o_perm) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return skiparse_scatter_launch(o_perm, o, *shape, sparse_k, mode, static_cast<cudaStream_t>(stream));
+}
+
+int osp_skiparse_attn(const void* q, const void* k, const void* v, void* o, const osp_shape* shape, int32_t sparse_k,
+                      int32_t mode, float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if ((rc = check_skiparse(shape, sparse_k, mode))) return rc;
+  if (mode == OSP_SKIP_GROUP && (sparse_k > 128 || (128 % sparse_k) != 0))
+    return set_error(OSP_ERR_UNSUPPORTED, "fused Group Skip needs k to divide 128 (got k=%d)", sparse_k);
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  const int layout = (sparse_k == 1) ? 0 : (mode == OSP_SKIP_SINGLE ? 1 : 2);
+  return attention_launch(q, k, v, o, *shape, layout, sparse_k, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+int osp_skiparse_index_map(int32_t n_video, int32_t sparse_k, int32_t mode, int32_t* dev_out, void* stream) {
+  g_last_error[0] = 0;
+  if (n_video < 1) return set_error(OSP_ERR_INVALID_ARG, "n_video=%d < 1", n_video);
+  if (!dev_out) return set_error(OSP_ERR_INVALID_ARG, "dev_out is NULL");
+  osp_shape s{1, 0, 1, 1, n_video, 1, 8};
+  int rc = check_skiparse(&s, sparse_k, mode);
+  if (rc) return rc;
+  return index_map_launch(n_video, sparse_k, mode, dev_out, static_cast<cudaStream_t>(stream));
+}
+
+int osp_check_status(void* stream) {
+  g_last_error[0] = 0;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return set_error(OSP_ERR_CUDA, "stream synchronize failed: %s", cudaGetErrorString(e));
+  unsigned* w = device_status_word();
+  if (!w) return OSP_ERR_CUDA;
+  unsigned h = 0;
+  if (cudaMemcpy(&h, w, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemset(w, 0, sizeof(unsigned)) != cudaSuccess)
+    return set_error(OSP_ERR_CUDA, "status word read failed");
+  if (h & kDevTimeout) return set_error(OSP_ERR_TIMEOUT, "a device-side bounded wait timed out");
+  if (h & kDevBounds) return set_error(OSP_ERR_BOUNDS, "a device-side index check failed");
+  return OSP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,42 @@
+// Internal declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/osp.h"
+#include "osp_device.cuh"
+
+namespace osp {
+
+// Sets the calling thread's last-error message; returns `code`.
+int set_error(int code, const char* fmt, ...);
+
+// OSP_ERR_CUDA with the kernel's name if the last launch failed, else OSP_OK.
+int check_launch(const char* what);
+
+// SM count of the current device (cached per device).
+int device_sm_count();
+
+// Per-device status word (allocated on first use, kept until exit).
+unsigned* device_status_word();
+
+// Bounded-wait limit for the attention kernels, in nanoseconds.
+uint64_t wait_timeout_ns();
+
+int rope3d_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_shape& s,
+                  const osp_rope& rope, cudaStream_t stream);
+int skiparse_gather_launch(const void* const src[3], void* const dst[3], int n_tensors, const osp_shape& s,
+                           int k, int mode, const osp_rope* rope, cudaStream_t stream);
+int skiparse_scatter_launch(const void* o_perm, void* o, const osp_shape& s, int k, int mode,
+                            cudaStream_t stream);
+int index_map_launch(int n_video, int k, int mode, int32_t* out, cudaStream_t stream);
+
+// Attention over `G` token sets per sample (G = 1: dense over all N tokens; G = k: Skiparse).
+//   layout: 0 dense, OSP_SKIP_SINGLE + 1, OSP_SKIP_GROUP + 1
+int attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
+                     int sparse_k, float scale, cudaStream_t stream);
+
+}  // namespace osp

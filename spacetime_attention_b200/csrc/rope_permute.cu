@@ -1,0 +1,280 @@
+// 3D RoPE and the Skiparse k-fold permutation (gather / scatter), fused into one streaming
+// kernel, plus the Skiparse index-map kernel.
+//
+// Sources: "CogVideoX: Text-to-Video Diffusion Models with an Expert Transformer" section 2.2
+// "3D-RoPE" (one 1D RoPE per axis on its own channel share, concatenated) and section 3.1
+// (raw integer positions, extrapolated); RoFormer for the pairwise rotation with frequencies
+// theta^(-2j/d_axis); "Open-Sora Plan" section 2.2.2 for the Skiparse sets and the k-fold batch.
+//
+// Work decomposition: a CTA owns a tile of whole token rows (heads * head_dim contiguous bf16,
+// 1-8 KB each), so every load and store is a coalesced 16-byte vector.  Per tile it first
+// computes each row's source/destination row and (t, h, w) position, then one cos/sin pair
+// per (row, channel pair) into shared memory, then streams the rows of every tensor.
+
+#include "osp_internal.h"
+
+namespace osp {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxPairs = 128;   // head_dim <= 256
+
+enum MapKind { kMapIdentity = 0, kMapGather = 1, kMapScatter = 2 };
+
+struct PermuteParams {
+  const uint4* src[3];
+  uint4* dst[3];
+  int n_tensors;
+  unsigned rope_mask;      // bit i: rotate tensor i
+  long long rows;          // rows to process (per tensor)
+  int vpr;                 // 16-byte vectors per row = heads * head_dim / 8
+  int head_dim;
+  int N;                   // tokens per sample in the natural-order tensor
+  int text_len;
+  int H, W;
+  int sparse_k, mode;      // Skiparse (gather / scatter only)
+  int d_t, d_h, d_w;
+  double log2_theta;
+  int rows_per_tile;
+  long long n_tiles;
+};
+
+// Token index of slot s of set g (Open-Sora Plan section 2.2.2; reading in osp.h).
+__device__ __forceinline__ int skiparse_token(int g, int s, int k, int mode) {
+  if (mode == OSP_SKIP_SINGLE) return s * k + g;
+  const int o = s / k, r = s - o * k;
+  return (o * k + g) * k + r;
+}
+
+template <int MAP>
+__global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* omega = reinterpret_cast<double*>(smem_raw);                       // [head_dim/2]
+  long long* src_row = reinterpret_cast<long long*>(omega + kMaxPairs);      // [rows_per_tile]
+  long long* dst_row = src_row + p.rows_per_tile;                            // [rows_per_tile]
+  int* vid = reinterpret_cast<int*>(dst_row + p.rows_per_tile);              // video index or -1
+  float2* cs = reinterpret_cast<float2*>(vid + ((p.rows_per_tile + 3) & ~3)); // [tile][pairs]
+
+  const int npairs = p.head_dim >> 1;
+  // Frequencies of every channel pair: pair j of a chunk of size d_a -> theta^(-2j/d_a).
+  for (int i = threadIdx.x; i < npairs; i += kThreads) {
+    const int c = 2 * i;
+    int j, da;
+    if (c < p.d_t) { j = i; da = p.d_t; }
+    else if (c < p.d_t + p.d_h) { j = i - p.d_t / 2; da = p.d_h; }
+    else { j = i - (p.d_t + p.d_h) / 2; da = p.d_w; }
+    omega[i] = exp2(-(2.0 * j / da) * p.log2_theta);
+  }
+  const int HW = p.H * p.W;
+  const int per_set = (MAP == kMapIdentity) ? 0 : p.N / p.sparse_k;
+
+  for (long long tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+    __syncthreads();  // previous tile's table fully consumed (and omega ready on the first pass)
+    const long long row0 = tile * p.rows_per_tile;
+    const int nrows = (int)min((long long)p.rows_per_tile, p.rows - row0);
+    for (int i = threadIdx.x; i < nrows; i += kThreads) {
+      const long long r = row0 + i;
+      long long s_row, d_row;
+      int token;
+      if (MAP == kMapIdentity) {
+        s_row = d_row = r;
+        token = (int)(r % p.N);
+      } else {
+        const long long bk = r / per_set;           // b*k + g
+        const int s = (int)(r - bk * per_set);
+        const int g = (int)(bk % p.sparse_k);
+        const long long b = bk / p.sparse_k;
+        token = skiparse_token(g, s, p.sparse_k, p.mode);
+        if (MAP == kMapGather) { s_row = b * p.N + token; d_row = r; }
+        else { s_row = r; d_row = b * p.N + token; }
+      }
+      src_row[i] = s_row;
+      dst_row[i] = d_row;
+      vid[i] = token - p.text_len;  // < 0 for text tokens
+    }
+    __syncthreads();
+    if (p.rope_mask) {
+      for (int idx = threadIdx.x; idx < nrows * npairs; idx += kThreads) {
+        const int i = idx / npairs, pr = idx - i * npairs;
+        const int v = vid[i];
+        float2 c_s = make_float2(1.f, 0.f);
+        if (v >= 0) {
+          const int c = 2 * pr;
+          int pos;
+          if (c < p.d_t) pos = v / HW;
+          else if (c < p.d_t + p.d_h) pos = (v / p.W) % p.H;
+          else pos = v % p.W;
+          float sn, cn;
+          sincosf((float)((double)pos * omega[pr]), &sn, &cn);
+          c_s = make_float2(cn, sn);
+        }
+        cs[idx] = c_s;
+      }
+      __syncthreads();
+    }
+    const int per_head_vec = p.head_dim >> 3;
+    for (int t = 0; t < p.n_tensors; ++t) {
+      const uint4* __restrict__ src = p.src[t];
+      uint4* dst = p.dst[t];
+      const bool rot = (p.rope_mask >> t) & 1u;
+      const bool inplace = (const void*)src == (const void*)dst;
+      const int total = nrows * p.vpr;
+      // 4 independent vectors in flight per thread
+      for (int base = threadIdx.x; base < total; base += 4 * kThreads) {
+        uint4 val[4];
+        int rowi[4], col[4];
+        bool live[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = base + u * kThreads;
+          live[u] = idx < total;
+          rowi[u] = live[u] ? idx / p.vpr : 0;
+          col[u] = live[u] ? idx - rowi[u] * p.vpr : 0;
+          if (live[u] && inplace && vid[rowi[u]] < 0) live[u] = false;  // text row, in place
+          if (live[u]) val[u] = src[src_row[rowi[u]] * p.vpr + col[u]];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (!live[u]) continue;
+          if (rot && vid[rowi[u]] >= 0) {
+            const int pair0 = (col[u] % per_head_vec) * 4;
+            const float2* tab = cs + rowi[u] * npairs + pair0;
+            uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x = __uint_as_float(w[e] << 16);
+              const float y = __uint_as_float(w[e] & 0xFFFF0000u);
+              const float2 c_s = tab[e];
+              const float xr = x * c_s.x - y * c_s.y;
+              const float yr = x * c_s.y + y * c_s.x;
+              w[e] = pack_bf16x2(xr, yr);
+            }
+            val[u] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          dst[dst_row[rowi[u]] * p.vpr + col[u]] = val[u];
+        }
+      }
+    }
+  }
+}
+
+__global__ void index_map_kernel(int n_video, int k, int mode, int* out) {
+  const int per_set = n_video / k;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_video; i += gridDim.x * blockDim.x) {
+    const int g = i / per_set, s = i - g * per_set;
+    out[i] = skiparse_token(g, s, k, mode);
+  }
+}
+
+int launch_permute(int map, PermuteParams& p, cudaStream_t stream) {
+  const int npairs = p.head_dim / 2;
+  p.rows_per_tile = (int)std::max(1, std::min(32, (1024 + p.vpr - 1) / p.vpr));
+  p.n_tiles = (p.rows + p.rows_per_tile - 1) / p.rows_per_tile;
+  const size_t smem = kMaxPairs * sizeof(double) + 2 * p.rows_per_tile * sizeof(long long) +
+                      ((p.rows_per_tile + 3) & ~3) * sizeof(int) +
+                      (size_t)p.rows_per_tile * npairs * sizeof(float2);
+  const int sms = device_sm_count();
+  const long long grid = std::min<long long>(p.n_tiles, (long long)sms * 8);
+  if (grid <= 0) return OSP_OK;
+  switch (map) {
+    case kMapIdentity:
+      permute_rope_kernel<kMapIdentity><<<(unsigned)grid, kThreads, smem, stream>>>(p);
+      break;
+    case kMapGather:
+      permute_rope_kernel<kMapGather><<<(unsigned)grid, kThreads, smem, stream>>>(p);
+      break;
+    default:
+      permute_rope_kernel<kMapScatter><<<(unsigned)grid, kThreads, smem, stream>>>(p);
+      break;
+  }
+  return check_launch("permute_rope_kernel");
+}
+
+void fill_rope(PermuteParams& p, const osp_rope* rope) {
+  if (rope) {
+    p.d_t = rope->d_t;
+    p.d_h = rope->d_h;
+    p.d_w = rope->d_w;
+    p.log2_theta = std::log2(rope->theta);
+  } else {
+    p.d_t = p.head_dim;
+    p.d_h = p.d_w = 0;
+    p.log2_theta = 0.0;
+  }
+}
+
+}  // namespace
+
+int rope3d_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_shape& s,
+                  const osp_rope& rope, cudaStream_t stream) {
+  PermuteParams p{};
+  p.src[0] = static_cast<const uint4*>(q);
+  p.dst[0] = static_cast<uint4*>(q_out);
+  p.src[1] = static_cast<const uint4*>(k);
+  p.dst[1] = static_cast<uint4*>(k_out);
+  p.n_tensors = 2;
+  p.rope_mask = 3u;
+  p.head_dim = s.head_dim;
+  p.N = s.text_len + s.T * s.H * s.W;
+  p.rows = (long long)s.B * p.N;
+  p.vpr = s.heads * s.head_dim / 8;
+  p.text_len = s.text_len;
+  p.H = s.H;
+  p.W = s.W;
+  p.sparse_k = 1;
+  p.mode = 0;
+  fill_rope(p, &rope);
+  return launch_permute(kMapIdentity, p, stream);
+}
+
+int skiparse_gather_launch(const void* const src[3], void* const dst[3], int n_tensors, const osp_shape& s,
+                           int k, int mode, const osp_rope* rope, cudaStream_t stream) {
+  PermuteParams p{};
+  for (int i = 0; i < n_tensors; ++i) {
+    p.src[i] = static_cast<const uint4*>(src[i]);
+    p.dst[i] = static_cast<uint4*>(dst[i]);
+  }
+  p.n_tensors = n_tensors;
+  p.rope_mask = rope ? (n_tensors >= 2 ? 3u : 1u) : 0u;
+  p.head_dim = s.head_dim;
+  p.N = s.T * s.H * s.W;
+  p.rows = (long long)s.B * p.N;
+  p.vpr = s.heads * s.head_dim / 8;
+  p.text_len = 0;
+  p.H = s.H;
+  p.W = s.W;
+  p.sparse_k = k;
+  p.mode = mode;
+  fill_rope(p, rope);
+  return launch_permute(kMapGather, p, stream);
+}
+
+int skiparse_scatter_launch(const void* o_perm, void* o, const osp_shape& s, int k, int mode,
+                            cudaStream_t stream) {
+  PermuteParams p{};
+  p.src[0] = static_cast<const uint4*>(o_perm);
+  p.dst[0] = static_cast<uint4*>(o);
+  p.n_tensors = 1;
+  p.rope_mask = 0u;
+  p.head_dim = s.head_dim;
+  p.N = s.T * s.H * s.W;
+  p.rows = (long long)s.B * p.N;
+  p.vpr = s.heads * s.head_dim / 8;
+  p.text_len = 0;
+  p.H = s.H;
+  p.W = s.W;
+  p.sparse_k = k;
+  p.mode = mode;
+  fill_rope(p, nullptr);
+  return launch_permute(kMapScatter, p, stream);
+}
+
+int index_map_launch(int n_video, int k, int mode, int32_t* out, cudaStream_t stream) {
+  const int threads = 256;
+  const int blocks = std::max(1, std::min((n_video + threads - 1) / threads, device_sm_count() * 4));
+  index_map_kernel<<<blocks, threads, 0, stream>>>(n_video, k, mode, out);
+  return check_launch("index_map_kernel");
+}
+
+}  // namespace osp

@@ -1,0 +1,195 @@
+"""ctypes binding over libosp.so (declared in include/osp.h).
+
+Argument marshalling only: every function takes torch CUDA tensors, checks dtype/layout/device,
+passes raw device pointers, the shape structs and the current CUDA stream to the C entry point
+of the same name, and raises on a non-zero status.  All computation happens in the library's
+CUDA kernels; there is no fallback of any kind.  If the library is missing or cannot be loaded,
+every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libosp.so")
+
+OSP_SKIP_SINGLE = 0
+OSP_SKIP_GROUP = 1
+
+STATUS_NAMES = {0: "OSP_OK", 1: "OSP_ERR_INVALID_ARG", 2: "OSP_ERR_UNSUPPORTED", 3: "OSP_ERR_DIVISIBILITY",
+                4: "OSP_ERR_CUDA", 5: "OSP_ERR_TIMEOUT", 6: "OSP_ERR_BOUNDS"}
+
+# Every symbol include/osp.h declares (tests check the library exports all of them).
+EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_scatter", "osp_skiparse_attn",
+            "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version")
+
+
+class OspShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("text_len", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("W", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32)]
+
+
+class OspRope(ctypes.Structure):
+    _fields_ = [("d_t", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_w", ctypes.c_int32),
+                ("theta", ctypes.c_double)]
+
+
+class OspError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} -> {STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libosp.so (once).  Raises if it is missing: there is no fallback path."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m spacetime_attention_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32, sp, rp = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(OspShape), ctypes.POINTER(OspRope)
+        sig = {
+            "osp_rope3d": [vp, vp, vp, vp, sp, rp, vp],
+            "osp_attn_full": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_skiparse_gather": [vp, vp, vp, vp, vp, vp, sp, i32, i32, rp, vp],
+            "osp_skiparse_scatter": [vp, vp, sp, i32, i32, vp],
+            "osp_skiparse_attn": [vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
+            "osp_skiparse_index_map": [i32, i32, i32, vp, vp],
+            "osp_check_status": [vp],
+            "osp_get_last_error": [],
+            "osp_version": [],
+        }
+        for name, args in sig.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = ctypes.c_char_p if name == "osp_get_last_error" else ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise OspError(fn, rc, library().osp_get_last_error().decode())
+
+
+def _stream_handle(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _bshd(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, N, heads, head_dim] tensor")
+
+
+def make_shape(B: int, text_len: int, grid: Sequence[int], heads: int, head_dim: int) -> OspShape:
+    T, H, W = (int(x) for x in grid)
+    return OspShape(int(B), int(text_len), T, H, W, int(heads), int(head_dim))
+
+
+def make_rope(split: Sequence[int], theta: float = 10000.0) -> OspRope:
+    d_t, d_h, d_w = (int(x) for x in split)
+    return OspRope(d_t, d_h, d_w, float(theta))
+
+
+def _shape_of(t: torch.Tensor, grid, text_len: int) -> OspShape:
+    B, N, heads, d = t.shape
+    return make_shape(B, text_len, grid, heads, d)
+
+
+def rope3d(q: torch.Tensor, k: torch.Tensor, grid, text_len: int, split, theta: float = 10000.0,
+           q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None):
+    """osp_rope3d: 3D RoPE of q and k; returns (q_out, k_out) (new tensors unless given)."""
+    _bshd(q, "q"); _bshd(k, "k")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    shp, rp = _shape_of(q, grid, text_len), make_rope(split, theta)
+    _check("osp_rope3d", library().osp_rope3d(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), ctypes.byref(shp),
+                                              ctypes.byref(rp), _stream_handle(q)))
+    return q_out, k_out
+
+
+def attn_full(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, scale: float = 0.0,
+              o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """osp_attn_full: dense 3D full attention over text_len + T*H*W tokens."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    shp = _shape_of(q, grid, text_len)
+    _check("osp_attn_full", library().osp_attn_full(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
+                                                    ctypes.c_float(scale), _stream_handle(q)))
+    return o
+
+
+def skiparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, sparse_k: int, mode: int,
+                  scale: float = 0.0, o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """osp_skiparse_attn: fused Skiparse attention in natural token order."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    shp = _shape_of(q, grid, 0)
+    _check("osp_skiparse_attn", library().osp_skiparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
+                                                            int(sparse_k), int(mode), ctypes.c_float(scale),
+                                                            _stream_handle(q)))
+    return o
+
+
+def skiparse_gather(q: torch.Tensor, k: Optional[torch.Tensor], v: Optional[torch.Tensor], grid, sparse_k: int,
+                    mode: int, split=None, theta: float = 10000.0):
+    """osp_skiparse_gather: returns (q_out, k_out, v_out) in the k-fold batch layout; RoPE on q, k
+    with the tokens' own positions when ``split`` is given."""
+    _bshd(q, "q")
+    B, N, heads, d = q.shape
+    outs = []
+    for t in (q, k, v):
+        outs.append(None if t is None else torch.empty((B * sparse_k, N // sparse_k, heads, d), dtype=t.dtype,
+                                                          device=t.device))
+    shp = _shape_of(q, grid, 0)
+    rp = make_rope(split, theta) if split is not None else None
+    _check("osp_skiparse_gather",
+           library().osp_skiparse_gather(_ptr(q), _ptr(k), _ptr(v), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
+                                         ctypes.byref(shp), int(sparse_k), int(mode),
+                                         ctypes.byref(rp) if rp is not None else None, _stream_handle(q)))
+    return tuple(outs)
+
+
+def skiparse_scatter(o_perm: torch.Tensor, grid, sparse_k: int, mode: int,
+                     o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """osp_skiparse_scatter: inverse of the gather for one tensor."""
+    _bshd(o_perm, "o_perm")
+    Bk, n_set, heads, d = o_perm.shape
+    B, N = Bk // sparse_k, n_set * sparse_k
+    o = torch.empty((B, N, heads, d), dtype=o_perm.dtype, device=o_perm.device) if o is None else o
+    shp = make_shape(B, 0, grid, heads, d)
+    _check("osp_skiparse_scatter", library().osp_skiparse_scatter(_ptr(o_perm), _ptr(o), ctypes.byref(shp),
+                                                                  int(sparse_k), int(mode), _stream_handle(o)))
+    return o
+
+
+def skiparse_index_map(n_video: int, sparse_k: int, mode: int, device="cuda") -> torch.Tensor:
+    """osp_skiparse_index_map: int32 [n_video] map, entry g*(n/k)+s = token of slot s of set g."""
+    out = torch.empty(n_video, dtype=torch.int32, device=device)
+    _check("osp_skiparse_index_map", library().osp_skiparse_index_map(int(n_video), int(sparse_k), int(mode),
+                                                                      _ptr(out), _stream_handle(out)))
+    return out
+
+
+def check_status(device=None) -> None:
+    """osp_check_status on the current stream: raises OspError on a device-side timeout."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check("osp_check_status", library().osp_check_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))

@@ -1,0 +1,95 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol include/osp.h declares,
+and rejects bad arguments on the host before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from spacetime_attention_b200 import build as B
+from spacetime_attention_b200 import ops
+
+HEADER = os.path.join(B.INCLUDE, "osp.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return ops.library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(osp_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for n in ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_scatter", "osp_skiparse_attn",
+              "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error"):
+        assert n in names
+    assert set(names) == set(ops.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+    assert lib.osp_version() >= 100
+
+
+def shp(B=1, L=0, T=4, H=8, W=8, heads=2, d=64):
+    return ctypes.byref(ops.OspShape(B, L, T, H, W, heads, d))
+
+
+def rc_msg(lib, rc):
+    return rc, lib.osp_get_last_error().decode()
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(B=0), 1), (dict(T=0), 1), (dict(heads=0), 1), (dict(L=-1), 1), (dict(d=80), 2), (dict(d=60), 2)])
+def test_attention_rejects_bad_shapes(lib, args, code):
+    p = ctypes.c_void_p(256)
+    rc, msg = rc_msg(lib, lib.osp_attn_full(p, p, p, p, shp(**args), 0.0, None))
+    assert rc == code and msg
+
+
+def test_rejects_null_and_misaligned(lib):
+    p, bad = ctypes.c_void_p(256), ctypes.c_void_p(258)
+    assert lib.osp_attn_full(None, p, p, p, shp(), 0.0, None) == 1
+    assert lib.osp_attn_full(p, p, bad, p, shp(), 0.0, None) == 1
+    assert "aligned" in lib.osp_get_last_error().decode()
+
+
+def test_rope_split_validation(lib):
+    p = ctypes.c_void_p(256)
+    for split, code in [((16, 24, 16), 1), ((15, 25, 24), 1), ((-2, 34, 32), 1)]:
+        r = ops.make_rope(split)
+        assert lib.osp_rope3d(p, p, p, p, shp(), ctypes.byref(r), None) == code
+    r = ops.make_rope((16, 24, 24), theta=0.0)
+    assert lib.osp_rope3d(p, p, p, p, shp(), ctypes.byref(r), None) == 1
+    assert lib.osp_rope3d(p, p, p, p, shp(), None, None) == 1
+
+
+def test_skiparse_validation(lib):
+    p = ctypes.c_void_p(256)
+    # text tokens with Skiparse -> unsupported
+    assert lib.osp_skiparse_attn(p, p, p, p, shp(L=3), 2, 0, 0.0, None) == 2
+    # 4*8*8 = 256 not divisible by 3 / by 9
+    assert lib.osp_skiparse_attn(p, p, p, p, shp(), 3, 0, 0.0, None) == 3
+    assert lib.osp_skiparse_gather(p, p, p, p, p, p, shp(T=3, H=3, W=3), 2, 1, None, None) == 3
+    # group needs k | 128 in the fused kernel
+    assert lib.osp_skiparse_attn(p, p, p, p, shp(T=9, H=6, W=6), 3, 1, 0.0, None) == 2
+    assert lib.osp_skiparse_attn(p, p, p, p, shp(), 0, 0, 0.0, None) == 1
+    assert lib.osp_skiparse_attn(p, p, p, p, shp(), 2, 7, 0.0, None) == 1
+    assert lib.osp_skiparse_index_map(10, 4, 0, p, None) == 3
+    assert lib.osp_skiparse_index_map(16, 2, 1, None, None) == 1
+    assert lib.osp_skiparse_gather(p, p, None, p, None, None, shp(), 2, 0, None, None) == 1  # k w/o k_out
+    assert lib.osp_skiparse_scatter(None, p, shp(), 2, 0, None) == 1
+
+
+def test_binding_refuses_non_cuda_tensors():
+    import torch
+    x = torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.attn_full(x, x, x, (4, 8, 8), 0)
