@@ -1,0 +1,418 @@
+"""Benchmark: attention TFLOP/s on one workload, as a fraction of B200 dense bf16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch of synthetic input: 3D RoPE of q and k
+(osp_rope3d) followed by attention (osp_attn_full for dense workloads; for Skiparse workloads
+osp_skiparse_attn, Single then Group Skip as an alternating pair).  The default workload is the
+CogVideoX-2B-shaped joint attention: B=1, 30 heads, head_dim 64, 13x30x45 video tokens after
+226 text tokens.  `value` counts attention flops (4*B*heads*Nq*Nkv*d, summed over sets) per
+second of the whole step (RoPE included), with q/k/v resident in HBM.
+
+N > 1 (one process per GPU, launched by torch.distributed.run): every rank runs its own
+independent copy of the workload (the (sample, head) units of attention share nothing), so
+per-GPU work is fixed ("weak" scaling) and the only collectives are the timing barrier and the
+max-over-ranks reduction.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0 only), on a
+bounded sample of the same workload per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from spacetime_attention_b200 import ops, synthetic as syn  # noqa: E402
+
+METRIC = "attention TFLOP/s and % of B200 BF16 tensor peak per config (1 GPU)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "osp_device.cuh"):
+        with open(os.path.join(ROOT, "spacetime_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith(" "):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+
+def step_fns(w, q, k, v, qr, kr, o, launch_events=None):
+    """Returns step() running one pass of the hot path (all launches on torch's current stream)."""
+    def attn():
+        if sparse(w):
+            ops.skiparse_attn(qr, kr, v, w.grid, w.skiparse_k, ops.OSP_SKIP_SINGLE, o=o)
+            ops.skiparse_attn(qr, kr, v, w.grid, w.skiparse_k, ops.OSP_SKIP_GROUP, o=o)
+        else:
+            ops.attn_full(qr, kr, v, w.grid, w.text_len, o=o)
+
+    def step():
+        ops.rope3d(q, k, w.grid, w.text_len, w.split, q_out=qr, k_out=kr)
+        if launch_events is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn()
+            e1.record()
+            launch_events.append((e0, e1))
+        else:
+            attn()
+    return step
+
+
+ATTN_MODE = {"value": "auto"}
+
+
+def sparse(w) -> bool:
+    """Skiparse pair (Single + Group) for workloads that define k, unless --attn dense."""
+    return bool(w.skiparse_k) and ATTN_MODE["value"] != "dense"
+
+
+def launches_per_step(w) -> int:
+    return 1 + (2 if sparse(w) else 1)
+
+
+def step_flops(w) -> float:
+    return 2 * w.skiparse_flops() if sparse(w) else w.dense_flops()
+
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = syn.WORKLOADS[args.workload]
+    q_h, k_h, v_h = syn.make_qkv(w, w.seed + 17 * rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    qr, kr, o = torch.empty_like(q), torch.empty_like(k), torch.empty_like(q)
+    step = step_fns(w, q, k, v, qr, kr, o)
+    for _ in range(args.warmup):
+        step()
+    ops.check_status(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    events = []
+    step_timed = step_fns(w, q, k, v, qr, kr, o, launch_events=events)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step_timed()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ops.check_status(dev)
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in events]))
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # ---- end to end through the public API: pinned host inputs -> device -> hot path -> host
+    qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
+    op = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    e2e_steps = max(3, min(20, args.steps))
+    stream = torch.cuda.current_stream(dev)
+
+    def e2e_step():
+        q.copy_(qp, non_blocking=True)
+        k.copy_(kp, non_blocking=True)
+        v.copy_(vp, non_blocking=True)
+        step()
+        op.copy_(o, non_blocking=True)
+
+    e2e_step()
+    stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    ops.check_status(dev)
+
+    flops = step_flops(w)
+    ms_step = ms_total / args.steps
+    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+    peaks, peaks_src = load_peaks()
+    # the attention kernels run back to back for the whole timed region: sustained peak
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    traffic = profiled_traffic(w.name)
+    in_bytes = 3 * q.numel() * q.element_size()
+    out_bytes = o.numel() * o.element_size()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(w.describe(), ops=("rope3d+skiparse_single+skiparse_group" if sparse(w)
+                                          else "rope3d+attn_full"),
+                       skiparse_k=w.skiparse_k if sparse(w) else None, parallelism=f"replicas x{world} (independent samples)",
+                       l2=f"inputs {in_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB, no flush",
+                       flops_per_step=flops),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "attn_fwd_kernel", "peak_source": f"{peaks_src} (sustained bf16 GEMM)",
+                     "frac_of_burst_peak": round(achieved / float(peaks["bf16_tflops"]), 4),
+                     "avg_launch_ms": round(attn_ms, 4)},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step(w) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------------------------------------------
+# the oracle on the host cores
+# ------------------------------------------------------------------------------------------
+
+def oracle_sample(w, heads, rows: int, q, k, v):
+    """One bounded sample of the hot path on the CPU oracle, for the given heads: RoPE of q and k
+    (all tokens of those heads), then attention for the first `rows` query tokens (dense), or the
+    first rows/k slots of every set for Single and Group Skip (Skiparse).  Returns
+    (attention flops done, seconds in RoPE, seconds in attention)."""
+    import oracle as O
+    heads = list(heads)
+    t0 = time.perf_counter()
+    qf = q[:, :, heads].to(torch.float64).numpy()
+    kf = k[:, :, heads].to(torch.float64).numpy()
+    vf = v[:, :, heads].to(torch.float64).numpy()
+    qr = O.round_to_bf16(O.rope3d_ref(qf, w.grid, w.text_len, w.split, w.theta))
+    kr = O.round_to_bf16(O.rope3d_ref(kf, w.grid, w.text_len, w.split, w.theta))
+    t1 = time.perf_counter()
+    nh = len(heads)
+    if not sparse(w):
+        O.attn_ref(qr, kr, vf, rows=np.arange(rows))
+        fl = 4.0 * w.B * nh * rows * w.seq_len * w.head_dim
+    else:
+        fl = 0.0
+        n_set = w.n_video // w.skiparse_k
+        per = max(1, rows // w.skiparse_k)
+        for mode in (O.SKIP_SINGLE, O.SKIP_GROUP):
+            sets = O.skiparse_sets(w.n_video, w.skiparse_k, mode)
+            sel = [t for st in sets for t in st[:per]]
+            O.skiparse_attn_ref(qr, kr, vf, w.skiparse_k, mode, rows=sel)
+            fl += 4.0 * w.B * nh * len(sel) * n_set * w.head_dim
+    return fl, t1 - t0, time.perf_counter() - t1
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:  # noqa: BLE001
+        return os.cpu_count()
+
+
+def _fit_rows(w, q, k, v, nheads: int, budget_s: float):
+    """Query rows per head such that RoPE of `nheads` heads plus their attention rows take about
+    `budget_s` seconds, from a 32-row probe on one head."""
+    _, tr, ta = oracle_sample(w, [0], 32, q, k, v)
+    per_row = ta / 32
+    rows = (budget_s - nheads * tr) / max(nheads * per_row, 1e-9)
+    return int(max(8, min(w.seq_len, rows)))
+
+
+def cpu_baseline(w, budget_s: float = 15.0):
+    q, k, v = syn.make_qkv(w)
+    heads = range(w.heads)
+    rows = _fit_rows(w, q, k, v, w.heads, budget_s)
+    fl, tr, ta = oracle_sample(w, heads, rows, q, k, v)
+    return {"value": round(fl / (tr + ta) / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{w.name}: RoPE of all q/k tokens of all {w.heads} heads + fp64 attention of "
+                      + (f"the first {rows // w.skiparse_k} slots of every set (Single and Group Skip)"
+                         if sparse(w) else f"the first {rows} query tokens")
+                      + f" of every head; {tr + ta:.1f} s ({tr:.1f} s RoPE)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = syn.WORKLOADS[args.workload]
+    q, k, v = syn.make_qkv(w)
+    # one head per step (rotating), rows sized so that warm-up + timed steps end in ~2.5 minutes
+    per_step_s = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    rows = _fit_rows(w, q, k, v, 1, per_step_s)
+    for i in range(args.warmup):
+        oracle_sample(w, [i % w.heads], rows, q, k, v)
+    fl = tt = 0.0
+    for i in range(args.steps):
+        f, tr, ta = oracle_sample(w, [i % w.heads], rows, q, k, v)
+        fl += f
+        tt += tr + ta
+    value = fl / tt / 1e12
+    sample = (f"{w.name}, per step: one head (rotating), RoPE of its q/k tokens + fp64 attention of "
+              + (f"the first {rows // w.skiparse_k} slots of every set (Single and Group Skip)" if sparse(w)
+                 else f"the first {rows} query tokens"))
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(w.describe(), ops="oracle: rope3d_ref + attn_ref (sampled)"),
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="cogvideox_2b", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse"],
+                    help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ATTN_MODE["value"] = args.attn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE", file=sys.stderr)
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

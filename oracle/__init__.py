@@ -13,6 +13,7 @@ from .spacetime_oracle import (  # noqa: F401
     rope3d_positions_ref,
     rope3d_ref,
     rope_frequencies,
+    round_to_bf16,
     skiparse_attn_ref,
     skiparse_gather_ref,
     skiparse_index_map,

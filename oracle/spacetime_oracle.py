@@ -53,6 +53,30 @@ SKIP_GROUP = 1
 
 
 # ----------------------------------------------------------------------------------------------
+# Storage precision
+# ----------------------------------------------------------------------------------------------
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value, ties to even, returned as fp64.
+
+    bf16 is the storage format of every tensor at the library's boundary (the pages run their
+    models in bf16, CogVideoX Tables 7 and 8), so a RoPE output that feeds attention is rounded
+    to bf16 once.  Done in two exact steps: fp64 -> fp32 rounded to odd (truncate toward zero,
+    then set the lowest bit when anything was dropped), then fp32 -> bf16 to nearest even on the
+    bit pattern.  fp32 keeps 16 more significand bits than bf16, so the result is the single
+    correct rounding of x.  Finite inputs only.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    f = x.astype(np.float32)
+    over = np.abs(f.astype(np.float64)) > np.abs(x)
+    f = np.where(over, np.nextafter(f, np.float32(0)), f).astype(np.float32)
+    bits = f.view(np.uint32) | (f.astype(np.float64) != x).astype(np.uint32)
+    lsb = (bits >> np.uint32(16)) & np.uint32(1)
+    rounded = ((bits + np.uint32(0x7FFF) + lsb) >> np.uint32(16)) << np.uint32(16)
+    return rounded.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------------------------
 # Token positions
 # ----------------------------------------------------------------------------------------------
 

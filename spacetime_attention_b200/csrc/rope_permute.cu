@@ -47,6 +47,17 @@ __device__ __forceinline__ int skiparse_token(int g, int s, int k, int mode) {
   return (o * k + g) * k + r;
 }
 
+// fp64 -> bf16 with a single round-to-nearest-even: first fp64 -> fp32 rounded to odd (truncate,
+// then set the last bit if anything was dropped; Boldo & Melquiond, "When double rounding is odd"),
+// then fp32 -> bf16 RNE.  fp32 keeps 16 more significand bits than bf16, so the second rounding
+// sees the exact tie/no-tie information.
+__device__ __forceinline__ uint32_t bf16_rn_from_f64(double x) {
+  const float t = __double2float_rz(x);
+  uint32_t b = __float_as_uint(t);
+  if ((double)t != x) b |= 1u;
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(b)));
+}
+
 template <int MAP>
 __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -54,7 +65,7 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
   long long* src_row = reinterpret_cast<long long*>(omega + kMaxPairs);      // [rows_per_tile]
   long long* dst_row = src_row + p.rows_per_tile;                            // [rows_per_tile]
   int* vid = reinterpret_cast<int*>(dst_row + p.rows_per_tile);              // video index or -1
-  float2* cs = reinterpret_cast<float2*>(vid + ((p.rows_per_tile + 3) & ~3)); // [tile][pairs]
+  double2* cs = reinterpret_cast<double2*>(vid + ((p.rows_per_tile + 3) & ~3)); // [tile][pairs]
 
   const int npairs = p.head_dim >> 1;
   // Frequencies of every channel pair: pair j of a chunk of size d_a -> theta^(-2j/d_a).
@@ -98,16 +109,16 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
       for (int idx = threadIdx.x; idx < nrows * npairs; idx += kThreads) {
         const int i = idx / npairs, pr = idx - i * npairs;
         const int v = vid[i];
-        float2 c_s = make_float2(1.f, 0.f);
+        double2 c_s = make_double2(1.0, 0.0);
         if (v >= 0) {
           const int c = 2 * pr;
           int pos;
           if (c < p.d_t) pos = v / HW;
           else if (c < p.d_t + p.d_h) pos = (v / p.W) % p.H;
           else pos = v % p.W;
-          float sn, cn;
-          sincosf((float)((double)pos * omega[pr]), &sn, &cn);
-          c_s = make_float2(cn, sn);
+          double sn, cn;
+          sincos((double)pos * omega[pr], &sn, &cn);
+          c_s = make_double2(cn, sn);
         }
         cs[idx] = c_s;
       }
@@ -139,16 +150,17 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
           if (!live[u]) continue;
           if (rot && vid[rowi[u]] >= 0) {
             const int pair0 = (col[u] % per_head_vec) * 4;
-            const float2* tab = cs + rowi[u] * npairs + pair0;
+            const double2* tab = cs + rowi[u] * npairs + pair0;
             uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float x = __uint_as_float(w[e] << 16);
-              const float y = __uint_as_float(w[e] & 0xFFFF0000u);
-              const float2 c_s = tab[e];
-              const float xr = x * c_s.x - y * c_s.y;
-              const float yr = x * c_s.y + y * c_s.x;
-              w[e] = pack_bf16x2(xr, yr);
+              // bf16 -> fp64 is exact; the rotation runs in fp64 and is rounded once to bf16
+              const double x = (double)__uint_as_float(w[e] << 16);
+              const double y = (double)__uint_as_float(w[e] & 0xFFFF0000u);
+              const double2 c_s = tab[e];
+              const double xr = fma(x, c_s.x, -y * c_s.y);
+              const double yr = fma(x, c_s.y, y * c_s.x);
+              w[e] = bf16_rn_from_f64(xr) | (bf16_rn_from_f64(yr) << 16);
             }
             val[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
@@ -169,11 +181,13 @@ __global__ void index_map_kernel(int n_video, int k, int mode, int* out) {
 
 int launch_permute(int map, PermuteParams& p, cudaStream_t stream) {
   const int npairs = p.head_dim / 2;
-  p.rows_per_tile = (int)std::max(1, std::min(32, (1024 + p.vpr - 1) / p.vpr));
+  // ~1024 vectors per tile, at most 32 rows, and the cos/sin table within 40 KB of shared memory
+  const int table_rows = (40 * 1024) / (npairs * (int)sizeof(double2));
+  p.rows_per_tile = (int)std::max(1, std::min(std::min(32, table_rows), (1024 + p.vpr - 1) / p.vpr));
   p.n_tiles = (p.rows + p.rows_per_tile - 1) / p.rows_per_tile;
   const size_t smem = kMaxPairs * sizeof(double) + 2 * p.rows_per_tile * sizeof(long long) +
                       ((p.rows_per_tile + 3) & ~3) * sizeof(int) +
-                      (size_t)p.rows_per_tile * npairs * sizeof(float2);
+                      (size_t)p.rows_per_tile * npairs * sizeof(double2);
   const int sms = device_sm_count();
   const long long grid = std::min<long long>(p.n_tiles, (long long)sms * 8);
   if (grid <= 0) return OSP_OK;

@@ -13,10 +13,17 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
 
 
 def bf16_round(x: np.ndarray) -> torch.Tensor:
-    """fp64 values -> bf16 with one round-to-nearest-even step (bit manipulation on fp64 is
-    avoided: fp64 -> fp32 is exact for the values compared here only up to rounding, so round
-    through fp32 and accept the rare double-rounding tie as a 1-ulp difference)."""
-    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.float32).to(torch.bfloat16)
+    """fp64 values -> bf16 tensor, correctly rounded (the oracle's storage rounding)."""
+    from oracle import round_to_bf16
+    return torch.from_numpy(round_to_bf16(x).astype(np.float32)).to(torch.bfloat16)
+
+
+def assert_bf16_close(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
+    """Correctly rounded results: at most 1 ulp apart anywhere, and almost all identical."""
+    dist = bf16_ulp_distance(got, ref)
+    mx = int(dist.max()) if dist.numel() else 0
+    frac = float((dist != 0).double().mean()) if dist.numel() else 0.0
+    assert mx <= 1 and frac <= 1e-4, f"{what}: max ulp distance {mx}, mismatch fraction {frac:.2e}"
 
 
 def bf16_ulp_distance(a: torch.Tensor, b: torch.Tensor) -> torch.Tensor:

@@ -1,7 +1,9 @@
 """GPU parity of 3D RoPE, the Skiparse index map and the k-fold gather / scatter.
 
-Index maps and pure copies: bit-exact.  RoPE outputs: within 1 bf16 ulp of the fp64 oracle
-rounded to bf16 (the kernel rotates in fp32 and rounds once)."""
+Index maps and pure copies: bit-exact.  RoPE outputs: the kernel rotates in fp64 and rounds
+once to bf16, so it is compared with the fp64 oracle correctly rounded to bf16: at most 1 ulp
+apart anywhere (fp64 cos/sin of the two sides may differ in the last bits, which can flip a
+rounding that sits on a tie boundary) and identical in all but a 1e-4 fraction of elements."""
 
 import numpy as np
 import pytest
@@ -10,7 +12,7 @@ import torch
 import oracle as O
 from spacetime_attention_b200 import ops, synthetic as syn
 from tests.gpu_common import gpu  # noqa: F401
-from tests.helpers import bf16_round, bf16_ulp_distance, to_f64
+from tests.helpers import assert_bf16_close, bf16_round, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +39,7 @@ def _rope_case(dev, B, heads, d, grid, L, split, seed=7, inplace=False):
     torch.cuda.synchronize()
     for x, xo in ((q, qo), (k, ko)):
         ref = bf16_round(O.rope3d_ref(to_f64(x), grid, L, split))
-        dist = bf16_ulp_distance(xo, ref)
-        assert int(dist.max()) <= 1, f"max ulp distance {int(dist.max())}"
+        assert_bf16_close(xo, ref, "rope3d")
         # text tokens are bit-exact copies
         assert torch.equal(xo[:, :L].cpu(), x[:, :L])
 
@@ -63,7 +64,7 @@ def test_rope3d_full_size(gpu, name):
     heads = sorted({0, w.heads // 2, w.heads - 1})
     for x, xo in ((q, qo), (k, ko)):
         ref = bf16_round(O.rope3d_ref(to_f64(x[:, :, heads]), w.grid, w.text_len, w.split))
-        assert int(bf16_ulp_distance(xo[:, :, heads], ref).max()) <= 1
+        assert_bf16_close(xo[:, :, heads], ref, name)
 
 
 @pytest.mark.parametrize("n,k,mode", [(256, 2, 0), (256, 2, 1), (28800, 4, 0), (28800, 4, 1), (36864, 4, 0),
@@ -102,7 +103,7 @@ def test_gather_scatter(gpu, case, mode):
     assert torch.equal(vr, vo)
     for x, xr in ((q, qr), (kk, kr)):
         ref = bf16_round(O.skiparse_gather_ref(O.rope3d_ref(to_f64(x), grid, 0, split), k, mode))
-        assert int(bf16_ulp_distance(xr, ref).max()) <= 1
+        assert_bf16_close(xr, ref, "gather+rope")
     # q only
     q_only, none_k, none_v = ops.skiparse_gather(qg, None, None, grid, k, mode, split=split)
     assert none_k is None and none_v is None and torch.equal(q_only, qr)
@@ -117,5 +118,5 @@ def test_gather_full_size_open_sora_plan(gpu):
         ref_v = O.skiparse_gather_ref(to_f64(v[:, :, :2]), 4, mode)
         assert np.array_equal(to_f64(vo[:, :, :2]), ref_v)
         ref_q = bf16_round(O.skiparse_gather_ref(O.rope3d_ref(to_f64(q[:, :, :2]), w.grid, 0, w.split), 4, mode))
-        assert int(bf16_ulp_distance(qo[:, :, :2], ref_q).max()) <= 1
+        assert_bf16_close(qo[:, :, :2], ref_q, "gather+rope full size")
         assert torch.equal(ops.skiparse_scatter(vo, w.grid, 4, mode).cpu(), v)

@@ -323,3 +323,35 @@ def test_skiparse_equals_gather_dense_scatter():
         g = [O.skiparse_gather_ref(t, 2, mode) for t in (q, k, v)]
         o = O.skiparse_scatter_ref(O.attn_ref(*g), 2, mode)
         np.testing.assert_allclose(o, O.skiparse_attn_ref(q, k, v, 2, mode), rtol=0, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------------------------
+# bf16 storage rounding
+# ----------------------------------------------------------------------------------------------
+
+def test_round_to_bf16_hand_values():
+    # bf16 has 8 significand bits: spacing 2^-7 on [1, 2), 2^-6 on [2, 4)
+    cases = [
+        (1.0, 1.0),
+        (1.0 + 2 ** -8, 1.0),                        # tie -> even (1.0)
+        (1.0 + 3 * 2 ** -8, 1.0 + 2 ** -6),          # tie -> even (1 + 2^-6 has even last bit)
+        (1.0 + 2 ** -8 + 2 ** -40, 1.0 + 2 ** -7),   # just above the tie: up (needs the sticky bit)
+        (1.0 + 2 ** -8 - 2 ** -40, 1.0),             # just below: down
+        (-(1.0 + 2 ** -8 + 2 ** -40), -(1.0 + 2 ** -7)),
+        (3.0 + 2 ** -7, 3.0),                        # tie on [2,4) -> even
+        (0.0, 0.0),
+        (2.0 ** -130, 2.0 ** -130),                  # subnormal in fp32, exact in bf16
+    ]
+    got = O.round_to_bf16(np.array([c[0] for c in cases]))
+    np.testing.assert_array_equal(got, [c[1] for c in cases])
+
+
+def test_round_to_bf16_is_nearest():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))
+    r = O.round_to_bf16(x)
+    # result has at most 8 significant bits and is within half a bf16 spacing of x
+    m, e = np.frexp(r)
+    assert np.all(m * 2 ** 8 == np.round(m * 2 ** 8))
+    spacing = 2.0 ** (np.floor(np.log2(np.abs(x))) - 7)
+    assert np.all(np.abs(r - x) <= spacing / 2)
