@@ -263,7 +263,7 @@ def run_ours(args, rank, world, local_rank):
         "config": dict(w.describe(), ops=("rope3d+skiparse_single+skiparse_group" if sparse(w)
                                           else "rope3d+attn_full"),
                        skiparse_k=w.skiparse_k if sparse(w) else None, parallelism=f"replicas x{world} (independent samples)",
-                       l2=f"inputs {in_bytes / 1e6:.0f} MB > L2 {L2_BYTES / 1e6:.0f} MB, no flush",
+                       l2=f"inputs {in_bytes / 1e6:.0f} MB > L2 126 MiB, no flush",
                        flops_per_step=flops),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
