@@ -126,6 +126,27 @@ int osp_skiparse_attn(const void* q, const void* k, const void* v, void* o, cons
 int osp_skiparse_index_map(int32_t n_video, int32_t sparse_k, int32_t mode, int32_t* dev_out,
                            void* stream);
 
+/* Dense 3D full attention exactly like osp_attn_full, for callers that cannot allocate device
+ * memory. The pages have no counterpart: this exists only for how the library is called.
+ * Who needs it: callers whose device memory is entirely owned by another allocator (a
+ * framework's caching pool or a serving runtime that reserves the GPU's memory up front), and
+ * latency-critical callers, for whom cudaMalloc's implicit device synchronisation would stall
+ * every stream. osp_attn_full allocates one status word with cudaMalloc on its first call per
+ * device; this entry point never calls cudaMalloc, cudaFree or any allocating routine.
+ *  Scratch: the kernel's only scratch, its 4-byte status word, lives in a file-scope
+ *    __device__ array of 256 bytes (the maximum; every problem size needs the same 4 bytes, and
+ *    a call whose scratch would exceed the array is rejected with OSP_ERR_UNSUPPORTED). Every
+ *    GPU that loads the library holds the array until the process exits.
+ *  First call per device: looks up the array's device address (cudaGetSymbolAddress) with that
+ *    device current and caches it; make that first call before any stream capture.
+ *  Sharing: all calls on a device share the array, and each call clears the status word on
+ *    `stream` before its kernel. Calls that overlap on the GPU (different streams) race on it.
+ *  Errors: as osp_attn_full. A bounded-wait timeout inside this call is recorded in the static
+ *    word, which osp_check_status does not read: the kernel still ends, its output is invalid.
+ *  Arguments, layout, arithmetic and results are those of osp_attn_full (bit-identical). */
+int osp_attn_full_noalloc(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                          float softmax_scale, void* stream);
+
 /* Synchronises `stream`, then reads and clears this device's status word.
  * Returns OSP_OK, OSP_ERR_TIMEOUT (a kernel's bounded wait gave up; its output is invalid),
  * OSP_ERR_BOUNDS, or OSP_ERR_CUDA (the synchronisation itself failed). */

@@ -26,6 +26,8 @@
 
 #include <cuda.h>
 
+#include <mutex>
+
 #include "osp_internal.h"
 
 namespace osp {
@@ -427,8 +429,11 @@ int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
 
 }  // namespace
 
-int attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
-                     int sparse_k, float scale, cudaStream_t stream) {
+namespace {
+
+// Attention launch with an explicit status word (the kernel's only global scratch).
+int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
+                       int sparse_k, float scale, cudaStream_t stream, unsigned* status) {
   const int N = s.text_len + s.T * s.H * s.W;
   const int G = (layout == 0) ? 1 : sparse_k;
   const int n = N / G;
@@ -441,8 +446,7 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
   p.layout = layout;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
-  p.status = device_status_word();
-  if (!p.status) return OSP_ERR_CUDA;
+  p.status = status;
   p.timeout_ns = wait_timeout_ns();
   CUtensorMap tq, tk, tv;
   int rc;
@@ -462,4 +466,87 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
   }
 }
 
+}  // namespace
+
+int attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
+                     int sparse_k, float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status);
+}
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free dense attention (osp_attn_full_noalloc)
+// ------------------------------------------------------------------------------------------
+// The attention kernel's only global scratch is its status word, into which its bounded waits
+// report a timeout.  osp_attn_full keeps that word in memory the library obtains with cudaMalloc
+// on first use.  This variant keeps it in the file-scope device array below instead, so a call
+// allocates nothing.  Every GPU that loads the library holds the array until the process exits.
+// In host code `g_noalloc_scratch` names a host-side shadow, not device memory: the kernel gets
+// the device address obtained with cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocScratchBytes = 256;   // maximum scratch a call may use
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Scratch bytes the kernel needs for a problem: its status word, whatever the shape.
+size_t noalloc_scratch_bytes(const osp_shape&) { return sizeof(unsigned); }
+
+// Device address of g_noalloc_scratch on the current device; looked up on the first call per
+// device (with that device current) and cached.
+int noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+    return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: no usable current CUDA device");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: cudaGetSymbolAddress failed: %s",
+                       cudaGetErrorString(e));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return OSP_OK;
+}
+
+}  // namespace
+
 }  // namespace osp
+
+extern "C" int osp_attn_full_noalloc(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                                     float softmax_scale, void* stream) {
+  using namespace osp;
+  set_error(OSP_OK, "");
+  if (!shape) return set_error(OSP_ERR_INVALID_ARG, "shape is NULL");
+  const osp_shape& s = *shape;
+  if (s.B < 1 || s.text_len < 0 || s.T < 1 || s.H < 1 || s.W < 1 || s.heads < 1)
+    return set_error(OSP_ERR_INVALID_ARG, "bad shape: B=%d text_len=%d T=%d H=%d W=%d heads=%d", s.B, s.text_len,
+                     s.T, s.H, s.W, s.heads);
+  if (s.head_dim != 64 && s.head_dim != 96 && s.head_dim != 128)
+    return set_error(OSP_ERR_UNSUPPORTED, "attention head_dim %d not in {64, 96, 128}", s.head_dim);
+  if ((long long)s.text_len + (long long)s.T * s.H * s.W > (1LL << 30))
+    return set_error(OSP_ERR_UNSUPPORTED, "sequence length too large");
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  const uintptr_t a = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                      reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o);
+  if (a & 15u) return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t need = noalloc_scratch_bytes(s);
+  if (need > kNoAllocScratchBytes)
+    return set_error(OSP_ERR_UNSUPPORTED, "osp_attn_full_noalloc needs %zu bytes of scratch, more than its %zu-byte "
+                     "static array", need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  int rc = noalloc_scratch_address(&scratch);
+  if (rc) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: the status word must start at zero
+  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess)
+    return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: clearing the scratch word failed");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)s.head_dim);
+  return launch_with_status(q, k, v, o, s, 0, 1, softmax_scale, st, static_cast<unsigned*>(scratch));
+}
