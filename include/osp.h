@@ -69,7 +69,7 @@ typedef struct {
  * (2j, 2j+1) rotates by angle pos * theta^(-2j/d_a) (RoFormer). Positions are raw integer grid
  * indices (extrapolation, CogVideoX section 3.1). Text tokens are not rotated. */
 typedef struct {
-  int32_t d_t, d_h, d_w;  /* each even and > 0... or 0; d_t + d_h + d_w == head_dim */
+  int32_t d_t, d_h, d_w;  /* each even and >= 0 (0: that axis is not rotated); sum == head_dim */
   double theta;           /* frequency base, > 0 (10000 on the pages) */
 } osp_rope;
 
@@ -77,7 +77,8 @@ typedef struct {
  *  q, k:          [B][N][heads][head_dim] bf16, device.
  *  q_out, k_out:  same shape; may equal q / k (in place) but must not overlap them otherwise.
  *  Text tokens are copied unchanged (nothing is written for them when out == in).
- *  Arithmetic: fp32 rotation of the bf16 inputs, rounded to bf16 (RNE).
+ *  Arithmetic: fp64 rotation of the bf16 inputs (fp64 cos/sin), rounded once to bf16 (RNE):
+ *    outputs are the correctly rounded rotation up to the last bits of fp64 cos/sin.
  *  Errors: OSP_ERR_INVALID_ARG (null, bad shape or split), OSP_ERR_CUDA (launch failed). */
 int osp_rope3d(const void* q, const void* k, void* q_out, void* k_out, const osp_shape* shape,
                const osp_rope* rope, void* stream);
