@@ -6,11 +6,14 @@
 // folded into the TMA tensor maps: a Single Skip set is a strided view of the token axis and a
 // Group Skip set a 2-level view, so the k-fold permuted tensor never exists in memory.
 //
-// CTA = 2 query tiles of 128 rows sharing one K/V stream (320 threads):
+// CTA = 2 query tiles of 128 rows sharing one K/V stream (384 threads, 3 warpgroups):
 //   warps 0-3  softmax for query tile 0 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax for query tile 1
 //   warp 8     TMA producer: Q once, then K/V tiles into a ring of shared-memory stages
 //   warp 9     tensor-memory allocator and MMA issuer (one elected thread)
+//   warps 10-11 idle (they complete the third warpgroup for the register split)
+// Registers: launched at 168 per thread (384 x 168 = 64,512); the producer/MMA warpgroup drops
+// to 104 and the two softmax warpgroups rise to 200 (2 x 128 x 200 + 128 x 104 = 64,512).
 // Tensor memory (512 columns x 128 lanes x 32 bit): S0 [0,128), S1 [128,256) fp32 scores,
 // O0 [256, 256+D), O1 [384, 384+D) fp32 output accumulators.  The softmax overwrites the first
 // 64 columns of S_i with P_i in bf16 pairs, and the PV product reads P_i from tensor memory as
@@ -36,7 +39,12 @@ namespace {
 constexpr int kBM = 128;               // query rows per tile
 constexpr int kBN = 128;               // keys per KV tile
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 channels (one 128-byte swizzle atom wide)
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsLaunch = 168;   // ptxas' count for __launch_bounds__(384, 1)
+constexpr uint32_t kRegsSoftmax = 200;
+constexpr uint32_t kRegsSupport = 104;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSupport == kThreads * kRegsLaunch,
+              "register split must equal the launch allocation");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -47,13 +55,17 @@ struct Cfg {
   static constexpr int kChunks = (D + 63) / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStages = (D == 64) ? 4 : 2;
+  // d <= 64: S0, S1, O0, O1 and separate P0, P1 buffers fit the 512 TMEM columns, so the softmax
+  // releases S as soon as it is in registers and QK^T of the next tile overlaps the exponentials.
+  // Larger d: P aliases the first 64 columns of S.
+  static constexpr bool kSepP = (D <= 64);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
-  // o_full[2], mma_done
-  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  // o_full[2], mma_done, s_free[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 9;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -105,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + S, B_VFULL = 1 + 2 * S, B_VEMPTY = 1 + 3 * S;
   const int B_SFULL = 1 + 4 * S, B_PREADY = B_SFULL + 2, B_OFULL = B_PREADY + 2, B_MMADONE = B_OFULL + 2;
+  const int B_SFREE = B_MMADONE + 1;  // separate-P layout: softmax has S_i in registers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -129,6 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_OFULL + i), 1);
     }
     mbar_init(bar(B_MMADONE), 1);
+    mbar_init(bar(B_SFREE + 0), 128);
+    mbar_init(bar(B_SFREE + 1), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -151,9 +166,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sK = [&](int s) { return sbase + C::kKOff + (uint32_t)(s * C::kTileBytes); };
   auto sV = [&](int s) { return sbase + C::kVOff + (uint32_t)(s * C::kTileBytes); };
   auto colS = [](int i) { return i ? 128u : 0u; };
-  auto colO = [](int i) { return i ? 384u : 256u; };
+  auto colO = [](int i) { return i ? (C::kSepP ? 320u : 384u) : 256u; };
+  auto colP = [](int i) { return C::kSepP ? (i ? 448u : 384u) : (i ? 128u : 0u); };
 
-  if (warp == kLoadWarp) {
+  if (warp >= kLoadWarp) {
+   // each warpgroup's register budget change dominates its own role code
+   regs_dec<kRegsSupport>();
+   if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
@@ -200,17 +219,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                  idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      // O_i += P_i V: P_i from tensor memory (bf16 pairs in S_i's first 64 columns), V MN-major
-      // (channels contiguous), 16 keys per MMA.
+      // O_i += P_i V: P_i from tensor memory (bf16 pairs, 64 columns), V MN-major (channels
+      // contiguous), 16 keys per MMA.
       auto issue_pv = [&](int i, int s, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + colO(i), tmem + colS(i) + 8u * kk, sdesc_sw128(sV(s) + 2048u * kk, kChunkBytes, 1024),
+          mma_ts(tmem + colO(i), tmem + colP(i) + 8u * kk, sdesc_sw128(sV(s) + 2048u * kk, kChunkBytes, 1024),
                  idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(B_QFULL), 0, wc) && mbar_wait(bar(B_KFULL), 0, wc);
-      if (ok) {
+      if (ok && C::kSepP) {
+        // Order per KV tile j: S0(j+1) as soon as softmax 0 holds S0(j) in registers, S1(j+1)
+        // likewise, then PV0(j), PV1(j) as their P tiles arrive.  O_full[i] completes after every
+        // PV_i(j): the softmax waits on it before overwriting P_i and before touching O_i.
+        tc_fence_after();
+        issue_s(0, 0);
+        tc_commit(bar(B_SFULL + 0));
+        issue_s(1, 0);
+        tc_commit(bar(B_SFULL + 1));
+        tc_commit(bar(B_KEMPTY + 0));
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j % S, u = j / S;
+          const bool more = j + 1 < n_kv;
+          const int s1 = (j + 1) % S, u1 = (j + 1) / S;
+          if (more) {
+            if (!mbar_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
+            if (!mbar_wait(bar(B_SFREE + 0), j & 1, wc)) break;
+            tc_fence_after();
+            issue_s(0, s1);
+            tc_commit(bar(B_SFULL + 0));
+            if (!mbar_wait(bar(B_SFREE + 1), j & 1, wc)) break;
+            tc_fence_after();
+            issue_s(1, s1);
+            tc_commit(bar(B_SFULL + 1));
+            tc_commit(bar(B_KEMPTY + s1));
+          }
+          if (!mbar_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          if (!mbar_wait(bar(B_PREADY + 0), j & 1, wc)) break;
+          tc_fence_after();
+          issue_pv(0, s, j > 0);
+          tc_commit(bar(B_OFULL + 0));
+          if (!mbar_wait(bar(B_PREADY + 1), j & 1, wc)) break;
+          tc_fence_after();
+          issue_pv(1, s, j > 0);
+          tc_commit(bar(B_OFULL + 1));
+          tc_commit(bar(B_VEMPTY + s));
+        }
+      } else if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         tc_commit(bar(B_SFULL + 0));
@@ -250,7 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_drain(bar(B_MMADONE), 0, p.timeout_ns);
     }
     __syncwarp();
+   }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax / epilogue
     const int i = warp >> 2;                       // query tile
     const int quarter = warp & 3;                  // TMEM lane quarter this warp may access
@@ -258,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + colS(i);
     const uint32_t tO = tmem + lane_base + colO(i);
+    const uint32_t tP = tmem + lane_base + colP(i);
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -270,6 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
+      if constexpr (C::kSepP) {
+        tc_fence_before();
+        mbar_arrive(bar(B_SFREE + i));   // S_i may now be overwritten by the next QK^T
+      }
       float sv[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
@@ -297,18 +360,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float neg_m = -m;
       float rs0 = 0.f, rs1 = 0.f;
+      if constexpr (C::kSepP) {
+        uint32_t pk[64];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float e0 = ex2_approx(fmaf(sv[64 * half + 2 * c], sl2, neg_m));
-          const float e1 = ex2_approx(fmaf(sv[64 * half + 2 * c + 1], sl2, neg_m));
+        for (int c = 0; c < 64; ++c) {
+          const float e0 = ex2_approx(fmaf(sv[2 * c], sl2, neg_m));
+          const float e1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, neg_m));
           rs0 += e0;
           rs1 += e1;
           pk[c] = pack_bf16x2(e0, e1);
         }
-        tmem_st32(tS + 32 * half, pk);
+        // P_i and O_i are free once PV_i(j-1) has completed
+        if (j > 0 && !warp_wait(bar(B_OFULL + i), (j - 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(tP + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      } else {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float e0 = ex2_approx(fmaf(sv[64 * half + 2 * c], sl2, neg_m));
+            const float e1 = ex2_approx(fmaf(sv[64 * half + 2 * c + 1], sl2, neg_m));
+            rs0 += e0;
+            rs1 += e1;
+            pk[c] = pack_bf16x2(e0, e1);
+          }
+          tmem_st32(tP + 32 * half, pk);
+        }
       }
       l = l * alpha + (rs0 + rs1);
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
@@ -326,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_PREADY + i));
     }
-    if (ok && warp_wait(bar(B_OFULL + i), 0, wc)) {
+    if (ok && warp_wait(bar(B_OFULL + i), C::kSepP ? (uint32_t)((n_kv - 1) & 1) : 0u, wc)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const int slot = q0 + i * kBM + row;
@@ -419,6 +499,14 @@ int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
   constexpr int smem = Cfg<D>::kSmemBytes;
   static bool attr_done = false;  // per process; the attribute is per function, not per device
   if (!attr_done) {
+    // The warpgroup register split only adds up if the kernel is launched with exactly
+    // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>) != cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "cudaFuncGetAttributes(attn_fwd_kernel<%d>) failed", D);
+    if ((uint32_t)fa.numRegs != kRegsLaunch)
+      return set_error(OSP_ERR_CUDA, "attn_fwd_kernel<%d> compiled to %d registers per thread, expected %u", D,
+                       fa.numRegs, kRegsLaunch);
     if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_fwd_kernel<%d>) failed", D);
     attr_done = true;
