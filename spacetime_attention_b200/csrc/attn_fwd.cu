@@ -50,6 +50,25 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Tuning switches (compile-time; the defaults are the measured best on B200: alternating the
+// softmax groups cost 4 % at d=64; the polynomial share pays only at d=128, where MUFU and the
+// tensor core are balanced: 1 pair in 16 there, +6 %).
+#ifndef OSP_SOFTMAX_TURNS
+#define OSP_SOFTMAX_TURNS 0     // 1: the two softmax groups alternate their exponential phases
+#endif
+#ifndef OSP_POLY16_D64
+#define OSP_POLY16_D64 0        // exp2 pairs (of 16) on the FMA pipe at d = 64
+#endif
+#ifndef OSP_POLY16_D96
+#define OSP_POLY16_D96 0
+#endif
+#ifndef OSP_POLY16_D128
+#define OSP_POLY16_D128 1
+#endif
+#ifndef OSP_F32X2
+#define OSP_F32X2 1             // packed fp32 pairs for the scale/subtract and the row sum
+#endif
+
 template <int D>
 struct Cfg {
   static constexpr int kChunks = (D + 63) / 64;
@@ -59,13 +78,16 @@ struct Cfg {
   // releases S as soon as it is in registers and QK^T of the next tile overlaps the exponentials.
   // Larger d: P aliases the first 64 columns of S.
   static constexpr bool kSepP = (D <= 64);
+  // Of every 16 exponential pairs, this many run as a polynomial on the FMA/ALU pipes instead of
+  // MUFU (whose 16 ex2/clk/SM bound the softmax at small d); the rest use ex2.approx.
+  static constexpr int kPolyPer16 = (D <= 64) ? OSP_POLY16_D64 : (D <= 96 ? OSP_POLY16_D96 : OSP_POLY16_D128);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
-  // o_full[2], mma_done, s_free[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 9;
+  // o_full[2], mma_done, s_free[2], turn[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 11;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -97,6 +119,67 @@ __device__ __forceinline__ int slot_token(int layout, int s, int g, int k) {
   return (o * k + g) * k + (s - o * k);
 }
 
+// exp2 of two values on the FMA and ALU pipes: 2^x = 2^n * 2^f with n = round(x) (added to the
+// exponent field) and f = x - n in [-1/2, 1/2]; 2^f is the degree-3 minimax polynomial derived
+// by csrc/exp2_poly.py (Remez, relative error 7.5e-5, far below the bf16 step of P).  Inputs
+// are clamped at -125 so that the exponent field cannot underflow (2^-125 is negligible next to
+// the row maximum's 1).
+__device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds round(x) in its low bits
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(xc, f2_pack(kRound, kRound));
+  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+  uint64_t q = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f, f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  q = f2_fma(q, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  q = f2_fma(q, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// p = exp2(s * sl2 - m) for the 128 scores of one row, packed to bf16 pairs; returns the row sum.
+// kPoly: whether the polynomial takes its share (never on a tile with masked (-inf) columns).
+template <int kPolyPer16, bool kPoly>
+__device__ __forceinline__ float softmax_exp_row(const float (&sv)[128], float sl2, float m, uint32_t (&pk)[64]) {
+  if (!OSP_F32X2 && (!kPoly || kPolyPer16 == 0)) {
+    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const float e0 = ex2_approx(fmaf(sv[2 * c], sl2, -m));
+      const float e1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, -m));
+      r0 += e0;
+      r1 += e1;
+      pk[c] = pack_bf16x2(e0, e1);
+    }
+    return r0 + r1;
+  }
+  const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
+  uint64_t sum2 = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const uint64_t x2 = f2_fma(f2_pack(sv[2 * c], sv[2 * c + 1]), scale2, negm2);
+    float e0, e1;
+    if (kPoly && (c % 16) < kPolyPer16) {
+      ex2_poly2(x2, e0, e1);
+    } else {
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
+    }
+    sum2 = f2_add(sum2, f2_pack(e0, e1));
+    pk[c] = pack_bf16x2(e0, e1);
+  }
+  float lo, hi;
+  f2_unpack(sum2, lo, hi);
+  return lo + hi;
+}
+
 // Warp-uniform bounded wait (tcgen05.ld/st that follow are warp-collective).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const bool ok = mbar_wait(bar, parity, w);
@@ -118,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 1 + S, B_VFULL = 1 + 2 * S, B_VEMPTY = 1 + 3 * S;
   const int B_SFULL = 1 + 4 * S, B_PREADY = B_SFULL + 2, B_OFULL = B_PREADY + 2, B_MMADONE = B_OFULL + 2;
   const int B_SFREE = B_MMADONE + 1;  // separate-P layout: softmax has S_i in registers
+  const int B_TURN = B_SFREE + 2;     // softmax i may start its exponentials (MUFU hand-off)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -144,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_MMADONE), 1);
     mbar_init(bar(B_SFREE + 0), 128);
     mbar_init(bar(B_SFREE + 1), 128);
+    mbar_init(bar(B_TURN + 0), 128);
+    mbar_init(bar(B_TURN + 1), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -210,22 +296,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
-      // S_i = Q_i K^T: both operands K-major (channels contiguous), 16 channels per MMA.
+      // Descriptors are built once; a K step moves the start address (bits [0,14), 16-byte units)
+      // within the tile, so each MMA only adds a small constant to a precomputed base.
+      // Tiles of one kind are contiguous, kTileBytes apart, so tile t's descriptor is the first
+      // one's plus t * kTileBytes / 16.
+      const uint64_t dq = sdesc_sw128(sQ(0), 16, 1024), dk = sdesc_sw128(sK(0), 16, 1024);
+      const uint64_t dv = sdesc_sw128(sV(0), kChunkBytes, 1024);
+      constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
+      // S_i = Q_i K^T: both operands K-major (channels contiguous), 16 channels per MMA: step kk
+      // starts (kk / 4) 64-channel chunks and (kk % 4) * 32 bytes into the tile.
       auto issue_s = [&](int i, int s) {
+        const uint64_t a0 = dq + (uint64_t)i * kTileStep, b0 = dk + (uint64_t)s * kTileStep;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * kChunkBytes + (kk & 3) * 32);
-          mma_ss(tmem + colS(i), sdesc_sw128(sQ(i) + off, 16, 1024), sdesc_sw128(sK(s) + off, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+          mma_ss(tmem + colS(i), a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       // O_i += P_i V: P_i from tensor memory (bf16 pairs, 64 columns), V MN-major (channels
-      // contiguous), 16 keys per MMA.
+      // contiguous), 16 keys (2048 bytes of V) per MMA.
       auto issue_pv = [&](int i, int s, bool acc) {
+        const uint64_t b0 = dv + (uint64_t)s * kTileStep;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + colO(i), tmem + colP(i) + 8u * kk, sdesc_sw128(sV(s) + 2048u * kk, kChunkBytes, 1024),
-                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + colO(i), tmem + colP(i) + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(B_QFULL), 0, wc) && mbar_wait(bar(B_KFULL), 0, wc);
@@ -337,20 +432,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
       const int valid = p.n - j * kBN;
-      if (valid < kBN) {
+      const bool masked = valid < kBN;
+      if (masked) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= valid) sv[c] = -INFINITY;
       }
-      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, sv[c]);
-        mx1 = fmaxf(mx1, sv[c + 1]);
-        mx2 = fmaxf(mx2, sv[c + 2]);
-        mx3 = fmaxf(mx3, sv[c + 3]);
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = fmax3(mx0, sv[c], sv[c + 1]);
+        mx1 = fmax3(mx1, sv[c + 2], sv[c + 3]);
+        mx2 = fmax3(mx2, sv[c + 4], sv[c + 5]);
+        mx3 = fmax3(mx3, sv[c + 6], sv[c + 7]);
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
       const float m_cand = fmaxf(m, mx);
       const bool rescale = m_cand > m + kRescaleThreshold;
       float alpha = 1.f;
@@ -358,39 +454,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = ex2_approx(m - m_cand);
         m = m_cand;
       }
-      const float neg_m = -m;
-      float rs0 = 0.f, rs1 = 0.f;
+      // The two softmax groups take turns on MUFU: group 0 runs the exponentials of tile j after
+      // group 1 finished those of tile j-1, group 1 after group 0 finished tile j.  Each group's
+      // load / max / store phases overlap the other group's exponentials.
+      if (OSP_SOFTMAX_TURNS && (i == 1 || j > 0)) {
+        if (!warp_wait(bar(B_TURN + i), (uint32_t)((i == 0 ? j - 1 : j) & 1), wc)) { ok = false; break; }
+      }
+      uint32_t pk[64];
+      const float rs = masked ? softmax_exp_row<C::kPolyPer16, false>(sv, sl2, m, pk)
+                              : softmax_exp_row<C::kPolyPer16, true>(sv, sl2, m, pk);
+      if (OSP_SOFTMAX_TURNS) mbar_arrive(bar(B_TURN + (1 - i)));
+      l = l * alpha + rs;
+      // P_i (and O_i) are free once PV_i(j-1) has completed (separate-P layout; with P inside S
+      // the MMA warp already ordered it)
       if constexpr (C::kSepP) {
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float e0 = ex2_approx(fmaf(sv[2 * c], sl2, neg_m));
-          const float e1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, neg_m));
-          rs0 += e0;
-          rs1 += e1;
-          pk[c] = pack_bf16x2(e0, e1);
-        }
-        // P_i and O_i are free once PV_i(j-1) has completed
         if (j > 0 && !warp_wait(bar(B_OFULL + i), (j - 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        tmem_st32(tP + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-      } else {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float e0 = ex2_approx(fmaf(sv[64 * half + 2 * c], sl2, neg_m));
-            const float e1 = ex2_approx(fmaf(sv[64 * half + 2 * c + 1], sl2, neg_m));
-            rs0 += e0;
-            rs1 += e1;
-            pk[c] = pack_bf16x2(e0, e1);
-          }
-          tmem_st32(tP + 32 * half, pk);
-        }
       }
-      l = l * alpha + (rs0 + rs1);
+      tmem_st32(tP + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
