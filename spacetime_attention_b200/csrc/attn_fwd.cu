@@ -144,39 +144,45 @@ __device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
 
 // p = exp2(s * sl2 - m) for the 128 scores of one row, packed to bf16 pairs; returns the row sum.
 // kPoly: whether the polynomial takes its share (never on a tile with masked (-inf) columns).
+#ifndef OSP_EXP_BATCH
+#define OSP_EXP_BATCH 8         // exponential pairs issued before any result is consumed
+#endif
+
+// p = exp2(s * sl2 - m) for the 128 scores of one row, packed to bf16 pairs; returns the row sum.
+// The pairs are processed in batches: all exponentials of a batch are issued before any result
+// is consumed, and the row sum uses four independent accumulators, so MUFU latency overlaps
+// instead of serialising the loop.  kPoly: whether the polynomial takes its share (never on a
+// tile with masked (-inf) columns).
 template <int kPolyPer16, bool kPoly>
 __device__ __forceinline__ float softmax_exp_row(const float (&sv)[128], float sl2, float m, uint32_t (&pk)[64]) {
-  if (!OSP_F32X2 && (!kPoly || kPolyPer16 == 0)) {
-    float r0 = 0.f, r1 = 0.f;
-#pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      const float e0 = ex2_approx(fmaf(sv[2 * c], sl2, -m));
-      const float e1 = ex2_approx(fmaf(sv[2 * c + 1], sl2, -m));
-      r0 += e0;
-      r1 += e1;
-      pk[c] = pack_bf16x2(e0, e1);
-    }
-    return r0 + r1;
-  }
+  constexpr int kB = OSP_EXP_BATCH;
   const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
-  uint64_t sum2 = f2_pack(0.f, 0.f);
+  uint64_t sum2[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
-    const uint64_t x2 = f2_fma(f2_pack(sv[2 * c], sv[2 * c + 1]), scale2, negm2);
-    float e0, e1;
-    if (kPoly && (c % 16) < kPolyPer16) {
-      ex2_poly2(x2, e0, e1);
-    } else {
-      float x0, x1;
-      f2_unpack(x2, x0, x1);
-      e0 = ex2_approx(x0);
-      e1 = ex2_approx(x1);
+  for (int c0 = 0; c0 < 64; c0 += kB) {
+    float e[2 * kB];
+#pragma unroll
+    for (int t = 0; t < kB; ++t) {
+      const int c = c0 + t;
+      const uint64_t x2 = f2_fma(f2_pack(sv[2 * c], sv[2 * c + 1]), scale2, negm2);
+      if (kPoly && (c % 16) < kPolyPer16) {
+        ex2_poly2(x2, e[2 * t], e[2 * t + 1]);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        e[2 * t] = ex2_approx(x0);
+        e[2 * t + 1] = ex2_approx(x1);
+      }
     }
-    sum2 = f2_add(sum2, f2_pack(e0, e1));
-    pk[c] = pack_bf16x2(e0, e1);
+#pragma unroll
+    for (int t = 0; t < kB; ++t) {
+      sum2[t & 3] = f2_add(sum2[t & 3], f2_pack(e[2 * t], e[2 * t + 1]));
+      pk[c0 + t] = pack_bf16x2(e[2 * t], e[2 * t + 1]);
+    }
   }
+  const uint64_t s01 = f2_add(sum2[0], sum2[1]), s23 = f2_add(sum2[2], sum2[3]);
   float lo, hi;
-  f2_unpack(sum2, lo, hi);
+  f2_unpack(f2_add(s01, s23), lo, hi);
   return lo + hi;
 }
 
@@ -258,32 +264,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= kLoadWarp) {
    // each warpgroup's register budget change dominates its own role code
    regs_dec<kRegsSupport>();
+   // The producer and MMA warps run their loops with all 32 lanes converged (so addresses and
+   // descriptors stay warp-uniform) and one elected lane issues the TMA / tcgen05 instructions.
+   const bool leader = elect_one_sync();
    if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    {
       int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
-      mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
-      for (int i = 0; i < 2; ++i)
-        for (int c = 0; c < C::kChunks; ++c)
-          load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, q0 + i * kBM, g, b,
-                    p.k);
+      if (leader) {
+        mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
+        for (int i = 0; i < 2; ++i)
+          for (int c = 0; c < C::kChunks; ++c)
+            load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, q0 + i * kBM, g, b,
+                      p.k);
+      }
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % S, u = j / S;
-        if (j >= S && !mbar_wait(bar(B_KEMPTY + s), (u - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
-                    p.k);
+        if (j >= S && !warp_wait(bar(B_KEMPTY + s), (u - 1) & 1, wc)) break;
+        if (leader) {
+          mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
+                      p.k);
+        }
         k_issued = j + 1;
-        if (j >= S && !mbar_wait(bar(B_VEMPTY + s), (u - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
-                    p.k);
+        if (j >= S && !warp_wait(bar(B_VEMPTY + s), (u - 1) & 1, wc)) break;
+        if (leader) {
+          mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
+                      p.k);
+        }
         v_issued = j + 1;
       }
-      // Drain: every load this thread issued has landed before the CTA may exit.  Only the
-      // last S tiles of each ring can still be in flight.
+      // Drain: every load issued has landed before the CTA may exit.  Only the last S tiles of
+      // each ring can still be in flight.
       mbar_drain(bar(B_QFULL), 0, p.timeout_ns);
       for (int t = (k_issued > S ? k_issued - S : 0); t < k_issued; ++t)
         mbar_drain(bar(B_KFULL + t % S), (t / S) & 1, p.timeout_ns);
@@ -293,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
       // Descriptors are built once; a K step moves the start address (bits [0,14), 16-byte units)
@@ -310,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-          mma_ss(tmem + colS(i), a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+          if (leader) mma_ss(tmem + colS(i), a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       // O_i += P_i V: P_i from tensor memory (bf16 pairs, 64 columns), V MN-major (channels
@@ -319,85 +334,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t b0 = dv + (uint64_t)s * kTileStep;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + colO(i), tmem + colP(i) + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_pv,
-                 (acc || kk > 0) ? 1u : 0u);
+          if (leader)
+            mma_ts(tmem + colO(i), tmem + colP(i) + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_pv,
+                   (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(B_QFULL), 0, wc) && mbar_wait(bar(B_KFULL), 0, wc);
+      bool ok = warp_wait(bar(B_QFULL), 0, wc) && warp_wait(bar(B_KFULL), 0, wc);
       if (ok && C::kSepP) {
         // Order per KV tile j: S0(j+1) as soon as softmax 0 holds S0(j) in registers, S1(j+1)
         // likewise, then PV0(j), PV1(j) as their P tiles arrive.  O_full[i] completes after every
         // PV_i(j): the softmax waits on it before overwriting P_i and before touching O_i.
         tc_fence_after();
         issue_s(0, 0);
-        tc_commit(bar(B_SFULL + 0));
+        if (leader) tc_commit(bar(B_SFULL + 0));
         issue_s(1, 0);
-        tc_commit(bar(B_SFULL + 1));
-        tc_commit(bar(B_KEMPTY + 0));
+        if (leader) tc_commit(bar(B_SFULL + 1));
+        if (leader) tc_commit(bar(B_KEMPTY + 0));
         for (int j = 0; j < n_kv; ++j) {
           const int s = j % S, u = j / S;
           const bool more = j + 1 < n_kv;
           const int s1 = (j + 1) % S, u1 = (j + 1) / S;
           if (more) {
-            if (!mbar_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
-            if (!mbar_wait(bar(B_SFREE + 0), j & 1, wc)) break;
+            if (!warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
+            if (!warp_wait(bar(B_SFREE + 0), j & 1, wc)) break;
             tc_fence_after();
             issue_s(0, s1);
-            tc_commit(bar(B_SFULL + 0));
-            if (!mbar_wait(bar(B_SFREE + 1), j & 1, wc)) break;
+            if (leader) tc_commit(bar(B_SFULL + 0));
+            if (!warp_wait(bar(B_SFREE + 1), j & 1, wc)) break;
             tc_fence_after();
             issue_s(1, s1);
-            tc_commit(bar(B_SFULL + 1));
-            tc_commit(bar(B_KEMPTY + s1));
+            if (leader) tc_commit(bar(B_SFULL + 1));
+            if (leader) tc_commit(bar(B_KEMPTY + s1));
           }
-          if (!mbar_wait(bar(B_VFULL + s), u & 1, wc)) break;
-          if (!mbar_wait(bar(B_PREADY + 0), j & 1, wc)) break;
+          if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          if (!warp_wait(bar(B_PREADY + 0), j & 1, wc)) break;
           tc_fence_after();
           issue_pv(0, s, j > 0);
-          tc_commit(bar(B_OFULL + 0));
-          if (!mbar_wait(bar(B_PREADY + 1), j & 1, wc)) break;
+          if (leader) tc_commit(bar(B_OFULL + 0));
+          if (!warp_wait(bar(B_PREADY + 1), j & 1, wc)) break;
           tc_fence_after();
           issue_pv(1, s, j > 0);
-          tc_commit(bar(B_OFULL + 1));
-          tc_commit(bar(B_VEMPTY + s));
+          if (leader) tc_commit(bar(B_OFULL + 1));
+          if (leader) tc_commit(bar(B_VEMPTY + s));
         }
       } else if (ok) {
         tc_fence_after();
         issue_s(0, 0);
-        tc_commit(bar(B_SFULL + 0));
+        if (leader) tc_commit(bar(B_SFULL + 0));
         issue_s(1, 0);
-        tc_commit(bar(B_SFULL + 1));
-        tc_commit(bar(B_KEMPTY + 0));
+        if (leader) tc_commit(bar(B_SFULL + 1));
+        if (leader) tc_commit(bar(B_KEMPTY + 0));
         for (int j = 0; j < n_kv; ++j) {
           const int s = j % S, u = j / S;
           const bool more = j + 1 < n_kv;
           const int s1 = (j + 1) % S, u1 = (j + 1) / S;
-          if (!mbar_wait(bar(B_VFULL + s), u & 1, wc)) break;
-          if (more && !mbar_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
-          if (!mbar_wait(bar(B_PREADY + 0), j & 1, wc)) break;
+          if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          if (more && !warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
+          if (!warp_wait(bar(B_PREADY + 0), j & 1, wc)) break;
           tc_fence_after();
           issue_pv(0, s, j > 0);
           if (more) {
             issue_s(0, s1);
-            tc_commit(bar(B_SFULL + 0));
+            if (leader) tc_commit(bar(B_SFULL + 0));
           } else {
-            tc_commit(bar(B_OFULL + 0));
+            if (leader) tc_commit(bar(B_OFULL + 0));
           }
-          if (!mbar_wait(bar(B_PREADY + 1), j & 1, wc)) break;
+          if (!warp_wait(bar(B_PREADY + 1), j & 1, wc)) break;
           tc_fence_after();
           issue_pv(1, s, j > 0);
-          tc_commit(bar(B_VEMPTY + s));
+          if (leader) tc_commit(bar(B_VEMPTY + s));
           if (more) {
             issue_s(1, s1);
-            tc_commit(bar(B_SFULL + 1));
-            tc_commit(bar(B_KEMPTY + s1));
+            if (leader) tc_commit(bar(B_SFULL + 1));
+            if (leader) tc_commit(bar(B_KEMPTY + s1));
           } else {
-            tc_commit(bar(B_OFULL + 1));
+            if (leader) tc_commit(bar(B_OFULL + 1));
           }
         }
       }
       // Drain: all issued MMAs complete before tensor memory is freed.
-      tc_commit(bar(B_MMADONE));
+      if (leader) tc_commit(bar(B_MMADONE));
       mbar_drain(bar(B_MMADONE), 0, p.timeout_ns);
     }
     __syncwarp();

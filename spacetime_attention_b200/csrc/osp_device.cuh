@@ -61,16 +61,26 @@ struct WaitCtx {
   uint64_t timeout_ns;
 };
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes or `ns` pass,
+// instead of spinning and taking issue slots from the other warps of its sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0; it < (1u << 28); ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 31u) {
-      if (*w.abort) return false;
-      // another CTA already gave up: this launch's output is invalid anyway
-      if (*reinterpret_cast<volatile unsigned*>(w.status) & kDevTimeout) break;
-      if (global_timer_ns() - t0 > w.timeout_ns) break;
-    }
+  for (uint32_t it = 0; it < (1u << 24); ++it) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (*w.abort) return false;
+    // another CTA already gave up: this launch's output is invalid anyway
+    if (*reinterpret_cast<volatile unsigned*>(w.status) & kDevTimeout) break;
+    if (global_timer_ns() - t0 > w.timeout_ns) break;
   }
   *w.abort = 1;
   atomicOr(w.status, kDevTimeout);
@@ -85,11 +95,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 // Bounded wait that ignores the abort flag (used on the exit path to drain in-flight work).
 static __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0; it < (1u << 28); ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 31u && global_timer_ns() - t0 > timeout_ns) return false;
+  for (uint32_t it = 0; it < (1u << 24); ++it) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (global_timer_ns() - t0 > timeout_ns) return false;
   }
   return false;
+}
+
+// One lane of a converged warp (the same lane every time for a full mask).
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred;
+  asm volatile("{ .reg .pred p; .reg .b32 r; elect.sync r|p, 0xffffffff; selp.u32 %0, 1, 0, p; }" : "=r"(pred));
+  return pred != 0;
 }
 
 // ------------------------------------------------------------------------------------------
