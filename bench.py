@@ -128,6 +128,15 @@ class ClockSampler:
 # our arm
 # ------------------------------------------------------------------------------------------
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank float over the process group (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def step_fns(w, q, k, v, qr, kr, o, launch_events=None):
     """Returns step() running one pass of the hot path (all launches on torch's current stream)."""
     def attn():
@@ -166,6 +175,65 @@ def step_flops(w) -> float:
     return 2 * w.skiparse_flops() if sparse(w) else w.dense_flops()
 
 
+def run_hbm_op(args, rank, world, local_rank):
+    """Time one HBM-bound row of the path alone: osp_rope3d, osp_skiparse_gather (q, k, v with
+    RoPE) or osp_skiparse_scatter.  Several input sets rotate so that every launch streams its
+    bytes from DRAM rather than L2.  value = algorithmic bytes / time (GB/s)."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = syn.WORKLOADS[args.workload]
+    nset = 3
+    sets = []
+    for r in range(nset):
+        q, k, v = (t.to(dev) for t in syn.make_qkv(w, w.seed + 101 * r))
+        sets.append((q, k, v))
+    esz = 2
+    if args.op == "rope":
+        outs = [(torch.empty_like(q), torch.empty_like(k)) for q, k, _ in sets]
+        nbytes = w.rope_bytes() + (4 * w.B * w.text_len * w.heads * w.head_dim * esz)  # text rows copied
+        def launch(i):
+            q, k, _ = sets[i % nset]
+            ops.rope3d(q, k, w.grid, w.text_len, w.split, q_out=outs[i % nset][0], k_out=outs[i % nset][1])
+    else:
+        if not w.skiparse_k or w.text_len:
+            raise SystemExit(f"--op {args.op} needs a Skiparse workload without text tokens")
+        kk = w.skiparse_k
+        if args.op == "gather":
+            nbytes = 3 * 2 * w.B * w.n_video * w.heads * w.head_dim * esz
+            def launch(i):
+                q, k, v = sets[i % nset]
+                ops.skiparse_gather(q, k, v, w.grid, kk, ops.OSP_SKIP_GROUP, split=w.split)
+        else:
+            nbytes = 2 * w.B * w.n_video * w.heads * w.head_dim * esz
+            outs = [torch.empty_like(v) for _, _, v in sets]
+            def launch(i):
+                _, _, v = sets[i % nset]
+                ops.skiparse_scatter(v.view(w.B * kk, w.n_video // kk, w.heads, w.head_dim), w.grid, kk,
+                                     ops.OSP_SKIP_GROUP, o=outs[i % nset])
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        launch(i)
+    t1.record()
+    torch.cuda.synchronize()
+    ops.check_status(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    peaks, src = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"metric": f"{args.op} GB/s (HBM-bound row of the path)", "value": round(world * gbs, 1), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(w.describe(), op=args.op, bytes_per_launch=nbytes,
+                           l2=f"{nset} input sets rotated ({nbytes * nset / 1e6:.0f} MB)"),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                         "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "traffic": None,
+                         "peak_source": f"{src} (copy bandwidth)"},
+            "gpu_launches": args.steps}
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -199,12 +267,8 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clocks = sampler.stop()
     ops.check_status(dev)
-    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     attn_ms = float(np.mean([a.elapsed_time(b) for a, b in events]))
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
 
     # ---- end to end through the public API: pinned host inputs -> device -> hot path -> host
     qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
@@ -230,11 +294,7 @@ def run_ours(args, rank, world, local_rank):
     b.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dev)
     ops.check_status(dev)
 
     flops = step_flops(w)
@@ -381,6 +441,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse"],
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
+    ap.add_argument("--op", default="step", choices=["step", "rope", "gather", "scatter"],
+                    help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -406,7 +468,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = run_ours(args, rank, world, local_rank) if args.op == "step" else run_hbm_op(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

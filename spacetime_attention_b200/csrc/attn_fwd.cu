@@ -102,6 +102,7 @@ struct AttnParams {
   __nv_bfloat16* o;
   unsigned* status;
   unsigned long long timeout_ns;
+  int debug_withhold_q;   // test knob: never load Q, so every consumer's bounded wait runs out
 };
 
 __device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
@@ -271,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     {
       int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
-      if (leader) {
+      const bool q_armed = !p.debug_withhold_q;
+      if (leader && q_armed) {
         mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
         for (int i = 0; i < 2; ++i)
           for (int c = 0; c < C::kChunks; ++c)
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: every load issued has landed before the CTA may exit.  Only the last S tiles of
       // each ring can still be in flight.
-      mbar_drain(bar(B_QFULL), 0, p.timeout_ns);
+      if (q_armed) mbar_drain(bar(B_QFULL), 0, p.timeout_ns);
       for (int t = (k_issued > S ? k_issued - S : 0); t < k_issued; ++t)
         mbar_drain(bar(B_KFULL + t % S), (t / S) & 1, p.timeout_ns);
       for (int t = (v_issued > S ? v_issued - S : 0); t < v_issued; ++t)
@@ -634,6 +636,7 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.o = static_cast<__nv_bfloat16*>(o);
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
+  p.debug_withhold_q = debug_withhold_q();
   CUtensorMap tq, tk, tv;
   int rc;
   if ((rc = make_tmap(&tq, q, s, N, layout, p.k)) != OSP_OK) return rc;

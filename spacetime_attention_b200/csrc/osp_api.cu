@@ -112,12 +112,14 @@ unsigned* device_status_word() {
 }
 
 uint64_t wait_timeout_ns() {
-  static const uint64_t ns = [] {
-    const char* e = getenv("OSP_WAIT_TIMEOUT_MS");
-    const long long ms = e ? atoll(e) : 2000;
-    return (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
-  }();
-  return ns;
+  const char* e = getenv("OSP_WAIT_TIMEOUT_MS");
+  const long long ms = e ? atoll(e) : 2000;
+  return (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
+}
+
+int debug_withhold_q() {
+  const char* e = getenv("OSP_DEBUG_WITHHOLD_Q");
+  return (e && e[0] == '1') ? 1 : 0;
 }
 
 }  // namespace osp

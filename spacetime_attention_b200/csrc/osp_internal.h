@@ -23,8 +23,13 @@ int device_sm_count();
 // Per-device status word (allocated on first use, kept until exit).
 unsigned* device_status_word();
 
-// Bounded-wait limit for the attention kernels, in nanoseconds.
+// Bounded-wait limit for the attention kernels, in nanoseconds (OSP_WAIT_TIMEOUT_MS, default
+// 2000 ms; read on every launch).
 uint64_t wait_timeout_ns();
+
+// Test knob (OSP_DEBUG_WITHHOLD_Q=1, read on every launch): the attention kernel never loads Q,
+// so its bounded waits run out and the launch reports OSP_ERR_TIMEOUT through osp_check_status.
+int debug_withhold_q();
 
 int rope3d_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_shape& s,
                   const osp_rope& rope, cudaStream_t stream);

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
   long long* dst_row = src_row + p.rows_per_tile;                            // [rows_per_tile]
   int* vid = reinterpret_cast<int*>(dst_row + p.rows_per_tile);              // video index or -1
   double2* cs = reinterpret_cast<double2*>(vid + ((p.rows_per_tile + 3) & ~3)); // [tile][pairs]
+  uint16_t* colpair = reinterpret_cast<uint16_t*>(cs + p.rows_per_tile * (p.head_dim >> 1));  // [vpr]
 
   const int npairs = p.head_dim >> 1;
   // Frequencies of every channel pair: pair j of a chunk of size d_a -> theta^(-2j/d_a).
@@ -77,6 +78,8 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
     else { j = i - (p.d_t + p.d_h) / 2; da = p.d_w; }
     omega[i] = exp2(-(2.0 * j / da) * p.log2_theta);
   }
+  // first channel pair of every 16-byte column of a token row (8 channels = 4 pairs per column)
+  for (int c = threadIdx.x; c < p.vpr; c += kThreads) colpair[c] = (uint16_t)((c % (p.head_dim >> 3)) * 4);
   const int HW = p.H * p.W;
   const int per_set = (MAP == kMapIdentity) ? 0 : p.N / p.sparse_k;
 
@@ -124,33 +127,35 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
       }
       __syncthreads();
     }
-    const int per_head_vec = p.head_dim >> 3;
+    // Flattened (row, 16-byte column) walk over the tile: thread i starts at vector i and
+    // advances by kThreads vectors; (row, col) is stepped incrementally (no division per vector).
+    const int drow = kThreads / p.vpr, dcol = kThreads - drow * p.vpr;
+    const int total = nrows * p.vpr;
     for (int t = 0; t < p.n_tensors; ++t) {
       const uint4* __restrict__ src = p.src[t];
       uint4* dst = p.dst[t];
       const bool rot = (p.rope_mask >> t) & 1u;
       const bool inplace = (const void*)src == (const void*)dst;
-      const int total = nrows * p.vpr;
-      // 4 independent vectors in flight per thread
+      int row = threadIdx.x / p.vpr, col = threadIdx.x - (threadIdx.x / p.vpr) * p.vpr;
       for (int base = threadIdx.x; base < total; base += 4 * kThreads) {
         uint4 val[4];
-        int rowi[4], col[4];
+        int rowi[4], coli[4];
         bool live[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx = base + u * kThreads;
-          live[u] = idx < total;
-          rowi[u] = live[u] ? idx / p.vpr : 0;
-          col[u] = live[u] ? idx - rowi[u] * p.vpr : 0;
-          if (live[u] && inplace && vid[rowi[u]] < 0) live[u] = false;  // text row, in place
-          if (live[u]) val[u] = src[src_row[rowi[u]] * p.vpr + col[u]];
+        for (int u = 0; u < 4; ++u) {  // 4 independent 16-byte loads in flight per thread
+          rowi[u] = row;
+          coli[u] = col;
+          live[u] = base + u * kThreads < total && !(inplace && vid[row] < 0);  // text row in place: skip
+          if (live[u]) val[u] = src[src_row[row] * p.vpr + col];
+          col += dcol;
+          row += drow;
+          if (col >= p.vpr) { col -= p.vpr; ++row; }
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (!live[u]) continue;
           if (rot && vid[rowi[u]] >= 0) {
-            const int pair0 = (col[u] % per_head_vec) * 4;
-            const double2* tab = cs + rowi[u] * npairs + pair0;
+            const double2* tab = cs + rowi[u] * npairs + colpair[coli[u]];
             uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
             }
             val[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          dst[dst_row[rowi[u]] * p.vpr + col[u]] = val[u];
+          dst[dst_row[rowi[u]] * p.vpr + coli[u]] = val[u];
         }
       }
     }
@@ -181,13 +186,14 @@ __global__ void index_map_kernel(int n_video, int k, int mode, int* out) {
 
 int launch_permute(int map, PermuteParams& p, cudaStream_t stream) {
   const int npairs = p.head_dim / 2;
-  // ~1024 vectors per tile, at most 32 rows, and the cos/sin table within 40 KB of shared memory
+  // ~4096 vectors (64 KB of one tensor) per tile, at most 64 rows, and the cos/sin table within
+  // 40 KB of shared memory
   const int table_rows = (40 * 1024) / (npairs * (int)sizeof(double2));
-  p.rows_per_tile = (int)std::max(1, std::min(std::min(32, table_rows), (1024 + p.vpr - 1) / p.vpr));
+  p.rows_per_tile = (int)std::max(1, std::min(std::min(64, table_rows), (4096 + p.vpr - 1) / p.vpr));
   p.n_tiles = (p.rows + p.rows_per_tile - 1) / p.rows_per_tile;
   const size_t smem = kMaxPairs * sizeof(double) + 2 * p.rows_per_tile * sizeof(long long) +
                       ((p.rows_per_tile + 3) & ~3) * sizeof(int) +
-                      (size_t)p.rows_per_tile * npairs * sizeof(double2);
+                      (size_t)p.rows_per_tile * npairs * sizeof(double2) + (size_t)p.vpr * sizeof(uint16_t);
   const int sms = device_sm_count();
   const long long grid = std::min<long long>(p.n_tiles, (long long)sms * 8);
   if (grid <= 0) return OSP_OK;
