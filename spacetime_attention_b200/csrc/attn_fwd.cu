@@ -45,8 +45,16 @@ constexpr uint32_t kRegsSoftmax = 200;
 constexpr uint32_t kRegsSupport = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSupport == kThreads * kRegsLaunch,
               "register split must equal the launch allocation");
+#ifndef OSP_MMA_WARP
+#define OSP_MMA_WARP 9          // warp 8 loads; the MMA warp is 9, 10 or 11 (the idle ones fill the warpgroup)
+#endif
+#ifndef OSP_SPLIT_MMA
+#define OSP_SPLIT_MMA 2         // separate-P layout: 1 = QK^T on warp 10, PV on warp 9;
+#endif                          // 2 = QK^T on warp 10, PV of tile 0 on warp 9, of tile 1 on warp 11
 constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = OSP_MMA_WARP;
+constexpr int kQkWarp = 10;
+constexpr int kPv1Warp = 11;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -87,7 +95,7 @@ struct Cfg {
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
   // o_full[2], mma_done, s_free[2], turn[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 11;
+  static constexpr int kNumBars = 1 + 4 * kStages + 13;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -209,6 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_SFULL = 1 + 4 * S, B_PREADY = B_SFULL + 2, B_OFULL = B_PREADY + 2, B_MMADONE = B_OFULL + 2;
   const int B_SFREE = B_MMADONE + 1;  // separate-P layout: softmax has S_i in registers
   const int B_TURN = B_SFREE + 2;     // softmax i may start its exponentials (MUFU hand-off)
+  const int B_QKDONE = B_TURN + 2;    // split MMA issue: the QK^T warp's final commit
+  const int B_PV1DONE = B_QKDONE + 1; // split MMA issue: the tile-1 PV warp's final commit
+  constexpr bool kSplitMma = C::kSepP && OSP_SPLIT_MMA > 0;
+  constexpr bool kSplitPv = C::kSepP && OSP_SPLIT_MMA > 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -225,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_KEMPTY + s), 1);
       mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_VEMPTY + s), 1);
+      mbar_init(bar(B_VEMPTY + s), kSplitPv ? 2 : 1);   // both PV issuers release a V stage
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
@@ -235,6 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_MMADONE), 1);
     mbar_init(bar(B_SFREE + 0), 128);
     mbar_init(bar(B_SFREE + 1), 128);
+    mbar_init(bar(B_QKDONE), 1);
+    mbar_init(bar(B_PV1DONE), 1);
     mbar_init(bar(B_TURN + 0), 128);
     mbar_init(bar(B_TURN + 1), 128);
     *abort_flag = 0;
@@ -308,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(bar(B_VFULL + t % S), (t / S) & 1, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || (kSplitMma && warp == kQkWarp) || (kSplitPv && warp == kPv1Warp)) {
     // ------------------------------------------------------------------ MMA issuer
     {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
@@ -342,21 +356,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       bool ok = warp_wait(bar(B_QFULL), 0, wc) && warp_wait(bar(B_KFULL), 0, wc);
+      // which MMAs this warp issues (one warp issues all of them unless the issue is split)
+      const bool do_qk = !kSplitMma || warp == kQkWarp;
+      const bool do_pv0 = !kSplitMma || warp == kMmaWarp;
+      const bool do_pv1 = !kSplitMma || (kSplitPv ? warp == kPv1Warp : warp == kMmaWarp);
       if (ok && C::kSepP) {
         // Order per KV tile j: S0(j+1) as soon as softmax 0 holds S0(j) in registers, S1(j+1)
         // likewise, then PV0(j), PV1(j) as their P tiles arrive.  O_full[i] completes after every
         // PV_i(j): the softmax waits on it before overwriting P_i and before touching O_i.
         tc_fence_after();
-        issue_s(0, 0);
-        if (leader) tc_commit(bar(B_SFULL + 0));
-        issue_s(1, 0);
-        if (leader) tc_commit(bar(B_SFULL + 1));
-        if (leader) tc_commit(bar(B_KEMPTY + 0));
+        if (do_qk) {
+          issue_s(0, 0);
+          if (leader) tc_commit(bar(B_SFULL + 0));
+          issue_s(1, 0);
+          if (leader) tc_commit(bar(B_SFULL + 1));
+          if (leader) tc_commit(bar(B_KEMPTY + 0));
+        }
         for (int j = 0; j < n_kv; ++j) {
           const int s = j % S, u = j / S;
           const bool more = j + 1 < n_kv;
           const int s1 = (j + 1) % S, u1 = (j + 1) / S;
-          if (more) {
+          if (do_qk && more) {
             if (!warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
             if (!warp_wait(bar(B_SFREE + 0), j & 1, wc)) break;
             tc_fence_after();
@@ -368,16 +388,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) tc_commit(bar(B_SFULL + 1));
             if (leader) tc_commit(bar(B_KEMPTY + s1));
           }
-          if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
-          if (!warp_wait(bar(B_PREADY + 0), j & 1, wc)) break;
-          tc_fence_after();
-          issue_pv(0, s, j > 0);
-          if (leader) tc_commit(bar(B_OFULL + 0));
-          if (!warp_wait(bar(B_PREADY + 1), j & 1, wc)) break;
-          tc_fence_after();
-          issue_pv(1, s, j > 0);
-          if (leader) tc_commit(bar(B_OFULL + 1));
-          if (leader) tc_commit(bar(B_VEMPTY + s));
+          if (do_pv0 || do_pv1) {
+            if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          }
+          if (do_pv0) {
+            if (!warp_wait(bar(B_PREADY + 0), j & 1, wc)) break;
+            tc_fence_after();
+            issue_pv(0, s, j > 0);
+            if (leader) tc_commit(bar(B_OFULL + 0));
+            if (kSplitPv && leader) tc_commit(bar(B_VEMPTY + s));
+          }
+          if (do_pv1) {
+            if (!warp_wait(bar(B_PREADY + 1), j & 1, wc)) break;
+            tc_fence_after();
+            issue_pv(1, s, j > 0);
+            if (leader) tc_commit(bar(B_OFULL + 1));
+            if (leader) tc_commit(bar(B_VEMPTY + s));
+          }
         }
       } else if (ok) {
         tc_fence_after();
@@ -415,8 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Drain: all issued MMAs complete before tensor memory is freed.
-      if (leader) tc_commit(bar(B_MMADONE));
-      mbar_drain(bar(B_MMADONE), 0, p.timeout_ns);
+      const int done_bar = (kSplitMma && warp == kQkWarp) ? B_QKDONE : (kSplitPv && warp == kPv1Warp) ? B_PV1DONE : B_MMADONE;
+      if (leader) tc_commit(bar(done_bar));
+      mbar_drain(bar(done_bar), 0, p.timeout_ns);
     }
     __syncwarp();
    }
