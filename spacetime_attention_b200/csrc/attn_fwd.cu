@@ -51,6 +51,9 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsSupport == kThreads * kRegsLau
 #ifndef OSP_SPLIT_MMA
 #define OSP_SPLIT_MMA 2         // separate-P layout: 1 = QK^T on warp 10, PV on warp 9;
 #endif                          // 2 = QK^T on warp 10, PV of tile 0 on warp 9, of tile 1 on warp 11
+#ifndef OSP_SPLIT_MMA_TILES
+#define OSP_SPLIT_MMA_TILES 1   // P inside S at d = 96: tile 0's MMAs on warp 9, tile 1's on warp 11
+#endif
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = OSP_MMA_WARP;
 constexpr int kQkWarp = 10;
@@ -221,6 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_PV1DONE = B_QKDONE + 1; // split MMA issue: the tile-1 PV warp's final commit
   constexpr bool kSplitMma = C::kSepP && OSP_SPLIT_MMA > 0;
   constexpr bool kSplitPv = C::kSepP && OSP_SPLIT_MMA > 1;
+  // per-tile issuers (9 and 11) pay at d = 96 (+2 %); at d = 128 the tensor pipe is the bottleneck
+  // and interleaving the two tiles' MMA streams delays each tile (-7 %)
+  constexpr bool kSplitTiles = !C::kSepP && D == 96 && OSP_SPLIT_MMA_TILES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -235,9 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_QFULL), 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_KEMPTY + s), kSplitTiles ? 2 : 1);   // per-tile issuers both release K
       mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_VEMPTY + s), kSplitPv ? 2 : 1);   // both PV issuers release a V stage
+      mbar_init(bar(B_VEMPTY + s), (kSplitPv || kSplitTiles) ? 2 : 1);   // both PV issuers release V
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
@@ -322,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(bar(B_VFULL + t % S), (t / S) & 1, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp || (kSplitMma && warp == kQkWarp) || (kSplitPv && warp == kPv1Warp)) {
+  } else if (warp == kMmaWarp || (kSplitMma && warp == kQkWarp) || ((kSplitPv || kSplitTiles) && warp == kPv1Warp)) {
     // ------------------------------------------------------------------ MMA issuer
     {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
@@ -406,6 +412,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) tc_commit(bar(B_VEMPTY + s));
           }
         }
+      } else if (ok && kSplitTiles) {
+        // P inside S: per tile, PV_i(j) must precede S_i(j+1) (the tensor pipe runs one thread's
+        // MMAs in order); the two tiles are independent, so each has its own issuing warp.
+        const int ti = (warp == kPv1Warp) ? 1 : 0;
+        tc_fence_after();
+        issue_s(ti, 0);
+        if (leader) tc_commit(bar(B_SFULL + ti));
+        if (leader) tc_commit(bar(B_KEMPTY + 0));
+        for (int j = 0; j < n_kv; ++j) {
+          const int s = j % S, u = j / S;
+          const bool more = j + 1 < n_kv;
+          const int s1 = (j + 1) % S, u1 = (j + 1) / S;
+          if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          if (more && !warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
+          if (!warp_wait(bar(B_PREADY + ti), j & 1, wc)) break;
+          tc_fence_after();
+          issue_pv(ti, s, j > 0);
+          if (leader) tc_commit(bar(B_VEMPTY + s));
+          if (more) {
+            issue_s(ti, s1);
+            if (leader) tc_commit(bar(B_SFULL + ti));
+            if (leader) tc_commit(bar(B_KEMPTY + s1));
+          } else {
+            if (leader) tc_commit(bar(B_OFULL + ti));
+          }
+        }
       } else if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -442,7 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Drain: all issued MMAs complete before tensor memory is freed.
-      const int done_bar = (kSplitMma && warp == kQkWarp) ? B_QKDONE : (kSplitPv && warp == kPv1Warp) ? B_PV1DONE : B_MMADONE;
+      const int done_bar = (kSplitMma && warp == kQkWarp) ? B_QKDONE
+                         : ((kSplitPv || kSplitTiles) && warp == kPv1Warp) ? B_PV1DONE : B_MMADONE;
       if (leader) tc_commit(bar(done_bar));
       mbar_drain(bar(done_bar), 0, p.timeout_ns);
     }
