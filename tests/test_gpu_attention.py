@@ -148,3 +148,21 @@ def test_full_size_skiparse_sampled(gpu, name, mode):
     rows = _sample_rows(w.n_video, 24, w.seed + mode)
     ref = O.skiparse_attn_ref(to_f64(q), to_f64(k), to_f64(v), w.skiparse_k, mode, rows=rows)
     assert_attn_close(o[:, rows], ref, f"{name} mode {mode}")
+
+
+@pytest.mark.parametrize("jump", [12.0, 40.0, 200.0])
+def test_row_max_jump_in_a_late_kv_tile(gpu, jump):
+    """A key in the third KV tile scores far above everything before it (jump in log2 units of
+    the scaled score): the running max must be raised and P, O and the row sum rescaled exactly,
+    however large the jump."""
+    B, heads, d, grid = 1, 2, 64, (2, 16, 16)     # 512 tokens = 4 KV tiles
+    q, k, v, _, _, _ = _qkv(gpu, B, heads, d, grid, 0, seed=13)
+    q = q.float(); k = k.float()
+    q[:, :, :, 0] = 8.0                             # every query has a large first channel
+    key = 300                                        # token in KV tile 2
+    k[:, key, :, 0] = jump / (8.0 * 1.4426950408889634) * 8.0   # score * scale * log2(e) ~ jump
+    q = q.to(torch.bfloat16); k = k.to(torch.bfloat16)
+    o = ops.attn_full(q.to(gpu), k.to(gpu), v.to(gpu), grid, 0)
+    ops.check_status()
+    ref = O.attn_ref(to_f64(q), to_f64(k), to_f64(v))
+    assert_attn_close(o, ref, f"jump {jump}")
