@@ -25,7 +25,10 @@
  *    enqueued and osp_get_last_error() describes the problem. Device-side faults of the
  *    bounded-wait kind (OSP_ERR_TIMEOUT) are reported later by osp_check_status().
  *  Scratch. On first use per device the library allocates (cudaMalloc) one small status
- *    word and caches it until process exit. No other allocation happens in any call.
+ *    word and caches it until process exit. Attention calls whose last partial wave of work
+ *    is split over several KV ranges (see osp_attn_full) take a stream-ordered workspace
+ *    (a few MB) from a library-owned per-device memory pool created on first use; freed
+ *    blocks stay cached in that pool, so steady-state calls do not allocate from the driver.
  *  Threads. Entry points may be called from several host threads; the last-error message is
  *    per thread.
  */
@@ -90,6 +93,10 @@ int osp_rope3d(const void* q, const void* k, void* q_out, void* k_out, const osp
  *  softmax_scale: <= 0 selects 1/sqrt(head_dim).
  *  Arithmetic: bf16 operands on tcgen05 tensor cores, fp32 accumulation in tensor memory,
  *    fp32 online softmax, probabilities rounded to bf16 for the PV product, O rounded to bf16.
+ *  Work split: the (sample, head, 256-query block) units run one per SM; when the last wave
+ *    would leave SMs idle, its units are split into 2-8 KV ranges whose fp32 partials are merged
+ *    exactly (log-sum-exp) by a second kernel. Results then differ from the unsplit order only
+ *    in fp32 summation order. OSP_SPLIT_KV=0 in the environment disables the split.
  *  Errors: OSP_ERR_INVALID_ARG, OSP_ERR_UNSUPPORTED (head_dim not 64/96/128), OSP_ERR_CUDA. */
 int osp_attn_full(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                   float softmax_scale, void* stream);
@@ -144,7 +151,9 @@ int osp_skiparse_index_map(int32_t n_video, int32_t sparse_k, int32_t mode, int3
  *    `stream` before its kernel. Calls that overlap on the GPU (different streams) race on it.
  *  Errors: as osp_attn_full. A bounded-wait timeout inside this call is recorded in the static
  *    word, which osp_check_status does not read: the kernel still ends, its output is invalid.
- *  Arguments, layout, arithmetic and results are those of osp_attn_full (bit-identical). */
+ *  Arguments, layout and arithmetic are those of osp_attn_full, without its split of the last
+ *    wave (which needs a workspace): results are bit-identical whenever osp_attn_full does not
+ *    split, and otherwise differ only in fp32 summation order. */
 int osp_attn_full_noalloc(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                           float softmax_scale, void* stream);
 

@@ -114,6 +114,15 @@ struct AttnParams {
   unsigned* status;
   unsigned long long timeout_ns;
   int debug_withhold_q;   // test knob: never load Q, so every consumer's bounded wait runs out
+  // Work items (1-D grid): units are (sample*set, head, query block) with the query block fastest.
+  // CTAs [0, n_full) process whole units; every later unit is split into n_split KV ranges whose
+  // CTAs write fp32 partials (unnormalised O, running max m, row sum l) to ws_o / ws_ml, merged
+  // by attn_combine_kernel.
+  int qblocks;            // 256-row query blocks per (sample*set, head)
+  int n_full;
+  int n_split;
+  float* ws_o;            // [split units][n_split][256][D]
+  float2* ws_ml;          // [split units][n_split][256]
 };
 
 __device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
@@ -231,11 +240,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z / p.G, g = blockIdx.z % p.G;
-  const int q0 = blockIdx.x * (2 * kBM);
-  const int n_kv = (p.n + kBN - 1) / kBN;
-  const int chan0 = h * D;
+  // work item -> unit (sample*set, head, query block) and KV tile range [kv_lo, kv_lo + n_kv).
+  // Recomputed where needed (cheap integer math) rather than kept live across the main loops.
+  struct Work { int unit, part, h, b, g, q0, kv_lo, n_kv; };
+  auto decode = [&]() {
+    Work w;
+    w.unit = blockIdx.x;
+    w.part = -1;
+    if (w.unit >= p.n_full) {
+      const int t = w.unit - p.n_full;
+      w.unit = p.n_full + t / p.n_split;
+      w.part = t % p.n_split;
+    }
+    const int qb = w.unit % p.qblocks, hb = w.unit / p.qblocks;
+    w.h = hb % p.heads;
+    const int bg = hb / p.heads;
+    w.b = bg / p.G;
+    w.g = bg % p.G;
+    w.q0 = qb * (2 * kBM);
+    const int n_kv_all = (p.n + kBN - 1) / kBN;
+    w.kv_lo = w.part < 0 ? 0 : (int)((long long)w.part * n_kv_all / p.n_split);
+    w.n_kv = (w.part < 0 ? n_kv_all : (int)((long long)(w.part + 1) * n_kv_all / p.n_split)) - w.kv_lo;
+    return w;
+  };
+  const Work wk = decode();
+  const int n_kv = wk.n_kv;
+  const int chan0 = wk.h * D;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -297,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
         for (int i = 0; i < 2; ++i)
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, q0 + i * kBM, g, b,
+            load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, wk.q0 + i * kBM, wk.g, wk.b,
                       p.k);
       }
       for (int j = 0; j < n_kv; ++j) {
@@ -306,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
+            load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, (wk.kv_lo + j) * kBN, wk.g, wk.b,
                       p.k);
         }
         k_issued = j + 1;
@@ -314,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, j * kBN, g, b,
+            load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, (wk.kv_lo + j) * kBN, wk.g, wk.b,
                       p.k);
         }
         v_issued = j + 1;
@@ -494,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    const int valid0 = p.n - wk.kv_lo * kBN;   // valid keys from this CTA's first KV tile on
     for (int j = 0; j < n_kv; ++j) {
       if (!warp_wait(bar(B_SFULL + i), j & 1, wc)) { ok = false; break; }
       tc_fence_after();
@@ -510,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sv[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-      const int valid = p.n - j * kBN;
+      const int valid = valid0 - j * kBN;
       const bool masked = valid < kBN;
       if (masked) {
 #pragma unroll
@@ -569,9 +600,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && warp_wait(bar(B_OFULL + i), C::kSepP ? (uint32_t)((n_kv - 1) & 1) : 0u, wc)) {
       tc_fence_after();
+      const Work w = decode();
+      const int unit = w.unit, part = w.part, h = w.h, b = w.b, g = w.g;
       const float inv_l = 1.f / l;
-      const int slot = q0 + i * kBM + row;
+      const int slot = w.q0 + i * kBM + row;
       const bool live = slot < p.n;
+      if (part >= 0) {
+        // split unit: unnormalised fp32 O (relative to m) and (m, l) for the combine kernel
+        const size_t prow = ((size_t)(unit - p.n_full) * p.n_split + part) * (2 * kBM) + i * kBM + row;
+        float4* wo = reinterpret_cast<float4*>(p.ws_o + prow * D);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * cc, o);
+          tmem_wait_ld();
+          if (live) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              wo[8 * cc + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                           __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          }
+        }
+        if (live) p.ws_ml[prow] = make_float2(m, l);
+      } else {
       const int token = slot_token(p.layout, live ? slot : 0, g, p.k);
       uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N + token) * p.heads + h) * D);
 #pragma unroll
@@ -588,6 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int v = 0; v < 4; ++v) dst[4 * cc + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
       }
+      }
     }
   }
   tc_fence_before();
@@ -596,6 +648,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Merges the n_split partials of every split unit: with m_s, l_s, O_s (O_s unnormalised,
+// relative to 2^m_s, m in log2 units), M = max m_s, w_s = 2^(m_s - M):
+//   O = sum_s w_s O_s / sum_s w_s l_s.
+// One warp per query row; lanes cover the head's D channels.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, int n_units) {
+  constexpr int kPer = D / 32;
+  const int wid = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (wid >= n_units * 2 * kBM) return;
+  const int su = wid / (2 * kBM), r = wid % (2 * kBM);
+  const int unit = p.n_full + su;
+  const int qb = unit % p.qblocks, hb = unit / p.qblocks;
+  const int h = hb % p.heads, bg = hb / p.heads;
+  const int b = bg / p.G, g = bg % p.G;
+  const int slot = qb * 2 * kBM + r;
+  if (slot >= p.n) return;
+  float mmax = -INFINITY;
+  for (int s = 0; s < p.n_split; ++s)
+    mmax = fmaxf(mmax, p.ws_ml[((size_t)su * p.n_split + s) * (2 * kBM) + r].x);
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float lsum = 0.f;
+  for (int s = 0; s < p.n_split; ++s) {
+    const size_t prow = ((size_t)su * p.n_split + s) * (2 * kBM) + r;
+    const float2 ml = p.ws_ml[prow];
+    const float wgt = exp2f(ml.x - mmax);
+    lsum += wgt * ml.y;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] += wgt * p.ws_o[prow * D + e * 32 + lane];
+  }
+  const float inv = 1.f / lsum;
+  const int token = slot_token(p.layout, slot, g, p.k);
+  __nv_bfloat16* dst = p.o + (((size_t)b * p.N + token) * p.heads + h) * D;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) dst[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -682,7 +772,7 @@ namespace {
 
 // Attention launch with an explicit status word (the kernel's only global scratch).
 int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
-                       int sparse_k, float scale, cudaStream_t stream, unsigned* status) {
+                       int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split) {
   const int N = s.text_len + s.T * s.H * s.W;
   const int G = (layout == 0) ? 1 : sparse_k;
   const int n = N / G;
@@ -704,16 +794,53 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   if ((rc = make_tmap(&tk, k, s, N, layout, p.k)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tv, v, s, N, layout, p.k)) != OSP_OK) return rc;
   const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
-  if ((long long)s.B * G > 65535 || s.heads > 65535)
-    return set_error(OSP_ERR_UNSUPPORTED, "B*sets (%lld) or heads (%d) exceeds the grid limit 65535",
-                     (long long)s.B * G, s.heads);
-  dim3 grid((unsigned)qblocks, (unsigned)s.heads, (unsigned)(s.B * G));
-  switch (s.head_dim) {
-    case 64: return launch_d<64>(tq, tk, tv, p, grid, stream);
-    case 96: return launch_d<96>(tq, tk, tv, p, grid, stream);
-    case 128: return launch_d<128>(tq, tk, tv, p, grid, stream);
-    default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  const long long units = qblocks * s.heads * (long long)s.B * G;
+  if (units > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld attention work units is too many", units);
+  p.qblocks = (int)qblocks;
+  p.n_full = (int)units;
+  p.n_split = 1;
+  // Split-KV for the last partial wave (one CTA per SM): its R units are split into KV ranges so
+  // that about one wave of CTAs runs them.  Needs a workspace, so only where allocation is allowed.
+  const int n_kv = (n + kBN - 1) / kBN;
+  const int sms = device_sm_count();
+  const int rem = (int)(units % sms);
+  if (allow_split && split_kv_enabled() && rem > 0) {
+    const int ns = std::min(std::min(sms / rem, n_kv / 2), 8);
+    if (ns >= 2) {
+      p.n_full = (int)(units - rem);
+      p.n_split = ns;
+    }
   }
+  void* ws = nullptr;
+  if (p.n_split > 1) {
+    const size_t rows = (size_t)(units - p.n_full) * p.n_split * 2 * kBM;
+    const size_t bytes = rows * (size_t)s.head_dim * sizeof(float) + rows * sizeof(float2);
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", bytes);
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_ml = reinterpret_cast<float2*>(p.ws_o + rows * (size_t)s.head_dim);
+  }
+  const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
+  dim3 grid((unsigned)ctas);
+  switch (s.head_dim) {
+    case 64: rc = launch_d<64>(tq, tk, tv, p, grid, stream); break;
+    case 96: rc = launch_d<96>(tq, tk, tv, p, grid, stream); break;
+    case 128: rc = launch_d<128>(tq, tk, tv, p, grid, stream); break;
+    default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  }
+  if (rc == OSP_OK && p.n_split > 1) {
+    const int su = (int)(units - p.n_full);
+    const unsigned blocks = (unsigned)(((size_t)su * 2 * kBM + 7) / 8);
+    switch (s.head_dim) {
+      case 64: attn_combine_kernel<64><<<blocks, 256, 0, stream>>>(p, su); break;
+      case 96: attn_combine_kernel<96><<<blocks, 256, 0, stream>>>(p, su); break;
+      default: attn_combine_kernel<128><<<blocks, 256, 0, stream>>>(p, su); break;
+    }
+    rc = check_launch("attn_combine_kernel");
+  }
+  if (ws) cudaFreeAsync(ws, stream);
+  return rc;
 }
 
 }  // namespace
@@ -722,7 +849,7 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
                      int sparse_k, float scale, cudaStream_t stream) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
-  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status);
+  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -798,5 +925,5 @@ extern "C" int osp_attn_full_noalloc(const void* q, const void* k, const void* v
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess)
     return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: clearing the scratch word failed");
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)s.head_dim);
-  return launch_with_status(q, k, v, o, s, 0, 1, softmax_scale, st, static_cast<unsigned*>(scratch));
+  return launch_with_status(q, k, v, o, s, 0, 1, softmax_scale, st, static_cast<unsigned*>(scratch), false);
 }

@@ -16,6 +16,7 @@ thread_local char g_last_error[512] = "";
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned* g_status[kMaxDevices] = {};
+cudaMemPool_t g_pool[kMaxDevices] = {};
 int g_sms[kMaxDevices] = {};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -111,10 +112,35 @@ unsigned* device_status_word() {
   return g_status[dev];
 }
 
+cudaMemPool_t workspace_pool() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    // keep freed workspace cached in the pool instead of returning it at every synchronisation
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pool[dev] = pool;
+  }
+  return g_pool[dev];
+}
+
 uint64_t wait_timeout_ns() {
   const char* e = getenv("OSP_WAIT_TIMEOUT_MS");
   const long long ms = e ? atoll(e) : 2000;
   return (uint64_t)(ms > 0 ? ms : 2000) * 1000000ull;
+}
+
+int split_kv_enabled() {
+  const char* e = getenv("OSP_SPLIT_KV");
+  return (e && e[0] == '0') ? 0 : 1;
 }
 
 int debug_withhold_q() {

@@ -31,6 +31,13 @@ uint64_t wait_timeout_ns();
 // so its bounded waits run out and the launch reports OSP_ERR_TIMEOUT through osp_check_status.
 int debug_withhold_q();
 
+// Per-device memory pool of the library's stream-ordered workspaces (created on first use; keeps
+// freed blocks cached until process exit).
+cudaMemPool_t workspace_pool();
+
+// Split-KV of the last partial wave of attention CTAs (OSP_SPLIT_KV=0 disables; read per launch).
+int split_kv_enabled();
+
 int rope3d_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_shape& s,
                   const osp_rope& rope, cudaStream_t stream);
 int skiparse_gather_launch(const void* const src[3], void* const dst[3], int n_tensors, const osp_shape& s,

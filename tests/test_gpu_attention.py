@@ -166,3 +166,28 @@ def test_row_max_jump_in_a_late_kv_tile(gpu, jump):
     ops.check_status()
     ref = O.attn_ref(to_f64(q), to_f64(k), to_f64(v))
     assert_attn_close(o, ref, f"jump {jump}")
+
+
+@pytest.mark.parametrize("d,grid,L,sparse", [(64, (4, 15, 16), 40, None), (96, (4, 15, 16), 40, None),
+                                             (128, (4, 15, 16), 40, None), (64, (4, 16, 16), 0, (2, 1)),
+                                             (128, (8, 16, 16), 0, (4, 0))])
+def test_split_kv_tail_matches_oracle_and_unsplit(gpu, monkeypatch, d, grid, L, sparse):
+    """Few work units (fewer than SMs): the kernel splits each unit's KV range into parts whose
+    fp32 partials are merged by the combine kernel.  Same result as the unsplit kernel (up to
+    summation order) and as the oracle."""
+    q, k, v, qg, kg, vg = _qkv(gpu, 1, 2, d, grid, L, seed=17)
+    if sparse is None:
+        run = lambda: ops.attn_full(qg, kg, vg, grid, L)
+        ref = O.attn_ref(to_f64(q), to_f64(k), to_f64(v))
+    else:
+        kk, mode = sparse
+        run = lambda: ops.skiparse_attn(qg, kg, vg, grid, kk, mode)
+        ref = O.skiparse_attn_ref(to_f64(q), to_f64(k), to_f64(v), kk, mode)
+    split = run()
+    ops.check_status()
+    monkeypatch.setenv("OSP_SPLIT_KV", "0")
+    plain = run()
+    ops.check_status()
+    assert_attn_close(split, ref, "split")
+    assert_attn_close(plain, ref, "unsplit")
+    assert float((split.float() - plain.float()).abs().max()) <= 1e-2
