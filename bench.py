@@ -167,8 +167,22 @@ def sparse(w) -> bool:
     return bool(w.skiparse_k) and ATTN_MODE["value"] != "dense"
 
 
-def launches_per_step(w) -> int:
-    return 1 + (2 if sparse(w) else 1)
+def attention_launches(w, sms: int) -> int:
+    """Kernel launches of one attention call: the attention kernel, plus the combine kernel when
+    the library splits the last partial wave of (sample*set, head, 256-row block) units over KV
+    ranges (the rule of osp_attn_full: units mod SMs = R > 0 and min(SMs / R, KV tiles / 2, 8) >= 2)."""
+    k = w.skiparse_k if sparse(w) else 1
+    n = (w.seq_len if not sparse(w) else w.n_video // k)
+    units = -(-n // 256) * w.heads * w.B * k
+    rem = units % sms
+    if rem == 0:
+        return 1
+    ns = min(sms // rem, (-(-n // 128)) // 2, 8)
+    return 2 if ns >= 2 else 1
+
+
+def launches_per_step(w, sms: int = 148) -> int:
+    return 1 + (2 * attention_launches(w, sms) if sparse(w) else attention_launches(w, sms))
 
 
 def step_flops(w) -> float:
@@ -350,14 +364,16 @@ def run_ours(args, rank, world, local_rank):
                        flops_per_step=flops),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "attn_fwd_kernel", "peak_source": f"{peaks_src} (sustained bf16 GEMM)",
+                     "kernel": "attn_fwd_kernel" + (" + attn_combine_kernel (split tail)" if attention_launches(
+                         w, torch.cuda.get_device_properties(dev).multi_processor_count) > 1 else ""),
+                     "peak_source": f"{peaks_src} (sustained bf16 GEMM)",
                      "frac_of_burst_peak": round(achieved / float(peaks["bf16_tflops"]), 4),
                      "avg_launch_ms": round(attn_ms, 4)},
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "ms_per_step": round(e2e_ms, 4),
                 "steps": e2e_steps, "copies": "pinned host <-> device on two copy streams, double-buffered, "
                                               "overlapping the previous/next step's kernels"},
-        "gpu_launches": launches_per_step(w) * args.steps,
+        "gpu_launches": launches_per_step(w, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

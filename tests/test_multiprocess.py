@@ -53,7 +53,10 @@ def test_weak_scaling_value_counts_all_ranks():
     from spacetime_attention_b200 import synthetic as syn
     w = syn.WORKLOADS["cogvideox_2b"]
     assert bench.step_flops(w) == w.dense_flops()
-    assert bench.launches_per_step(w) == 2
+    # 2100 units on 148 SMs: the last 28 are split 5 ways -> attention + combine kernel + RoPE
+    assert bench.attention_launches(w, 148) == 2 and bench.launches_per_step(w, 148) == 3
+    assert bench.attention_launches(w, 150) == 1          # 2100 = 14 * 150: no partial wave
     w2 = syn.WORKLOADS["long_video"]
     assert bench.step_flops(w2) == 2 * w2.skiparse_flops()
-    assert bench.launches_per_step(w2) == 3
+    # 4608 Skiparse units: 20 left over on 148 SMs, split 7 ways, for each of the two calls
+    assert bench.launches_per_step(w2, 148) == 5
