@@ -9,6 +9,7 @@ from .spacetime_oracle import (  # noqa: F401
     SKIP_SINGLE,
     attention_head_ref,
     attn_ref,
+    cross_attn_ref,
     default_scale,
     rope3d_positions_ref,
     rope3d_ref,

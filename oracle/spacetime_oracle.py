@@ -287,6 +287,26 @@ def attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float | None = 
     return out
 
 
+def cross_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float | None = None,
+                   rows=None, heads=None) -> np.ndarray:
+    """Video -> text cross-attention ("Open-Sora Plan" section 2.2.1: each block attends from the
+    video tokens to the text embeddings): o_i = softmax_j(q_i . k_j * scale) v_j with queries from
+    the video sequence and keys/values from the text sequence, per sample and head.
+
+    q: [B, N_q, n_h, d]; k, v: [B, N_kv, n_h, d] (N_q and N_kv independent).  ``rows`` optionally
+    selects query tokens; the result is [B, len(rows), len(heads), d].
+    """
+    B, Nq, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    rows_ = np.arange(Nq) if rows is None else np.asarray(rows)
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    out = np.empty((B, len(rows_), len(heads_), d), dtype=np.float64)
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            out[b, :, hi] = attention_head_ref(q[b, :, h], k[b, :, h], v[b, :, h], scale, rows_)
+    return out
+
+
 def skiparse_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, k_ratio: int, mode: int,
                       scale: float | None = None, rows=None, heads=None) -> np.ndarray:
     """Skiparse attention: each token attends only to the tokens of its own set

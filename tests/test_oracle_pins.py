@@ -355,3 +355,30 @@ def test_round_to_bf16_is_nearest():
     assert np.all(m * 2 ** 8 == np.round(m * 2 ** 8))
     spacing = 2.0 ** (np.floor(np.log2(np.abs(x))) - 7)
     assert np.all(np.abs(r - x) <= spacing / 2)
+
+
+# ----------------------------------------------------------------------------------------------
+# cross-attention (video queries, text keys/values)
+# ----------------------------------------------------------------------------------------------
+
+def test_cross_attention_brute_force_and_special_cases():
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal((2, 6, 2, 4))
+    k = rng.standard_normal((2, 3, 2, 4))
+    v = rng.standard_normal((2, 3, 2, 4))
+    got = O.cross_attn_ref(q, k, v)
+    for b in range(2):
+        for h in range(2):
+            ref = _brute_masked_attention(q[b, :, h].tolist(), k[b, :, h].tolist(), v[b, :, h].tolist(),
+                                          lambda i, j: True, 0.5)
+            np.testing.assert_allclose(got[b, :, h], ref, rtol=1e-12, atol=1e-13)
+    # one text token: every video query returns that token's value
+    np.testing.assert_allclose(O.cross_attn_ref(q, k[:, :1], v[:, :1]), np.broadcast_to(v[:, :1], q.shape), atol=1e-15)
+    # closed form with 3 video queries and 2 text keys: q.k0 - q.k1 = ln 3 -> weights 3/4, 1/4
+    q3 = np.zeros((1, 3, 1, 2)); q3[0, :, 0, 0] = 1.0
+    k2 = np.zeros((1, 2, 1, 2)); k2[0, 0, 0, 0] = math.log(3.0)
+    v2 = np.zeros((1, 2, 1, 2)); v2[0, 0, 0] = [4.0, 0.0]; v2[0, 1, 0] = [0.0, 8.0]
+    np.testing.assert_allclose(O.cross_attn_ref(q3, k2, v2, scale=1.0)[0, :, 0], [[3.0, 2.0]] * 3, rtol=1e-14)
+    # rows / heads subsets agree with the full result
+    np.testing.assert_allclose(O.cross_attn_ref(q, k, v, rows=[5, 0], heads=[1]), got[:, [5, 0]][:, :, [1]],
+                               rtol=0, atol=1e-15)
