@@ -248,6 +248,79 @@ def run_hbm_op(args, rank, world, local_rank):
             "gpu_launches": args.steps}
 
 
+def cross_launches(w, text_len: int, sms: int = 148) -> int:
+    """Kernel launches of one osp_attn_cross call (same split rule as attention_launches, with the
+    video tokens as queries and the text tokens as keys)."""
+    units = -(-w.n_video // 256) * w.heads * w.B
+    rem = units % sms
+    if rem == 0:
+        return 1
+    return 2 if min(sms // rem, (-(-text_len // 128)) // 2, 8) >= 2 else 1
+
+
+def run_cross_op(args, rank, world, local_rank):
+    """Time video -> text cross-attention (osp_attn_cross) alone: the workload's video tokens as
+    queries, --text-len text tokens as keys and values.  Three input sets rotate (q alone is
+    larger than L2 for the full-size workloads).  value = attention flops / time."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = syn.WORKLOADS[args.workload]
+    L = args.text_len
+    nset = 3
+    sets = []
+    for r in range(nset):
+        s = w.seed + 7 + 101 * r + 17 * rank
+        sets.append(tuple(syn.randn_bf16(shape, s + i).to(dev) for i, shape in enumerate(
+            [(w.B, w.n_video, w.heads, w.head_dim), (w.B, L, w.heads, w.head_dim), (w.B, L, w.heads, w.head_dim)])))
+    outs = [torch.empty_like(q) for q, _, _ in sets]
+
+    def launch(i):
+        q, k, v = sets[i % nset]
+        ops.attn_cross(q, k, v, w.grid, o=outs[i % nset])
+
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        launch(i)
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ops.check_status(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    peaks, src = load_peaks()
+    flops = 4.0 * w.B * w.heads * w.n_video * L * w.head_dim
+    nbytes = 2 * 2 * w.B * w.heads * w.head_dim * (w.n_video + L)      # q read + o written, k and v read
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    t_tensor = flops / (float(peaks["bf16_tflops_sustained"]) * 1e12)
+    t_hbm = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": float(peaks["bf16_tflops_sustained"]),
+                "unit": "TFLOP/s", "frac": round(tflops / float(peaks["bf16_tflops_sustained"]), 4),
+                "peak_source": f"{src} (cuBLAS bf16, sustained)"}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": f"{src} (copy bandwidth)"}
+    roof.update(traffic=None, time_bound_frac=round(max(t_tensor, t_hbm) / (ms * 1e-3), 4),
+                hbm_gb_s=round(gbs, 1), bytes_per_launch=nbytes)
+    n_launch = cross_launches(w, L)
+    return {"metric": "cross-attention TFLOP/s (video queries, text keys)", "value": round(world * tflops, 1),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(w.describe(), op="cross", text_len=L, queries=w.n_video, flops_per_launch=flops,
+                           l2=f"{nset} input sets rotated ({nset * nbytes / 1e6:.0f} MB)"),
+            "roofline": roof, "clocks": clocks, "gpu_launches": n_launch * args.steps}
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -482,8 +555,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse"],
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
-    ap.add_argument("--op", default="step", choices=["step", "rope", "gather", "scatter"],
-                    help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone")
+    ap.add_argument("--op", default="step", choices=["step", "rope", "gather", "scatter", "cross"],
+                    help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone; "
+                         "cross: video -> text cross-attention alone")
+    ap.add_argument("--text-len", type=int, default=226, help="--op cross: text tokens (keys)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -509,7 +584,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank) if args.op == "step" else run_hbm_op(args, rank, world, local_rank)
+        runner = {"step": run_ours, "cross": run_cross_op}.get(args.op, run_hbm_op)
+        line = runner(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

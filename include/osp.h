@@ -101,6 +101,17 @@ int osp_rope3d(const void* q, const void* k, void* q_out, void* k_out, const osp
 int osp_attn_full(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                   float softmax_scale, void* stream);
 
+/* Video -> text cross-attention ("Open-Sora Plan" section 2.2.1: every block attends from the
+ * video tokens to the mT5 text embeddings): for every sample b and head h,
+ *   O = softmax(Q K^T * scale) V  with Q the video tokens and K, V the text tokens.
+ *  q, o:  [B][T*H*W][heads][head_dim] bf16, device (video tokens only; o must not overlap q, k, v).
+ *  k, v:  [B][text_len][heads][head_dim] bf16, device (text_len >= 1 key/value tokens).
+ *  No RoPE is involved (text tokens have no grid position). Same kernel, arithmetic, scale
+ *  convention and work split as osp_attn_full.
+ *  Errors: OSP_ERR_INVALID_ARG (null, text_len < 1), OSP_ERR_UNSUPPORTED, OSP_ERR_CUDA. */
+int osp_attn_cross(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                   float softmax_scale, void* stream);
+
 /* Skiparse gather ("Open-Sora Plan" section 2.2.2: sequence cut to 1/k, batch grown k-fold):
  *   x_out[b*k + g][s] = RoPE(x[b][token(g, s)])   for q and k (RoPE skipped if rope == NULL),
  *   v_out[b*k + g][s] = v[b][token(g, s)]         (exact copy).

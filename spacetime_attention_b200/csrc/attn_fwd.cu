@@ -103,8 +103,9 @@ struct Cfg {
 };
 
 struct AttnParams {
-  int n;          // tokens per set (query rows = key rows)
-  int N;          // tokens per sample in the natural-order tensors
+  int n_q;        // query rows per set
+  int n_kv;       // key / value rows per set (= n_q for self-attention)
+  int N_q;        // tokens per sample of the natural-order q and o tensors
   int heads;
   int G;          // sets per sample
   int k;          // sparse ratio (1 for dense)
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     w.b = bg / p.G;
     w.g = bg % p.G;
     w.q0 = qb * (2 * kBM);
-    const int n_kv_all = (p.n + kBN - 1) / kBN;
+    const int n_kv_all = (p.n_kv + kBN - 1) / kBN;
     w.kv_lo = w.part < 0 ? 0 : (int)((long long)w.part * n_kv_all / p.n_split);
     w.n_kv = (w.part < 0 ? n_kv_all : (int)((long long)(w.part + 1) * n_kv_all / p.n_split)) - w.kv_lo;
     return w;
@@ -524,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    const int valid0 = p.n - wk.kv_lo * kBN;   // valid keys from this CTA's first KV tile on
+    const int valid0 = p.n_kv - wk.kv_lo * kBN;   // valid keys from this CTA's first KV tile on
     for (int j = 0; j < n_kv; ++j) {
       if (!warp_wait(bar(B_SFULL + i), j & 1, wc)) { ok = false; break; }
       tc_fence_after();
@@ -604,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int unit = w.unit, part = w.part, h = w.h, b = w.b, g = w.g;
       const float inv_l = 1.f / l;
       const int slot = w.q0 + i * kBM + row;
-      const bool live = slot < p.n;
+      const bool live = slot < p.n_q;
       if (part >= 0) {
         // split unit: unnormalised fp32 O (relative to m) and (m, l) for the combine kernel
         const size_t prow = ((size_t)(unit - p.n_full) * p.n_split + part) * (2 * kBM) + i * kBM + row;
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (live) p.ws_ml[prow] = make_float2(m, l);
       } else {
       const int token = slot_token(p.layout, live ? slot : 0, g, p.k);
-      uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N + token) * p.heads + h) * D);
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -665,7 +666,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, i
   const int h = hb % p.heads, bg = hb / p.heads;
   const int b = bg / p.G, g = bg % p.G;
   const int slot = qb * 2 * kBM + r;
-  if (slot >= p.n) return;
+  if (slot >= p.n_q) return;
   float mmax = -INFINITY;
   for (int s = 0; s < p.n_split; ++s)
     mmax = fmaxf(mmax, p.ws_ml[((size_t)su * p.n_split + s) * (2 * kBM) + r].x);
@@ -683,7 +684,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, i
   }
   const float inv = 1.f / lsum;
   const int token = slot_token(p.layout, slot, g, p.k);
-  __nv_bfloat16* dst = p.o + (((size_t)b * p.N + token) * p.heads + h) * D;
+  __nv_bfloat16* dst = p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) dst[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
 }
@@ -771,14 +772,18 @@ int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
 namespace {
 
 // Attention launch with an explicit status word (the kernel's only global scratch).
+// N_kv: tokens per sample of k and v; < 0 means the same sequence as q (self-attention).
 int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
-                       int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split) {
-  const int N = s.text_len + s.T * s.H * s.W;
+                       int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
+                       int N_kv = -1) {
+  const int N = (N_kv < 0) ? s.text_len + s.T * s.H * s.W : s.T * s.H * s.W;   // q / o tokens per sample
+  if (N_kv < 0) N_kv = N;
   const int G = (layout == 0) ? 1 : sparse_k;
   const int n = N / G;
   AttnParams p{};
-  p.n = n;
-  p.N = N;
+  p.n_q = n;
+  p.n_kv = N_kv / G;
+  p.N_q = N;
   p.heads = s.heads;
   p.G = G;
   p.k = (layout == 0) ? 1 : sparse_k;
@@ -791,8 +796,8 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   CUtensorMap tq, tk, tv;
   int rc;
   if ((rc = make_tmap(&tq, q, s, N, layout, p.k)) != OSP_OK) return rc;
-  if ((rc = make_tmap(&tk, k, s, N, layout, p.k)) != OSP_OK) return rc;
-  if ((rc = make_tmap(&tv, v, s, N, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tk, k, s, N_kv, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tv, v, s, N_kv, layout, p.k)) != OSP_OK) return rc;
   const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
   const long long units = qblocks * s.heads * (long long)s.B * G;
   if (units > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld attention work units is too many", units);
@@ -801,7 +806,7 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.n_split = 1;
   // Split-KV for the last partial wave (one CTA per SM): its R units are split into KV ranges so
   // that about one wave of CTAs runs them.  Needs a workspace, so only where allocation is allowed.
-  const int n_kv = (n + kBN - 1) / kBN;
+  const int n_kv = (p.n_kv + kBN - 1) / kBN;
   const int sms = device_sm_count();
   const int rem = (int)(units % sms);
   if (allow_split && split_kv_enabled() && rem > 0) {
@@ -850,6 +855,13 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true);
+}
+
+int cross_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, float scale,
+                           cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  return launch_with_status(q, k, v, o, s, 0, 1, scale, stream, status, true, s.text_len);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -182,6 +182,20 @@ int osp_attn_full(const void* q, const void* k, const void* v, void* o, const os
   return attention_launch(q, k, v, o, *shape, 0, 1, softmax_scale, static_cast<cudaStream_t>(stream));
 }
 
+int osp_attn_cross(const void* q, const void* k, const void* v, void* o, const osp_shape* shape, float softmax_scale,
+                   void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (shape->text_len < 1)
+    return set_error(OSP_ERR_INVALID_ARG, "cross-attention needs text_len >= 1 key/value tokens");
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return cross_attention_launch(q, k, v, o, *shape, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
 int osp_skiparse_gather(const void* q, const void* k, const void* v, void* q_out, void* k_out, void* v_out,
                         const osp_shape* shape, int32_t sparse_k, int32_t mode, const osp_rope* rope, void* stream) {
   g_last_error[0] = 0;

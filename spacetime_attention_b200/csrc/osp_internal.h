@@ -51,4 +51,9 @@ int index_map_launch(int n_video, int k, int mode, int32_t* out, cudaStream_t st
 int attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
                      int sparse_k, float scale, cudaStream_t stream);
 
+// Cross-attention: queries are the T*H*W video tokens of q, keys/values the text_len tokens of
+// k and v; o has q's shape.
+int cross_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, float scale,
+                           cudaStream_t stream);
+
 }  // namespace osp

@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "OSP_OK", 1: "OSP_ERR_INVALID_ARG", 2: "OSP_ERR_UNSUPPORTED",
 # Every symbol include/osp.h declares (tests check the library exports all of them).
 EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_scatter", "osp_skiparse_attn",
             "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version",
-            "osp_attn_full_noalloc")
+            "osp_attn_full_noalloc", "osp_attn_cross")
 
 
 class OspShape(ctypes.Structure):
@@ -61,6 +61,7 @@ def library() -> ctypes.CDLL:
             "osp_rope3d": [vp, vp, vp, vp, sp, rp, vp],
             "osp_attn_full": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_full_noalloc": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_cross": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_skiparse_gather": [vp, vp, vp, vp, vp, vp, sp, i32, i32, rp, vp],
             "osp_skiparse_scatter": [vp, vp, sp, i32, i32, vp],
             "osp_skiparse_attn": [vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
@@ -135,6 +136,20 @@ def attn_full(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len:
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_full", library().osp_attn_full(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                     ctypes.c_float(scale), _stream_handle(q)))
+    return o
+
+
+def attn_cross(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, scale: float = 0.0,
+               o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """osp_attn_cross: video queries q [B, T*H*W, heads, d] attend to text keys/values
+    k, v [B, text_len, heads, d]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    B, _, heads, d = q.shape
+    shp = make_shape(B, k.shape[1], grid, heads, d)
+    _check("osp_attn_cross", library().osp_attn_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
+                                                      ctypes.c_float(scale), _stream_handle(q)))
     return o
 
 

@@ -60,3 +60,12 @@ def test_weak_scaling_value_counts_all_ranks():
     assert bench.step_flops(w2) == 2 * w2.skiparse_flops()
     # 4608 Skiparse units: 20 left over on 148 SMs, split 7 ways, for each of the two calls
     assert bench.launches_per_step(w2, 148) == 5
+
+
+def test_cross_launch_count():
+    import bench
+    from spacetime_attention_b200 import synthetic as syn
+    # 113 blocks * 24 heads = 2712 units, 48 left for the last wave, 2 KV tiles: no split
+    assert bench.cross_launches(syn.WORKLOADS["open_sora_plan"], 226, 148) == 1
+    # 1 block * 2 heads, 8 KV tiles: the two units are split over KV ranges (+ combine kernel)
+    assert bench.cross_launches(syn.custom("x", 1, 2, 64, (1, 3, 5), 1000, (16, 24, 24)), 1000, 148) == 2
