@@ -11,10 +11,13 @@ from .spacetime_oracle import (  # noqa: F401
     attn_ref,
     cross_attn_ref,
     default_scale,
+    packed_attn_ref,
+    rope3d_packed_ref,
     rope3d_positions_ref,
     rope3d_ref,
     rope_frequencies,
     round_to_bf16,
+    segment_bounds,
     skiparse_attn_ref,
     skiparse_gather_ref,
     skiparse_index_map,

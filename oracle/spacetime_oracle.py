@@ -336,3 +336,71 @@ def skiparse_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, k_ratio: int,
                 out[b, sel, hi] = attention_head_ref(q[b, idx, h], k[b, idx, h], v[b, idx, h],
                                                      scale, slot_of[rows_[sel]])
     return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Packed batches of videos of different shapes
+# ----------------------------------------------------------------------------------------------
+#
+# "CogVideoX", section 3.1 "Multi-Resolution Frame Pack": videos of different durations and
+# resolutions are placed into one batch (after Patch'n Pack / NaViT), and each video's 3D RoPE
+# positions are its own grid coordinates (extrapolation: the front of one position table, never
+# rescaled).  Readings: the packed sequence is the concatenation of samples; sample i is its own
+# text_i tokens followed by its T_i*H_i*W_i video tokens; a token attends only to the tokens of its
+# own sample (Patch'n Pack's example masking), i.e. attention is block-diagonal over samples.
+
+def segment_bounds(lengths: Sequence[int]) -> np.ndarray:
+    """Start offsets of consecutive segments: [0, l_0, l_0 + l_1, ...] (n_seg + 1 entries)."""
+    out = np.zeros(len(lengths) + 1, dtype=np.int64)
+    out[1:] = np.cumsum(np.asarray(lengths, dtype=np.int64))
+    return out
+
+
+def rope3d_packed_ref(x: np.ndarray, samples: Sequence[Sequence[int]], split: Sequence[int],
+                      theta: float = 10000.0) -> np.ndarray:
+    """3D RoPE over a packed [1, sum_i (text_i + T_i*H_i*W_i), n_h, d] sequence.
+
+    ``samples`` lists (text_len, T, H, W) per packed sample.  Every sample is rotated exactly as
+    ``rope3d_ref`` rotates it on its own: its video positions start at (0, 0, 0) and follow its
+    own grid; its text tokens are left unrotated.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    lens = [int(L) + int(T) * int(H) * int(W) for L, T, H, W in samples]
+    bounds = segment_bounds(lens)
+    if x.shape[0] != 1 or x.shape[1] != bounds[-1]:
+        raise ValueError("packed tensor must be [1, sum of sample lengths, heads, d]")
+    out = np.empty_like(x)
+    for i, (L, T, H, W) in enumerate(samples):
+        a, b = bounds[i], bounds[i + 1]
+        out[:, a:b] = rope3d_ref(x[:, a:b], (T, H, W), int(L), split, theta)
+    return out
+
+
+def packed_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_bounds: Sequence[int],
+                    kv_bounds: Sequence[int] | None = None, scale: float | None = None,
+                    rows=None, heads=None) -> np.ndarray:
+    """Block-diagonal attention over a packed batch: query token r of segment i attends to the
+    key/value tokens of segment i only, per head.
+
+    q: [1, N_q, n_h, d]; k, v: [1, N_kv, n_h, d].  Segment i owns query rows
+    [q_bounds[i], q_bounds[i+1]) and key rows [kv_bounds[i], kv_bounds[i+1]) (the same rows
+    when ``kv_bounds`` is None: self-attention within each sample).  ``rows`` optionally
+    selects query rows (packed indices); the result is [1, len(rows), len(heads), d].
+    """
+    qb = np.asarray(q_bounds, dtype=np.int64)
+    kb = qb if kv_bounds is None else np.asarray(kv_bounds, dtype=np.int64)
+    _, Nq, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    rows_ = np.arange(Nq) if rows is None else np.asarray(rows)
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    seg_of = np.searchsorted(qb, rows_, side="right") - 1
+    out = np.empty((1, len(rows_), len(heads_), d), dtype=np.float64)
+    for i in range(len(qb) - 1):
+        sel = np.nonzero(seg_of == i)[0]
+        if sel.size == 0:
+            continue
+        kk = slice(kb[i], kb[i + 1])
+        for hi, h in enumerate(heads_):
+            out[0, sel, hi] = attention_head_ref(q[0, qb[i]:qb[i + 1], h], k[0, kk, h], v[0, kk, h], scale,
+                                                 rows_[sel] - qb[i])
+    return out

@@ -382,3 +382,69 @@ def test_cross_attention_brute_force_and_special_cases():
     # rows / heads subsets agree with the full result
     np.testing.assert_allclose(O.cross_attn_ref(q, k, v, rows=[5, 0], heads=[1]), got[:, [5, 0]][:, :, [1]],
                                rtol=0, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------------------------
+# packed batches (Multi-Resolution Frame Pack)
+# ----------------------------------------------------------------------------------------------
+
+def test_segment_bounds():
+    assert O.segment_bounds([3, 1, 4]).tolist() == [0, 3, 4, 8]
+    assert O.segment_bounds([]).tolist() == [0]
+
+
+def test_packed_attention_is_block_diagonal_brute_force():
+    rng = np.random.default_rng(21)
+    seg = [0, 0, 0, 1, 2, 2, 2, 2]          # sample of each packed token, written out by hand
+    q, k, v = (rng.standard_normal((1, 8, 2, 3)) for _ in range(3))
+    got = O.packed_attn_ref(q, k, v, [0, 3, 4, 8])
+    for h in range(2):
+        ref = _brute_masked_attention(q[0, :, h].tolist(), k[0, :, h].tolist(), v[0, :, h].tolist(),
+                                      lambda i, j: seg[i] == seg[j], 1 / math.sqrt(3))
+        np.testing.assert_allclose(got[0, :, h], ref, rtol=1e-12, atol=1e-13)
+    # the one-token sample returns its own value
+    np.testing.assert_allclose(got[0, 3], v[0, 3], atol=1e-15)
+    # row / head subsets agree with the full result
+    np.testing.assert_allclose(O.packed_attn_ref(q, k, v, [0, 3, 4, 8], rows=[7, 3, 0], heads=[1]),
+                               got[:, [7, 3, 0]][:, :, [1]], rtol=0, atol=1e-15)
+
+
+def test_packed_cross_attention_pairs_segments_brute_force():
+    rng = np.random.default_rng(22)
+    qseg = [0, 0, 1, 1, 1]                   # 2 samples: 2 and 3 queries
+    kseg = [0, 0, 0, 1]                      # 3 and 1 keys
+    q = rng.standard_normal((1, 5, 1, 4))
+    k = rng.standard_normal((1, 4, 1, 4))
+    v = rng.standard_normal((1, 4, 1, 4))
+    got = O.packed_attn_ref(q, k, v, [0, 2, 5], [0, 3, 4], scale=0.7)
+    ref = _brute_masked_attention(q[0, :, 0].tolist(), k[0, :, 0].tolist(), v[0, :, 0].tolist(),
+                                  lambda i, j: qseg[i] == kseg[j], 0.7)
+    np.testing.assert_allclose(got[0, :, 0], ref, rtol=1e-12, atol=1e-13)
+    # sample 1 has one key: its queries all return that value
+    np.testing.assert_allclose(got[0, 2:, 0], np.broadcast_to(v[0, 3, 0], (3, 4)), atol=1e-15)
+
+
+def test_packed_rope_restarts_positions_per_sample():
+    # sample 0: 2 text tokens + a 1x2x3 grid; sample 1: no text + a 2x1x2 grid.  Positions written
+    # by hand (t, h, w), w fastest, restarting at the origin for every sample.
+    samples = [(2, 1, 2, 3), (0, 2, 1, 2)]
+    pos0 = [(0, 0, 0), (0, 0, 1), (0, 0, 2), (0, 1, 0), (0, 1, 1), (0, 1, 2)]
+    pos1 = [(0, 0, 0), (0, 0, 1), (1, 0, 0), (1, 0, 1)]
+    split = (8, 8, 8)
+    rng = np.random.default_rng(23)
+    x = rng.standard_normal((1, 2 + 6 + 4, 2, 24))
+    y = O.rope3d_packed_ref(x, samples, split)
+    np.testing.assert_array_equal(y[0, :2], x[0, :2])                  # text untouched
+    np.testing.assert_array_equal(y[0, 2], x[0, 2])                    # sample 0 origin
+    np.testing.assert_array_equal(y[0, 8], x[0, 8])                    # sample 1 origin
+    for base, pos in ((2, pos0), (8, pos1)):
+        for r, (t, h, w) in enumerate(pos):
+            # a 1D rotation per axis pair (RoFormer) checked through complex multiplication
+            for c in range(0, 24, 2):
+                axis, j = divmod(c, 8)
+                p = (t, h, w)[axis]
+                ang = p * 10000.0 ** (-(j / 2) * 2 / 8)
+                for hd in range(2):
+                    z = complex(x[0, base + r, hd, c], x[0, base + r, hd, c + 1]) * complex(math.cos(ang), math.sin(ang))
+                    assert abs(y[0, base + r, hd, c] - z.real) < 1e-12
+                    assert abs(y[0, base + r, hd, c + 1] - z.imag) < 1e-12
