@@ -321,6 +321,65 @@ def run_cross_op(args, rank, world, local_rank):
             "roofline": roof, "clocks": clocks, "gpu_launches": n_launch * args.steps}
 
 
+def run_packed_op(args, rank, world, local_rank):
+    """Time a packed batch of samples of different shapes (Multi-Resolution Frame Pack):
+    osp_rope3d_packed then osp_attn_packed (block-diagonal), inputs resident in HBM (larger
+    than L2).  value = block-diagonal attention flops / step time."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = syn.PACKED_WORKLOADS[args.packed]
+    q, k, v = (t.to(dev) for t in syn.make_packed_qkv(w.heads, w.head_dim, w.total, w.seed + 17 * rank))
+    qr, kr, o = torch.empty_like(q), torch.empty_like(k), torch.empty_like(q)
+    bounds = w.bounds
+    events = []
+
+    def step(record=False):
+        ops.rope3d_packed(q, k, w.samples, w.split, q_out=qr, k_out=kr)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+        ops.attn_packed(qr, kr, v, bounds, o=o)
+        if record:
+            e1.record()
+            events.append((e0, e1))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ops.check_status(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    attn_ms = sum(a.elapsed_time(b) for a, b in events) / len(events)
+    peaks, src = load_peaks()
+    flops = w.flops()
+    tflops = flops / (ms * 1e-3) / 1e12
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops_sustained"])
+    nbytes = 2 * w.total * w.heads * w.head_dim
+    return {"metric": "packed-batch attention TFLOP/s (Multi-Resolution Frame Pack, 1 GPU)",
+            "value": round(world * tflops, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(w.describe(), ops="rope3d_packed+attn_packed", flops_per_step=flops,
+                           l2=f"inputs {3 * nbytes / 1e6:.0f} MB > L2 126 MiB, no flush"),
+            "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(attn_tflops / peak, 4), "traffic": None,
+                         "kernel": "attn_fwd_kernel (packed segment table)",
+                         "peak_source": f"{src} (sustained bf16 GEMM)", "avg_launch_ms": round(attn_ms, 4)},
+            "clocks": clocks, "gpu_launches": 2 * args.steps}
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -555,9 +614,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse"],
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
-    ap.add_argument("--op", default="step", choices=["step", "rope", "gather", "scatter", "cross"],
+    ap.add_argument("--op", default="step", choices=["step", "rope", "gather", "scatter", "cross", "packed"],
                     help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone; "
-                         "cross: video -> text cross-attention alone")
+                         "cross: video -> text cross-attention alone; packed: a packed batch of mixed shapes")
+    ap.add_argument("--packed", default="frame_pack_cog2b", choices=sorted(syn.PACKED_WORKLOADS),
+                    help="--op packed: the packed batch")
     ap.add_argument("--text-len", type=int, default=226, help="--op cross: text tokens (keys)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -584,7 +645,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        runner = {"step": run_ours, "cross": run_cross_op}.get(args.op, run_hbm_op)
+        runner = {"step": run_ours, "cross": run_cross_op, "packed": run_packed_op}.get(args.op, run_hbm_op)
         line = runner(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)

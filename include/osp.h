@@ -10,7 +10,10 @@
  *   - dense 3D full attention over text + video tokens (CogVideoX section 2 and section 2.2
  *     "3D Full Attention");
  *   - Skiparse sparse attention, Single Skip and Group Skip with sparse ratio k
- *     ("Open-Sora Plan: Open-Source Large Video Generation Model", section 2.2.2).
+ *     ("Open-Sora Plan: Open-Source Large Video Generation Model", section 2.2.2);
+ *   - video -> text cross-attention (Open-Sora Plan section 2.2.1);
+ *   - packed batches of videos of different shapes, with per-sample RoPE grids and
+ *     block-diagonal attention (CogVideoX section 3.1 "Multi-Resolution Frame Pack").
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -76,6 +79,19 @@ typedef struct {
   double theta;           /* frequency base, > 0 (10000 on the pages) */
 } osp_rope;
 
+/* Packed batches ("CogVideoX" section 3.1 "Multi-Resolution Frame Pack": videos of different
+ * durations and resolutions share one batch, after Patch'n Pack).  A packed tensor is
+ * [total][heads][head_dim] bf16, the samples' rows one after another; sample i is its text_len
+ * text tokens followed by its T*H*W video tokens (row-major, w fastest).  Offsets ("bounds") are
+ * HOST arrays of n + 1 int32 values: bounds[0] = 0, non-decreasing, sample i owning rows
+ * [bounds[i], bounds[i+1]). */
+#define OSP_MAX_SEGMENTS 256   /* samples per packed call */
+
+typedef struct {
+  int32_t text_len;  /* >= 0 */
+  int32_t T, H, W;   /* >= 1 each */
+} osp_sample_grid;
+
 /* 3D RoPE of q and k.
  *  q, k:          [B][N][heads][head_dim] bf16, device.
  *  q_out, k_out:  same shape; may equal q / k (in place) but must not overlap them otherwise.
@@ -111,6 +127,37 @@ int osp_attn_full(const void* q, const void* k, const void* v, void* o, const os
  *  Errors: OSP_ERR_INVALID_ARG (null, text_len < 1), OSP_ERR_UNSUPPORTED, OSP_ERR_CUDA. */
 int osp_attn_cross(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                    float softmax_scale, void* stream);
+
+/* 3D RoPE of a packed batch (CogVideoX section 3.1: every video keeps its own position grid,
+ * starting at (0, 0, 0); extrapolation, never rescaled).
+ *  samples:       HOST array of n_samples (1 .. OSP_MAX_SEGMENTS) sample grids, read during the call.
+ *  q, k:          packed [sum_i (text_len_i + T_i*H_i*W_i)][heads][head_dim] bf16, device.
+ *  q_out, k_out:  same shape; may equal q / k. Text rows are copied (skipped in place).
+ *  Arithmetic as osp_rope3d: sample i's rows equal what osp_rope3d gives for that sample alone.
+ *  Errors: OSP_ERR_INVALID_ARG (null, n_samples out of range, bad grid or split), OSP_ERR_CUDA. */
+int osp_rope3d_packed(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
+                      int32_t n_samples, int32_t heads, int32_t head_dim, const osp_rope* rope, void* stream);
+
+/* Block-diagonal attention over a packed batch (CogVideoX section 3.1; Patch'n Pack masks
+ * attention to each example): query row r of sample i attends to the key/value rows of sample
+ * i only, per head, O = softmax(Q_i K_i^T * scale) V_i.
+ *  q_bounds:  HOST, n_seg + 1 offsets of the samples' rows in q and o.
+ *  kv_bounds: HOST, n_seg + 1 offsets in k and v, or NULL for q_bounds (self-attention within
+ *             each sample; with different bounds: per-sample cross-attention, e.g. each video's
+ *             queries against its own prompt's text tokens).
+ *  q, o:      [q_bounds[n_seg]][heads][head_dim] bf16, device; o must not overlap q, k, v.
+ *  k, v:      [kv_bounds[n_seg]][heads][head_dim] bf16, device.
+ *  n_seg:     1 .. OSP_MAX_SEGMENTS. A sample with query rows needs >= 1 key row; samples with
+ *             no query rows are skipped.
+ *  softmax_scale: <= 0 selects 1/sqrt(head_dim).
+ *  Same kernel and arithmetic as osp_attn_full; work units (sample, head, 256-query block) are
+ *  never split over KV ranges here. The bounds are copied into the launch's parameters, so the
+ *  host arrays may be reused as soon as the call returns.
+ *  Errors: OSP_ERR_INVALID_ARG (null, bad bounds, a sample with queries but no keys),
+ *  OSP_ERR_UNSUPPORTED (head_dim, n_seg > OSP_MAX_SEGMENTS, > 2^30 rows), OSP_ERR_CUDA. */
+int osp_attn_packed(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
+                    const int32_t* kv_bounds, int32_t n_seg, int32_t heads, int32_t head_dim,
+                    float softmax_scale, void* stream);
 
 /* Skiparse gather ("Open-Sora Plan" section 2.2.2: sequence cut to 1/k, batch grown k-fold):
  *   x_out[b*k + g][s] = RoPE(x[b][token(g, s)])   for q and k (RoPE skipped if rope == NULL),

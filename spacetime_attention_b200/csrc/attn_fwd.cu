@@ -30,6 +30,7 @@
 #include <cuda.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "osp_internal.h"
 
@@ -126,6 +127,20 @@ struct AttnParams {
   float2* ws_ml;          // [split units][n_split][256]
 };
 
+// Packed batch of samples of different lengths (block-diagonal attention).  Segment i owns query
+// rows [q[i], q[i+1]) and key rows [kv[i], kv[i+1]) of the packed tensors and the work units
+// [heads * blk[i], heads * blk[i+1]) (one per head and 256-row query block, block fastest).
+// Passed by value as a kernel parameter, so a launch carries its own table.
+struct SegTable {
+  int n_seg;
+  int blk[kMaxSegments + 1];
+  int q[kMaxSegments + 1];
+  int kv[kMaxSegments + 1];
+};
+struct NoSegTable {};
+template <bool kPacked>
+using SegParam = typename std::conditional<kPacked, SegTable, NoSegTable>::type;
+
 __device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
                                           int chan, int row0, int g, int b, int k) {
   if (layout == 0) tma_load_3d(dst, tm, bar, chan, row0, b);
@@ -214,10 +229,11 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D>
+template <int D, bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p,
+                    const __grid_constant__ SegParam<kPacked> seg) {
   using C = Cfg<D>;
   constexpr int S = C::kStages;
   extern __shared__ unsigned char smem_raw[];
@@ -239,34 +255,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kSplitTiles = !C::kSepP && D == 96 && OSP_SPLIT_MMA_TILES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* seg_slot = reinterpret_cast<int*>(tmem_slot + 2);   // packed batches: this CTA's segment
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // work item -> unit (sample*set, head, query block) and KV tile range [kv_lo, kv_lo + n_kv).
-  // Recomputed where needed (cheap integer math) rather than kept live across the main loops.
-  struct Work { int unit, part, h, b, g, q0, kv_lo, n_kv; };
+  // q_row0 / kv_row0 offset the rows of a packed segment; nq / nkv are the set's query and key
+  // rows.  Recomputed where needed (cheap integer math) rather than kept live across the main loops.
+  struct Work { int unit, part, h, b, g, q0, kv_lo, n_kv, q_row0, kv_row0, nq, nkv; };
   auto decode = [&]() {
     Work w;
     w.unit = blockIdx.x;
     w.part = -1;
-    if (w.unit >= p.n_full) {
-      const int t = w.unit - p.n_full;
-      w.unit = p.n_full + t / p.n_split;
-      w.part = t % p.n_split;
+    int qb;
+    if constexpr (kPacked) {
+      const int sg = *seg_slot;
+      const int nqb = seg.blk[sg + 1] - seg.blk[sg];
+      const int local = w.unit - p.heads * seg.blk[sg];
+      w.h = local / nqb;
+      qb = local - w.h * nqb;
+      w.b = 0;
+      w.g = 0;
+      w.q_row0 = seg.q[sg];
+      w.kv_row0 = seg.kv[sg];
+      w.nq = seg.q[sg + 1] - w.q_row0;
+      w.nkv = seg.kv[sg + 1] - w.kv_row0;
+    } else {
+      if (w.unit >= p.n_full) {
+        const int t = w.unit - p.n_full;
+        w.unit = p.n_full + t / p.n_split;
+        w.part = t % p.n_split;
+      }
+      qb = w.unit % p.qblocks;
+      const int hb = w.unit / p.qblocks;
+      w.h = hb % p.heads;
+      const int bg = hb / p.heads;
+      w.b = bg / p.G;
+      w.g = bg % p.G;
+      w.q_row0 = 0;
+      w.kv_row0 = 0;
+      w.nq = p.n_q;
+      w.nkv = p.n_kv;
     }
-    const int qb = w.unit % p.qblocks, hb = w.unit / p.qblocks;
-    w.h = hb % p.heads;
-    const int bg = hb / p.heads;
-    w.b = bg / p.G;
-    w.g = bg % p.G;
     w.q0 = qb * (2 * kBM);
-    const int n_kv_all = (p.n_kv + kBN - 1) / kBN;
+    const int n_kv_all = (w.nkv + kBN - 1) / kBN;
     w.kv_lo = w.part < 0 ? 0 : (int)((long long)w.part * n_kv_all / p.n_split);
     w.n_kv = (w.part < 0 ? n_kv_all : (int)((long long)(w.part + 1) * n_kv_all / p.n_split)) - w.kv_lo;
     return w;
   };
-  const Work wk = decode();
-  const int n_kv = wk.n_kv;
-  const int chan0 = wk.h * D;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
@@ -291,6 +326,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if constexpr (kPacked) {
+    if (warp == 0) {
+      // segment of this CTA's unit: the number of i in [1, n_seg] with heads * blk[i] <= unit
+      // (blk is non-decreasing and unit < heads * blk[n_seg]); 32 lanes test 8 entries each
+      int c = 0;
+#pragma unroll
+      for (int t = 0; t < (kMaxSegments + 31) / 32; ++t) {
+        const int i = 1 + lane + 32 * t;
+        if (i <= seg.n_seg && p.heads * seg.blk[i] <= (int)blockIdx.x) ++c;
+      }
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) *seg_slot = c;
+    }
+  }
   if (warp == kLoadWarp && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
@@ -305,6 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+  const Work wk = decode();
+  const int n_kv = wk.n_kv;
+  const int chan0 = wk.h * D;
 
   auto sQ = [&](int i) { return sbase + C::kQOff + (uint32_t)(i * C::kTileBytes); };
   auto sK = [&](int s) { return sbase + C::kKOff + (uint32_t)(s * C::kTileBytes); };
@@ -328,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
         for (int i = 0; i < 2; ++i)
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, wk.q0 + i * kBM, wk.g, wk.b,
+            load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, wk.q_row0 + wk.q0 + i * kBM, wk.g, wk.b,
                       p.k);
       }
       for (int j = 0; j < n_kv; ++j) {
@@ -337,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, (wk.kv_lo + j) * kBN, wk.g, wk.b,
+            load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, wk.kv_row0 + (wk.kv_lo + j) * kBN, wk.g, wk.b,
                       p.k);
         }
         k_issued = j + 1;
@@ -345,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, (wk.kv_lo + j) * kBN, wk.g, wk.b,
+            load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, wk.kv_row0 + (wk.kv_lo + j) * kBN, wk.g, wk.b,
                       p.k);
         }
         v_issued = j + 1;
@@ -525,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    const int valid0 = p.n_kv - wk.kv_lo * kBN;   // valid keys from this CTA's first KV tile on
+    const int valid0 = wk.nkv - wk.kv_lo * kBN;   // valid keys from this CTA's first KV tile on
     for (int j = 0; j < n_kv; ++j) {
       if (!warp_wait(bar(B_SFULL + i), j & 1, wc)) { ok = false; break; }
       tc_fence_after();
@@ -605,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int unit = w.unit, part = w.part, h = w.h, b = w.b, g = w.g;
       const float inv_l = 1.f / l;
       const int slot = w.q0 + i * kBM + row;
-      const bool live = slot < p.n_q;
+      const bool live = slot < w.nq;
       if (part >= 0) {
         // split unit: unnormalised fp32 O (relative to m) and (m, l) for the combine kernel
         const size_t prow = ((size_t)(unit - p.n_full) * p.n_split + part) * (2 * kBM) + i * kBM + row;
@@ -624,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (live) p.ws_ml[prow] = make_float2(m, l);
       } else {
-      const int token = slot_token(p.layout, live ? slot : 0, g, p.k);
+      const int token = w.q_row0 + slot_token(p.layout, live ? slot : 0, g, p.k);
       uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -745,25 +797,25 @@ int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int l
   return OSP_OK;
 }
 
-template <int D>
+template <int D, bool kPacked>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
-             dim3 grid, cudaStream_t stream) {
+             const SegParam<kPacked>& seg, dim3 grid, cudaStream_t stream) {
   constexpr int smem = Cfg<D>::kSmemBytes;
   static bool attr_done = false;  // per process; the attribute is per function, not per device
   if (!attr_done) {
     // The warpgroup register split only adds up if the kernel is launched with exactly
     // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kPacked>) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncGetAttributes(attn_fwd_kernel<%d>) failed", D);
     if ((uint32_t)fa.numRegs != kRegsLaunch)
       return set_error(OSP_ERR_CUDA, "attn_fwd_kernel<%d> compiled to %d registers per thread, expected %u", D,
                        fa.numRegs, kRegsLaunch);
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_fwd_kernel<%d>) failed", D);
     attr_done = true;
   }
-  attn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  attn_fwd_kernel<D, kPacked><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
   return check_launch("attn_fwd_kernel");
 }
 
@@ -829,9 +881,9 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
   dim3 grid((unsigned)ctas);
   switch (s.head_dim) {
-    case 64: rc = launch_d<64>(tq, tk, tv, p, grid, stream); break;
-    case 96: rc = launch_d<96>(tq, tk, tv, p, grid, stream); break;
-    case 128: rc = launch_d<128>(tq, tk, tv, p, grid, stream); break;
+    case 64: rc = launch_d<64, false>(tq, tk, tv, p, NoSegTable{}, grid, stream); break;
+    case 96: rc = launch_d<96, false>(tq, tk, tv, p, NoSegTable{}, grid, stream); break;
+    case 128: rc = launch_d<128, false>(tq, tk, tv, p, NoSegTable{}, grid, stream); break;
     default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
   }
   if (rc == OSP_OK && p.n_split > 1) {
@@ -862,6 +914,54 @@ int cross_attention_launch(const void* q, const void* k, const void* v, void* o,
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   return launch_with_status(q, k, v, o, s, 0, 1, scale, stream, status, true, s.text_len);
+}
+
+int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
+                            const int32_t* kv_bounds, int n_seg, int heads, int head_dim, float scale,
+                            cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  SegTable seg{};
+  seg.n_seg = n_seg;
+  long long blocks = 0;
+  for (int i = 0; i <= n_seg; ++i) {
+    seg.q[i] = q_bounds[i];
+    seg.kv[i] = kv_bounds[i];
+    seg.blk[i] = (int)blocks;
+    if (i < n_seg) blocks += (q_bounds[i + 1] - q_bounds[i] + 2 * kBM - 1) / (2 * kBM);
+  }
+  const long long units = blocks * heads;
+  if (units == 0) return OSP_OK;   // no query rows at all
+  if (units > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld attention work units is too many", units);
+  const int n_q_total = q_bounds[n_seg], n_kv_total = kv_bounds[n_seg];
+  AttnParams p{};
+  p.N_q = n_q_total;
+  p.heads = heads;
+  p.G = 1;
+  p.k = 1;
+  p.layout = 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.status = status;
+  p.timeout_ns = wait_timeout_ns();
+  p.debug_withhold_q = debug_withhold_q();
+  p.qblocks = 1;
+  p.n_full = (int)units;
+  p.n_split = 1;
+  // the packed tensors are one sample of n_q_total (q, o) / n_kv_total (k, v) rows
+  const osp_shape sh{1, 0, 1, 1, 1, heads, head_dim};
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap(&tq, q, sh, n_q_total, 0, 1)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tk, k, sh, n_kv_total, 0, 1)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tv, v, sh, n_kv_total, 0, 1)) != OSP_OK) return rc;
+  const dim3 grid((unsigned)units);
+  switch (head_dim) {
+    case 64: return launch_d<64, true>(tq, tk, tv, p, seg, grid, stream);
+    case 96: return launch_d<96, true>(tq, tk, tv, p, seg, grid, stream);
+    case 128: return launch_d<128, true>(tq, tk, tv, p, seg, grid, stream);
+    default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
+  }
 }
 
 // ------------------------------------------------------------------------------------------

@@ -148,6 +148,17 @@ int debug_withhold_q() {
   return (e && e[0] == '1') ? 1 : 0;
 }
 
+// Offsets of a packed batch: n + 1 host values, bounds[0] = 0, non-decreasing, total <= 2^30.
+int check_bounds(const int32_t* b, int n, const char* what) {
+  if (!b) return set_error(OSP_ERR_INVALID_ARG, "%s is NULL", what);
+  if (b[0] != 0) return set_error(OSP_ERR_INVALID_ARG, "%s[0] = %d, must be 0", what, b[0]);
+  for (int i = 0; i < n; ++i)
+    if (b[i + 1] < b[i])
+      return set_error(OSP_ERR_INVALID_ARG, "%s decreases at %d (%d -> %d)", what, i, b[i], b[i + 1]);
+  if (b[n] > (1 << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%s: %d rows is too many", what, b[n]);
+  return OSP_OK;
+}
+
 }  // namespace osp
 
 using namespace osp;
@@ -194,6 +205,61 @@ int osp_attn_cross(const void* q, const void* k, const void* v, void* o, const o
     return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
   return cross_attention_launch(q, k, v, o, *shape, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+int osp_rope3d_packed(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
+                      int32_t n_samples, int32_t heads, int32_t head_dim, const osp_rope* rope, void* stream) {
+  g_last_error[0] = 0;
+  if (!samples) return set_error(OSP_ERR_INVALID_ARG, "samples is NULL");
+  if (n_samples < 1 || n_samples > OSP_MAX_SEGMENTS)
+    return set_error(n_samples < 1 ? OSP_ERR_INVALID_ARG : OSP_ERR_UNSUPPORTED, "n_samples = %d not in [1, %d]",
+                     n_samples, OSP_MAX_SEGMENTS);
+  long long total = 0;
+  for (int i = 0; i < n_samples; ++i) {
+    const osp_sample_grid& g = samples[i];
+    const osp_shape one{1, g.text_len, g.T, g.H, g.W, heads, head_dim};
+    int rc = check_shape(&one, false);
+    if (rc) {
+      char msg[256];
+      snprintf(msg, sizeof(msg), "%s", g_last_error);
+      return set_error(rc, "sample %d: %s", i, msg);
+    }
+    total += (long long)g.text_len + (long long)g.T * g.H * g.W;
+  }
+  if (total > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "packed batch of %lld rows is too large", total);
+  int rc = check_rope(rope, head_dim);
+  if (rc) return rc;
+  if (!q || !k || !q_out || !k_out) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return rope3d_packed_launch(q, k, q_out, k_out, samples, n_samples, heads, head_dim, *rope,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int osp_attn_packed(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
+                    const int32_t* kv_bounds, int32_t n_seg, int32_t heads, int32_t head_dim, float softmax_scale,
+                    void* stream) {
+  g_last_error[0] = 0;
+  if (n_seg < 1 || n_seg > OSP_MAX_SEGMENTS)
+    return set_error(n_seg < 1 ? OSP_ERR_INVALID_ARG : OSP_ERR_UNSUPPORTED, "n_seg = %d not in [1, %d]", n_seg,
+                     OSP_MAX_SEGMENTS);
+  if (heads < 1) return set_error(OSP_ERR_INVALID_ARG, "heads = %d", heads);
+  if (head_dim != 64 && head_dim != 96 && head_dim != 128)
+    return set_error(OSP_ERR_UNSUPPORTED, "attention head_dim %d not in {64, 96, 128}", head_dim);
+  int rc = check_bounds(q_bounds, n_seg, "q_bounds");
+  if (rc) return rc;
+  if (!kv_bounds) kv_bounds = q_bounds;
+  if ((rc = check_bounds(kv_bounds, n_seg, "kv_bounds"))) return rc;
+  for (int i = 0; i < n_seg; ++i)
+    if (q_bounds[i + 1] > q_bounds[i] && kv_bounds[i + 1] == kv_bounds[i])
+      return set_error(OSP_ERR_INVALID_ARG, "sample %d has %d query rows and no key rows", i,
+                       q_bounds[i + 1] - q_bounds[i]);
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)head_dim);
+  return packed_attention_launch(q, k, v, o, q_bounds, kv_bounds, n_seg, heads, head_dim, softmax_scale,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 int osp_skiparse_gather(const void* q, const void* k, const void* v, void* q_out, void* k_out, void* v_out,

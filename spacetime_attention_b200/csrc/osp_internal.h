@@ -11,6 +11,8 @@
 
 namespace osp {
 
+constexpr int kMaxSegments = OSP_MAX_SEGMENTS;
+
 // Sets the calling thread's last-error message; returns `code`.
 int set_error(int code, const char* fmt, ...);
 
@@ -55,5 +57,15 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
 // k and v; o has q's shape.
 int cross_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, float scale,
                            cudaStream_t stream);
+
+// Packed batch (block-diagonal attention): segment i owns q/o rows [q_bounds[i], q_bounds[i+1])
+// and k/v rows [kv_bounds[i], kv_bounds[i+1]); host arrays of n_seg + 1 validated offsets.
+int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
+                            const int32_t* kv_bounds, int n_seg, int heads, int head_dim, float scale,
+                            cudaStream_t stream);
+
+// 3D RoPE of a packed batch: sample i is text_len_i unrotated tokens then its own T_i x H_i x W_i grid.
+int rope3d_packed_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
+                         int n_samples, int heads, int head_dim, const osp_rope& rope, cudaStream_t stream);
 
 }  // namespace osp

@@ -11,6 +11,8 @@
 // computes each row's source/destination row and (t, h, w) position, then one cos/sin pair
 // per (row, channel pair) into shared memory, then streams the rows of every tensor.
 
+#include <type_traits>
+
 #include "osp_internal.h"
 
 namespace osp {
@@ -20,7 +22,9 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxPairs = 128;   // head_dim <= 256
 
-enum MapKind { kMapIdentity = 0, kMapGather = 1, kMapScatter = 2 };
+// identity: RoPE in natural order; gather / scatter: the Skiparse k-fold permutation;
+// packed: RoPE of a packed batch (identity order, every sample with its own grid)
+enum MapKind { kMapIdentity = 0, kMapGather = 1, kMapScatter = 2, kMapPacked = 3 };
 
 struct PermuteParams {
   const uint4* src[3];
@@ -39,6 +43,19 @@ struct PermuteParams {
   int rows_per_tile;
   long long n_tiles;
 };
+
+// Samples of a packed batch: sample i owns rows [start[i], start[i+1]), its first text[i] rows
+// are text, the rest an H[i] x W[i]-wide grid.  A kernel parameter (copied at launch).
+struct PackTable {
+  int n;
+  int start[kMaxSegments + 1];
+  int text[kMaxSegments];
+  int H[kMaxSegments];
+  int W[kMaxSegments];
+};
+struct NoPackTable {};
+template <int MAP>
+using PackParam = typename std::conditional<MAP == kMapPacked, PackTable, NoPackTable>::type;
 
 // Token index of slot s of set g (Open-Sora Plan section 2.2.2; reading in osp.h).
 __device__ __forceinline__ int skiparse_token(int g, int s, int k, int mode) {
@@ -59,13 +76,15 @@ __device__ __forceinline__ uint32_t bf16_rn_from_f64(double x) {
 }
 
 template <int MAP>
-__global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteParams p) {
+__global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteParams p,
+                                                                const __grid_constant__ PackParam<MAP> tab) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* omega = reinterpret_cast<double*>(smem_raw);                       // [head_dim/2]
   long long* src_row = reinterpret_cast<long long*>(omega + kMaxPairs);      // [rows_per_tile]
   long long* dst_row = src_row + p.rows_per_tile;                            // [rows_per_tile]
   int* vid = reinterpret_cast<int*>(dst_row + p.rows_per_tile);              // video index or -1
-  double2* cs = reinterpret_cast<double2*>(vid + ((p.rows_per_tile + 3) & ~3)); // [tile][pairs]
+  int4* tpos = reinterpret_cast<int4*>(vid + ((p.rows_per_tile + 3) & ~3));  // (t, h, w) per row
+  double2* cs = reinterpret_cast<double2*>(tpos + p.rows_per_tile);          // [tile][pairs]
   uint16_t* colpair = reinterpret_cast<uint16_t*>(cs + p.rows_per_tile * (p.head_dim >> 1));  // [vpr]
 
   const int npairs = p.head_dim >> 1;
@@ -80,7 +99,6 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
   }
   // first channel pair of every 16-byte column of a token row (8 channels = 4 pairs per column)
   for (int c = threadIdx.x; c < p.vpr; c += kThreads) colpair[c] = (uint16_t)((c % (p.head_dim >> 3)) * 4);
-  const int HW = p.H * p.W;
   const int per_set = (MAP == kMapIdentity) ? 0 : p.N / p.sparse_k;
 
   for (long long tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
@@ -90,10 +108,23 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
     for (int i = threadIdx.x; i < nrows; i += kThreads) {
       const long long r = row0 + i;
       long long s_row, d_row;
-      int token;
-      if (MAP == kMapIdentity) {
+      int token, text_len = p.text_len, H = p.H, W = p.W;
+      if constexpr (MAP == kMapIdentity) {
         s_row = d_row = r;
         token = (int)(r % p.N);
+      } else if constexpr (MAP == kMapPacked) {
+        // sample of row r: the largest s with start[s] <= r (starts strictly increase)
+        int lo = 0, hi = tab.n;
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (tab.start[mid] <= r) lo = mid;
+          else hi = mid;
+        }
+        s_row = d_row = r;
+        token = (int)(r - tab.start[lo]);
+        text_len = tab.text[lo];
+        H = tab.H[lo];
+        W = tab.W[lo];
       } else {
         const long long bk = r / per_set;           // b*k + g
         const int s = (int)(r - bk * per_set);
@@ -105,7 +136,9 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
       }
       src_row[i] = s_row;
       dst_row[i] = d_row;
-      vid[i] = token - p.text_len;  // < 0 for text tokens
+      const int v = token - text_len;  // < 0 for text tokens
+      vid[i] = v;
+      if (v >= 0) tpos[i] = make_int4(v / (H * W), (v / W) % H, v % W, 0);
     }
     __syncthreads();
     if (p.rope_mask) {
@@ -115,10 +148,8 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
         double2 c_s = make_double2(1.0, 0.0);
         if (v >= 0) {
           const int c = 2 * pr;
-          int pos;
-          if (c < p.d_t) pos = v / HW;
-          else if (c < p.d_t + p.d_h) pos = (v / p.W) % p.H;
-          else pos = v % p.W;
+          const int4 tp = tpos[i];
+          const int pos = c < p.d_t ? tp.x : (c < p.d_t + p.d_h ? tp.y : tp.z);
           double sn, cn;
           sincos((double)pos * omega[pr], &sn, &cn);
           c_s = make_double2(cn, sn);
@@ -184,7 +215,7 @@ __global__ void index_map_kernel(int n_video, int k, int mode, int* out) {
   }
 }
 
-int launch_permute(int map, PermuteParams& p, cudaStream_t stream) {
+int launch_permute(int map, PermuteParams& p, cudaStream_t stream, const PackTable* tab = nullptr) {
   const int npairs = p.head_dim / 2;
   // ~4096 vectors (64 KB of one tensor) per tile, at most 64 rows, and the cos/sin table within
   // 40 KB of shared memory
@@ -192,20 +223,23 @@ int launch_permute(int map, PermuteParams& p, cudaStream_t stream) {
   p.rows_per_tile = (int)std::max(1, std::min(std::min(64, table_rows), (4096 + p.vpr - 1) / p.vpr));
   p.n_tiles = (p.rows + p.rows_per_tile - 1) / p.rows_per_tile;
   const size_t smem = kMaxPairs * sizeof(double) + 2 * p.rows_per_tile * sizeof(long long) +
-                      ((p.rows_per_tile + 3) & ~3) * sizeof(int) +
+                      ((p.rows_per_tile + 3) & ~3) * sizeof(int) + p.rows_per_tile * sizeof(int4) +
                       (size_t)p.rows_per_tile * npairs * sizeof(double2) + (size_t)p.vpr * sizeof(uint16_t);
   const int sms = device_sm_count();
   const long long grid = std::min<long long>(p.n_tiles, (long long)sms * 8);
   if (grid <= 0) return OSP_OK;
   switch (map) {
     case kMapIdentity:
-      permute_rope_kernel<kMapIdentity><<<(unsigned)grid, kThreads, smem, stream>>>(p);
+      permute_rope_kernel<kMapIdentity><<<(unsigned)grid, kThreads, smem, stream>>>(p, NoPackTable{});
       break;
     case kMapGather:
-      permute_rope_kernel<kMapGather><<<(unsigned)grid, kThreads, smem, stream>>>(p);
+      permute_rope_kernel<kMapGather><<<(unsigned)grid, kThreads, smem, stream>>>(p, NoPackTable{});
+      break;
+    case kMapPacked:
+      permute_rope_kernel<kMapPacked><<<(unsigned)grid, kThreads, smem, stream>>>(p, *tab);
       break;
     default:
-      permute_rope_kernel<kMapScatter><<<(unsigned)grid, kThreads, smem, stream>>>(p);
+      permute_rope_kernel<kMapScatter><<<(unsigned)grid, kThreads, smem, stream>>>(p, NoPackTable{});
       break;
   }
   return check_launch("permute_rope_kernel");
@@ -246,6 +280,36 @@ int rope3d_launch(const void* q, const void* k, void* q_out, void* k_out, const 
   p.mode = 0;
   fill_rope(p, &rope);
   return launch_permute(kMapIdentity, p, stream);
+}
+
+int rope3d_packed_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
+                         int n_samples, int heads, int head_dim, const osp_rope& rope, cudaStream_t stream) {
+  PackTable tab{};
+  tab.n = n_samples;
+  long long rows = 0;
+  for (int i = 0; i < n_samples; ++i) {
+    tab.start[i] = (int)rows;
+    tab.text[i] = samples[i].text_len;
+    tab.H[i] = samples[i].H;
+    tab.W[i] = samples[i].W;
+    rows += (long long)samples[i].text_len + (long long)samples[i].T * samples[i].H * samples[i].W;
+  }
+  tab.start[n_samples] = (int)rows;
+  PermuteParams p{};
+  p.src[0] = static_cast<const uint4*>(q);
+  p.dst[0] = static_cast<uint4*>(q_out);
+  p.src[1] = static_cast<const uint4*>(k);
+  p.dst[1] = static_cast<uint4*>(k_out);
+  p.n_tensors = 2;
+  p.rope_mask = 3u;
+  p.head_dim = head_dim;
+  p.N = (int)rows;
+  p.rows = rows;
+  p.vpr = heads * head_dim / 8;
+  p.H = p.W = 1;
+  p.sparse_k = 1;
+  fill_rope(p, &rope);
+  return launch_permute(kMapPacked, p, stream, &tab);
 }
 
 int skiparse_gather_launch(const void* const src[3], void* const dst[3], int n_tensors, const osp_shape& s,

@@ -26,7 +26,9 @@ STATUS_NAMES = {0: "OSP_OK", 1: "OSP_ERR_INVALID_ARG", 2: "OSP_ERR_UNSUPPORTED",
 # Every symbol include/osp.h declares (tests check the library exports all of them).
 EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_scatter", "osp_skiparse_attn",
             "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version",
-            "osp_attn_full_noalloc", "osp_attn_cross")
+            "osp_attn_full_noalloc", "osp_attn_cross", "osp_rope3d_packed", "osp_attn_packed")
+
+MAX_SEGMENTS = 256   # OSP_MAX_SEGMENTS
 
 
 class OspShape(ctypes.Structure):
@@ -38,6 +40,10 @@ class OspShape(ctypes.Structure):
 class OspRope(ctypes.Structure):
     _fields_ = [("d_t", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_w", ctypes.c_int32),
                 ("theta", ctypes.c_double)]
+
+
+class OspSampleGrid(ctypes.Structure):
+    _fields_ = [("text_len", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32)]
 
 
 class OspError(RuntimeError):
@@ -62,6 +68,9 @@ def library() -> ctypes.CDLL:
             "osp_attn_full": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_full_noalloc": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_cross": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_rope3d_packed": [vp, vp, vp, vp, ctypes.POINTER(OspSampleGrid), i32, i32, i32, rp, vp],
+            "osp_attn_packed": [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
+                                i32, i32, ctypes.c_float, vp],
             "osp_skiparse_gather": [vp, vp, vp, vp, vp, vp, sp, i32, i32, rp, vp],
             "osp_skiparse_scatter": [vp, vp, sp, i32, i32, vp],
             "osp_skiparse_attn": [vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
@@ -150,6 +159,42 @@ def attn_cross(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, scale: f
     shp = make_shape(B, k.shape[1], grid, heads, d)
     _check("osp_attn_cross", library().osp_attn_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                       ctypes.c_float(scale), _stream_handle(q)))
+    return o
+
+
+def _bounds(b) -> ctypes.Array:
+    vals = [int(x) for x in b]
+    return (ctypes.c_int32 * len(vals))(*vals)
+
+
+def rope3d_packed(q: torch.Tensor, k: torch.Tensor, samples, split, theta: float = 10000.0,
+                  q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None):
+    """osp_rope3d_packed: 3D RoPE of a packed batch [1, total, heads, d]; ``samples`` lists
+    (text_len, T, H, W) per sample.  Returns (q_out, k_out)."""
+    _bshd(q, "q"); _bshd(k, "k")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    arr = (OspSampleGrid * max(1, len(samples)))(*[OspSampleGrid(*(int(x) for x in s)) for s in samples])
+    rp = make_rope(split, theta)
+    _, _, heads, d = q.shape
+    _check("osp_rope3d_packed", library().osp_rope3d_packed(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), arr,
+                                                            len(samples), heads, d, ctypes.byref(rp),
+                                                            _stream_handle(q)))
+    return q_out, k_out
+
+
+def attn_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_bounds, kv_bounds=None, scale: float = 0.0,
+                o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """osp_attn_packed: block-diagonal attention over a packed batch q [1, total_q, heads, d],
+    k, v [1, total_kv, heads, d]; sample i owns rows [bounds[i], bounds[i+1])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    _, _, heads, d = q.shape
+    qb = _bounds(q_bounds)
+    kb = _bounds(kv_bounds) if kv_bounds is not None else None
+    _check("osp_attn_packed", library().osp_attn_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(o), qb, kb, len(qb) - 1,
+                                                        heads, d, ctypes.c_float(scale), _stream_handle(q)))
     return o
 
 

@@ -98,3 +98,62 @@ def custom(name: str, B: int, heads: int, head_dim: int, grid, text_len: int, sp
            skiparse_k: int = 0, index: int = 100) -> Workload:
     """An ad-hoc workload (tests use these for ragged and edge-case shapes)."""
     return Workload(name, index, B, heads, head_dim, tuple(grid), text_len, tuple(split), skiparse_k)
+
+
+@dataclass(frozen=True)
+class PackedWorkload:
+    """A packed batch of samples of different shapes (CogVideoX section 3.1, Multi-Resolution
+    Frame Pack): each sample is (text_len, T, H, W); all share heads and head_dim."""
+    name: str
+    index: int
+    heads: int
+    head_dim: int
+    samples: tuple          # ((text_len, T, H, W), ...)
+    split: tuple
+    theta: float = 10000.0
+
+    @property
+    def lengths(self) -> list:
+        return [L + T * H * W for L, T, H, W in self.samples]
+
+    @property
+    def total(self) -> int:
+        return sum(self.lengths)
+
+    @property
+    def bounds(self) -> list:
+        out = [0]
+        for n in self.lengths:
+            out.append(out[-1] + n)
+        return out
+
+    @property
+    def seed(self) -> int:
+        return 2000 + self.index
+
+    def flops(self) -> float:
+        """4 * heads * d * sum_i N_i^2 (block-diagonal attention, QK^T and PV)."""
+        return 4.0 * self.heads * self.head_dim * sum(n * n for n in self.lengths)
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "heads": self.heads, "head_dim": self.head_dim,
+                "samples": ["%d+%dx%dx%d" % s for s in self.samples], "tokens": self.total,
+                "rope_split": "/".join(str(s) for s in self.split)}
+
+
+# CogVideoX-2B-shaped heads; 49- and 25-frame clips at 480x720, a 49-frame clip at 384x640, a
+# 960x1440 image and a 480x720 image, each with a 226-token prompt
+PACKED_WORKLOADS = {
+    w.name: w for w in [
+        PackedWorkload("frame_pack_cog2b", 0, 30, 64,
+                       ((226, 13, 30, 45), (226, 7, 30, 45), (226, 13, 24, 40), (226, 1, 60, 90), (226, 1, 30, 45)),
+                       (16, 24, 24)),
+    ]
+}
+
+
+def make_packed_qkv(heads: int, head_dim: int, total: int, seed: int, total_kv: int | None = None):
+    """q [1, total, heads, d] and k, v [1, total_kv (default total), heads, d], CPU bf16."""
+    nkv = total if total_kv is None else total_kv
+    return (randn_bf16((1, total, heads, head_dim), seed), randn_bf16((1, nkv, heads, head_dim), seed + 1),
+            randn_bf16((1, nkv, heads, head_dim), seed + 2))

@@ -93,3 +93,37 @@ def test_binding_refuses_non_cuda_tensors():
     x = torch.zeros(1, 256, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.attn_full(x, x, x, (4, 8, 8), 0)
+
+
+def _i32(vals):
+    return (ctypes.c_int32 * len(vals))(*vals)
+
+
+def test_packed_attention_validation(lib):
+    p = ctypes.c_void_p(256)
+    ok = _i32([0, 5, 9])
+    call = lambda qb, kb, n, heads=2, d=64: lib.osp_attn_packed(p, p, p, p, qb, kb, n, heads, d, 0.0, None)
+    assert call(ok, None, 0) == 1                       # no segments
+    assert call(ok, None, 257) == 2                     # more than OSP_MAX_SEGMENTS
+    assert call(None, None, 2) == 1                     # no bounds
+    assert call(_i32([1, 5, 9]), None, 2) == 1          # must start at 0
+    assert call(_i32([0, 5, 4]), None, 2) == 1          # decreasing
+    assert "decreases" in lib.osp_get_last_error().decode()
+    assert call(ok, _i32([0, 3, 3]), 2) == 1            # sample 1: 4 queries, no keys
+    assert "no key rows" in lib.osp_get_last_error().decode()
+    assert call(ok, None, 2, d=80) == 2
+    assert call(ok, None, 2, heads=0) == 1
+    assert lib.osp_attn_packed(None, p, p, p, ok, None, 2, 2, 64, 0.0, None) == 1
+    assert lib.osp_attn_packed(p, p, p, ctypes.c_void_p(260), ok, None, 2, 2, 64, 0.0, None) == 1
+
+
+def test_packed_rope_validation(lib):
+    p = ctypes.c_void_p(256)
+    r = ops.make_rope((16, 24, 24))
+    grids = (ops.OspSampleGrid * 2)(ops.OspSampleGrid(3, 2, 4, 4), ops.OspSampleGrid(0, 1, 0, 5))
+    assert lib.osp_rope3d_packed(p, p, p, p, grids, 2, 2, 64, ctypes.byref(r), None) == 1   # H = 0
+    assert "sample 1" in lib.osp_get_last_error().decode()
+    assert lib.osp_rope3d_packed(p, p, p, p, grids, 0, 2, 64, ctypes.byref(r), None) == 1
+    assert lib.osp_rope3d_packed(p, p, p, p, None, 1, 2, 64, ctypes.byref(r), None) == 1
+    bad = ops.make_rope((16, 24, 16))
+    assert lib.osp_rope3d_packed(p, p, p, p, grids, 1, 2, 64, ctypes.byref(bad), None) == 1
