@@ -11,6 +11,8 @@ from .spacetime_oracle import (  # noqa: F401
     attn_ref,
     cross_attn_ref,
     default_scale,
+    frame_causal_attn_ref,
+    frame_causal_limit,
     packed_attn_ref,
     rope3d_packed_ref,
     rope3d_positions_ref,
@@ -24,5 +26,7 @@ from .spacetime_oracle import (  # noqa: F401
     skiparse_scatter_ref,
     skiparse_sets,
     softmax_rows,
+    spatial_attn_ref,
+    temporal_attn_ref,
     video_positions,
 )

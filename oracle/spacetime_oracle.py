@@ -404,3 +404,91 @@ def packed_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_bounds: Seque
             out[0, sel, hi] = attention_head_ref(q[0, qb[i]:qb[i + 1], h], k[0, kk, h], v[0, kk, h], scale,
                                                  rows_[sel] - qb[i])
     return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Factorized and frame-causal attention masks
+# ----------------------------------------------------------------------------------------------
+#
+# "CogVideoX" section 2.2 and Table 8 compare 3D full attention with "2D + 1D" attention:
+# separate spatial attention (within one frame) and temporal attention (across frames).  The
+# Sora page ("Video DiT Diffusion Model") names Local Spatial Attention (patches of the same
+# frame; a block-diagonal 0/1 mask over frames), Causal Time Attention (previous frames), and
+# brute-force long-time attention (frame i attends to all earlier frames).  Readings: spatial
+# and temporal attention act on the video tokens only (no text); temporal attention of token
+# (t, h, w) covers the tokens (t', h, w) of the same spatial position, every t' (bidirectional)
+# or t' <= t (causal); frame-causal attention lets a token of frame t attend to every token of
+# frames 0..t, with a text prefix forming a block before frame 0 (text attends to text only,
+# every video token attends to the text).
+
+def spatial_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: Sequence[int],
+                     scale: float | None = None) -> np.ndarray:
+    """Per-frame attention: token (t, h, w) attends to the H*W tokens of frame t.
+    q, k, v: [B, T*H*W, n_h, d] video tokens (no text)."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    if N != T * H * W:
+        raise ValueError("spatial attention takes the T*H*W video tokens only")
+    scale = default_scale(d) if scale is None else scale
+    out = np.empty((B, N, nh, d), dtype=np.float64)
+    HW = H * W
+    for b in range(B):
+        for t in range(T):
+            f = slice(t * HW, (t + 1) * HW)
+            for h in range(nh):
+                out[b, f, h] = attention_head_ref(q[b, f, h], k[b, f, h], v[b, f, h], scale)
+    return out
+
+
+def temporal_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: Sequence[int],
+                      causal: bool = False, scale: float | None = None) -> np.ndarray:
+    """Per-position attention over time: token (t, h, w) attends to the tokens (t', h, w),
+    all t' or (causal) t' <= t.  q, k, v: [B, T*H*W, n_h, d] video tokens (no text)."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    if N != T * H * W:
+        raise ValueError("temporal attention takes the T*H*W video tokens only")
+    scale = default_scale(d) if scale is None else scale
+    HW = H * W
+    out = np.empty((B, N, nh, d), dtype=np.float64)
+    for b in range(B):
+        for pos in range(HW):
+            idx = pos + HW * np.arange(T)          # the position's token in every frame
+            for h in range(nh):
+                if not causal:
+                    out[b, idx, h] = attention_head_ref(q[b, idx, h], k[b, idx, h], v[b, idx, h], scale)
+                else:
+                    for t in range(T):
+                        sub = idx[:t + 1]
+                        out[b, idx[t], h] = attention_head_ref(q[b, idx[t:t + 1], h], k[b, sub, h], v[b, sub, h],
+                                                               scale)[0]
+    return out
+
+
+def frame_causal_limit(token: int, text_len: int, HW: int) -> int:
+    """Number of leading tokens a query token may attend to under the frame-causal mask: the
+    text block for a text token, the text and frames 0..t for a token of frame t."""
+    if token < text_len:
+        return text_len
+    return text_len + ((token - text_len) // HW + 1) * HW
+
+
+def frame_causal_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: Sequence[int], text_len: int,
+                          scale: float | None = None, rows=None, heads=None) -> np.ndarray:
+    """Frame-causal attention over [B, text_len + T*H*W, n_h, d]: query token r attends to the
+    first frame_causal_limit(r) tokens.  ``rows`` / ``heads`` select a subset as in attn_ref."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    if N != text_len + T * H * W:
+        raise ValueError("sequence length does not match text_len + T*H*W")
+    scale = default_scale(d) if scale is None else scale
+    rows_ = np.arange(N) if rows is None else np.asarray(rows)
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    lim = np.array([frame_causal_limit(int(r), text_len, H * W) for r in rows_])
+    out = np.empty((B, len(rows_), len(heads_), d), dtype=np.float64)
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            for L in np.unique(lim):
+                sel = np.nonzero(lim == L)[0]
+                out[b, sel, hi] = attention_head_ref(q[b, :L, h], k[b, :L, h], v[b, :L, h], scale, rows_[sel])
+    return out

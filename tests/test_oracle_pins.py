@@ -448,3 +448,81 @@ def test_packed_rope_restarts_positions_per_sample():
                     z = complex(x[0, base + r, hd, c], x[0, base + r, hd, c + 1]) * complex(math.cos(ang), math.sin(ang))
                     assert abs(y[0, base + r, hd, c] - z.real) < 1e-12
                     assert abs(y[0, base + r, hd, c + 1] - z.imag) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------------
+# factorized (2D + 1D) and frame-causal masks
+# ----------------------------------------------------------------------------------------------
+
+def _coords(T, H, W):
+    """(t, h, w) of every video token by nested loops (w fastest), written independently."""
+    out = []
+    for t in range(T):
+        for h in range(H):
+            for w in range(W):
+                out.append((t, h, w))
+    return out
+
+
+@pytest.mark.parametrize("grid", [(3, 2, 2), (2, 1, 3)])
+def test_spatial_and_temporal_attention_brute_force(grid):
+    T, H, W = grid
+    N = T * H * W
+    c = _coords(T, H, W)
+    rng = np.random.default_rng(40)
+    q, k, v = (rng.standard_normal((1, N, 2, 3)) for _ in range(3))
+    sp = O.spatial_attn_ref(q, k, v, grid)
+    te = O.temporal_attn_ref(q, k, v, grid)
+    tc = O.temporal_attn_ref(q, k, v, grid, causal=True)
+    for h in range(2):
+        args = (q[0, :, h].tolist(), k[0, :, h].tolist(), v[0, :, h].tolist())
+        np.testing.assert_allclose(sp[0, :, h], _brute_masked_attention(*args, lambda i, j: c[i][0] == c[j][0],
+                                                                         1 / math.sqrt(3)), rtol=1e-12, atol=1e-13)
+        same_pos = lambda i, j: c[i][1:] == c[j][1:]
+        np.testing.assert_allclose(te[0, :, h], _brute_masked_attention(*args, same_pos, 1 / math.sqrt(3)),
+                                   rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(tc[0, :, h], _brute_masked_attention(
+            *args, lambda i, j: same_pos(i, j) and c[j][0] <= c[i][0], 1 / math.sqrt(3)), rtol=1e-12, atol=1e-13)
+    # causal: the first frame sees only itself -> its own value
+    HW = H * W
+    np.testing.assert_allclose(tc[0, :HW], v[0, :HW], atol=1e-15)
+
+
+def test_factorized_special_cases():
+    rng = np.random.default_rng(41)
+    q, k, v = (rng.standard_normal((2, 12, 2, 4)) for _ in range(3))
+    # one frame: spatial = full attention, temporal = each token alone (its own value)
+    np.testing.assert_allclose(O.spatial_attn_ref(q, k, v, (1, 3, 4)), O.attn_ref(q, k, v), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(O.temporal_attn_ref(q, k, v, (1, 3, 4)), v, atol=1e-15)
+    # one position per frame: temporal = full attention, spatial = each token alone
+    np.testing.assert_allclose(O.temporal_attn_ref(q, k, v, (12, 1, 1)), O.attn_ref(q, k, v), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(O.spatial_attn_ref(q, k, v, (12, 1, 1)), v, atol=1e-15)
+
+
+def test_frame_causal_limit_values():
+    # text_len 3, frames of 4 tokens: text -> 3; frame 0 (tokens 3..6) -> 7; frame 1 -> 11
+    assert [O.frame_causal_limit(r, 3, 4) for r in range(11)] == [3, 3, 3, 7, 7, 7, 7, 11, 11, 11, 11]
+    assert [O.frame_causal_limit(r, 0, 2) for r in range(6)] == [2, 2, 4, 4, 6, 6]
+
+
+def test_frame_causal_attention_brute_force():
+    T, H, W, L = 3, 1, 2, 2
+    N = L + T * H * W
+    # block of each token written out: text 0, frame t -> t + 1
+    block = [0, 0, 1, 1, 2, 2, 3, 3]
+    rng = np.random.default_rng(42)
+    q, k, v = (rng.standard_normal((1, N, 2, 5)) for _ in range(3))
+    got = O.frame_causal_attn_ref(q, k, v, (T, H, W), L)
+    for h in range(2):
+        ref = _brute_masked_attention(q[0, :, h].tolist(), k[0, :, h].tolist(), v[0, :, h].tolist(),
+                                      lambda i, j: block[j] <= block[i], 1 / math.sqrt(5))
+        np.testing.assert_allclose(got[0, :, h], ref, rtol=1e-12, atol=1e-13)
+    # the last frame sees everything: full attention there
+    full = O.attn_ref(q, k, v)
+    np.testing.assert_allclose(got[:, -2:], full[:, -2:], rtol=1e-13, atol=1e-14)
+    # rows / heads subsets
+    np.testing.assert_allclose(O.frame_causal_attn_ref(q, k, v, (T, H, W), L, rows=[7, 2, 0], heads=[1]),
+                               got[:, [7, 2, 0]][:, :, [1]], rtol=0, atol=1e-15)
+    # one frame, no text: plain full attention
+    np.testing.assert_allclose(O.frame_causal_attn_ref(q[:, :6], k[:, :6], v[:, :6], (1, 2, 3), 0),
+                               O.attn_ref(q[:, :6], k[:, :6], v[:, :6]), rtol=1e-13, atol=1e-14)
