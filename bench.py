@@ -380,6 +380,75 @@ def run_packed_op(args, rank, world, local_rank):
             "clocks": clocks, "gpu_launches": 2 * args.steps}
 
 
+def run_variant_op(args, rank, world, local_rank):
+    """Time one attention variant alone on the workload's full video grid: spatial (per-frame,
+    tensor-bound), temporal (per-position over frames, HBM-bound; --causal for t' <= t) or
+    frame_causal (text block + frames, tensor-bound).  Three rotating input sets."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = syn.WORKLOADS[args.workload]
+    T, H, W = w.grid
+    HW = H * W
+    L = w.text_len if args.op == "frame_causal" else 0
+    N = L + w.n_video
+    nset = 3
+    sets = [tuple(syn.randn_bf16((w.B, N, w.heads, w.head_dim), w.seed + 11 + 101 * r + 17 * rank + i).to(dev)
+                  for i in range(3)) for r in range(nset)]
+    outs = [torch.empty_like(q) for q, _, _ in sets]
+    if args.op == "spatial":
+        launch = lambda i: ops.attn_spatial(*sets[i % nset], w.grid, o=outs[i % nset])
+        pairs = w.B * T * HW * HW
+    elif args.op == "temporal":
+        launch = lambda i: ops.attn_temporal(*sets[i % nset], w.grid, causal=args.causal, o=outs[i % nset])
+        pairs = w.B * HW * (T * (T + 1) // 2 if args.causal else T * T)
+    else:
+        launch = lambda i: ops.attn_frame_causal(*sets[i % nset], w.grid, L, o=outs[i % nset])
+        pairs = w.B * (L * L + sum(HW * (L + (t + 1) * HW) for t in range(T)))
+    flops = 4.0 * w.heads * w.head_dim * pairs            # unmasked (query, key) pairs only
+    nbytes = 4 * w.B * N * w.heads * w.head_dim * 2       # q, k, v read once, o written once
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        launch(i)
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ops.check_status(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    peaks, src = load_peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    peak_t, peak_b = float(peaks["bf16_tflops_sustained"]), float(peaks["hbm_gbs"])
+    if args.op == "temporal":
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_b, "unit": "GB/s",
+                "frac": round(gbs / peak_b, 4), "peak_source": f"{src} (copy bandwidth)",
+                "kernel": "attn_temporal_kernel" if T <= 64 else "attn_fwd_kernel (Single Skip, k = H*W)"}
+        metric, value, unit = "temporal attention GB/s (2D+1D, 1D part)", gbs, "GB/s"
+    else:
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_t, "unit": "TFLOP/s",
+                "frac": round(tflops / peak_t, 4), "peak_source": f"{src} (sustained bf16 GEMM)",
+                "kernel": "attn_fwd_kernel"}
+        metric = ("spatial attention TFLOP/s (2D+1D, 2D part)" if args.op == "spatial"
+                  else "frame-causal attention TFLOP/s (unmasked pairs)")
+        value, unit = tflops, "TFLOP/s"
+    roof.update(traffic=None, bytes_per_launch=nbytes, flops_per_launch=flops)
+    cfg = dict(w.describe(), op=args.op, text_len=L, l2=f"{nset} input sets rotated ({nset * nbytes / 1e6:.0f} MB)")
+    if args.op == "temporal":
+        cfg["causal"] = bool(args.causal)
+    return {"metric": metric, "value": round(world * value, 1), "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roof,
+            "clocks": clocks, "gpu_launches": args.steps, "tflops": round(tflops, 1), "hbm_gbs": round(gbs, 1)}
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -614,12 +683,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse"],
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
-    ap.add_argument("--op", default="step", choices=["step", "rope", "gather", "scatter", "cross", "packed"],
+    ap.add_argument("--op", default="step",
+                    choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
+                             "frame_causal"],
                     help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone; "
                          "cross: video -> text cross-attention alone; packed: a packed batch of mixed shapes")
     ap.add_argument("--packed", default="frame_pack_cog2b", choices=sorted(syn.PACKED_WORKLOADS),
                     help="--op packed: the packed batch")
     ap.add_argument("--text-len", type=int, default=226, help="--op cross: text tokens (keys)")
+    ap.add_argument("--causal", action="store_true", help="--op temporal: causal in time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -645,7 +717,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        runner = {"step": run_ours, "cross": run_cross_op, "packed": run_packed_op}.get(args.op, run_hbm_op)
+        runner = {"step": run_ours, "cross": run_cross_op, "packed": run_packed_op, "spatial": run_variant_op,
+                  "temporal": run_variant_op, "frame_causal": run_variant_op}.get(args.op, run_hbm_op)
         line = runner(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -128,6 +128,37 @@ int osp_attn_full(const void* q, const void* k, const void* v, void* o, const os
 int osp_attn_cross(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                    float softmax_scale, void* stream);
 
+/* Factorized "2D + 1D" attention ("CogVideoX" section 2.2 and Table 8: separate spatial and
+ * temporal attention, the baseline 3D full attention replaces; the Sora page, "Video DiT
+ * Diffusion Model": Local Spatial Attention and Causal Time Attention).  Video tokens only:
+ * shape->text_len must be 0 (OSP_ERR_UNSUPPORTED otherwise); q, k, v, o as osp_attn_full.
+ *
+ * osp_attn_spatial: token (t, h, w) attends to the H*W tokens of frame t (block-diagonal over
+ *   frames). Runs osp_attn_full's kernel on the B*T frames (same arithmetic and work split). */
+int osp_attn_spatial(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                     float softmax_scale, void* stream);
+
+/* osp_attn_temporal: token (t, h, w) attends to the tokens (t', h, w) of its spatial position,
+ *   every t' (causal = 0) or t' <= t (causal = 1).
+ *   T <= 64: a shared-memory-staged kernel with mma.sync tiles (the sets are too small for
+ *   128-row tensor-memory tiles; the work is bound by HBM traffic), P rounded to bf16, fp32
+ *   accumulation.  T > 64 (causal = 0 only): the osp_skiparse_attn kernel with the position's
+ *   tokens as Single Skip set pos, k = H*W.
+ *   Errors: OSP_ERR_INVALID_ARG (causal not 0/1, ...), OSP_ERR_UNSUPPORTED (text, causal with
+ *   T > 64, head_dim), OSP_ERR_CUDA. */
+int osp_attn_temporal(const void* q, const void* k, const void* v, void* o, const osp_shape* shape, int32_t causal,
+                      float softmax_scale, void* stream);
+
+/* Frame-causal attention (the Sora page, "Long-Time Consistency Strategies": during generation of
+ * frame i the model attends to all previous frames): over N = text_len + T*H*W tokens, query
+ * token r attends to the first limit(r) tokens, limit = text_len for a text token and
+ * text_len + (t + 1)*H*W for a token of frame t (text is one block before frame 0; it sees
+ * itself, every video token sees it).  q, k, v, o as osp_attn_full; same kernel and arithmetic,
+ * with key tiles past a query block's last limit skipped; no KV-range split.
+ *  Errors: as osp_attn_full. */
+int osp_attn_frame_causal(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                          float softmax_scale, void* stream);
+
 /* 3D RoPE of a packed batch (CogVideoX section 3.1: every video keeps its own position grid,
  * starting at (0, 0, 0); extrapolation, never rescaled).
  *  samples:       HOST array of n_samples (1 .. OSP_MAX_SEGMENTS) sample grids, read during the call.

@@ -116,6 +116,11 @@ struct AttnParams {
   unsigned* status;
   unsigned long long timeout_ns;
   int debug_withhold_q;   // test knob: never load Q, so every consumer's bounded wait runs out
+  // Frame-causal mask (dense layout only; 0 = off): query token r attends to the first
+  // limit(r) keys, limit = text_len for a text token and text_len + (t + 1) * frame_hw for a
+  // token of frame t.  Query blocks then run heaviest (latest) first.
+  int frame_hw;
+  int text_len;
   // Work items (1-D grid): units are (sample*set, head, query block) with the query block fastest.
   // CTAs [0, n_full) process whole units; every later unit is split into n_split KV ranges whose
   // CTAs write fp32 partials (unnormalised O, running max m, row sum l) to ws_o / ws_ml, merged
@@ -138,14 +143,21 @@ struct SegTable {
   int kv[kMaxSegments + 1];
 };
 struct NoSegTable {};
-template <bool kPacked>
-using SegParam = typename std::conditional<kPacked, SegTable, NoSegTable>::type;
+// Kernel variants: plain (dense / Skiparse / cross), packed batch, frame-causal mask.
+enum AttnMode { kModePlain = 0, kModePacked = 1, kModeFrameCausal = 2 };
+template <int kMode>
+using SegParam = typename std::conditional<kMode == kModePacked, SegTable, NoSegTable>::type;
 
 __device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
                                           int chan, int row0, int g, int b, int k) {
   if (layout == 0) tma_load_3d(dst, tm, bar, chan, row0, b);
   else if (layout == 1) tma_load_4d(dst, tm, bar, chan, g, row0, b);
   else tma_load_5d(dst, tm, bar, chan, 0, g, row0 / k, b);
+}
+
+// Keys visible to query token r under the frame-causal mask (text block, then one block per frame).
+__device__ __forceinline__ int frame_causal_limit(int r, int text_len, int hw) {
+  return r < text_len ? text_len : text_len + ((r - text_len) / hw + 1) * hw;
 }
 
 // Natural token index of slot s of set g.
@@ -229,11 +241,13 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, bool kPacked>
+template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p,
-                    const __grid_constant__ SegParam<kPacked> seg) {
+                    const __grid_constant__ SegParam<kMode> seg) {
+  constexpr bool kPacked = kMode == kModePacked;
+  constexpr bool kFrameCausal = kMode == kModeFrameCausal;
   using C = Cfg<D>;
   constexpr int S = C::kStages;
   extern __shared__ unsigned char smem_raw[];
@@ -295,6 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       w.kv_row0 = 0;
       w.nq = p.n_q;
       w.nkv = p.n_kv;
+    }
+    if constexpr (kFrameCausal) {
+      qb = p.qblocks - 1 - qb;   // latest (longest) query blocks first
+      // keys up to the limit of the block's last query row
+      const int last = min(qb * (2 * kBM) + 2 * kBM, w.nq) - 1;
+      w.nkv = min(w.nkv, frame_causal_limit(last, p.text_len, p.frame_hw));
     }
     w.q0 = qb * (2 * kBM);
     const int n_kv_all = (w.nkv + kBN - 1) / kBN;
@@ -577,7 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    const int valid0 = wk.nkv - wk.kv_lo * kBN;   // valid keys from this CTA's first KV tile on
+    int lim = wk.nkv;                                // keys this row may see
+    if constexpr (kFrameCausal)
+      lim = min(lim, frame_causal_limit(wk.q0 + i * kBM + row, p.text_len, p.frame_hw));
+    const int valid0 = lim - wk.kv_lo * kBN;         // valid keys from this CTA's first KV tile on
     for (int j = 0; j < n_kv; ++j) {
       if (!warp_wait(bar(B_SFULL + i), j & 1, wc)) { ok = false; break; }
       tc_fence_after();
@@ -797,25 +820,25 @@ int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int l
   return OSP_OK;
 }
 
-template <int D, bool kPacked>
+template <int D, int kMode>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
-             const SegParam<kPacked>& seg, dim3 grid, cudaStream_t stream) {
+             const SegParam<kMode>& seg, dim3 grid, cudaStream_t stream) {
   constexpr int smem = Cfg<D>::kSmemBytes;
   static bool attr_done = false;  // per process; the attribute is per function, not per device
   if (!attr_done) {
     // The warpgroup register split only adds up if the kernel is launched with exactly
     // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kPacked>) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode>) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncGetAttributes(attn_fwd_kernel<%d>) failed", D);
     if ((uint32_t)fa.numRegs != kRegsLaunch)
       return set_error(OSP_ERR_CUDA, "attn_fwd_kernel<%d> compiled to %d registers per thread, expected %u", D,
                        fa.numRegs, kRegsLaunch);
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_fwd_kernel<%d>) failed", D);
     attr_done = true;
   }
-  attn_fwd_kernel<D, kPacked><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
+  attn_fwd_kernel<D, kMode><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
   return check_launch("attn_fwd_kernel");
 }
 
@@ -825,9 +848,10 @@ namespace {
 
 // Attention launch with an explicit status word (the kernel's only global scratch).
 // N_kv: tokens per sample of k and v; < 0 means the same sequence as q (self-attention).
+// frame_causal: dense layout only; the frame-causal mask over s's text block and frames.
 int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
                        int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
-                       int N_kv = -1) {
+                       int N_kv = -1, bool frame_causal = false) {
   const int N = (N_kv < 0) ? s.text_len + s.T * s.H * s.W : s.T * s.H * s.W;   // q / o tokens per sample
   if (N_kv < 0) N_kv = N;
   const int G = (layout == 0) ? 1 : sparse_k;
@@ -845,6 +869,9 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
   p.debug_withhold_q = debug_withhold_q();
+  p.frame_hw = frame_causal ? s.H * s.W : 0;
+  p.text_len = s.text_len;
+  if (frame_causal) allow_split = false;   // a KV range could hold no visible key for some rows
   CUtensorMap tq, tk, tv;
   int rc;
   if ((rc = make_tmap(&tq, q, s, N, layout, p.k)) != OSP_OK) return rc;
@@ -881,9 +908,18 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
   dim3 grid((unsigned)ctas);
   switch (s.head_dim) {
-    case 64: rc = launch_d<64, false>(tq, tk, tv, p, NoSegTable{}, grid, stream); break;
-    case 96: rc = launch_d<96, false>(tq, tk, tv, p, NoSegTable{}, grid, stream); break;
-    case 128: rc = launch_d<128, false>(tq, tk, tv, p, NoSegTable{}, grid, stream); break;
+    case 64:
+      rc = frame_causal ? launch_d<64, kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, grid, stream)
+                        : launch_d<64, kModePlain>(tq, tk, tv, p, NoSegTable{}, grid, stream);
+      break;
+    case 96:
+      rc = frame_causal ? launch_d<96, kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, grid, stream)
+                        : launch_d<96, kModePlain>(tq, tk, tv, p, NoSegTable{}, grid, stream);
+      break;
+    case 128:
+      rc = frame_causal ? launch_d<128, kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, grid, stream)
+                        : launch_d<128, kModePlain>(tq, tk, tv, p, NoSegTable{}, grid, stream);
+      break;
     default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
   }
   if (rc == OSP_OK && p.n_split > 1) {
@@ -914,6 +950,13 @@ int cross_attention_launch(const void* q, const void* k, const void* v, void* o,
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   return launch_with_status(q, k, v, o, s, 0, 1, scale, stream, status, true, s.text_len);
+}
+
+int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
+                                  float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  return launch_with_status(q, k, v, o, s, 0, 1, scale, stream, status, false, -1, true);
 }
 
 int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
@@ -957,9 +1000,9 @@ int packed_attention_launch(const void* q, const void* k, const void* v, void* o
   if ((rc = make_tmap(&tv, v, sh, n_kv_total, 0, 1)) != OSP_OK) return rc;
   const dim3 grid((unsigned)units);
   switch (head_dim) {
-    case 64: return launch_d<64, true>(tq, tk, tv, p, seg, grid, stream);
-    case 96: return launch_d<96, true>(tq, tk, tv, p, seg, grid, stream);
-    case 128: return launch_d<128, true>(tq, tk, tv, p, seg, grid, stream);
+    case 64: return launch_d<64, kModePacked>(tq, tk, tv, p, seg, grid, stream);
+    case 96: return launch_d<96, kModePacked>(tq, tk, tv, p, seg, grid, stream);
+    case 128: return launch_d<128, kModePacked>(tq, tk, tv, p, seg, grid, stream);
     default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
   }
 }

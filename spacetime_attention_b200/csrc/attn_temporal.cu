@@ -1,0 +1,299 @@
+// Temporal attention of the factorized "2D + 1D" scheme: token (t, h, w) attends to the tokens
+// (t', h, w) of the same spatial position, every t' or (causal) t' <= t.
+//
+// Sources: "CogVideoX: Text-to-Video Diffusion Models with an Expert Transformer", section 2.2
+// (separated spatial and temporal attention of earlier video models) and Table 8 (3D full vs
+// 2D + 1D attention); the Sora page, "Video DiT Diffusion Model" (Causal Time Attention).
+//
+// The work is many independent tiny problems: one (sample, spatial position, head) set of T
+// tokens (T <= 64) at a stride of H*W rows, T x T scores over head_dim channels.  Per token and
+// head it reads q, k, v and writes o once (8 * head_dim bytes) for 4 * T * head_dim flops:
+// 6.5 flop/byte at T = 13, d = 64, far below the balance point, so the kernel is bound by HBM.
+// The design therefore follows the memory: each warp owns one set at a time and stages its
+// q/k/v rows in shared memory with 16-byte cp.async copies; many resident warps (one staging
+// buffer each, ~100 KB of shared memory per CTA, two CTAs per SM) keep enough copies in flight,
+// which measured faster than fewer warps with double buffers.  The small contractions run on mma.sync
+// (m16n8k16, bf16 in, fp32 accumulate) so that the arithmetic costs a few dozen instructions
+// per set instead of thousands of scalar FMAs.  The 128-row tcgen05 tiles of the main kernel
+// would leave more than 85 % of every tile empty here.
+
+#include "osp_internal.h"
+
+// Staging buffers per warp (2: the next set's copies overlap the current set's arithmetic) and
+// the shared memory a CTA may take (bounds the warps per CTA).  Measured on B200 (GB/s, CogVideoX
+// / Open-Sora Plan / long grids): 1 buffer, 100 KB: 5270 / 5260 / 5740; 2 buffers, 200 KB:
+// 5160 / 3930 / 5620.
+#ifndef OSP_TEMPORAL_BUFS
+#define OSP_TEMPORAL_BUFS 1
+#endif
+#ifndef OSP_TEMPORAL_SMEM_KB
+#define OSP_TEMPORAL_SMEM_KB 100
+#endif
+
+namespace osp {
+
+namespace {
+
+struct TemporalParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  __nv_bfloat16* o;
+  int T, HW, heads;
+  long long n_sets;     // B * HW * heads, set s = (b * HW + pos) * heads + h
+  float scale_log2;
+  int causal;
+  int warps;            // warps per CTA (each with its own staging buffers)
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool fill) {
+  // src-size 0 writes 16 zero bytes and reads nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(fill ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D, int MT>
+struct TemporalCfg {
+  static constexpr int kRows = 16 * MT;              // token rows per set, padded
+  static constexpr int kRowBytes = D * 2 + 16;       // padded row: conflict-free ldmatrix
+  static constexpr int kTensorBytes = kRows * kRowBytes;
+  static constexpr int kBufBytes = 3 * kTensorBytes; // q, k, v
+  static constexpr int kBufs = OSP_TEMPORAL_BUFS;
+  static constexpr int kWarpBytes = kBufs * kBufBytes;
+};
+
+template <int D, int MT>
+__global__ void __launch_bounds__(256) attn_temporal_kernel(const TemporalParams p) {
+  using C = TemporalCfg<D, MT>;
+  constexpr int kChunks = D / 8;                     // 16-byte chunks per row
+  extern __shared__ __align__(128) unsigned char smem_t[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t wbase = smem_u32(smem_t) + (uint32_t)(warp * C::kWarpBytes);
+  const long long step = (long long)gridDim.x * p.warps;
+  long long set = (long long)blockIdx.x * p.warps + warp;
+  const int g = lane >> 2, c = lane & 3;
+
+  // global element offset of row t = 0 of a set (the host checks n_sets < 2^31); row t adds
+  // t * tstride
+  const long long tstride = (long long)p.HW * p.heads * D;
+  auto set_base = [&](long long s) -> long long {
+    const int si = (int)s;
+    const int h = si % p.heads, bp = si / p.heads;
+    const int pos = bp % p.HW, b = bp / p.HW;
+    return ((long long)b * p.T * p.HW + pos) * p.heads * D + (long long)h * D;
+  };
+  auto prefetch = [&](long long s, int buf) {
+    const uint32_t base = wbase + (uint32_t)(buf * C::kBufBytes);
+    const long long sb = set_base(s);
+    for (int ch = lane; ch < C::kRows * kChunks; ch += 32) {
+      const int r = ch / kChunks, cc = ch - r * kChunks;
+      const bool live = r < p.T;
+      const long long off = live ? sb + r * tstride + cc * 8 : 0;
+      const uint32_t dst = base + (uint32_t)(r * C::kRowBytes + cc * 16);
+      cp_async16(dst, p.q + off, live);
+      cp_async16(dst + C::kTensorBytes, p.k + off, live);
+      cp_async16(dst + 2 * C::kTensorBytes, p.v + off, live);
+    }
+    cp_async_commit();
+  };
+
+  int buf = 0;
+  if (C::kBufs == 2 && set < p.n_sets) prefetch(set, 0);
+  for (; set < p.n_sets; set += step, buf ^= (C::kBufs - 1)) {
+    if constexpr (C::kBufs == 2) {
+      const bool more = set + step < p.n_sets;
+      if (more) prefetch(set + step, buf ^ 1);
+      if (more) cp_async_wait<1>();
+      else cp_async_wait<0>();
+    } else {
+      prefetch(set, 0);
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const uint32_t sq = wbase + (uint32_t)(buf * C::kBufBytes);
+    const uint32_t sk = sq + C::kTensorBytes, sv = sq + 2 * C::kTensorBytes;
+
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      // ---- S = Q K^T for query rows mt*16 .. mt*16+15, all kRows keys
+      float s[2 * MT][4];
+#pragma unroll
+      for (int nt = 0; nt < 2 * MT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(sq + (uint32_t)((mt * 16 + (lane & 15)) * C::kRowBytes + (kk * 16 + (lane >> 4) * 8) * 2), a[0], a[1],
+                a[2], a[3]);
+#pragma unroll
+        for (int n2 = 0; n2 < MT; ++n2) {   // 16 keys per ldmatrix.x4
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sk + (uint32_t)((n2 * 16 + (lane & 7) + ((lane >> 4) << 3)) * C::kRowBytes +
+                                  (kk * 16 + ((lane >> 3) & 1) * 8) * 2),
+                  b0, b1, b2, b3);
+          mma_bf16_16816(s[2 * n2], a, b0, b1);
+          mma_bf16_16816(s[2 * n2 + 1], a, b2, b3);
+        }
+      }
+      // ---- mask, row max, exponentials, row sums (rows r0 = mt*16 + g and r1 = r0 + 8)
+      const int r0 = mt * 16 + g, r1 = r0 + 8;
+      float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2 * MT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = nt * 8 + 2 * c + e;
+          const bool ok0 = key < p.T && (!p.causal || key <= r0);
+          const bool ok1 = key < p.T && (!p.causal || key <= r1);
+          s[nt][e] = ok0 ? s[nt][e] * p.scale_log2 : -INFINITY;
+          s[nt][2 + e] = ok1 ? s[nt][2 + e] * p.scale_log2 : -INFINITY;
+          m0 = fmaxf(m0, s[nt][e]);
+          m1 = fmaxf(m1, s[nt][2 + e]);
+        }
+      }
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+      // rows past T with the causal mask still see key 0, so m is finite on every row
+      float l0 = 0.f, l1 = 0.f;
+      uint32_t pa[MT][4];   // P as A fragments, one per 16 keys
+#pragma unroll
+      for (int nt = 0; nt < 2 * MT; ++nt) {
+        const float e0 = ex2_approx(s[nt][0] - m0), e1 = ex2_approx(s[nt][1] - m0);
+        const float e2 = ex2_approx(s[nt][2] - m1), e3 = ex2_approx(s[nt][3] - m1);
+        l0 += e0 + e1;
+        l1 += e2 + e3;
+        pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(e0, e1);
+        pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(e2, e3);
+      }
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      // ---- O = P V
+      float o[D / 8][4];
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < MT; ++kk) {
+        // A fragment of keys kk*16..+15: (row g, keys 2c..) from n-tile 2kk, (row g+8) likewise,
+        // then the same rows for keys +8 from n-tile 2kk+1
+        const uint32_t a[4] = {pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3]};
+#pragma unroll
+        for (int n2 = 0; n2 < D / 16; ++n2) {   // 16 channels per ldmatrix.x4.trans
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(sv + (uint32_t)((kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::kRowBytes +
+                                    (n2 * 16 + (lane >> 4) * 8) * 2),
+                    b0, b1, b2, b3);
+          mma_bf16_16816(o[2 * n2], a, b0, b1);
+          mma_bf16_16816(o[2 * n2 + 1], a, b2, b3);
+        }
+      }
+      // ---- normalise and park the bf16 rows in the (consumed) Q rows of this m-tile
+      const float i0 = 1.f / l0, i1 = 1.f / l1;
+      __syncwarp();
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt) {
+        const uint32_t col = (uint32_t)((nt * 8 + 2 * c) * 2);
+        const uint32_t w0 = pack_bf16x2(o[nt][0] * i0, o[nt][1] * i0);
+        const uint32_t w1 = pack_bf16x2(o[nt][2] * i1, o[nt][3] * i1);
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sq + (uint32_t)(r0 * C::kRowBytes) + col), "r"(w0) : "memory");
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sq + (uint32_t)(r1 * C::kRowBytes) + col), "r"(w1) : "memory");
+      }
+    }
+    __syncwarp();
+    // ---- coalesced 16-byte stores of the T output rows
+    const long long ob = set_base(set);
+    for (int ch = lane; ch < p.T * kChunks; ch += 32) {
+      const int r = ch / kChunks, cc = ch - r * kChunks;
+      uint4 val;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                   : "r"(sq + (uint32_t)(r * C::kRowBytes + cc * 16)));
+      *reinterpret_cast<uint4*>(p.o + ob + r * tstride + cc * 8) = val;
+    }
+    __syncwarp();   // this buffer is refilled by the prefetch two sets later
+  }
+}
+
+template <int D, int MT>
+int launch_temporal_t(TemporalParams& p, cudaStream_t stream) {
+  using C = TemporalCfg<D, MT>;
+  // as many warps per CTA (<= 8) as fit the shared-memory budget
+  p.warps = std::max(1, std::min(8, (OSP_TEMPORAL_SMEM_KB * 1024) / C::kWarpBytes));
+  const int smem = p.warps * C::kWarpBytes;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(attn_temporal_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_temporal_kernel) failed");
+    attr_done = true;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_temporal_kernel<D, MT>, p.warps * 32, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const long long ctas_needed = (p.n_sets + p.warps - 1) / p.warps;
+  const long long grid = std::min<long long>(ctas_needed, (long long)device_sm_count() * per_sm);
+  attn_temporal_kernel<D, MT><<<(unsigned)grid, p.warps * 32, smem, stream>>>(p);
+  return check_launch("attn_temporal_kernel");
+}
+
+template <int D>
+int launch_temporal_d(TemporalParams& p, cudaStream_t stream) {
+  switch ((p.T + 15) / 16) {
+    case 1: return launch_temporal_t<D, 1>(p, stream);
+    case 2: return launch_temporal_t<D, 2>(p, stream);
+    case 3: return launch_temporal_t<D, 3>(p, stream);
+    default: return launch_temporal_t<D, 4>(p, stream);
+  }
+}
+
+}  // namespace
+
+int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
+                              float scale, cudaStream_t stream) {
+  TemporalParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.T = s.T;
+  p.HW = s.H * s.W;
+  p.heads = s.heads;
+  p.n_sets = (long long)s.B * p.HW * s.heads;
+  if (p.n_sets > 0x7fffffffLL) return set_error(OSP_ERR_UNSUPPORTED, "%lld temporal sets is too many", p.n_sets);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  switch (s.head_dim) {
+    case 64: return launch_temporal_d<64>(p, stream);
+    case 96: return launch_temporal_d<96>(p, stream);
+    case 128: return launch_temporal_d<128>(p, stream);
+    default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  }
+}
+
+}  // namespace osp

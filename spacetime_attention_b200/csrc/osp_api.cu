@@ -207,6 +207,54 @@ int osp_attn_cross(const void* q, const void* k, const void* v, void* o, const o
   return cross_attention_launch(q, k, v, o, *shape, softmax_scale, static_cast<cudaStream_t>(stream));
 }
 
+int osp_attn_spatial(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                     float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (shape->text_len != 0) return set_error(OSP_ERR_UNSUPPORTED, "spatial attention takes video tokens only (text_len 0)");
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if ((long long)shape->B * shape->T > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "too many frames");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  // [B][T*H*W][heads][d] is [B*T][H*W][heads][d]: one dense problem per frame
+  const osp_shape frames{shape->B * shape->T, 0, 1, 1, shape->H * shape->W, shape->heads, shape->head_dim};
+  return attention_launch(q, k, v, o, frames, 0, 1, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+int osp_attn_temporal(const void* q, const void* k, const void* v, void* o, const osp_shape* shape, int32_t causal,
+                      float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (shape->text_len != 0)
+    return set_error(OSP_ERR_UNSUPPORTED, "temporal attention takes video tokens only (text_len 0)");
+  if (causal != 0 && causal != 1) return set_error(OSP_ERR_INVALID_ARG, "causal must be 0 or 1 (got %d)", causal);
+  if (causal && shape->T > 64)
+    return set_error(OSP_ERR_UNSUPPORTED, "causal temporal attention supports T <= 64 (got %d)", shape->T);
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (shape->T <= 64) return temporal_attention_launch(q, k, v, o, *shape, causal, softmax_scale, st);
+  // longer sets: the position's tokens t*H*W + pos are Single Skip set pos with k = H*W
+  return attention_launch(q, k, v, o, *shape, OSP_SKIP_SINGLE + 1, shape->H * shape->W, softmax_scale, st);
+}
+
+int osp_attn_frame_causal(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
+                          float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return frame_causal_attention_launch(q, k, v, o, *shape, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
 int osp_rope3d_packed(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
                       int32_t n_samples, int32_t heads, int32_t head_dim, const osp_rope* rope, void* stream) {
   g_last_error[0] = 0;

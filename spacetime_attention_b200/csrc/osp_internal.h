@@ -58,6 +58,14 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
 int cross_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, float scale,
                            cudaStream_t stream);
 
+// Frame-causal attention (dense layout): token r attends to the text block and the frames up to its own.
+int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
+                                  float scale, cudaStream_t stream);
+
+// Temporal attention of 2D + 1D (T <= 64): sets of T tokens at stride H*W, optionally causal in t.
+int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
+                              float scale, cudaStream_t stream);
+
 // Packed batch (block-diagonal attention): segment i owns q/o rows [q_bounds[i], q_bounds[i+1])
 // and k/v rows [kv_bounds[i], kv_bounds[i+1]); host arrays of n_seg + 1 validated offsets.
 int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,

@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "OSP_OK", 1: "OSP_ERR_INVALID_ARG", 2: "OSP_ERR_UNSUPPORTED",
 # Every symbol include/osp.h declares (tests check the library exports all of them).
 EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_scatter", "osp_skiparse_attn",
             "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version",
-            "osp_attn_full_noalloc", "osp_attn_cross", "osp_rope3d_packed", "osp_attn_packed")
+            "osp_attn_full_noalloc", "osp_attn_cross", "osp_rope3d_packed", "osp_attn_packed",
+            "osp_attn_spatial", "osp_attn_temporal", "osp_attn_frame_causal")
 
 MAX_SEGMENTS = 256   # OSP_MAX_SEGMENTS
 
@@ -68,6 +69,9 @@ def library() -> ctypes.CDLL:
             "osp_attn_full": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_full_noalloc": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_cross": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_spatial": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_temporal": [vp, vp, vp, vp, sp, i32, ctypes.c_float, vp],
+            "osp_attn_frame_causal": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_rope3d_packed": [vp, vp, vp, vp, ctypes.POINTER(OspSampleGrid), i32, i32, i32, rp, vp],
             "osp_attn_packed": [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
                                 i32, i32, ctypes.c_float, vp],
@@ -160,6 +164,32 @@ def attn_cross(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, scale: f
     _check("osp_attn_cross", library().osp_attn_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                       ctypes.c_float(scale), _stream_handle(q)))
     return o
+
+
+def _attn3(fn: str, q, k, v, grid, text_len, scale, o, *extra):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    shp = _shape_of(q, grid, text_len)
+    f = getattr(library(), fn)
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp), *extra, ctypes.c_float(scale), _stream_handle(q)]
+    _check(fn, f(*args))
+    return o
+
+
+def attn_spatial(q, k, v, grid, scale: float = 0.0, o=None) -> torch.Tensor:
+    """osp_attn_spatial: per-frame attention over the H*W tokens of each frame (no text)."""
+    return _attn3("osp_attn_spatial", q, k, v, grid, 0, scale, o)
+
+
+def attn_temporal(q, k, v, grid, causal: bool = False, scale: float = 0.0, o=None) -> torch.Tensor:
+    """osp_attn_temporal: per-position attention over the T frames (causal: t' <= t)."""
+    return _attn3("osp_attn_temporal", q, k, v, grid, 0, scale, o, int(bool(causal)))
+
+
+def attn_frame_causal(q, k, v, grid, text_len: int, scale: float = 0.0, o=None) -> torch.Tensor:
+    """osp_attn_frame_causal: token of frame t attends to the text and frames 0..t."""
+    return _attn3("osp_attn_frame_causal", q, k, v, grid, text_len, scale, o)
 
 
 def _bounds(b) -> ctypes.Array:

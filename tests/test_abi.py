@@ -127,3 +127,14 @@ def test_packed_rope_validation(lib):
     assert lib.osp_rope3d_packed(p, p, p, p, None, 1, 2, 64, ctypes.byref(r), None) == 1
     bad = ops.make_rope((16, 24, 16))
     assert lib.osp_rope3d_packed(p, p, p, p, grids, 1, 2, 64, ctypes.byref(bad), None) == 1
+
+
+def test_factorized_validation(lib):
+    p = ctypes.c_void_p(256)
+    assert lib.osp_attn_spatial(p, p, p, p, shp(L=4), 0.0, None) == 2          # text not allowed
+    assert lib.osp_attn_temporal(p, p, p, p, shp(L=4), 0, 0.0, None) == 2
+    assert lib.osp_attn_temporal(p, p, p, p, shp(), 2, 0.0, None) == 1          # causal must be 0/1
+    assert lib.osp_attn_temporal(p, p, p, p, shp(T=65), 1, 0.0, None) == 2      # causal needs T <= 64
+    assert lib.osp_attn_temporal(p, p, p, p, shp(d=80), 0, 0.0, None) == 2
+    assert lib.osp_attn_frame_causal(None, p, p, p, shp(), 0.0, None) == 1
+    assert lib.osp_attn_frame_causal(p, p, p, p, shp(d=60), 0.0, None) == 2
