@@ -25,6 +25,7 @@ from .spacetime_oracle import (  # noqa: F401
     skiparse_index_map,
     skiparse_scatter_ref,
     skiparse_sets,
+    skiparse_text_attn_ref,
     softmax_rows,
     spatial_attn_ref,
     temporal_attn_ref,

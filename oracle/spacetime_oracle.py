@@ -492,3 +492,41 @@ def frame_causal_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: Seq
                 sel = np.nonzero(lim == L)[0]
                 out[b, sel, hi] = attention_head_ref(q[b, :L, h], k[b, :L, h], v[b, :L, h], scale, rows_[sel])
     return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Skiparse with a text prefix joined to every set
+# ----------------------------------------------------------------------------------------------
+#
+# Not on the pages (Open-Sora Plan feeds text through cross-attention; CogVideoX joins text and
+# video in dense attention).  Reading for a joint text + video sequence under Skiparse: the text
+# tokens are global tokens.  A video token of set g attends to every text token and to the video
+# tokens of set g; a text token attends to every token of its sample.
+
+def skiparse_text_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, text_len: int, k_ratio: int, mode: int,
+                           scale: float | None = None, rows=None, heads=None) -> np.ndarray:
+    """q, k, v: [B, text_len + N_v, n_h, d].  ``rows`` (token indices) / ``heads`` select a
+    subset as in attn_ref."""
+    B, N, nh, d = q.shape
+    L = int(text_len)
+    scale = default_scale(d) if scale is None else scale
+    sets = skiparse_sets(N - L, k_ratio, mode)
+    set_of = np.empty(N - L, dtype=np.int64)
+    for g, st in enumerate(sets):
+        set_of[st] = g
+    rows_ = np.arange(N) if rows is None else np.asarray(rows)
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    out = np.empty((B, len(rows_), len(heads_), d), dtype=np.float64)
+    text = np.arange(L)
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            sel = np.nonzero(rows_ < L)[0]
+            if sel.size:
+                out[b, sel, hi] = attention_head_ref(q[b, :, h], k[b, :, h], v[b, :, h], scale, rows_[sel])
+            for g, st in enumerate(sets):
+                sel = np.nonzero((rows_ >= L) & (set_of[np.maximum(rows_ - L, 0)] == g))[0]
+                if sel.size == 0:
+                    continue
+                keys = np.concatenate([text, L + np.asarray(st)])
+                out[b, sel, hi] = attention_head_ref(q[b, rows_[sel], h], k[b, keys, h], v[b, keys, h], scale)
+    return out

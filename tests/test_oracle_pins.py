@@ -526,3 +526,40 @@ def test_frame_causal_attention_brute_force():
     # one frame, no text: plain full attention
     np.testing.assert_allclose(O.frame_causal_attn_ref(q[:, :6], k[:, :6], v[:, :6], (1, 2, 3), 0),
                                O.attn_ref(q[:, :6], k[:, :6], v[:, :6]), rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------------------------
+# Skiparse with a joined text prefix (global text tokens)
+# ----------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [O.SKIP_SINGLE, O.SKIP_GROUP])
+def test_skiparse_text_brute_force(mode):
+    L, nv, kr = 3, 8, 2
+    N = L + nv
+    # set of video token u (0-based among the video tokens), from the mode's definition
+    set_of = (lambda u: u % kr) if mode == O.SKIP_SINGLE else (lambda u: (u // kr) % kr)
+
+    def allowed(i, j):
+        if i < L or j < L:
+            return True          # text queries see all; every query sees the text
+        return set_of(i - L) == set_of(j - L)
+
+    rng = np.random.default_rng(60)
+    q, k, v = (rng.standard_normal((1, N, 2, 3)) for _ in range(3))
+    got = O.skiparse_text_attn_ref(q, k, v, L, kr, mode)
+    for h in range(2):
+        ref = _brute_masked_attention(q[0, :, h].tolist(), k[0, :, h].tolist(), v[0, :, h].tolist(), allowed,
+                                      1 / math.sqrt(3))
+        np.testing.assert_allclose(got[0, :, h], ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(O.skiparse_text_attn_ref(q, k, v, L, kr, mode, rows=[10, 1, 4], heads=[1]),
+                               got[:, [10, 1, 4]][:, :, [1]], rtol=0, atol=1e-15)
+
+
+def test_skiparse_text_special_cases():
+    rng = np.random.default_rng(61)
+    q, k, v = (rng.standard_normal((2, 16, 2, 4)) for _ in range(3))
+    # no text: plain Skiparse; k = 1: full attention
+    np.testing.assert_allclose(O.skiparse_text_attn_ref(q, k, v, 0, 4, O.SKIP_GROUP),
+                               O.skiparse_attn_ref(q, k, v, 4, O.SKIP_GROUP), rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(O.skiparse_text_attn_ref(q, k, v, 5, 1, O.SKIP_SINGLE), O.attn_ref(q, k, v),
+                               rtol=1e-13, atol=1e-14)
