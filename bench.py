@@ -389,7 +389,7 @@ def run_variant_op(args, rank, world, local_rank):
     w = syn.WORKLOADS[args.workload]
     T, H, W = w.grid
     HW = H * W
-    L = w.text_len if args.op == "frame_causal" else 0
+    L = w.text_len if args.op == "frame_causal" else (args.text_len if args.op == "skiparse_text" else 0)
     N = L + w.n_video
     nset = 3
     sets = [tuple(syn.randn_bf16((w.B, N, w.heads, w.head_dim), w.seed + 11 + 101 * r + 17 * rank + i).to(dev)
@@ -401,6 +401,16 @@ def run_variant_op(args, rank, world, local_rank):
     elif args.op == "temporal":
         launch = lambda i: ops.attn_temporal(*sets[i % nset], w.grid, causal=args.causal, o=outs[i % nset])
         pairs = w.B * HW * (T * (T + 1) // 2 if args.causal else T * T)
+    elif args.op == "skiparse_text":
+        kk = w.skiparse_k
+        if not kk:
+            raise SystemExit("--op skiparse_text needs a Skiparse workload")
+
+        def launch(i):   # Single then Group Skip, text joined to every set
+            ops.skiparse_attn(*sets[i % nset], w.grid, kk, ops.OSP_SKIP_SINGLE, o=outs[i % nset], text_len=L)
+            ops.skiparse_attn(*sets[i % nset], w.grid, kk, ops.OSP_SKIP_GROUP, o=outs[i % nset], text_len=L)
+        n_set = w.n_video // kk
+        pairs = 2 * w.B * (w.n_video * (L + n_set) + L * N)
     else:
         launch = lambda i: ops.attn_frame_causal(*sets[i % nset], w.grid, L, o=outs[i % nset])
         pairs = w.B * (L * L + sum(HW * (L + (t + 1) * HW) for t in range(T)))
@@ -436,8 +446,9 @@ def run_variant_op(args, rank, world, local_rank):
         roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_t, "unit": "TFLOP/s",
                 "frac": round(tflops / peak_t, 4), "peak_source": f"{src} (sustained bf16 GEMM)",
                 "kernel": "attn_fwd_kernel"}
-        metric = ("spatial attention TFLOP/s (2D+1D, 2D part)" if args.op == "spatial"
-                  else "frame-causal attention TFLOP/s (unmasked pairs)")
+        metric = {"spatial": "spatial attention TFLOP/s (2D+1D, 2D part)",
+                  "frame_causal": "frame-causal attention TFLOP/s (unmasked pairs)",
+                  "skiparse_text": "Skiparse + joined text TFLOP/s (Single + Group pair, unmasked pairs)"}[args.op]
         value, unit = tflops, "TFLOP/s"
     roof.update(traffic=None, bytes_per_launch=nbytes, flops_per_launch=flops)
     cfg = dict(w.describe(), op=args.op, text_len=L, l2=f"{nset} input sets rotated ({nset * nbytes / 1e6:.0f} MB)")
@@ -446,7 +457,8 @@ def run_variant_op(args, rank, world, local_rank):
     return {"metric": metric, "value": round(world * value, 1), "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roof,
-            "clocks": clocks, "gpu_launches": args.steps, "tflops": round(tflops, 1), "hbm_gbs": round(gbs, 1)}
+            "clocks": clocks, "gpu_launches": args.steps * (4 if args.op == "skiparse_text" else 1),
+            "tflops": round(tflops, 1), "hbm_gbs": round(gbs, 1)}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -685,12 +697,12 @@ def main():
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
     ap.add_argument("--op", default="step",
                     choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
-                             "frame_causal"],
+                             "frame_causal", "skiparse_text"],
                     help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone; "
                          "cross: video -> text cross-attention alone; packed: a packed batch of mixed shapes")
     ap.add_argument("--packed", default="frame_pack_cog2b", choices=sorted(syn.PACKED_WORKLOADS),
                     help="--op packed: the packed batch")
-    ap.add_argument("--text-len", type=int, default=226, help="--op cross: text tokens (keys)")
+    ap.add_argument("--text-len", type=int, default=226, help="--op cross / skiparse_text: text tokens")
     ap.add_argument("--causal", action="store_true", help="--op temporal: causal in time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -718,7 +730,8 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     try:
         runner = {"step": run_ours, "cross": run_cross_op, "packed": run_packed_op, "spatial": run_variant_op,
-                  "temporal": run_variant_op, "frame_causal": run_variant_op}.get(args.op, run_hbm_op)
+                  "temporal": run_variant_op, "frame_causal": run_variant_op,
+                  "skiparse_text": run_variant_op}.get(args.op, run_hbm_op)
         line = runner(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
   OSP_OK = 0,
   OSP_ERR_INVALID_ARG = 1,  /* null pointer, bad dimension, RoPE split not summing to head_dim */
-  OSP_ERR_UNSUPPORTED = 2,  /* head_dim not in {64, 96, 128}; text tokens with Skiparse; ... */
+  OSP_ERR_UNSUPPORTED = 2,  /* head_dim not in {64, 96, 128}; text tokens in gather/scatter; ... */
   OSP_ERR_DIVISIBILITY = 3, /* T*H*W mod k != 0 (Single Skip) or mod k*k != 0 (Group Skip) */
   OSP_ERR_CUDA = 4,         /* a CUDA runtime/driver call or a kernel launch failed */
   OSP_ERR_TIMEOUT = 5,      /* a bounded device-side wait gave up (see osp_check_status) */
@@ -211,7 +211,12 @@ int osp_skiparse_scatter(const void* o_perm, void* o, const osp_shape* shape, in
 /* Fused Skiparse attention: every video token attends only to the tokens of its own set
  * ("Open-Sora Plan" section 2.2.2). The set structure is folded into the kernel's tile
  * address map, so no permuted copy of q/k/v/o is ever written.
- *  q, k, v, o: [B][T*H*W][heads][head_dim] bf16, device, natural token order; text_len == 0.
+ *  q, k, v, o: [B][text_len + T*H*W][heads][head_dim] bf16, device, natural token order.
+ *  Text prefix (text_len > 0; the pages give no joint text + Skiparse scheme, so the text tokens
+ *    are read as global tokens): a video token of set g attends to every text token and to the
+ *    video tokens of set g; a text token attends to every token of its sample.  Two launches of
+ *    the same kernel (video queries with the text rows prepended to every set's KV range, then
+ *    the text queries over all rows).
  *  Group Skip additionally needs k to divide 128 (a power of two up to 128).
  *  Same arithmetic and scale convention as osp_attn_full. k == 1 is dense attention.
  *  Errors: OSP_ERR_INVALID_ARG, OSP_ERR_UNSUPPORTED, OSP_ERR_DIVISIBILITY, OSP_ERR_CUDA. */

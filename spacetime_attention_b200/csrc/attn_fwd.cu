@@ -121,6 +121,10 @@ struct AttnParams {
   // token of frame t.  Query blocks then run heaviest (latest) first.
   int frame_hw;
   int text_len;
+  // Skiparse with a joined text prefix (mode kModeSkipText): every set's KV range is the
+  // text_len text rows (ceil(text_len / 128) tiles from the text maps) followed by the set's own
+  // tiles; the set's query tokens sit q_row_base (= text_len) rows into each sample.
+  int q_row_base;
   // Work items (1-D grid): units are (sample*set, head, query block) with the query block fastest.
   // CTAs [0, n_full) process whole units; every later unit is split into n_split KV ranges whose
   // CTAs write fp32 partials (unnormalised O, running max m, row sum l) to ws_o / ws_ml, merged
@@ -143,10 +147,18 @@ struct SegTable {
   int kv[kMaxSegments + 1];
 };
 struct NoSegTable {};
-// Kernel variants: plain (dense / Skiparse / cross), packed batch, frame-causal mask.
-enum AttnMode { kModePlain = 0, kModePacked = 1, kModeFrameCausal = 2 };
+// Tensor maps of the text rows of k and v (dense view, text_len rows per sample) for Skiparse
+// with a joined text prefix.
+struct TextMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+};
+// Kernel variants: plain (dense / Skiparse / cross), packed batch, frame-causal mask, Skiparse
+// with a joined text prefix.
+enum AttnMode { kModePlain = 0, kModePacked = 1, kModeFrameCausal = 2, kModeSkipText = 3 };
 template <int kMode>
-using SegParam = typename std::conditional<kMode == kModePacked, SegTable, NoSegTable>::type;
+using SegParam = typename std::conditional<
+    kMode == kModePacked, SegTable, typename std::conditional<kMode == kModeSkipText, TextMaps, NoSegTable>::type>::type;
 
 __device__ __forceinline__ void load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
                                           int chan, int row0, int g, int b, int k) {
@@ -248,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ SegParam<kMode> seg) {
   constexpr bool kPacked = kMode == kModePacked;
   constexpr bool kFrameCausal = kMode == kModeFrameCausal;
+  constexpr bool kSkipText = kMode == kModeSkipText;
   using C = Cfg<D>;
   constexpr int S = C::kStages;
   extern __shared__ unsigned char smem_raw[];
@@ -275,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // work item -> unit (sample*set, head, query block) and KV tile range [kv_lo, kv_lo + n_kv).
   // q_row0 / kv_row0 offset the rows of a packed segment; nq / nkv are the set's query and key
   // rows.  Recomputed where needed (cheap integer math) rather than kept live across the main loops.
-  struct Work { int unit, part, h, b, g, q0, kv_lo, n_kv, q_row0, kv_row0, nq, nkv; };
+  struct Work { int unit, part, h, b, g, q0, kv_lo, n_kv, q_row0, kv_row0, nq, nkv, q_out0; };
   auto decode = [&]() {
     Work w;
     w.unit = blockIdx.x;
@@ -290,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       w.b = 0;
       w.g = 0;
       w.q_row0 = seg.q[sg];
+      w.q_out0 = w.q_row0;
       w.kv_row0 = seg.kv[sg];
       w.nq = seg.q[sg + 1] - w.q_row0;
       w.nkv = seg.kv[sg + 1] - w.kv_row0;
@@ -306,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       w.b = bg / p.G;
       w.g = bg % p.G;
       w.q_row0 = 0;
+      w.q_out0 = p.q_row_base;   // the maps start at the set's rows; outputs sit past the text
       w.kv_row0 = 0;
       w.nq = p.n_q;
       w.nkv = p.n_kv;
@@ -317,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       w.nkv = min(w.nkv, frame_causal_limit(last, p.text_len, p.frame_hw));
     }
     w.q0 = qb * (2 * kBM);
-    const int n_kv_all = (w.nkv + kBN - 1) / kBN;
+    const int n_kv_all = (w.nkv + kBN - 1) / kBN + (kSkipText ? (p.text_len + kBN - 1) / kBN : 0);
     w.kv_lo = w.part < 0 ? 0 : (int)((long long)w.part * n_kv_all / p.n_split);
     w.n_kv = (w.part < 0 ? n_kv_all : (int)((long long)(w.part + 1) * n_kv_all / p.n_split)) - w.kv_lo;
     return w;
@@ -364,6 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    if constexpr (kSkipText) {
+      prefetch_tmap(&seg.k);
+      prefetch_tmap(&seg.v);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -377,6 +396,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Work wk = decode();
   const int n_kv = wk.n_kv;
   const int chan0 = wk.h * D;
+  // KV tile jj of this unit's range: with a joined text prefix the first tiles come from the
+  // text maps (dense rows), the rest from the set's own map.
+  auto load_kv_tile = [&](const CUtensorMap& tm, const SegParam<kMode>& sp, uint32_t dst, uint32_t mbar, int chan,
+                          int jj, const Work& w, bool is_k) {
+    if constexpr (kSkipText) {
+      const int ntt = (p.text_len + kBN - 1) / kBN;
+      if (jj < ntt) {
+        tma_load_3d(dst, is_k ? &sp.k : &sp.v, mbar, chan, jj * kBN, w.b);
+        return;
+      }
+      jj -= ntt;
+    }
+    load_tile(&tm, dst, mbar, p.layout, chan, w.kv_row0 + jj * kBN, w.g, w.b, p.k);
+  };
 
   auto sQ = [&](int i) { return sbase + C::kQOff + (uint32_t)(i * C::kTileBytes); };
   auto sK = [&](int s) { return sbase + C::kKOff + (uint32_t)(s * C::kTileBytes); };
@@ -409,16 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) {
           mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_k, sK(s) + c * kChunkBytes, bar(B_KFULL + s), p.layout, chan0 + 64 * c, wk.kv_row0 + (wk.kv_lo + j) * kBN, wk.g, wk.b,
-                      p.k);
+            load_kv_tile(tm_k, seg, sK(s) + c * kChunkBytes, bar(B_KFULL + s), chan0 + 64 * c, wk.kv_lo + j, wk, true);
         }
         k_issued = j + 1;
         if (j >= S && !warp_wait(bar(B_VEMPTY + s), (u - 1) & 1, wc)) break;
         if (leader) {
           mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_v, sV(s) + c * kChunkBytes, bar(B_VFULL + s), p.layout, chan0 + 64 * c, wk.kv_row0 + (wk.kv_lo + j) * kBN, wk.g, wk.b,
-                      p.k);
+            load_kv_tile(tm_v, seg, sV(s) + c * kChunkBytes, bar(B_VFULL + s), chan0 + 64 * c, wk.kv_lo + j, wk, false);
         }
         v_issued = j + 1;
       }
@@ -617,7 +648,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sv[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-      const int valid = valid0 - j * kBN;
+      int valid = valid0 - j * kBN;
+      if constexpr (kSkipText) {
+        // text tiles (ragged last one), then the set's tiles (ragged last one)
+        const int jj = wk.kv_lo + j, ntt = (p.text_len + kBN - 1) / kBN;
+        valid = jj < ntt ? p.text_len - jj * kBN : wk.nkv - (jj - ntt) * kBN;
+      }
       const bool masked = valid < kBN;
       if (masked) {
 #pragma unroll
@@ -699,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (live) p.ws_ml[prow] = make_float2(m, l);
       } else {
-      const int token = w.q_row0 + slot_token(p.layout, live ? slot : 0, g, p.k);
+      const int token = w.q_out0 + slot_token(p.layout, live ? slot : 0, g, p.k);
       uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -758,7 +794,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, i
     for (int e = 0; e < kPer; ++e) acc[e] += wgt * p.ws_o[prow * D + e * 32 + lane];
   }
   const float inv = 1.f / lsum;
-  const int token = slot_token(p.layout, slot, g, p.k);
+  const int token = p.q_row_base + slot_token(p.layout, slot, g, p.k);
   __nv_bfloat16* dst = p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) dst[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
@@ -788,29 +824,33 @@ EncodeTiledFn encode_fn() {
 //   single: (heads*D, k, N/k, B)               box (64, 1, 128, 1)   token = s*k + g
 //   group:  (heads*D, k, k, N/(k*k), B)         box (64, k, 1, 128/k, 1)  token = (o*k + g)*k + r
 // The channel axis merges heads and head_dim; a box starts at channel h*D + 64c.
-int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k) {
+// batch_rows: rows between samples (default N); a view of part of each sample (the text rows,
+// or the video rows from an offset pointer) keeps the full sample stride.
+int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k,
+              long long batch_rows = -1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return set_error(OSP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t HD = (cuuint64_t)s.heads * s.head_dim;
   const cuuint64_t row = HD * 2;  // bytes per token
+  const cuuint64_t bstride = row * (cuuint64_t)(batch_rows < 0 ? N : batch_rows);
   cuuint64_t dims[5], strides[4];
   cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
   cuuint32_t rank;
   if (layout == 0) {
     rank = 3;
     dims[0] = HD; dims[1] = (cuuint64_t)N; dims[2] = (cuuint64_t)s.B;
-    strides[0] = row; strides[1] = row * N;
+    strides[0] = row; strides[1] = bstride;
     box[0] = 64; box[1] = kBM; box[2] = 1;
   } else if (layout == 1) {
     rank = 4;
     dims[0] = HD; dims[1] = (cuuint64_t)k; dims[2] = (cuuint64_t)(N / k); dims[3] = (cuuint64_t)s.B;
-    strides[0] = row; strides[1] = row * k; strides[2] = row * N;
+    strides[0] = row; strides[1] = row * k; strides[2] = bstride;
     box[0] = 64; box[1] = 1; box[2] = kBM; box[3] = 1;
   } else {
     rank = 5;
     dims[0] = HD; dims[1] = (cuuint64_t)k; dims[2] = (cuuint64_t)k; dims[3] = (cuuint64_t)(N / (k * k));
     dims[4] = (cuuint64_t)s.B;
-    strides[0] = row; strides[1] = row * k; strides[2] = row * k * k; strides[3] = row * N;
+    strides[0] = row; strides[1] = row * k; strides[2] = row * k * k; strides[3] = bstride;
     box[0] = 64; box[1] = (cuuint32_t)k; box[2] = 1; box[3] = (cuuint32_t)(kBM / k); box[4] = 1;
   }
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -848,20 +888,63 @@ namespace {
 
 // Attention launch with an explicit status word (the kernel's only global scratch).
 // N_kv: tokens per sample of k and v; < 0 means the same sequence as q (self-attention).
-// frame_causal: dense layout only; the frame-causal mask over s's text block and frames.
-int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
-                       int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
-                       int N_kv = -1, bool frame_causal = false) {
-  const int N = (N_kv < 0) ? s.text_len + s.T * s.H * s.W : s.T * s.H * s.W;   // q / o tokens per sample
-  if (N_kv < 0) N_kv = N;
-  const int G = (layout == 0) ? 1 : sparse_k;
-  const int n = N / G;
+// Runs the attention kernel over `units` work units of n_kv_tiles KV tiles each: the split of
+// the last partial wave over KV ranges (when allowed), its workspace and the combine kernel.
+template <int kMode>
+int run_units(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, AttnParams& p,
+              const SegParam<kMode>& extra, long long units, int n_kv_tiles, bool allow_split, int head_dim,
+              cudaStream_t stream) {
+  if (units > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld attention work units is too many", units);
+  p.n_full = (int)units;
+  p.n_split = 1;
+  // Split-KV for the last partial wave (one CTA per SM): its R units are split into KV ranges so
+  // that about one wave of CTAs runs them.  Needs a workspace, so only where allocation is allowed.
+  const int sms = device_sm_count();
+  const int rem = (int)(units % sms);
+  if (allow_split && split_kv_enabled() && rem > 0) {
+    const int ns = std::min(std::min(sms / rem, n_kv_tiles / 2), 8);
+    if (ns >= 2) {
+      p.n_full = (int)(units - rem);
+      p.n_split = ns;
+    }
+  }
+  void* ws = nullptr;
+  if (p.n_split > 1) {
+    const size_t rows = (size_t)(units - p.n_full) * p.n_split * 2 * kBM;
+    const size_t bytes = rows * (size_t)head_dim * sizeof(float) + rows * sizeof(float2);
+    cudaMemPool_t pool = workspace_pool();
+    if (!pool || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", bytes);
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_ml = reinterpret_cast<float2*>(p.ws_o + rows * (size_t)head_dim);
+  }
+  const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
+  dim3 grid((unsigned)ctas);
+  int rc;
+  switch (head_dim) {
+    case 64: rc = launch_d<64, kMode>(tq, tk, tv, p, extra, grid, stream); break;
+    case 96: rc = launch_d<96, kMode>(tq, tk, tv, p, extra, grid, stream); break;
+    case 128: rc = launch_d<128, kMode>(tq, tk, tv, p, extra, grid, stream); break;
+    default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
+  }
+  if (rc == OSP_OK && p.n_split > 1) {
+    const int su = (int)(units - p.n_full);
+    const unsigned blocks = (unsigned)(((size_t)su * 2 * kBM + 7) / 8);
+    switch (head_dim) {
+      case 64: attn_combine_kernel<64><<<blocks, 256, 0, stream>>>(p, su); break;
+      case 96: attn_combine_kernel<96><<<blocks, 256, 0, stream>>>(p, su); break;
+      default: attn_combine_kernel<128><<<blocks, 256, 0, stream>>>(p, su); break;
+    }
+    rc = check_launch("attn_combine_kernel");
+  }
+  if (ws) cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+AttnParams base_params(const osp_shape& s, int layout, int sparse_k, float scale, void* o, unsigned* status) {
   AttnParams p{};
-  p.n_q = n;
-  p.n_kv = N_kv / G;
-  p.N_q = N;
   p.heads = s.heads;
-  p.G = G;
+  p.G = (layout == 0) ? 1 : sparse_k;
   p.k = (layout == 0) ? 1 : sparse_k;
   p.layout = layout;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -869,6 +952,21 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
   p.debug_withhold_q = debug_withhold_q();
+  return p;
+}
+
+// frame_causal: dense layout only; the frame-causal mask over s's text block and frames.
+int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
+                       int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
+                       int N_kv = -1, bool frame_causal = false) {
+  const int N = (N_kv < 0) ? s.text_len + s.T * s.H * s.W : s.T * s.H * s.W;   // q / o tokens per sample
+  if (N_kv < 0) N_kv = N;
+  AttnParams p = base_params(s, layout, sparse_k, scale, o, status);
+  const int G = p.G;
+  const int n = N / G;
+  p.n_q = n;
+  p.n_kv = N_kv / G;
+  p.N_q = N;
   p.frame_hw = frame_causal ? s.H * s.W : 0;
   p.text_len = s.text_len;
   if (frame_causal) allow_split = false;   // a KV range could hold no visible key for some rows
@@ -878,62 +976,12 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   if ((rc = make_tmap(&tk, k, s, N_kv, layout, p.k)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tv, v, s, N_kv, layout, p.k)) != OSP_OK) return rc;
   const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
-  const long long units = qblocks * s.heads * (long long)s.B * G;
-  if (units > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld attention work units is too many", units);
   p.qblocks = (int)qblocks;
-  p.n_full = (int)units;
-  p.n_split = 1;
-  // Split-KV for the last partial wave (one CTA per SM): its R units are split into KV ranges so
-  // that about one wave of CTAs runs them.  Needs a workspace, so only where allocation is allowed.
-  const int n_kv = (p.n_kv + kBN - 1) / kBN;
-  const int sms = device_sm_count();
-  const int rem = (int)(units % sms);
-  if (allow_split && split_kv_enabled() && rem > 0) {
-    const int ns = std::min(std::min(sms / rem, n_kv / 2), 8);
-    if (ns >= 2) {
-      p.n_full = (int)(units - rem);
-      p.n_split = ns;
-    }
-  }
-  void* ws = nullptr;
-  if (p.n_split > 1) {
-    const size_t rows = (size_t)(units - p.n_full) * p.n_split * 2 * kBM;
-    const size_t bytes = rows * (size_t)s.head_dim * sizeof(float) + rows * sizeof(float2);
-    cudaMemPool_t pool = workspace_pool();
-    if (!pool || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess)
-      return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", bytes);
-    p.ws_o = static_cast<float*>(ws);
-    p.ws_ml = reinterpret_cast<float2*>(p.ws_o + rows * (size_t)s.head_dim);
-  }
-  const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
-  dim3 grid((unsigned)ctas);
-  switch (s.head_dim) {
-    case 64:
-      rc = frame_causal ? launch_d<64, kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, grid, stream)
-                        : launch_d<64, kModePlain>(tq, tk, tv, p, NoSegTable{}, grid, stream);
-      break;
-    case 96:
-      rc = frame_causal ? launch_d<96, kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, grid, stream)
-                        : launch_d<96, kModePlain>(tq, tk, tv, p, NoSegTable{}, grid, stream);
-      break;
-    case 128:
-      rc = frame_causal ? launch_d<128, kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, grid, stream)
-                        : launch_d<128, kModePlain>(tq, tk, tv, p, NoSegTable{}, grid, stream);
-      break;
-    default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
-  }
-  if (rc == OSP_OK && p.n_split > 1) {
-    const int su = (int)(units - p.n_full);
-    const unsigned blocks = (unsigned)(((size_t)su * 2 * kBM + 7) / 8);
-    switch (s.head_dim) {
-      case 64: attn_combine_kernel<64><<<blocks, 256, 0, stream>>>(p, su); break;
-      case 96: attn_combine_kernel<96><<<blocks, 256, 0, stream>>>(p, su); break;
-      default: attn_combine_kernel<128><<<blocks, 256, 0, stream>>>(p, su); break;
-    }
-    rc = check_launch("attn_combine_kernel");
-  }
-  if (ws) cudaFreeAsync(ws, stream);
-  return rc;
+  const long long units = qblocks * s.heads * (long long)s.B * G;
+  const int n_kv_tiles = (p.n_kv + kBN - 1) / kBN;
+  if (frame_causal)
+    return run_units<kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, units, n_kv_tiles, false, s.head_dim, stream);
+  return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, units, n_kv_tiles, allow_split, s.head_dim, stream);
 }
 
 }  // namespace
@@ -950,6 +998,56 @@ int cross_attention_launch(const void* q, const void* k, const void* v, void* o,
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   return launch_with_status(q, k, v, o, s, 0, 1, scale, stream, status, true, s.text_len);
+}
+
+int skiparse_text_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
+                                   int sparse_k, int mode, float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  const int L = s.text_len, Nv = s.T * s.H * s.W, N = L + Nv;
+  const size_t row = (size_t)s.heads * s.head_dim * 2;
+  const osp_shape sv{s.B, 0, s.T, s.H, s.W, s.heads, s.head_dim};   // the video part of each sample
+  int rc;
+  // 1) video queries: set g attends to the text rows, then to the set's own rows
+  {
+    const int layout = mode + 1;
+    AttnParams p = base_params(sv, layout, sparse_k, scale, o, status);
+    const int n = Nv / sparse_k;
+    p.n_q = p.n_kv = n;
+    p.N_q = N;
+    p.text_len = L;
+    p.q_row_base = L;
+    CUtensorMap tq, tk, tv;
+    TextMaps tm{};
+    const char* qv = static_cast<const char*>(q) + L * row;
+    const char* kv = static_cast<const char*>(k) + L * row;
+    const char* vv = static_cast<const char*>(v) + L * row;
+    if ((rc = make_tmap(&tq, qv, sv, Nv, layout, sparse_k, N)) != OSP_OK) return rc;
+    if ((rc = make_tmap(&tk, kv, sv, Nv, layout, sparse_k, N)) != OSP_OK) return rc;
+    if ((rc = make_tmap(&tv, vv, sv, Nv, layout, sparse_k, N)) != OSP_OK) return rc;
+    if ((rc = make_tmap(&tm.k, k, s, L, 0, 1, N)) != OSP_OK) return rc;
+    if ((rc = make_tmap(&tm.v, v, s, L, 0, 1, N)) != OSP_OK) return rc;
+    const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
+    p.qblocks = (int)qblocks;
+    const long long units = qblocks * s.heads * (long long)s.B * sparse_k;
+    const int n_kv_tiles = (n + kBN - 1) / kBN + (L + kBN - 1) / kBN;
+    rc = run_units<kModeSkipText>(tq, tk, tv, p, tm, units, n_kv_tiles, true, s.head_dim, stream);
+    if (rc) return rc;
+  }
+  if (L == 0) return OSP_OK;
+  // 2) text queries: every text token attends to all N tokens of its sample
+  AttnParams p = base_params(s, 0, 1, scale, o, status);
+  p.n_q = L;
+  p.n_kv = N;
+  p.N_q = N;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_tmap(&tq, q, s, L, 0, 1, N)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tk, k, s, N, 0, 1)) != OSP_OK) return rc;
+  if ((rc = make_tmap(&tv, v, s, N, 0, 1)) != OSP_OK) return rc;
+  const long long qblocks = (L + 2 * kBM - 1) / (2 * kBM);
+  p.qblocks = (int)qblocks;
+  const long long units = qblocks * s.heads * (long long)s.B;
+  return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, units, (N + kBN - 1) / kBN, true, s.head_dim, stream);
 }
 
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,

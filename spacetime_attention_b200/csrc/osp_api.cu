@@ -55,12 +55,13 @@ int check_rope(const osp_rope* r, int head_dim) {
   return OSP_OK;
 }
 
-int check_skiparse(const osp_shape* s, int k, int mode) {
+int check_skiparse(const osp_shape* s, int k, int mode, bool allow_text = false) {
   if (k < 1) return set_error(OSP_ERR_INVALID_ARG, "sparse ratio k=%d < 1", k);
   if (mode != OSP_SKIP_SINGLE && mode != OSP_SKIP_GROUP)
     return set_error(OSP_ERR_INVALID_ARG, "mode %d is neither OSP_SKIP_SINGLE nor OSP_SKIP_GROUP", mode);
-  if (s->text_len != 0)
-    return set_error(OSP_ERR_UNSUPPORTED, "Skiparse with text tokens (text_len=%d) is not supported", s->text_len);
+  if (s->text_len != 0 && !allow_text)
+    return set_error(OSP_ERR_UNSUPPORTED, "Skiparse gather / scatter take video tokens only (text_len=%d)",
+                     s->text_len);
   const long long nv = (long long)s->T * s->H * s->W;
   const long long step = (mode == OSP_SKIP_SINGLE) ? k : (long long)k * k;
   if (nv % step)
@@ -357,7 +358,7 @@ int osp_skiparse_attn(const void* q, const void* k, const void* v, void* o, cons
   g_last_error[0] = 0;
   int rc = check_shape(shape, true);
   if (rc) return rc;
-  if ((rc = check_skiparse(shape, sparse_k, mode))) return rc;
+  if ((rc = check_skiparse(shape, sparse_k, mode, true))) return rc;
   if (mode == OSP_SKIP_GROUP && (sparse_k > 128 || (128 % sparse_k) != 0))
     return set_error(OSP_ERR_UNSUPPORTED, "fused Group Skip needs k to divide 128 (got k=%d)", sparse_k);
   if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
@@ -365,7 +366,10 @@ int osp_skiparse_attn(const void* q, const void* k, const void* v, void* o, cons
     return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
   const int layout = (sparse_k == 1) ? 0 : (mode == OSP_SKIP_SINGLE ? 1 : 2);
-  return attention_launch(q, k, v, o, *shape, layout, sparse_k, softmax_scale, static_cast<cudaStream_t>(stream));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (shape->text_len > 0 && layout != 0)
+    return skiparse_text_attention_launch(q, k, v, o, *shape, sparse_k, mode, softmax_scale, st);
+  return attention_launch(q, k, v, o, *shape, layout, sparse_k, softmax_scale, st);
 }
 
 int osp_skiparse_index_map(int32_t n_video, int32_t sparse_k, int32_t mode, int32_t* dev_out, void* stream) {

@@ -58,6 +58,11 @@ int attention_launch(const void* q, const void* k, const void* v, void* o, const
 int cross_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, float scale,
                            cudaStream_t stream);
 
+// Skiparse with a joined text prefix (text_len > 0, k > 1): video queries of set g attend to the
+// text rows and set g; text queries attend to every row.  Two launches of the attention kernel.
+int skiparse_text_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
+                                   int sparse_k, int mode, float scale, cudaStream_t stream);
+
 // Frame-causal attention (dense layout): token r attends to the text block and the frames up to its own.
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
                                   float scale, cudaStream_t stream);

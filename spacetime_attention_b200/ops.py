@@ -243,12 +243,13 @@ def attn_full_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, t
 
 
 def skiparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, sparse_k: int, mode: int,
-                  scale: float = 0.0, o: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """osp_skiparse_attn: fused Skiparse attention in natural token order."""
+                  scale: float = 0.0, o: Optional[torch.Tensor] = None, text_len: int = 0) -> torch.Tensor:
+    """osp_skiparse_attn: fused Skiparse attention in natural token order (text_len > 0: the text
+    prefix is joined to every set as global tokens)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _bshd(t, n)
     o = torch.empty_like(q) if o is None else o
-    shp = _shape_of(q, grid, 0)
+    shp = _shape_of(q, grid, text_len)
     _check("osp_skiparse_attn", library().osp_skiparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                             int(sparse_k), int(mode), ctypes.c_float(scale),
                                                             _stream_handle(q)))

@@ -73,8 +73,9 @@ def test_rope_split_validation(lib):
 
 def test_skiparse_validation(lib):
     p = ctypes.c_void_p(256)
-    # text tokens with Skiparse -> unsupported
-    assert lib.osp_skiparse_attn(p, p, p, p, shp(L=3), 2, 0, 0.0, None) == 2
+    # text tokens: gather / scatter take video tokens only; Skiparse attention still checks k
+    assert lib.osp_skiparse_gather(p, p, p, p, p, p, shp(L=3), 2, 0, None, None) == 2
+    assert lib.osp_skiparse_attn(p, p, p, p, shp(L=3), 3, 0, 0.0, None) == 3
     # 4*8*8 = 256 not divisible by 3 / by 9
     assert lib.osp_skiparse_attn(p, p, p, p, shp(), 3, 0, 0.0, None) == 3
     assert lib.osp_skiparse_gather(p, p, p, p, p, p, shp(T=3, H=3, W=3), 2, 1, None, None) == 3
