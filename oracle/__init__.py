@@ -7,7 +7,10 @@ CPU-baseline legs of ``bench.py``.  The CUDA library neither imports nor calls i
 from .spacetime_oracle import (  # noqa: F401
     SKIP_GROUP,
     SKIP_SINGLE,
+    attention_head_backward_ref,
+    attention_head_lse_ref,
     attention_head_ref,
+    attn_backward_ref,
     attn_ref,
     cross_attn_ref,
     default_scale,
@@ -21,6 +24,7 @@ from .spacetime_oracle import (  # noqa: F401
     round_to_bf16,
     segment_bounds,
     skiparse_attn_ref,
+    skiparse_backward_ref,
     skiparse_gather_ref,
     skiparse_index_map,
     skiparse_scatter_ref,

@@ -530,3 +530,62 @@ def skiparse_text_attn_ref(q: np.ndarray, k: np.ndarray, v: np.ndarray, text_len
                 keys = np.concatenate([text, L + np.asarray(st)])
                 out[b, sel, hi] = attention_head_ref(q[b, rows_[sel], h], k[b, keys, h], v[b, keys, h], scale)
     return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Backward pass (gradients of the attention output)
+# ----------------------------------------------------------------------------------------------
+#
+# Open-Sora Plan trains with Skiparse attention (section 2.2.2 and the sparse-tuning stage), so
+# the hot path has a backward pass.  For one head with S = q k^T * scale, P = softmax(S) (rows),
+# O = P v and an upstream gradient dO, the chain rule gives
+#   dV = P^T dO,   dP = dO v^T,   dS = P * (dP - rowsum(P * dP)),
+#   dQ = dS k * scale,   dK = dS^T q * scale,
+# and rowsum(P * dP) = rowsum(dO * O).  The log-sum-exp of a row, lse = log sum_j exp(S_ij), is
+# what the forward pass keeps so that P can be rebuilt as exp(S - lse).
+
+def attention_head_lse_ref(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """Natural log-sum-exp of every row of q k^T * scale (one head), fp64."""
+    s = (np.asarray(q, np.float64) @ np.asarray(k, np.float64).T) * scale
+    m = s.max(axis=1)
+    return m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+
+
+def attention_head_backward_ref(q, k, v, do, scale: float):
+    """(dq, dk, dv) of one head by the chain rule above, fp64."""
+    q, k, v, do = (np.asarray(a, np.float64) for a in (q, k, v, do))
+    p = softmax_rows((q @ k.T) * scale)
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    ds = p * (dp - (do * o).sum(axis=1, keepdims=True))
+    return ds @ k * scale, ds.T @ q * scale, dv
+
+
+def attn_backward_ref(q, k, v, do, scale: float | None = None):
+    """Gradients of 3D full attention (attn_ref) for [B, N, n_h, d] inputs: (dq, dk, dv)."""
+    B, N, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    out = [np.empty((B, N, nh, d)) for _ in range(3)]
+    for b in range(B):
+        for h in range(nh):
+            g = attention_head_backward_ref(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale)
+            for o_, g_ in zip(out, g):
+                o_[b, :, h] = g_
+    return tuple(out)
+
+
+def skiparse_backward_ref(q, k, v, do, k_ratio: int, mode: int, scale: float | None = None):
+    """Gradients of Skiparse attention (skiparse_attn_ref, no text): each set's own backward,
+    scattered back to natural token order."""
+    B, N, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    out = [np.empty((B, N, nh, d)) for _ in range(3)]
+    for st in skiparse_sets(N, k_ratio, mode):
+        idx = np.asarray(st)
+        for b in range(B):
+            for h in range(nh):
+                g = attention_head_backward_ref(q[b, idx, h], k[b, idx, h], v[b, idx, h], do[b, idx, h], scale)
+                for o_, g_ in zip(out, g):
+                    o_[b, idx, h] = g_
+    return tuple(out)

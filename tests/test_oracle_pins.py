@@ -563,3 +563,60 @@ def test_skiparse_text_special_cases():
                                O.skiparse_attn_ref(q, k, v, 4, O.SKIP_GROUP), rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(O.skiparse_text_attn_ref(q, k, v, 5, 1, O.SKIP_SINGLE), O.attn_ref(q, k, v),
                                rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------------------------
+# backward pass: central finite differences of a scalar loss through the forward oracle
+# ----------------------------------------------------------------------------------------------
+
+def _fd_grad(f, x, eps=1e-6):
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        xp, xm = x.copy(), x.copy()
+        xp[i] += eps
+        xm[i] -= eps
+        g[i] = (f(xp) - f(xm)) / (2 * eps)
+    return g
+
+
+def test_dense_backward_matches_finite_differences():
+    rng = np.random.default_rng(80)
+    q, k, v = (rng.standard_normal((1, 5, 2, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 5, 2, 3))           # loss = sum(O * G), so dO = G
+    loss = lambda q_, k_, v_: float((O.attn_ref(q_, k_, v_, scale=0.7) * G).sum())
+    dq, dk, dv = O.attn_backward_ref(q, k, v, G, scale=0.7)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("mode", [O.SKIP_SINGLE, O.SKIP_GROUP])
+def test_skiparse_backward_matches_finite_differences(mode):
+    rng = np.random.default_rng(81)
+    q, k, v = (rng.standard_normal((1, 8, 1, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 8, 1, 3))
+    loss = lambda q_, k_, v_: float((O.skiparse_attn_ref(q_, k_, v_, 2, mode) * G).sum())
+    dq, dk, dv = O.skiparse_backward_ref(q, k, v, G, 2, mode)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+
+
+def test_backward_closed_forms_and_lse():
+    rng = np.random.default_rng(82)
+    q, k, v = (rng.standard_normal((4, 3)) for _ in range(3))
+    # dO = 0: every gradient vanishes; equal keys: dQ = 0 (softmax is flat in q)
+    dq, dk, dv = O.attention_head_backward_ref(q, k, v, np.zeros((4, 3)), 0.5)
+    assert not dq.any() and not dk.any() and not dv.any()
+    kk = np.tile(k[:1], (4, 1))
+    dq, _, dv = O.attention_head_backward_ref(q, kk, v, rng.standard_normal((4, 3)), 0.5)
+    np.testing.assert_allclose(dq, 0, atol=1e-14)
+    # dV = P^T dO with uniform P = 1/4 when all keys are equal
+    do = rng.standard_normal((4, 3))
+    _, _, dv = O.attention_head_backward_ref(q, kk, v, do, 0.5)
+    np.testing.assert_allclose(dv, np.tile(do.sum(0) / 4, (4, 1)), rtol=1e-13)
+    # lse: two keys with scores 0 and ln 3 -> ln 4
+    lse = O.attention_head_lse_ref(np.array([[1.0, 0.0]]), np.array([[0.0, 0.0], [math.log(3.0), 0.0]]), 1.0)
+    np.testing.assert_allclose(lse, [math.log(4.0)], rtol=1e-15)
