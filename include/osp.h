@@ -159,6 +159,34 @@ int osp_attn_temporal(const void* q, const void* k, const void* v, void* o, cons
 int osp_attn_frame_causal(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                           float softmax_scale, void* stream);
 
+/* Training: forward with saved statistics, and the backward pass (Open-Sora Plan section 2.2.2:
+ * the model is trained with Skiparse attention).  sparse_k == 1: dense attention over
+ * N = text_len + T*H*W tokens (as osp_attn_full); sparse_k > 1: Skiparse Single / Group Skip
+ * (as osp_skiparse_attn, text_len must be 0, Group Skip needs k | 128).
+ *
+ * osp_attn_forward_train: o as the corresponding inference call (same kernel, arithmetic and work
+ *   split), plus lse, the log2-domain log-sum-exp of every query row's scaled scores:
+ *   lse[((b*G + g)*heads + h)*n_pad + s] = log2(sum_j exp2(score_sj * scale * log2(e))) for slot s
+ *   of set g (G = 1 and slot = token for dense; G = k for Skiparse), n = N / G,
+ *   n_pad = ceil(n / 128) * 128.  lse: device fp32 array of B * G * heads * n_pad values (the
+ *   padding entries are not written), 16-byte aligned; it is an opaque input of the backward. */
+int osp_attn_forward_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
+                           int32_t sparse_k, int32_t mode, float softmax_scale, void* stream);
+
+/* osp_attn_backward: gradients of the attention output o with respect to q, k, v, given the
+ *   upstream gradient dout (same shape as o) and the forward's o and lse:
+ *     dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)), dQ = scale * dS K,
+ *     dK = scale * dS^T Q, per (sample, set, head), with P = exp2(S * scale * log2(e) - lse).
+ *   dq, dk, dv: [B][N][heads][head_dim] bf16, device, written completely; must not overlap the
+ *   inputs.  Arithmetic: tcgen05 tensor cores, bf16 operands (P and dS rounded to bf16), fp32
+ *   accumulation in tensor memory, outputs rounded to bf16.  Scratch: rowsum(dO * O) in a
+ *   stream-ordered block (B * G * heads * n_pad floats) from the library's memory pool.
+ *   Three kernel launches (row sums, dK/dV, dQ).
+ *  Errors: as the forward, OSP_ERR_CUDA. */
+int osp_attn_backward(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                      void* dq, void* dk, void* dv, const osp_shape* shape, int32_t sparse_k, int32_t mode,
+                      float softmax_scale, void* stream);
+
 /* 3D RoPE of a packed batch (CogVideoX section 3.1: every video keeps its own position grid,
  * starting at (0, 0, 0); extrapolation, never rescaled).
  *  samples:       HOST array of n_samples (1 .. OSP_MAX_SEGMENTS) sample grids, read during the call.

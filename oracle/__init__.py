@@ -8,6 +8,7 @@ from .spacetime_oracle import (  # noqa: F401
     SKIP_GROUP,
     SKIP_SINGLE,
     attention_head_backward_ref,
+    attention_head_backward_rows_ref,
     attention_head_lse_ref,
     attention_head_ref,
     attn_backward_ref,

@@ -589,3 +589,32 @@ def skiparse_backward_ref(q, k, v, do, k_ratio: int, mode: int, scale: float | N
                 for o_, g_ in zip(out, g):
                     o_[b, idx, h] = g_
     return tuple(out)
+
+
+def attention_head_backward_rows_ref(q, k, v, do, scale: float, q_rows, k_rows, chunk: int = 2048):
+    """Selected rows of (dq, dk, dv) of one head, without forming the full score matrix: dq for
+    query rows ``q_rows``, dk and dv for key rows ``k_rows``.  Same chain rule as
+    attention_head_backward_ref; the row log-sum-exp and rowsum(dO * O) of every query come first
+    (query chunks of ``chunk`` rows)."""
+    q, k, v, do = (np.asarray(a, np.float64) for a in (q, k, v, do))
+    n = q.shape[0]
+    lse = np.empty(n)
+    dsum = np.empty(n)
+    for r0 in range(0, n, chunk):
+        s = (q[r0:r0 + chunk] @ k.T) * scale
+        m = s.max(axis=1)
+        e = np.exp(s - m[:, None])
+        z = e.sum(axis=1)
+        lse[r0:r0 + chunk] = m + np.log(z)
+        o = (e / z[:, None]) @ v
+        dsum[r0:r0 + chunk] = (do[r0:r0 + chunk] * o).sum(axis=1)
+    qr = np.asarray(q_rows)
+    p = np.exp((q[qr] @ k.T) * scale - lse[qr][:, None])
+    ds = p * (do[qr] @ v.T - dsum[qr][:, None])
+    dq = ds @ k * scale
+    kr = np.asarray(k_rows)
+    pt = np.exp((q @ k[kr].T) * scale - lse[:, None])              # [n, len(k_rows)]
+    dst = pt * (do @ v[kr].T - dsum[:, None])
+    dk = dst.T @ q * scale
+    dv = pt.T @ do
+    return dq, dk, dv

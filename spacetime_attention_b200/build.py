@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libosp.so")
 
-SOURCES = ["osp_api.cu", "rope_permute.cu", "attn_fwd.cu", "attn_temporal.cu"]
+SOURCES = ["osp_api.cu", "rope_permute.cu", "attn_fwd.cu", "attn_temporal.cu", "attn_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
               "-I", CSRC, "-I", INCLUDE]

@@ -1,0 +1,621 @@
+// Backward pass of dense and Skiparse attention on tcgen05 tensor cores.
+//
+// Source: "Open-Sora Plan: Open-Source Large Video Generation Model", section 2.2.2 (the model
+// is trained with Skiparse attention); the gradients are the chain rule of softmax attention.
+// For one (sample, set, head) with S = Q K^T * scale, P = softmax(S), O = P V and upstream dO:
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Dv),  Dv = rowsum(dO * O),
+//   dQ = scale * dS K,  dK = scale * dS^T Q.
+// P is rebuilt from the forward pass's row log-sum-exp: P = exp2(S * scale * log2(e) - lse).
+//
+// Three kernels:
+//   attn_bwd_dvec_kernel  Dv per query row (fp32), written in set-slot order like lse;
+//   attn_bwd_dkdv_kernel  one CTA per 128-key tile: K, V stay in shared memory while the set's
+//                         query tiles stream through; S^T = K Q^T and dP^T = V dO^T land in
+//                         tensor memory with the keys on the lanes, the compute warps turn them
+//                         into P^T and dS^T (bf16, written back over S^T / dP^T), and
+//                         dV += P^T dO, dK += dS^T Q accumulate in tensor memory;
+//   attn_bwd_dq_kernel    one CTA per 128-query tile: Q, dO stay resident while the key tiles
+//                         stream; S = Q K^T, dP = dO V^T, dS (bf16, over dP), dQ += dS K.
+// Rows are addressed through the same TMA maps as the forward kernel, so Skiparse sets are
+// never gathered.  Every wait is bounded (status word + abort flag, as in the forward kernel).
+
+#include "osp_internal.h"
+
+namespace osp {
+
+namespace {
+
+constexpr int kBT = 128;                 // rows per tile (queries or keys)
+constexpr int kChunkBytes = 128 * 128;   // 128 rows x 64 bf16 channels, one SW128 atom wide
+constexpr int kBwdThreads = 192;         // warps 0-3 compute, 4 TMA producer, 5 MMA issuer
+constexpr int kProdWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 512;
+// tensor memory columns: S (or S^T) 0..127, dP (dP^T) 128..255, accumulators at 256 and 384
+constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 384;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kChunks = (D + 63) / 64;
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kResOff = 0;                                 // two resident tiles
+  static constexpr int kStageOff = 2 * kTileBytes;                  // stages of two tiles each
+  static constexpr int kVecOff = kStageOff + kStages * 2 * kTileBytes;
+  static constexpr int kVecBytes = 2 * kBT * 4;                     // lse + Dv of one query tile
+  static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
+  static constexpr int kNumBars = 12;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+};
+
+struct BwdParams {
+  int n;            // rows per set (queries = keys)
+  int N;            // tokens per sample of the natural-order tensors
+  int heads, G, k, layout;
+  int n_tiles;      // ceil(n / 128)
+  int vec_stride;   // floats per (sample*set, head) row of lse / Dv (n rounded up to 128)
+  float scale_log2;
+  float scale;
+  const float* lse;
+  float* dvec;
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  unsigned* status;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ int bwd_slot_token(int layout, int s, int g, int k) {
+  if (layout == 0) return s;
+  if (layout == 1) return s * k + g;
+  const int o = s / k;
+  return (o * k + g) * k + (s - o * k);
+}
+
+__device__ __forceinline__ void bwd_load_tile(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int layout,
+                                              int chan, int row0, int g, int b, int k) {
+  if (layout == 0) tma_load_3d(dst, tm, bar, chan, row0, b);
+  else if (layout == 1) tma_load_4d(dst, tm, bar, chan, g, row0, b);
+  else tma_load_5d(dst, tm, bar, chan, 0, g, row0 / k, b);
+}
+
+__device__ __forceinline__ bool bwd_warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  const bool ok = mbar_wait(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// ------------------------------------------------------------------------------------------
+// Dv = rowsum(dO * O), one thread per (sample, token, head) row, stored at the row's set slot
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16* __restrict__ o,
+                                                            const __nv_bfloat16* __restrict__ dout,
+                                                            const BwdParams p, long long rows) {
+  for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < rows;
+       r += (long long)gridDim.x * blockDim.x) {
+    const int h = (int)(r % p.heads);
+    const long long bt = r / p.heads;
+    const int token = (int)(bt % p.N);
+    const int b = (int)(bt / p.N);
+    const uint4* a = reinterpret_cast<const uint4*>(o + r * D);
+    const uint4* c = reinterpret_cast<const uint4*>(dout + r * D);
+    float acc = 0.f;
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) {
+      const uint4 x = a[v], y = c[v];
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(xs[e] << 16), __uint_as_float(ys[e] << 16), acc);
+        acc = fmaf(__uint_as_float(xs[e] & 0xFFFF0000u), __uint_as_float(ys[e] & 0xFFFF0000u), acc);
+      }
+    }
+    int g = 0, slot = token;
+    if (p.layout == 1) {
+      g = token % p.k;
+      slot = token / p.k;
+    } else if (p.layout == 2) {
+      const int kk = p.k * p.k, ob = token / kk, rem = token - ob * kk;
+      g = rem / p.k;
+      slot = ob * p.k + (rem - g * p.k);
+    }
+    p.dvec[((size_t)(b * p.G + g) * p.heads + h) * p.vec_stride + slot] = acc;
+  }
+}
+
+// P and dS of one 32-column chunk for one TMEM lane (the thread's row).
+//   s, dp: raw scores / dP of the chunk; lse, dv: per-column (kCols) or per-row values.
+//   valid: columns [0, valid) of the chunk are real.
+template <bool kPerColumn>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
+                                          const float* lse_col, const float* dv_col, float lse_row, float dv_row,
+                                          int valid, uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pv[2], dsv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float l = kPerColumn ? lse_col[e + u] : lse_row;
+      const float dd = kPerColumn ? dv_col[e + u] : dv_row;
+      const float pe = ex2_approx(fmaf(__uint_as_float(s[e + u]), sl2, -l));
+      const float de = pe * (__uint_as_float(dp[e + u]) - dd);
+      const bool ok = e + u < valid;
+      pv[u] = ok ? pe : 0.f;
+      dsv[u] = ok ? de : 0.f;
+    }
+    pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+    dk[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+  }
+}
+
+// Writes one 128-row tile's fp32 accumulator row (TMEM columns [col, col + D)) as bf16, scaled.
+template <int D>
+__device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_bfloat16* dst, bool live) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 32 * cc, r);
+    tmem_wait_ld();
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * scale, __uint_as_float(r[2 * e + 1]) * scale);
+    if (live) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cc);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) d4[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// dK, dV: one CTA per (sample*set, head, 128-key tile)
+// ------------------------------------------------------------------------------------------
+// kKeysMajor = true: the kernel's "resident" tiles are K, V and the streamed ones Q, dO.
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 1,
+            B_DONE = B_PREADY + 1, B_FIN = B_DONE + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int tile = blockIdx.x % p.n_tiles;
+  const int hb = blockIdx.x / p.n_tiles;
+  const int h = hb % p.heads, bg = hb / p.heads;
+  const int b = bg / p.G, g = bg % p.G;
+  const int kv0 = tile * kBT;
+  const int nq = p.n_tiles;   // query tiles of the set
+  const int chan0 = h * D;
+  const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_RES), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_SFULL), 1);
+    mbar_init(bar(B_PREADY), 128);
+    mbar_init(bar(B_DONE), 1);
+    mbar_init(bar(B_FIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProdWarp && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+  auto sRes = [&](int i) { return sbase + C::kResOff + (uint32_t)(i * C::kTileBytes); };           // K, V
+  auto sStr = [&](int s, int i) { return sbase + C::kStageOff + (uint32_t)((2 * s + i) * C::kTileBytes); };  // Q, dO
+  auto sVec = [&](int s) { return sbase + C::kVecOff + (uint32_t)(s * C::kVecBytes); };
+
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    const bool leader = elect_one_sync();
+    int issued = 0;
+    if (leader) {
+      mbar_arrive_expect_tx(bar(B_RES), 2 * C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c) {
+        bwd_load_tile(&tm_k, sRes(0) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, kv0, g, b, p.k);
+        bwd_load_tile(&tm_v, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, kv0, g, b, p.k);
+      }
+    }
+    for (int i = 0; i < nq; ++i) {
+      const int s = i % kStages;
+      if (i >= kStages && !bwd_warp_wait(bar(B_EMPTY + s), ((i / kStages) - 1) & 1, wc)) break;
+      if (leader) {
+        mbar_arrive_expect_tx(bar(B_FULL + s), 2 * C::kTileBytes + C::kVecBytes);
+        for (int c = 0; c < C::kChunks; ++c) {
+          bwd_load_tile(&tm_q, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, i * kBT, g,
+                        b, p.k);
+          bwd_load_tile(&tm_do, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, i * kBT, g,
+                        b, p.k);
+        }
+        bulk_load(sVec(s), p.lse + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
+        bulk_load(sVec(s) + kBT * 4, p.dvec + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
+      }
+      issued = i + 1;
+    }
+    // every load issued lands before the CTA may exit
+    mbar_drain(bar(B_RES), 0, p.timeout_ns);
+    for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
+      mbar_drain(bar(B_FULL + t % kStages), (t / kStages) & 1, p.timeout_ns);
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    const bool leader = elect_one_sync();
+    constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kBT, false);   // M = 128, N = 128, both K-major
+    constexpr uint32_t idesc_ts = idesc_bf16_f32(kBT, D, true);      // M = 128, N = D, B MN-major
+    constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
+    const uint64_t dK = sdesc_sw128(sRes(0), 16, 1024), dV = sdesc_sw128(sRes(1), 16, 1024);
+    const uint64_t dQk = sdesc_sw128(sStr(0, 0), 16, 1024);             // Q as K-major B (N = queries)
+    const uint64_t dQmn = sdesc_sw128(sStr(0, 0), kChunkBytes, 1024);   // Q as MN-major B (N = channels)
+    const uint64_t dOk = sdesc_sw128(sStr(0, 1), 16, 1024);
+    const uint64_t dOmn = sdesc_sw128(sStr(0, 1), kChunkBytes, 1024);
+    // stage s's tiles sit 2*s tiles after stage 0's
+    auto stage_off = [&](int s) { return (uint64_t)(2 * s) * kTileStep; };
+    // D_t = A K-major (128 rows x D) times B K-major (128 rows x D)^T
+    auto issue_ss = [&](uint32_t d_col, uint64_t a0, uint64_t b0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+        if (leader) mma_ss(tmem + d_col, a0 + off, b0 + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+    };
+    // D_t (+)= A (tensor memory, bf16 pairs, 128 x 128) times B MN-major (128 rows x D)
+    auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
+#pragma unroll
+      for (int kk = 0; kk < kBT / 16; ++kk)
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_ts,
+                           (acc || kk > 0) ? 1u : 0u);
+    };
+    bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+    for (int i = 0; ok && i <= nq; ++i) {
+      const int s = i % kStages;
+      if (i < nq && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
+      if (i > 0) {
+        // tile i-1: P^T and dS^T are in tensor memory
+        if (!bwd_warp_wait(bar(B_PREADY), (i - 1) & 1, wc)) break;
+        tc_fence_after();
+        const int sp = (i - 1) % kStages;
+        issue_ts(kColAcc0, kColS, dOmn + stage_off(sp), i > 1);    // dV += P^T dO
+        issue_ts(kColAcc1, kColDP, dQmn + stage_off(sp), i > 1);   // dK += dS^T Q
+        if (leader) tc_commit(bar(B_EMPTY + sp));
+      }
+      if (i < nq) {
+        tc_fence_after();
+        issue_ss(kColS, dK, dQk + stage_off(s));    // S^T = K Q^T
+        issue_ss(kColDP, dV, dOk + stage_off(s));   // dP^T = V dO^T
+        if (leader) tc_commit(bar(B_SFULL));
+      } else if (leader) {
+        tc_commit(bar(B_DONE));
+      }
+    }
+    if (leader) tc_commit(bar(B_FIN));
+    mbar_drain(bar(B_FIN), 0, p.timeout_ns);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ compute warps 0-3
+    const int row = warp * 32 + lane;                       // key row = tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kColS, tP = tmem + lane_base + kColDP;
+    bool ok = true;
+    for (int i = 0; i < nq; ++i) {
+      if (!bwd_warp_wait(bar(B_SFULL), i & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (i % kStages) * C::kVecBytes);
+      const int valid_q = min(kBT, p.n - i * kBT);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tS + 32 * c, s);
+        tmem_ld32(tP + 32 * c, dp);
+        tmem_wait_ld();
+        uint32_t pk[16], dk[16];
+        bwd_chunk<true>(s, dp, p.scale_log2, vec + 32 * c, vec + kBT + 32 * c, 0.f, 0.f, valid_q - 32 * c, pk, dk);
+        tmem_st16(tS + 16 * c, pk);    // P^T over the consumed S^T columns
+        tmem_st16(tP + 16 * c, dk);    // dS^T over the consumed dP^T columns
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PREADY));
+    }
+    if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
+      tc_fence_after();
+      const int j = kv0 + row;
+      const bool live = j < p.n;
+      const int token = bwd_slot_token(p.layout, live ? j : 0, g, p.k);
+      const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
+      bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, live);
+      bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, live);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// dQ: one CTA per (sample*set, head, 128-query tile)
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 1,
+            B_DONE = B_PREADY + 1, B_FIN = B_DONE + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int tile = blockIdx.x % p.n_tiles;
+  const int hb = blockIdx.x / p.n_tiles;
+  const int h = hb % p.heads, bg = hb / p.heads;
+  const int b = bg / p.G, g = bg % p.G;
+  const int q0 = tile * kBT;
+  const int nk = p.n_tiles;   // key tiles of the set
+  const int chan0 = h * D;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_RES), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_SFULL), 1);
+    mbar_init(bar(B_PREADY), 128);
+    mbar_init(bar(B_DONE), 1);
+    mbar_init(bar(B_FIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProdWarp && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+  auto sRes = [&](int i) { return sbase + C::kResOff + (uint32_t)(i * C::kTileBytes); };           // Q, dO
+  auto sStr = [&](int s, int i) { return sbase + C::kStageOff + (uint32_t)((2 * s + i) * C::kTileBytes); };  // K, V
+
+  if (warp == kProdWarp) {
+    const bool leader = elect_one_sync();
+    int issued = 0;
+    if (leader) {
+      mbar_arrive_expect_tx(bar(B_RES), 2 * C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c) {
+        bwd_load_tile(&tm_q, sRes(0) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, q0, g, b, p.k);
+        bwd_load_tile(&tm_do, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, q0, g, b, p.k);
+      }
+    }
+    for (int j = 0; j < nk; ++j) {
+      const int s = j % kStages;
+      if (j >= kStages && !bwd_warp_wait(bar(B_EMPTY + s), ((j / kStages) - 1) & 1, wc)) break;
+      if (leader) {
+        mbar_arrive_expect_tx(bar(B_FULL + s), 2 * C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c) {
+          bwd_load_tile(&tm_k, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, j * kBT, g, b,
+                        p.k);
+          bwd_load_tile(&tm_v, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, j * kBT, g, b,
+                        p.k);
+        }
+      }
+      issued = j + 1;
+    }
+    mbar_drain(bar(B_RES), 0, p.timeout_ns);
+    for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
+      mbar_drain(bar(B_FULL + t % kStages), (t / kStages) & 1, p.timeout_ns);
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    const bool leader = elect_one_sync();
+    constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kBT, false);
+    constexpr uint32_t idesc_ts = idesc_bf16_f32(kBT, D, true);
+    constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
+    const uint64_t dQ = sdesc_sw128(sRes(0), 16, 1024), dO = sdesc_sw128(sRes(1), 16, 1024);
+    const uint64_t dKk = sdesc_sw128(sStr(0, 0), 16, 1024);             // K as K-major B (N = keys)
+    const uint64_t dKmn = sdesc_sw128(sStr(0, 0), kChunkBytes, 1024);   // K as MN-major B (N = channels)
+    const uint64_t dVk = sdesc_sw128(sStr(0, 1), 16, 1024);
+    auto stage_off = [&](int s) { return (uint64_t)(2 * s) * kTileStep; };
+    auto issue_ss = [&](uint32_t d_col, uint64_t a0, uint64_t b0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+        if (leader) mma_ss(tmem + d_col, a0 + off, b0 + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
+#pragma unroll
+      for (int kk = 0; kk < kBT / 16; ++kk)
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_ts,
+                           (acc || kk > 0) ? 1u : 0u);
+    };
+    bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+    for (int j = 0; ok && j <= nk; ++j) {
+      const int s = j % kStages;
+      if (j < nk && !bwd_warp_wait(bar(B_FULL + s), (j / kStages) & 1, wc)) break;
+      if (j > 0) {
+        if (!bwd_warp_wait(bar(B_PREADY), (j - 1) & 1, wc)) break;
+        tc_fence_after();
+        const int sp = (j - 1) % kStages;
+        issue_ts(kColAcc0, kColDP, dKmn + stage_off(sp), j > 1);   // dQ += dS K
+        if (leader) tc_commit(bar(B_EMPTY + sp));
+      }
+      if (j < nk) {
+        tc_fence_after();
+        issue_ss(kColS, dQ, dKk + stage_off(s));    // S = Q K^T
+        issue_ss(kColDP, dO, dVk + stage_off(s));   // dP = dO V^T
+        if (leader) tc_commit(bar(B_SFULL));
+      } else if (leader) {
+        tc_commit(bar(B_DONE));
+      }
+    }
+    if (leader) tc_commit(bar(B_FIN));
+    mbar_drain(bar(B_FIN), 0, p.timeout_ns);
+    __syncwarp();
+  } else {
+    const int row = warp * 32 + lane;                       // query row = tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kColS, tP = tmem + lane_base + kColDP;
+    const int qs = q0 + row;
+    const bool live = qs < p.n;
+    const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
+    const float lse_r = live ? p.lse[vec_row + qs] : 0.f;
+    const float dv_r = live ? p.dvec[vec_row + qs] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      if (!bwd_warp_wait(bar(B_SFULL), j & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      const int valid_k = min(kBT, p.n - j * kBT);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tS + 32 * c, s);
+        tmem_ld32(tP + 32 * c, dp);
+        tmem_wait_ld();
+        uint32_t pk[16], dk[16];
+        bwd_chunk<false>(s, dp, p.scale_log2, nullptr, nullptr, lse_r, dv_r, live ? valid_k - 32 * c : 0, pk, dk);
+        tmem_st16(tP + 16 * c, dk);    // dS over the consumed dP columns
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_PREADY));
+    }
+    if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
+      tc_fence_after();
+      const int token = bwd_slot_token(p.layout, live ? qs : 0, g, p.k);
+      const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
+      bwd_store_row<D>(tmem + lane_base + kColAcc0, p.scale, p.dq + off, live);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const CUtensorMap& tk,
+                 const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, long long rows, long long ctas,
+                 cudaStream_t stream) {
+  constexpr int smem = BwdCfg<D>::kSmemBytes;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attention backward, d=%d) failed", D);
+    attr_done = true;
+  }
+  const long long dblocks = std::min<long long>((rows + 255) / 256, (long long)device_sm_count() * 16);
+  attn_bwd_dvec_kernel<D><<<(unsigned)dblocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                                 static_cast<const __nv_bfloat16*>(dout), p, rows);
+  int rc = check_launch("attn_bwd_dvec_kernel");
+  if (rc) return rc;
+  attn_bwd_dkdv_kernel<D><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  if ((rc = check_launch("attn_bwd_dkdv_kernel"))) return rc;
+  attn_bwd_dq_kernel<D><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  return check_launch("attn_bwd_dq_kernel");
+}
+
+}  // namespace
+
+int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
+                              int sparse_k, float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  const int N = s.text_len + s.T * s.H * s.W;
+  const int G = (layout == 0) ? 1 : sparse_k;
+  const int n = N / G;
+  BwdParams p{};
+  p.n = n;
+  p.N = N;
+  p.heads = s.heads;
+  p.G = G;
+  p.k = (layout == 0) ? 1 : sparse_k;
+  p.layout = layout;
+  p.n_tiles = (n + kBT - 1) / kBT;
+  p.vec_stride = p.n_tiles * kBT;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = status;
+  p.timeout_ns = wait_timeout_ns();
+  const long long ctas = (long long)p.n_tiles * s.heads * s.B * G;
+  if (ctas > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld backward work units is too many", ctas);
+  CUtensorMap tq, tk, tv, tdo;
+  int rc;
+  if ((rc = make_attn_tmap(&tq, q, s, N, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_attn_tmap(&tk, k, s, N, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_attn_tmap(&tv, v, s, N, layout, p.k)) != OSP_OK) return rc;
+  if ((rc = make_attn_tmap(&tdo, dout, s, N, layout, p.k)) != OSP_OK) return rc;
+  // Dv scratch, [B*G][heads][vec_stride] fp32, from the library's stream-ordered pool; cleared so
+  // that the padding slots past n hold zeros
+  const size_t vec_bytes = (size_t)s.B * G * s.heads * p.vec_stride * sizeof(float);
+  void* ws = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool || cudaMallocFromPoolAsync(&ws, vec_bytes, pool, stream) != cudaSuccess)
+    return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", vec_bytes);
+  if (cudaMemsetAsync(ws, 0, vec_bytes, stream) != cudaSuccess) {
+    cudaFreeAsync(ws, stream);
+    return set_error(OSP_ERR_CUDA, "clearing the backward workspace failed");
+  }
+  p.dvec = static_cast<float*>(ws);
+  const long long rows = (long long)s.B * N * s.heads;
+  switch (s.head_dim) {
+    case 64: rc = launch_bwd_d<64>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
+    case 96: rc = launch_bwd_d<96>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
+    case 128: rc = launch_bwd_d<128>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
+    default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  }
+  cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+}  // namespace osp

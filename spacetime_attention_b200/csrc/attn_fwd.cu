@@ -125,6 +125,10 @@ struct AttnParams {
   // text_len text rows (ceil(text_len / 128) tiles from the text maps) followed by the set's own
   // tiles; the set's query tokens sit q_row_base (= text_len) rows into each sample.
   int q_row_base;
+  // Optional row log-sum-exp for the backward pass (plain mode): lse[(b*G + g)*heads + h][slot]
+  // = m + log2(l) in the log2 domain of the scaled scores, rows lse_stride apart.
+  float* lse;
+  int lse_stride;
   // Work items (1-D grid): units are (sample*set, head, query block) with the query block fastest.
   // CTAs [0, n_full) process whole units; every later unit is split into n_split KV ranges whose
   // CTAs write fp32 partials (unnormalised O, running max m, row sum l) to ws_o / ws_ml, merged
@@ -717,6 +721,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = 1.f / l;
       const int slot = w.q0 + i * kBM + row;
       const bool live = slot < w.nq;
+      if (!kPacked && part < 0 && p.lse && live)
+        p.lse[((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot] = m + __log2f(l);
       if (part >= 0) {
         // split unit: unnormalised fp32 O (relative to m) and (m, l) for the combine kernel
         const size_t prow = ((size_t)(unit - p.n_full) * p.n_split + part) * (2 * kBM) + i * kBM + row;
@@ -794,6 +800,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, i
     for (int e = 0; e < kPer; ++e) acc[e] += wgt * p.ws_o[prow * D + e * 32 + lane];
   }
   const float inv = 1.f / lsum;
+  if (p.lse && lane == 0) p.lse[((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot] = mmax + __log2f(lsum);
   const int token = p.q_row_base + slot_token(p.layout, slot, g, p.k);
   __nv_bfloat16* dst = p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D;
 #pragma unroll
@@ -884,6 +891,11 @@ int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
 
 }  // namespace
 
+int make_attn_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k,
+                   long long batch_rows) {
+  return make_tmap(tm, ptr, s, N, layout, k, batch_rows);
+}
+
 namespace {
 
 // Attention launch with an explicit status word (the kernel's only global scratch).
@@ -958,7 +970,7 @@ AttnParams base_params(const osp_shape& s, int layout, int sparse_k, float scale
 // frame_causal: dense layout only; the frame-causal mask over s's text block and frames.
 int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
                        int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
-                       int N_kv = -1, bool frame_causal = false) {
+                       int N_kv = -1, bool frame_causal = false, float* lse = nullptr) {
   const int N = (N_kv < 0) ? s.text_len + s.T * s.H * s.W : s.T * s.H * s.W;   // q / o tokens per sample
   if (N_kv < 0) N_kv = N;
   AttnParams p = base_params(s, layout, sparse_k, scale, o, status);
@@ -969,6 +981,8 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.N_q = N;
   p.frame_hw = frame_causal ? s.H * s.W : 0;
   p.text_len = s.text_len;
+  p.lse = lse;
+  p.lse_stride = (n + kBM - 1) / kBM * kBM;
   if (frame_causal) allow_split = false;   // a KV range could hold no visible key for some rows
   CUtensorMap tq, tk, tv;
   int rc;
@@ -1048,6 +1062,13 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
   p.qblocks = (int)qblocks;
   const long long units = qblocks * s.heads * (long long)s.B;
   return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, units, (N + kBN - 1) / kBN, true, s.head_dim, stream);
+}
+
+int attention_forward_lse_launch(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const osp_shape& s, int layout, int sparse_k, float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true, -1, false, lse);
 }
 
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,

@@ -256,6 +256,52 @@ int osp_attn_frame_causal(const void* q, const void* k, const void* v, void* o, 
   return frame_causal_attention_launch(q, k, v, o, *shape, softmax_scale, static_cast<cudaStream_t>(stream));
 }
 
+// Shared validation of the training entry points: dense (sparse_k == 1, text allowed) or
+// Skiparse (sparse_k > 1, video tokens only).
+static int check_train(const osp_shape* shape, int32_t sparse_k, int32_t mode, int* layout) {
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (sparse_k == 1) {
+    *layout = 0;
+    return OSP_OK;
+  }
+  if ((rc = check_skiparse(shape, sparse_k, mode, false))) return rc;
+  if (mode == OSP_SKIP_GROUP && (sparse_k > 128 || (128 % sparse_k) != 0))
+    return set_error(OSP_ERR_UNSUPPORTED, "fused Group Skip needs k to divide 128 (got k=%d)", sparse_k);
+  *layout = mode + 1;
+  return OSP_OK;
+}
+
+int osp_attn_forward_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
+                           int32_t sparse_k, int32_t mode, float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int layout = 0;
+  int rc = check_train(shape, sparse_k, mode, &layout);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse) return set_error(OSP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_forward_lse_launch(q, k, v, o, lse, *shape, layout, sparse_k, softmax_scale,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+int osp_attn_backward(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                      void* dq, void* dk, void* dv, const osp_shape* shape, int32_t sparse_k, int32_t mode,
+                      float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int layout = 0;
+  int rc = check_train(shape, sparse_k, mode, &layout);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return set_error(OSP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, layout, sparse_k, softmax_scale,
+                                   static_cast<cudaStream_t>(stream));
+}
+
 int osp_rope3d_packed(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
                       int32_t n_samples, int32_t heads, int32_t head_dim, const osp_rope* rope, void* stream) {
   g_last_error[0] = 0;

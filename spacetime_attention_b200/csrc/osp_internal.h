@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/osp.h"
@@ -70,6 +71,21 @@ int frame_causal_attention_launch(const void* q, const void* k, const void* v, v
 // Temporal attention of 2D + 1D (T <= 64): sets of T tokens at stride H*W, optionally causal in t.
 int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
                               float scale, cudaStream_t stream);
+
+// TMA map over a BSHD tensor for the attention kernels' 128-row x 64-channel SW128 tiles, viewed
+// per layout (0 dense, 1 Single Skip, 2 Group Skip); batch_rows = rows between samples (< 0: N).
+int make_attn_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k,
+                   long long batch_rows = -1);
+
+// Training forward: attention as attention_launch (layout 0 dense, or Skiparse) that also writes
+// the row log-sum-exp (log2 domain of the scaled scores) to lse, [B*G][heads][ceil(n/128)*128].
+int attention_forward_lse_launch(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 const osp_shape& s, int layout, int sparse_k, float scale, cudaStream_t stream);
+
+// Backward pass of attention_forward_lse_launch: dq, dk, dv from q, k, v, o, dout and lse.
+int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
+                              int sparse_k, float scale, cudaStream_t stream);
 
 // Packed batch (block-diagonal attention): segment i owns q/o rows [q_bounds[i], q_bounds[i+1])
 // and k/v rows [kv_bounds[i], kv_bounds[i+1]); host arrays of n_seg + 1 validated offsets.

@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "OSP_OK", 1: "OSP_ERR_INVALID_ARG", 2: "OSP_ERR_UNSUPPORTED",
 EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_scatter", "osp_skiparse_attn",
             "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version",
             "osp_attn_full_noalloc", "osp_attn_cross", "osp_rope3d_packed", "osp_attn_packed",
-            "osp_attn_spatial", "osp_attn_temporal", "osp_attn_frame_causal")
+            "osp_attn_spatial", "osp_attn_temporal", "osp_attn_frame_causal", "osp_attn_forward_train",
+            "osp_attn_backward")
 
 MAX_SEGMENTS = 256   # OSP_MAX_SEGMENTS
 
@@ -70,6 +71,8 @@ def library() -> ctypes.CDLL:
             "osp_attn_full_noalloc": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_cross": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_spatial": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_forward_train": [vp, vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
+            "osp_attn_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
             "osp_attn_temporal": [vp, vp, vp, vp, sp, i32, ctypes.c_float, vp],
             "osp_attn_frame_causal": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_rope3d_packed": [vp, vp, vp, vp, ctypes.POINTER(OspSampleGrid), i32, i32, i32, rp, vp],
@@ -190,6 +193,44 @@ def attn_temporal(q, k, v, grid, causal: bool = False, scale: float = 0.0, o=Non
 def attn_frame_causal(q, k, v, grid, text_len: int, scale: float = 0.0, o=None) -> torch.Tensor:
     """osp_attn_frame_causal: token of frame t attends to the text and frames 0..t."""
     return _attn3("osp_attn_frame_causal", q, k, v, grid, text_len, scale, o)
+
+
+def lse_shape(q: torch.Tensor, sparse_k: int = 1):
+    """Shape of the lse buffer of osp_attn_forward_train: [B*G, heads, ceil(n/128)*128]."""
+    B, N, heads, _ = q.shape
+    G = 1 if sparse_k == 1 else sparse_k
+    n = N // G
+    return (B * G, heads, (n + 127) // 128 * 128)
+
+
+def attn_forward_train(q, k, v, grid, text_len: int = 0, sparse_k: int = 1, mode: int = 0, scale: float = 0.0,
+                       o=None, lse=None):
+    """osp_attn_forward_train: returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(lse_shape(q, sparse_k), dtype=torch.float32, device=q.device) if lse is None else lse
+    shp = _shape_of(q, grid, text_len)
+    _check("osp_attn_forward_train",
+           library().osp_attn_forward_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
+                                            int(sparse_k), int(mode), ctypes.c_float(scale), _stream_handle(q)))
+    return o, lse
+
+
+def attn_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, sparse_k: int = 1, mode: int = 0,
+                  scale: float = 0.0, dq=None, dk=None, dv=None):
+    """osp_attn_backward: returns (dq, dk, dv)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _bshd(t, n)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    shp = _shape_of(q, grid, text_len)
+    _check("osp_attn_backward",
+           library().osp_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                       _ptr(dv), ctypes.byref(shp), int(sparse_k), int(mode), ctypes.c_float(scale),
+                                       _stream_handle(q)))
+    return dq, dk, dv
 
 
 def _bounds(b) -> ctypes.Array:

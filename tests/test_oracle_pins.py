@@ -620,3 +620,16 @@ def test_backward_closed_forms_and_lse():
     # lse: two keys with scores 0 and ln 3 -> ln 4
     lse = O.attention_head_lse_ref(np.array([[1.0, 0.0]]), np.array([[0.0, 0.0], [math.log(3.0), 0.0]]), 1.0)
     np.testing.assert_allclose(lse, [math.log(4.0)], rtol=1e-15)
+
+
+def test_backward_rows_agree_with_full_backward():
+    # the sampled-row form is the same chain rule evaluated row by row (pinned above by finite
+    # differences through the full form)
+    rng = np.random.default_rng(83)
+    q, k, v, do = (rng.standard_normal((40, 8)) for _ in range(4))
+    dq, dk, dv = O.attention_head_backward_ref(q, k, v, do, 0.3)
+    rq, rk = [0, 7, 39], [3, 4, 38]
+    sq, sk, sv = O.attention_head_backward_rows_ref(q, k, v, do, 0.3, rq, rk, chunk=16)
+    np.testing.assert_allclose(sq, dq[rq], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(sk, dk[rk], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(sv, dv[rk], rtol=1e-12, atol=1e-13)
