@@ -461,6 +461,60 @@ def run_variant_op(args, rank, world, local_rank):
             "tflops": round(tflops, 1), "hbm_gbs": round(gbs, 1)}
 
 
+def run_backward_op(args, rank, world, local_rank):
+    """Time the attention backward pass (osp_attn_backward: row sums, dK/dV kernel, dQ kernel)
+    on the workload (dense, or the Skiparse Single + Group pair with --attn skiparse), after a
+    training forward that saved o and lse.  value = backward flops / backward time, counting 2.5x
+    the forward's flops (the five matrix products of the standard backward: S recomputed, dV, dP,
+    dQ, dK)."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = syn.WORKLOADS[args.workload]
+    q, k, v = (t.to(dev) for t in syn.make_qkv(w, w.seed + 17 * rank))
+    do = syn.randn_bf16(tuple(q.shape), w.seed + 99 + 17 * rank).to(dev)
+    modes = [(w.skiparse_k, ops.OSP_SKIP_SINGLE), (w.skiparse_k, ops.OSP_SKIP_GROUP)] if sparse(w) else [(1, 0)]
+    L = 0 if sparse(w) else w.text_len
+    saved = [ops.attn_forward_train(q, k, v, w.grid, L, sparse_k=kk, mode=m) for kk, m in modes]
+    grads = [tuple(torch.empty_like(q) for _ in range(3)) for _ in modes]
+
+    def step():
+        for (kk, m), (o, lse), (dq, dk, dv) in zip(modes, saved, grads):
+            ops.attn_backward(q, k, v, o, do, lse, w.grid, L, sparse_k=kk, mode=m, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ops.check_status(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    peaks, src = load_peaks()
+    flops = 2.5 * step_flops(w)
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops_sustained"])
+    return {"metric": "attention backward TFLOP/s (2.5x forward flops)", "value": round(world * tflops, 1),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(w.describe(), op="backward", attn="skiparse pair" if sparse(w) else "dense",
+                           flops_per_step=flops, l2="inputs > L2, no flush"),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tflops / peak, 4), "traffic": None,
+                         "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel",
+                         "peak_source": f"{src} (sustained bf16 GEMM)"},
+            "clocks": clocks, "gpu_launches": 3 * len(modes) * args.steps}
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -697,7 +751,7 @@ def main():
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
     ap.add_argument("--op", default="step",
                     choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
-                             "frame_causal", "skiparse_text"],
+                             "frame_causal", "skiparse_text", "backward"],
                     help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone; "
                          "cross: video -> text cross-attention alone; packed: a packed batch of mixed shapes")
     ap.add_argument("--packed", default="frame_pack_cog2b", choices=sorted(syn.PACKED_WORKLOADS),
@@ -731,7 +785,7 @@ def main():
     try:
         runner = {"step": run_ours, "cross": run_cross_op, "packed": run_packed_op, "spatial": run_variant_op,
                   "temporal": run_variant_op, "frame_causal": run_variant_op,
-                  "skiparse_text": run_variant_op}.get(args.op, run_hbm_op)
+                  "skiparse_text": run_variant_op, "backward": run_backward_op}.get(args.op, run_hbm_op)
         line = runner(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
