@@ -27,9 +27,12 @@ namespace {
 
 constexpr int kBT = 128;                 // rows per tile (queries or keys)
 constexpr int kChunkBytes = 128 * 128;   // 128 rows x 64 bf16 channels, one SW128 atom wide
-constexpr int kBwdThreads = 192;         // warps 0-3 compute, 4 TMA producer, 5 MMA issuer
-constexpr int kProdWarp = 4;
-constexpr int kMmaWarp = 5;
+// warps 0-7 compute (warp w: tensor-memory lane quarter w % 4, column half w / 4; two warps per
+// SM sub-partition keep its MUFU busy), 8 TMA producer, 9 MMA issuer
+constexpr int kBwdThreads = 320;
+constexpr int kComputeThreads = 256;
+constexpr int kProdWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 // tensor memory columns: S (or S^T) 0..127, dP (dP^T) 128..255, accumulators at 256 and 384
@@ -78,6 +81,12 @@ __device__ __forceinline__ void bwd_load_tile(const CUtensorMap* tm, uint32_t ds
   else if (layout == 1) tma_load_4d(dst, tm, bar, chan, g, row0, b);
   else tma_load_5d(dst, tm, bar, chan, 0, g, row0 / k, b);
 }
+
+// Packed bf16 P / dS columns: compute warp half h writes the 64 query (key) columns it owns,
+// 64h .. 64h + 63, as 32 packed columns at 64h .. 64h + 31, i.e. over its own consumed S / dP
+// columns, so the two warps sharing a lane quarter never touch each other's unread columns.
+// The tensor-memory A operand of K-step kk (16 columns of P / dS) therefore starts at:
+__device__ __forceinline__ uint32_t packed_col(int kk) { return 8u * kk + (kk >= 4 ? 32u : 0u); }
 
 __device__ __forceinline__ bool bwd_warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const bool ok = mbar_wait(bar, parity, w);
@@ -149,10 +158,13 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_
 }
 
 // Writes one 128-row tile's fp32 accumulator row (TMEM columns [col, col + D)) as bf16, scaled.
+// part = 0 / 1: only the even / odd 32-column chunks (two warps share a row); -1: all.
 template <int D>
-__device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_bfloat16* dst, bool live) {
+__device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_bfloat16* dst, bool live,
+                                              int part = -1) {
 #pragma unroll
   for (int cc = 0; cc < D / 32; ++cc) {
+    if (part >= 0 && (cc & 1) != part) continue;
     uint32_t r[32];
     tmem_ld32(taddr + 32 * cc, r);
     tmem_wait_ld();
@@ -205,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(B_EMPTY + s), 1);
     }
     mbar_init(bar(B_SFULL), 1);
-    mbar_init(bar(B_PREADY), 128);
+    mbar_init(bar(B_PREADY), kComputeThreads);
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
@@ -287,7 +299,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < kBT / 16; ++kk)
-        if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_ts,
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
     bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
@@ -316,9 +328,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_drain(bar(B_FIN), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ compute warps 0-3
-    const int row = warp * 32 + lane;                       // key row = tensor-memory lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------------ compute warps 0-7
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;                    // key row = tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + kColS, tP = tmem + lane_base + kColDP;
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
@@ -327,15 +340,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (i % kStages) * C::kVecBytes);
       const int valid_q = min(kBT, p.n - i * kBT);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int u = 0; u < 2; ++u) {   // this warp's two 32-column chunks, in order
+        const int c = 2 * half + u;
         uint32_t s[32], dp[32];
         tmem_ld32(tS + 32 * c, s);
         tmem_ld32(tP + 32 * c, dp);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
         bwd_chunk<true>(s, dp, p.scale_log2, vec + 32 * c, vec + kBT + 32 * c, 0.f, 0.f, valid_q - 32 * c, pk, dk);
-        tmem_st16(tS + 16 * c, pk);    // P^T over the consumed S^T columns
-        tmem_st16(tP + 16 * c, dk);    // dS^T over the consumed dP^T columns
+        tmem_st16(tS + 64 * half + 16 * u, pk);    // P^T over this warp's consumed S^T columns
+        tmem_st16(tP + 64 * half + 16 * u, dk);    // dS^T over this warp's consumed dP^T columns
       }
       tmem_wait_st();
       tc_fence_before();
@@ -347,8 +361,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool live = j < p.n;
       const int token = bwd_slot_token(p.layout, live ? j : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
-      bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, live);
-      bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, live);
+      if (half == 0) bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, live);
+      else bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, live);
     }
   }
   tc_fence_before();
@@ -395,7 +409,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(B_EMPTY + s), 1);
     }
     mbar_init(bar(B_SFULL), 1);
-    mbar_init(bar(B_PREADY), 128);
+    mbar_init(bar(B_PREADY), kComputeThreads);
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
@@ -467,7 +481,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < kBT / 16; ++kk)
-        if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + (uint64_t)(128 * kk), idesc_ts,
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
     bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
@@ -494,8 +508,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_drain(bar(B_FIN), 0, p.timeout_ns);
     __syncwarp();
   } else {
-    const int row = warp * 32 + lane;                       // query row = tensor-memory lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;                    // query row = tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_base + kColS, tP = tmem + lane_base + kColDP;
     const int qs = q0 + row;
     const bool live = qs < p.n;
@@ -508,14 +523,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int valid_k = min(kBT, p.n - j * kBT);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int u = 0; u < 2; ++u) {   // this warp's two 32-column chunks, in order
+        const int c = 2 * half + u;
         uint32_t s[32], dp[32];
         tmem_ld32(tS + 32 * c, s);
         tmem_ld32(tP + 32 * c, dp);
         tmem_wait_ld();
         uint32_t pk[16], dk[16];
         bwd_chunk<false>(s, dp, p.scale_log2, nullptr, nullptr, lse_r, dv_r, live ? valid_k - 32 * c : 0, pk, dk);
-        tmem_st16(tP + 16 * c, dk);    // dS over the consumed dP columns
+        tmem_st16(tP + 64 * half + 16 * u, dk);    // dS over this warp's consumed dP columns
       }
       tmem_wait_st();
       tc_fence_before();
@@ -525,7 +541,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int token = bwd_slot_token(p.layout, live ? qs : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
-      bwd_store_row<D>(tmem + lane_base + kColAcc0, p.scale, p.dq + off, live);
+      bwd_store_row<D>(tmem + lane_base + kColAcc0, p.scale, p.dq + off, live, half);
     }
   }
   tc_fence_before();
