@@ -191,3 +191,16 @@ def test_split_kv_tail_matches_oracle_and_unsplit(gpu, monkeypatch, d, grid, L, 
     assert_attn_close(split, ref, "split")
     assert_attn_close(plain, ref, "unsplit")
     assert float((split.float() - plain.float()).abs().max()) <= 1e-2
+
+
+def test_maximum_sequence_length_sampled(gpu):
+    """A 2^20-token sequence (64 x 128 x 128 grid, one head, d = 64): 4,096 query blocks of 256
+    rows and 8,192 KV tiles per block; sampled rows against the oracle."""
+    grid = (64, 128, 128)
+    N = grid[0] * grid[1] * grid[2]
+    q, k, v = (syn.randn_bf16((1, N, 1, 64), 301 + i) for i in range(3))
+    o = ops.attn_full(q.to(gpu), k.to(gpu), v.to(gpu), grid, 0)
+    ops.check_status()
+    rows = _sample_rows(N, 8, 3)
+    ref = O.attn_ref(to_f64(q), to_f64(k), to_f64(v), rows=rows)
+    assert_attn_close(o[:, rows], ref, "2^20 tokens")

@@ -77,6 +77,7 @@ SPARSE = [
     (1, 2, 64, (4, 8, 8), 2),
     (1, 2, 96, (4, 10, 15), 2),       # sets of 300: ragged tiles
     (1, 1, 128, (4, 16, 18), 4),
+    (2, 1, 64, (2, 16, 16), 8),       # B = 2, sets of 64 (one partial tile each)
 ]
 
 
