@@ -35,8 +35,17 @@ constexpr int kProdWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
-// tensor memory columns: S (or S^T) 0..127, dP (dP^T) 128..255, accumulators at 256 and 384
-constexpr uint32_t kColS = 0, kColDP = 128, kColAcc0 = 256, kColAcc1 = 384;
+// The streamed 128-row tiles are processed as two 64-row sub-tiles, and the score buffers are
+// double-buffered across sub-tiles so that the products of sub-tile t+1 run on the tensor core
+// while the compute warps turn sub-tile t into P / dS.  Tensor-memory columns: buffer b holds S
+// (or S^T) at 128b .. 128b+63 and dP (dP^T) at 128b+64 .. 128b+127; accumulators at 256 and 384.
+constexpr int kSub = 64;
+constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
+__device__ __forceinline__ uint32_t col_s(int buf) { return 128u * buf; }
+__device__ __forceinline__ uint32_t col_dp(int buf) { return 128u * buf + 64u; }
+// descriptor offset (16-byte units) of the second 64-row sub-tile of a 128-row SW128 tile
+// (eight 1024-byte groups of 8 rows), for both K-major and MN-major use
+constexpr uint64_t kSubDescOff = (64 * 128) >> 4;
 
 template <int D>
 struct BwdCfg {
@@ -82,11 +91,11 @@ __device__ __forceinline__ void bwd_load_tile(const CUtensorMap* tm, uint32_t ds
   else tma_load_5d(dst, tm, bar, chan, 0, g, row0 / k, b);
 }
 
-// Packed bf16 P / dS columns: compute warp half h writes the 64 query (key) columns it owns,
-// 64h .. 64h + 63, as 32 packed columns at 64h .. 64h + 31, i.e. over its own consumed S / dP
-// columns, so the two warps sharing a lane quarter never touch each other's unread columns.
-// The tensor-memory A operand of K-step kk (16 columns of P / dS) therefore starts at:
-__device__ __forceinline__ uint32_t packed_col(int kk) { return 8u * kk + (kk >= 4 ? 32u : 0u); }
+// Packed bf16 P / dS columns: compute warp half h owns the 32 columns 32h .. 32h + 31 of a
+// 64-column sub-tile buffer and writes their 16 packed columns at 32h .. 32h + 15, i.e. over its
+// own consumed S / dP columns, so the two warps sharing a lane quarter never touch each other's
+// unread columns.  The tensor-memory A operand of K-step kk (16 rows of P / dS) starts at:
+__device__ __forceinline__ uint32_t packed_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
 __device__ __forceinline__ bool bwd_warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const bool ok = mbar_wait(bar, parity, w);
@@ -195,8 +204,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::kBarOff;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 1,
-            B_DONE = B_PREADY + 1, B_FIN = B_DONE + 1;
+  const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 2,
+            B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -216,8 +225,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(B_FULL + s), 1);
       mbar_init(bar(B_EMPTY + s), 1);
     }
-    mbar_init(bar(B_SFULL), 1);
-    mbar_init(bar(B_PREADY), kComputeThreads);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(B_SFULL + u), 1);
+      mbar_init(bar(B_PREADY + u), kComputeThreads);
+    }
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
@@ -277,7 +288,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     const bool leader = elect_one_sync();
-    constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kBT, false);   // M = 128, N = 128, both K-major
+    constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kSub, false);  // M = 128 keys, N = 64 queries, K-major
     constexpr uint32_t idesc_ts = idesc_bf16_f32(kBT, D, true);      // M = 128, N = D, B MN-major
     constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
     const uint64_t dK = sdesc_sw128(sRes(0), 16, 1024), dV = sdesc_sw128(sRes(1), 16, 1024);
@@ -295,34 +306,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) mma_ss(tmem + d_col, a0 + off, b0 + off, idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
-    // D_t (+)= A (tensor memory, bf16 pairs, 128 x 128) times B MN-major (128 rows x D)
+    // D_t (+)= A (tensor memory, packed bf16, 128 x 64) times B MN-major (64 rows x D)
     auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
 #pragma unroll
-      for (int kk = 0; kk < kBT / 16; ++kk)
+      for (int kk = 0; kk < kSub / 16; ++kk)
         if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
+    // Sub-tile t = 2i + hh is rows 64hh .. 64hh+63 of query tile i, in score buffer t & 1.  The
+    // products of sub-tile t are issued before waiting for the compute warps on sub-tile t-1:
+    // buffer t & 1 was last read by sub-tile t-2, whose P^T / dS^T products were issued (and so
+    // execute) before these.
+    const int n_sub = 2 * nq;
     bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
-    for (int i = 0; ok && i <= nq; ++i) {
-      const int s = i % kStages;
-      if (i < nq && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
-      if (i > 0) {
-        // tile i-1: P^T and dS^T are in tensor memory
-        if (!bwd_warp_wait(bar(B_PREADY), (i - 1) & 1, wc)) break;
+    for (int t = 0; ok && t <= n_sub; ++t) {
+      if (t < n_sub) {
+        const int i = t >> 1, hh = t & 1, s = i % kStages;
+        if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
         tc_fence_after();
-        const int sp = (i - 1) % kStages;
-        issue_ts(kColAcc0, kColS, dOmn + stage_off(sp), i > 1);    // dV += P^T dO
-        issue_ts(kColAcc1, kColDP, dQmn + stage_off(sp), i > 1);   // dK += dS^T Q
-        if (leader) tc_commit(bar(B_EMPTY + sp));
+        const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
+        issue_ss(col_s(t & 1), dK, dQk + sub);    // S^T = K Q_sub^T
+        issue_ss(col_dp(t & 1), dV, dOk + sub);   // dP^T = V dO_sub^T
+        if (leader) tc_commit(bar(B_SFULL + (t & 1)));
       }
-      if (i < nq) {
+      if (t > 0) {
+        const int tp = t - 1, ip = tp >> 1, hp = tp & 1, sp = ip % kStages;
+        if (!bwd_warp_wait(bar(B_PREADY + (tp & 1)), (tp >> 1) & 1, wc)) break;
         tc_fence_after();
-        issue_ss(kColS, dK, dQk + stage_off(s));    // S^T = K Q^T
-        issue_ss(kColDP, dV, dOk + stage_off(s));   // dP^T = V dO^T
-        if (leader) tc_commit(bar(B_SFULL));
-      } else if (leader) {
-        tc_commit(bar(B_DONE));
+        const uint64_t sub = stage_off(sp) + (hp ? kSubDescOff : 0);
+        issue_ts(kColAcc0, col_s(tp & 1), dOmn + sub, tp > 0);    // dV += P^T dO_sub
+        issue_ts(kColAcc1, col_dp(tp & 1), dQmn + sub, tp > 0);   // dK += dS^T Q_sub
+        if (hp == 1 && leader) tc_commit(bar(B_EMPTY + sp));    // both halves of tile ip consumed
       }
+      if (t == n_sub && leader) tc_commit(bar(B_DONE));
     }
     if (leader) tc_commit(bar(B_FIN));
     mbar_drain(bar(B_FIN), 0, p.timeout_ns);
@@ -332,28 +348,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;                    // key row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kColS, tP = tmem + lane_base + kColDP;
     bool ok = true;
-    for (int i = 0; i < nq; ++i) {
-      if (!bwd_warp_wait(bar(B_SFULL), i & 1, wc)) { ok = false; break; }
+    for (int t = 0; t < 2 * nq; ++t) {
+      const int i = t >> 1, hh = t & 1, bb = t & 1;
+      if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (i % kStages) * C::kVecBytes);
-      const int valid_q = min(kBT, p.n - i * kBT);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {   // this warp's two 32-column chunks, in order
-        const int c = 2 * half + u;
-        uint32_t s[32], dp[32];
-        tmem_ld32(tS + 32 * c, s);
-        tmem_ld32(tP + 32 * c, dp);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
-        bwd_chunk<true>(s, dp, p.scale_log2, vec + 32 * c, vec + kBT + 32 * c, 0.f, 0.f, valid_q - 32 * c, pk, dk);
-        tmem_st16(tS + 64 * half + 16 * u, pk);    // P^T over this warp's consumed S^T columns
-        tmem_st16(tP + 64 * half + 16 * u, dk);    // dS^T over this warp's consumed dP^T columns
-      }
+      const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (i % kStages) * C::kVecBytes) +
+                         kSub * hh + 32 * half;
+      const int valid_q = p.n - (i * kBT + kSub * hh + 32 * half);   // of this warp's 32 query columns
+      const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
+      uint32_t s[32], dp[32];
+      tmem_ld32(tS, s);
+      tmem_ld32(tP, dp);
+      tmem_wait_ld();
+      uint32_t pk[16], dk[16];
+      bwd_chunk<true>(s, dp, p.scale_log2, vec, vec + kBT, 0.f, 0.f, valid_q, pk, dk);
+      tmem_st16(tS, pk);    // P^T over this warp's consumed S^T columns
+      tmem_st16(tP, dk);    // dS^T over this warp's consumed dP^T columns
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_PREADY));
+      mbar_arrive(bar(B_PREADY + bb));
     }
     if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
       tc_fence_after();
@@ -388,8 +402,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::kBarOff;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 1,
-            B_DONE = B_PREADY + 1, B_FIN = B_DONE + 1;
+  const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 2,
+            B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -408,8 +422,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(B_FULL + s), 1);
       mbar_init(bar(B_EMPTY + s), 1);
     }
-    mbar_init(bar(B_SFULL), 1);
-    mbar_init(bar(B_PREADY), kComputeThreads);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(B_SFULL + u), 1);
+      mbar_init(bar(B_PREADY + u), kComputeThreads);
+    }
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
     *abort_flag = 0;
@@ -463,7 +479,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     const bool leader = elect_one_sync();
-    constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kBT, false);
+    constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kSub, false);  // M = 128 queries, N = 64 keys
     constexpr uint32_t idesc_ts = idesc_bf16_f32(kBT, D, true);
     constexpr uint64_t kTileStep = (uint64_t)(C::kTileBytes >> 4);
     const uint64_t dQ = sdesc_sw128(sRes(0), 16, 1024), dO = sdesc_sw128(sRes(1), 16, 1024);
@@ -480,29 +496,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
 #pragma unroll
-      for (int kk = 0; kk < kBT / 16; ++kk)
+      for (int kk = 0; kk < kSub / 16; ++kk)
         if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
+    // sub-tile t = 2j + hh: keys 64hh .. 64hh+63 of key tile j, score buffer t & 1 (as dK/dV)
+    const int n_sub = 2 * nk;
     bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
-    for (int j = 0; ok && j <= nk; ++j) {
-      const int s = j % kStages;
-      if (j < nk && !bwd_warp_wait(bar(B_FULL + s), (j / kStages) & 1, wc)) break;
-      if (j > 0) {
-        if (!bwd_warp_wait(bar(B_PREADY), (j - 1) & 1, wc)) break;
+    for (int t = 0; ok && t <= n_sub; ++t) {
+      if (t < n_sub) {
+        const int j = t >> 1, hh = t & 1, s = j % kStages;
+        if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (j / kStages) & 1, wc)) break;
         tc_fence_after();
-        const int sp = (j - 1) % kStages;
-        issue_ts(kColAcc0, kColDP, dKmn + stage_off(sp), j > 1);   // dQ += dS K
-        if (leader) tc_commit(bar(B_EMPTY + sp));
+        const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
+        issue_ss(col_s(t & 1), dQ, dKk + sub);    // S = Q K_sub^T
+        issue_ss(col_dp(t & 1), dO, dVk + sub);   // dP = dO V_sub^T
+        if (leader) tc_commit(bar(B_SFULL + (t & 1)));
       }
-      if (j < nk) {
+      if (t > 0) {
+        const int tp = t - 1, jp = tp >> 1, hp = tp & 1, sp = jp % kStages;
+        if (!bwd_warp_wait(bar(B_PREADY + (tp & 1)), (tp >> 1) & 1, wc)) break;
         tc_fence_after();
-        issue_ss(kColS, dQ, dKk + stage_off(s));    // S = Q K^T
-        issue_ss(kColDP, dO, dVk + stage_off(s));   // dP = dO V^T
-        if (leader) tc_commit(bar(B_SFULL));
-      } else if (leader) {
-        tc_commit(bar(B_DONE));
+        issue_ts(kColAcc0, col_dp(tp & 1), dKmn + stage_off(sp) + (hp ? kSubDescOff : 0), tp > 0);   // dQ += dS K_sub
+        if (hp == 1 && leader) tc_commit(bar(B_EMPTY + sp));
       }
+      if (t == n_sub && leader) tc_commit(bar(B_DONE));
     }
     if (leader) tc_commit(bar(B_FIN));
     mbar_drain(bar(B_FIN), 0, p.timeout_ns);
@@ -511,31 +529,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;                    // query row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_base + kColS, tP = tmem + lane_base + kColDP;
     const int qs = q0 + row;
     const bool live = qs < p.n;
     const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
     const float lse_r = live ? p.lse[vec_row + qs] : 0.f;
     const float dv_r = live ? p.dvec[vec_row + qs] : 0.f;
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
-      if (!bwd_warp_wait(bar(B_SFULL), j & 1, wc)) { ok = false; break; }
+    for (int t = 0; t < 2 * nk; ++t) {
+      const int j = t >> 1, hh = t & 1, bb = t & 1;
+      if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      const int valid_k = min(kBT, p.n - j * kBT);
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {   // this warp's two 32-column chunks, in order
-        const int c = 2 * half + u;
-        uint32_t s[32], dp[32];
-        tmem_ld32(tS + 32 * c, s);
-        tmem_ld32(tP + 32 * c, dp);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
-        bwd_chunk<false>(s, dp, p.scale_log2, nullptr, nullptr, lse_r, dv_r, live ? valid_k - 32 * c : 0, pk, dk);
-        tmem_st16(tP + 64 * half + 16 * u, dk);    // dS over this warp's consumed dP columns
-      }
+      const int valid_k = p.n - (j * kBT + kSub * hh + 32 * half);   // of this warp's 32 key columns
+      const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
+      uint32_t s[32], dp[32];
+      tmem_ld32(tS, s);
+      tmem_ld32(tP, dp);
+      tmem_wait_ld();
+      uint32_t pk[16], dk[16];
+      bwd_chunk<false>(s, dp, p.scale_log2, nullptr, nullptr, lse_r, dv_r, live ? valid_k : 0, pk, dk);
+      tmem_st16(tP, dk);    // dS over this warp's consumed dP columns
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_PREADY));
+      mbar_arrive(bar(B_PREADY + bb));
     }
     if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
       tc_fence_after();
