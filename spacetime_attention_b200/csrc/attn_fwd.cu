@@ -61,6 +61,7 @@ constexpr int kQkWarp = 10;
 constexpr int kPv1Warp = 11;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPersistMaxTiles = 32;       // KV tiles per item up to which CTAs run items in turn
 
 // Tuning switches (compile-time; the defaults are the measured best on B200: alternating the
 // softmax groups cost 4 % at d=64; the polynomial share pays only at d=128, where MUFU and the
@@ -99,7 +100,7 @@ struct Cfg {
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
   // o_full[2], mma_done, s_free[2], turn[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 13;
+  static constexpr int kNumBars = 1 + 4 * kStages + 16;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -136,6 +137,7 @@ struct AttnParams {
   int qblocks;            // 256-row query blocks per (sample*set, head)
   int n_full;
   int n_split;
+  int n_items;            // work items (whole units, then split parts); CTA c runs items c, c + grid, ...
   float* ws_o;            // [split units][n_split][256][D]
   float2* ws_ml;          // [split units][n_split][256]
 };
@@ -257,7 +259,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int kMode>
+// kLoop: the CTA runs work items blockIdx.x, blockIdx.x + gridDim.x, ... (grid smaller than the
+// item count); otherwise exactly item blockIdx.x, and every cross-item wait folds away.
+template <int D, int kMode, bool kLoop>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p,
@@ -279,6 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int B_TURN = B_SFREE + 2;     // softmax i may start its exponentials (MUFU hand-off)
   const int B_QKDONE = B_TURN + 2;    // split MMA issue: the QK^T warp's final commit
   const int B_PV1DONE = B_QKDONE + 1; // split MMA issue: the tile-1 PV warp's final commit
+  // A CTA may run several work items in turn (grid smaller than the item count):
+  const int B_QEMPTY = B_PV1DONE + 1; // Q may be overwritten: every QK^T of the item has completed
+  const int B_OFREE = B_QEMPTY + 1;   // [2] the softmax has read O_i out (the next item may overwrite it)
   constexpr bool kSplitMma = C::kSepP && OSP_SPLIT_MMA > 0;
   constexpr bool kSplitPv = C::kSepP && OSP_SPLIT_MMA > 1;
   // per-tile issuers (9 and 11) pay at d = 96 (+2 %); at d = 128 the tensor pipe is the bottleneck
@@ -293,9 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // q_row0 / kv_row0 offset the rows of a packed segment; nq / nkv are the set's query and key
   // rows.  Recomputed where needed (cheap integer math) rather than kept live across the main loops.
   struct Work { int unit, part, h, b, g, q0, kv_lo, n_kv, q_row0, kv_row0, nq, nkv, q_out0; };
-  auto decode = [&]() {
+  auto decode = [&](int item) {
     Work w;
-    w.unit = blockIdx.x;
+    w.unit = item;
     w.part = -1;
     int qb;
     if constexpr (kPacked) {
@@ -360,6 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_SFREE + 1), 128);
     mbar_init(bar(B_QKDONE), 1);
     mbar_init(bar(B_PV1DONE), 1);
+    mbar_init(bar(B_QEMPTY), kSplitTiles ? 2 : 1);   // each QK^T issuing warp commits once per item
+    mbar_init(bar(B_OFREE + 0), 128);
+    mbar_init(bar(B_OFREE + 1), 128);
     mbar_init(bar(B_TURN + 0), 128);
     mbar_init(bar(B_TURN + 1), 128);
     *abort_flag = 0;
@@ -397,9 +407,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
-  const Work wk = decode();
-  const int n_kv = wk.n_kv;
-  const int chan0 = wk.h * D;
   // KV tile jj of this unit's range: with a joined text prefix the first tiles come from the
   // text maps (dense rows), the rest from the set's own map.
   auto load_kv_tile = [&](const CUtensorMap& tm, const SegParam<kMode>& sp, uint32_t dst, uint32_t mbar, int chan,
@@ -431,35 +438,46 @@ __global__ void __launch_bounds__(kThreads, 1)
    if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
     {
-      int k_issued = 0, v_issued = 0;  // K / V tiles whose loads were issued
+      // K / V tiles are counted over all of this CTA's items (the rings continue across items)
+      int k_issued = 0, v_issued = 0, q_issued = 0, jb = 0;
       const bool q_armed = !p.debug_withhold_q;
-      if (leader && q_armed) {
-        mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
-        for (int i = 0; i < 2; ++i)
-          for (int c = 0; c < C::kChunks; ++c)
-            load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, chan0 + 64 * c, wk.q_row0 + wk.q0 + i * kBM, wk.g, wk.b,
-                      p.k);
-      }
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % S, u = j / S;
-        if (j >= S && !warp_wait(bar(B_KEMPTY + s), (u - 1) & 1, wc)) break;
-        if (leader) {
-          mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
-          for (int c = 0; c < C::kChunks; ++c)
-            load_kv_tile(tm_k, seg, sK(s) + c * kChunkBytes, bar(B_KFULL + s), chan0 + 64 * c, wk.kv_lo + j, wk, true);
+      bool ok = true;
+      for (int item = blockIdx.x, ub = 0; ok && (kLoop ? item < p.n_items : ub == 0); item += gridDim.x, ++ub) {
+        const Work w = decode(item);
+        const int c0 = w.h * D;
+        // the previous item's Q may be overwritten once its last QK^T has completed
+        if (ub > 0 && !warp_wait(bar(B_QEMPTY), (ub - 1) & 1, wc)) break;
+        if (leader && q_armed) {
+          mbar_arrive_expect_tx(bar(B_QFULL), 2 * C::kTileBytes);
+          for (int i = 0; i < 2; ++i)
+            for (int c = 0; c < C::kChunks; ++c)
+              load_tile(&tm_q, sQ(i) + c * kChunkBytes, bar(B_QFULL), p.layout, c0 + 64 * c,
+                        w.q_row0 + w.q0 + i * kBM, w.g, w.b, p.k);
         }
-        k_issued = j + 1;
-        if (j >= S && !warp_wait(bar(B_VEMPTY + s), (u - 1) & 1, wc)) break;
-        if (leader) {
-          mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
-          for (int c = 0; c < C::kChunks; ++c)
-            load_kv_tile(tm_v, seg, sV(s) + c * kChunkBytes, bar(B_VFULL + s), chan0 + 64 * c, wk.kv_lo + j, wk, false);
+        q_issued = ub + 1;
+        for (int j = 0; j < w.n_kv; ++j) {
+          const int jg = jb + j, s = jg % S, u = jg / S;
+          if (jg >= S && !warp_wait(bar(B_KEMPTY + s), (u - 1) & 1, wc)) { ok = false; break; }
+          if (leader) {
+            mbar_arrive_expect_tx(bar(B_KFULL + s), C::kTileBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              load_kv_tile(tm_k, seg, sK(s) + c * kChunkBytes, bar(B_KFULL + s), c0 + 64 * c, w.kv_lo + j, w, true);
+          }
+          k_issued = jg + 1;
+          if (jg >= S && !warp_wait(bar(B_VEMPTY + s), (u - 1) & 1, wc)) { ok = false; break; }
+          if (leader) {
+            mbar_arrive_expect_tx(bar(B_VFULL + s), C::kTileBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              load_kv_tile(tm_v, seg, sV(s) + c * kChunkBytes, bar(B_VFULL + s), c0 + 64 * c, w.kv_lo + j, w, false);
+          }
+          v_issued = jg + 1;
         }
-        v_issued = j + 1;
+        jb += w.n_kv;
       }
-      // Drain: every load issued has landed before the CTA may exit.  Only the last S tiles of
-      // each ring can still be in flight.
-      if (q_armed) mbar_drain(bar(B_QFULL), 0, p.timeout_ns);
+      // Drain: every load issued has landed before the CTA may exit.  A Q load is issued only
+      // after the previous one was consumed, and only the last S tiles of each ring can still be
+      // in flight.
+      if (q_armed && q_issued > 0) mbar_drain(bar(B_QFULL), (q_issued - 1) & 1, p.timeout_ns);
       for (int t = (k_issued > S ? k_issued - S : 0); t < k_issued; ++t)
         mbar_drain(bar(B_KFULL + t % S), (t / S) & 1, p.timeout_ns);
       for (int t = (v_issued > S ? v_issued - S : 0); t < v_issued; ++t)
@@ -499,117 +517,150 @@ __global__ void __launch_bounds__(kThreads, 1)
                    (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = warp_wait(bar(B_QFULL), 0, wc) && warp_wait(bar(B_KFULL), 0, wc);
       // which MMAs this warp issues (one warp issues all of them unless the issue is split)
       const bool do_qk = !kSplitMma || warp == kQkWarp;
       const bool do_pv0 = !kSplitMma || warp == kMmaWarp;
       const bool do_pv1 = !kSplitMma || (kSplitPv ? warp == kPv1Warp : warp == kMmaWarp);
-      if (ok && C::kSepP) {
-        // Order per KV tile j: S0(j+1) as soon as softmax 0 holds S0(j) in registers, S1(j+1)
-        // likewise, then PV0(j), PV1(j) as their P tiles arrive.  O_full[i] completes after every
-        // PV_i(j): the softmax waits on it before overwriting P_i and before touching O_i.
-        tc_fence_after();
-        if (do_qk) {
-          issue_s(0, 0);
-          if (leader) tc_commit(bar(B_SFULL + 0));
-          issue_s(1, 0);
-          if (leader) tc_commit(bar(B_SFULL + 1));
-          if (leader) tc_commit(bar(B_KEMPTY + 0));
+      // KV tiles are counted over all of this CTA's items (jg = jb + j), as by the producer and
+      // the softmax warps; per-item barriers (Q full / empty, O free) by the item count ub.
+      int jb = 0;
+      bool ok = true;
+      for (int item = blockIdx.x, ub = 0; ok && (kLoop ? item < p.n_items : ub == 0); item += gridDim.x, ++ub) {
+        const int n_kv = decode(item).n_kv;
+        const int s0 = jb % S;
+        // Q and the item's first K tile, for the warps that issue QK^T (a PV-only warp never reads
+        // them and must not wait on phases it could fall behind on)
+        if ((!C::kSepP || do_qk) &&
+            (!warp_wait(bar(B_QFULL), ub & 1, wc) || !warp_wait(bar(B_KFULL + s0), (jb / S) & 1, wc))) {
+          ok = false;
+          break;
         }
-        for (int j = 0; j < n_kv; ++j) {
-          const int s = j % S, u = j / S;
-          const bool more = j + 1 < n_kv;
-          const int s1 = (j + 1) % S, u1 = (j + 1) / S;
-          if (do_qk && more) {
-            if (!warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
-            if (!warp_wait(bar(B_SFREE + 0), j & 1, wc)) break;
+        if (C::kSepP) {
+          // Order per KV tile j: S0(j+1) as soon as softmax 0 holds S0(j) in registers, S1(j+1)
+          // likewise, then PV0(j), PV1(j) as their P tiles arrive.  O_full[i] completes after every
+          // PV_i(j): the softmax waits on it before overwriting P_i and before touching O_i.
+          tc_fence_after();
+          if (do_qk) {
+            // S_i of the previous item's last tile must be out of tensor memory
+            if (ub > 0 && !warp_wait(bar(B_SFREE + 0), (jb - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            issue_s(0, s1);
+            issue_s(0, s0);
             if (leader) tc_commit(bar(B_SFULL + 0));
-            if (!warp_wait(bar(B_SFREE + 1), j & 1, wc)) break;
+            if (ub > 0 && !warp_wait(bar(B_SFREE + 1), (jb - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            issue_s(1, s1);
+            issue_s(1, s0);
             if (leader) tc_commit(bar(B_SFULL + 1));
-            if (leader) tc_commit(bar(B_KEMPTY + s1));
+            if (leader) tc_commit(bar(B_KEMPTY + s0));
+            if (n_kv == 1 && leader) tc_commit(bar(B_QEMPTY));
           }
-          if (do_pv0 || do_pv1) {
-            if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
+          for (int j = 0; j < n_kv; ++j) {
+            const int jg = jb + j, s = jg % S, u = jg / S;
+            const bool more = j + 1 < n_kv;
+            const int s1 = (jg + 1) % S, u1 = (jg + 1) / S;
+            if (do_qk && more) {
+              if (!warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) { ok = false; break; }
+              if (!warp_wait(bar(B_SFREE + 0), jg & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(0, s1);
+              if (leader) tc_commit(bar(B_SFULL + 0));
+              if (!warp_wait(bar(B_SFREE + 1), jg & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(1, s1);
+              if (leader) tc_commit(bar(B_SFULL + 1));
+              if (leader) tc_commit(bar(B_KEMPTY + s1));
+              if (j + 2 == n_kv && leader) tc_commit(bar(B_QEMPTY));
+            }
+            if (do_pv0 || do_pv1) {
+              if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) { ok = false; break; }
+            }
+            if (do_pv0) {
+              if (!warp_wait(bar(B_PREADY + 0), jg & 1, wc)) { ok = false; break; }
+              // the first PV of an item overwrites O_0: the previous item's epilogue has read it
+              if (j == 0 && ub > 0 && !warp_wait(bar(B_OFREE + 0), (ub - 1) & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv(0, s, j > 0);
+              if (leader) tc_commit(bar(B_OFULL + 0));
+              if (kSplitPv && leader) tc_commit(bar(B_VEMPTY + s));
+            }
+            if (do_pv1) {
+              if (!warp_wait(bar(B_PREADY + 1), jg & 1, wc)) { ok = false; break; }
+              if (j == 0 && ub > 0 && !warp_wait(bar(B_OFREE + 1), (ub - 1) & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv(1, s, j > 0);
+              if (leader) tc_commit(bar(B_OFULL + 1));
+              if (leader) tc_commit(bar(B_VEMPTY + s));
+            }
           }
-          if (do_pv0) {
-            if (!warp_wait(bar(B_PREADY + 0), j & 1, wc)) break;
+        } else if (kSplitTiles) {
+          // P inside S: per tile, PV_i(j) must precede S_i(j+1) (the tensor pipe runs one thread's
+          // MMAs in order); the two tiles are independent, so each has its own issuing warp.
+          // The first S_i of an item follows the previous item's last PV_i in this warp's order.
+          const int ti = (warp == kPv1Warp) ? 1 : 0;
+          tc_fence_after();
+          issue_s(ti, s0);
+          if (leader) tc_commit(bar(B_SFULL + ti));
+          if (leader) tc_commit(bar(B_KEMPTY + s0));
+          if (n_kv == 1 && leader) tc_commit(bar(B_QEMPTY));
+          for (int j = 0; j < n_kv; ++j) {
+            const int jg = jb + j, s = jg % S, u = jg / S;
+            const bool more = j + 1 < n_kv;
+            const int s1 = (jg + 1) % S, u1 = (jg + 1) / S;
+            if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) { ok = false; break; }
+            if (more && !warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) { ok = false; break; }
+            if (!warp_wait(bar(B_PREADY + ti), jg & 1, wc)) { ok = false; break; }
+            if (j == 0 && ub > 0 && !warp_wait(bar(B_OFREE + ti), (ub - 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(ti, s, j > 0);
+            if (leader) tc_commit(bar(B_VEMPTY + s));
+            if (more) {
+              issue_s(ti, s1);
+              if (leader) tc_commit(bar(B_SFULL + ti));
+              if (leader) tc_commit(bar(B_KEMPTY + s1));
+              if (j + 2 == n_kv && leader) tc_commit(bar(B_QEMPTY));
+            } else {
+              if (leader) tc_commit(bar(B_OFULL + ti));
+            }
+          }
+        } else {
+          tc_fence_after();
+          issue_s(0, s0);
+          if (leader) tc_commit(bar(B_SFULL + 0));
+          issue_s(1, s0);
+          if (leader) tc_commit(bar(B_SFULL + 1));
+          if (leader) tc_commit(bar(B_KEMPTY + s0));
+          if (n_kv == 1 && leader) tc_commit(bar(B_QEMPTY));
+          for (int j = 0; j < n_kv; ++j) {
+            const int jg = jb + j, s = jg % S, u = jg / S;
+            const bool more = j + 1 < n_kv;
+            const int s1 = (jg + 1) % S, u1 = (jg + 1) / S;
+            if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) { ok = false; break; }
+            if (more && !warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) { ok = false; break; }
+            if (!warp_wait(bar(B_PREADY + 0), jg & 1, wc)) { ok = false; break; }
+            if (j == 0 && ub > 0 && !warp_wait(bar(B_OFREE + 0), (ub - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
             issue_pv(0, s, j > 0);
-            if (leader) tc_commit(bar(B_OFULL + 0));
-            if (kSplitPv && leader) tc_commit(bar(B_VEMPTY + s));
-          }
-          if (do_pv1) {
-            if (!warp_wait(bar(B_PREADY + 1), j & 1, wc)) break;
+            if (more) {
+              issue_s(0, s1);
+              if (leader) tc_commit(bar(B_SFULL + 0));
+            } else {
+              if (leader) tc_commit(bar(B_OFULL + 0));
+            }
+            if (!warp_wait(bar(B_PREADY + 1), jg & 1, wc)) { ok = false; break; }
+            if (j == 0 && ub > 0 && !warp_wait(bar(B_OFREE + 1), (ub - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
             issue_pv(1, s, j > 0);
-            if (leader) tc_commit(bar(B_OFULL + 1));
             if (leader) tc_commit(bar(B_VEMPTY + s));
+            if (more) {
+              issue_s(1, s1);
+              if (leader) tc_commit(bar(B_SFULL + 1));
+              if (leader) tc_commit(bar(B_KEMPTY + s1));
+              if (j + 2 == n_kv && leader) tc_commit(bar(B_QEMPTY));
+            } else {
+              if (leader) tc_commit(bar(B_OFULL + 1));
+            }
           }
         }
-      } else if (ok && kSplitTiles) {
-        // P inside S: per tile, PV_i(j) must precede S_i(j+1) (the tensor pipe runs one thread's
-        // MMAs in order); the two tiles are independent, so each has its own issuing warp.
-        const int ti = (warp == kPv1Warp) ? 1 : 0;
-        tc_fence_after();
-        issue_s(ti, 0);
-        if (leader) tc_commit(bar(B_SFULL + ti));
-        if (leader) tc_commit(bar(B_KEMPTY + 0));
-        for (int j = 0; j < n_kv; ++j) {
-          const int s = j % S, u = j / S;
-          const bool more = j + 1 < n_kv;
-          const int s1 = (j + 1) % S, u1 = (j + 1) / S;
-          if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
-          if (more && !warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
-          if (!warp_wait(bar(B_PREADY + ti), j & 1, wc)) break;
-          tc_fence_after();
-          issue_pv(ti, s, j > 0);
-          if (leader) tc_commit(bar(B_VEMPTY + s));
-          if (more) {
-            issue_s(ti, s1);
-            if (leader) tc_commit(bar(B_SFULL + ti));
-            if (leader) tc_commit(bar(B_KEMPTY + s1));
-          } else {
-            if (leader) tc_commit(bar(B_OFULL + ti));
-          }
-        }
-      } else if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        if (leader) tc_commit(bar(B_SFULL + 0));
-        issue_s(1, 0);
-        if (leader) tc_commit(bar(B_SFULL + 1));
-        if (leader) tc_commit(bar(B_KEMPTY + 0));
-        for (int j = 0; j < n_kv; ++j) {
-          const int s = j % S, u = j / S;
-          const bool more = j + 1 < n_kv;
-          const int s1 = (j + 1) % S, u1 = (j + 1) / S;
-          if (!warp_wait(bar(B_VFULL + s), u & 1, wc)) break;
-          if (more && !warp_wait(bar(B_KFULL + s1), u1 & 1, wc)) break;
-          if (!warp_wait(bar(B_PREADY + 0), j & 1, wc)) break;
-          tc_fence_after();
-          issue_pv(0, s, j > 0);
-          if (more) {
-            issue_s(0, s1);
-            if (leader) tc_commit(bar(B_SFULL + 0));
-          } else {
-            if (leader) tc_commit(bar(B_OFULL + 0));
-          }
-          if (!warp_wait(bar(B_PREADY + 1), j & 1, wc)) break;
-          tc_fence_after();
-          issue_pv(1, s, j > 0);
-          if (leader) tc_commit(bar(B_VEMPTY + s));
-          if (more) {
-            issue_s(1, s1);
-            if (leader) tc_commit(bar(B_SFULL + 1));
-            if (leader) tc_commit(bar(B_KEMPTY + s1));
-          } else {
-            if (leader) tc_commit(bar(B_OFULL + 1));
-          }
-        }
+        jb += n_kv;
       }
       // Drain: all issued MMAs complete before tensor memory is freed.
       const int done_bar = (kSplitMma && warp == kQkWarp) ? B_QKDONE
@@ -630,14 +681,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + colO(i);
     const uint32_t tP = tmem + lane_base + colP(i);
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
+    int jb = 0;   // KV tiles of this CTA's earlier items
+    for (int item = blockIdx.x, ub = 0; ok && (kLoop ? item < p.n_items : ub == 0); item += gridDim.x, ++ub) {
+    const Work wk = decode(item);
+    const int n_kv = wk.n_kv;
+    float m = -INFINITY, l = 0.f;
     int lim = wk.nkv;                                // keys this row may see
     if constexpr (kFrameCausal)
       lim = min(lim, frame_causal_limit(wk.q0 + i * kBM + row, p.text_len, p.frame_hw));
-    const int valid0 = lim - wk.kv_lo * kBN;         // valid keys from this CTA's first KV tile on
+    const int valid0 = lim - wk.kv_lo * kBN;         // valid keys from this item's first KV tile on
     for (int j = 0; j < n_kv; ++j) {
-      if (!warp_wait(bar(B_SFULL + i), j & 1, wc)) { ok = false; break; }
+      const int jg = jb + j;
+      if (!warp_wait(bar(B_SFULL + i), jg & 1, wc)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -683,8 +739,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The two softmax groups take turns on MUFU: group 0 runs the exponentials of tile j after
       // group 1 finished those of tile j-1, group 1 after group 0 finished tile j.  Each group's
       // load / max / store phases overlap the other group's exponentials.
-      if (OSP_SOFTMAX_TURNS && (i == 1 || j > 0)) {
-        if (!warp_wait(bar(B_TURN + i), (uint32_t)((i == 0 ? j - 1 : j) & 1), wc)) { ok = false; break; }
+      if (OSP_SOFTMAX_TURNS && (i == 1 || jg > 0)) {
+        if (!warp_wait(bar(B_TURN + i), (uint32_t)((i == 0 ? jg - 1 : jg) & 1), wc)) { ok = false; break; }
       }
       uint32_t pk[64];
       const float rs = masked ? softmax_exp_row<C::kPolyPer16, false>(sv, sl2, m, pk)
@@ -694,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P_i (and O_i) are free once PV_i(j-1) has completed (separate-P layout; with P inside S
       // the MMA warp already ordered it)
       if constexpr (C::kSepP) {
-        if (j > 0 && !warp_wait(bar(B_OFULL + i), (j - 1) & 1, wc)) { ok = false; break; }
+        if (j > 0 && !warp_wait(bar(B_OFULL + i), (jg - 1) & 1, wc)) { ok = false; break; }
         tc_fence_after();
       }
       tmem_st32(tP + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
@@ -714,9 +770,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(B_PREADY + i));
     }
-    if (ok && warp_wait(bar(B_OFULL + i), C::kSepP ? (uint32_t)((n_kv - 1) & 1) : 0u, wc)) {
+    if (!ok) break;
+    // O_i complete: per tile in the separate-P layout, once per item otherwise
+    if (!warp_wait(bar(B_OFULL + i), C::kSepP ? (uint32_t)((jb + n_kv - 1) & 1) : (uint32_t)(ub & 1), wc)) {
+      ok = false;
+      break;
+    }
+    {
       tc_fence_after();
-      const Work w = decode();
+      const Work w = decode(item);
       const int unit = w.unit, part = w.part, h = w.h, b = w.b, g = w.g;
       const float inv_l = 1.f / l;
       const int slot = w.q0 + i * kBM + row;
@@ -759,6 +821,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       }
     }
+    tc_fence_before();
+    mbar_arrive(bar(B_OFREE + i));   // O_i is read out: the next item's first PV may overwrite it
+    jb += n_kv;
+    }   // items
   }
   tc_fence_before();
   __syncthreads();
@@ -867,7 +933,7 @@ int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int l
   return OSP_OK;
 }
 
-template <int D, int kMode>
+template <int D, int kMode, bool kLoop = false>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
              const SegParam<kMode>& seg, dim3 grid, cudaStream_t stream) {
   constexpr int smem = Cfg<D>::kSmemBytes;
@@ -876,16 +942,16 @@ int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
     // The warpgroup register split only adds up if the kernel is launched with exactly
     // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode>) != cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode, kLoop>) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncGetAttributes(attn_fwd_kernel<%d>) failed", D);
     if ((uint32_t)fa.numRegs != kRegsLaunch)
       return set_error(OSP_ERR_CUDA, "attn_fwd_kernel<%d> compiled to %d registers per thread, expected %u", D,
                        fa.numRegs, kRegsLaunch);
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kMode, kLoop>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_fwd_kernel<%d>) failed", D);
     attr_done = true;
   }
-  attn_fwd_kernel<D, kMode><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
+  attn_fwd_kernel<D, kMode, kLoop><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
   return check_launch("attn_fwd_kernel");
 }
 
@@ -931,12 +997,31 @@ int run_units(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& t
     p.ws_ml = reinterpret_cast<float2*>(p.ws_o + rows * (size_t)head_dim);
   }
   const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
-  dim3 grid((unsigned)ctas);
+  p.n_items = (int)ctas;
+  // Short KV ranges: one CTA per SM runs items in turn, so an item's Q load and first QK^T
+  // overlap the previous item's softmax and epilogue (a fixed cost per item that a few KV tiles
+  // do not amortise).  Not with a split tail (its items differ in kind) or packed batches.
+  long long grid_ctas = ctas;
+  const int persist = persist_mode();
+  if (kMode != kModePacked && p.n_split == 1 &&
+      ((persist == 1 && n_kv_tiles <= kPersistMaxTiles && ctas >= 2LL * sms) || persist == 2))
+    grid_ctas = std::min<long long>(ctas, sms);
+  const bool loop = grid_ctas < ctas;
+  dim3 grid((unsigned)grid_ctas);
   int rc;
   switch (head_dim) {
-    case 64: rc = launch_d<64, kMode>(tq, tk, tv, p, extra, grid, stream); break;
-    case 96: rc = launch_d<96, kMode>(tq, tk, tv, p, extra, grid, stream); break;
-    case 128: rc = launch_d<128, kMode>(tq, tk, tv, p, extra, grid, stream); break;
+    case 64:
+      rc = loop ? launch_d<64, kMode, true>(tq, tk, tv, p, extra, grid, stream)
+                : launch_d<64, kMode, false>(tq, tk, tv, p, extra, grid, stream);
+      break;
+    case 96:
+      rc = loop ? launch_d<96, kMode, true>(tq, tk, tv, p, extra, grid, stream)
+                : launch_d<96, kMode, false>(tq, tk, tv, p, extra, grid, stream);
+      break;
+    case 128:
+      rc = loop ? launch_d<128, kMode, true>(tq, tk, tv, p, extra, grid, stream)
+                : launch_d<128, kMode, false>(tq, tk, tv, p, extra, grid, stream);
+      break;
     default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
   }
   if (rc == OSP_OK && p.n_split > 1) {
@@ -1110,6 +1195,7 @@ int packed_attention_launch(const void* q, const void* k, const void* v, void* o
   p.qblocks = 1;
   p.n_full = (int)units;
   p.n_split = 1;
+  p.n_items = (int)units;
   // the packed tensors are one sample of n_q_total (q, o) / n_kv_total (k, v) rows
   const osp_shape sh{1, 0, 1, 1, 1, heads, head_dim};
   CUtensorMap tq, tk, tv;

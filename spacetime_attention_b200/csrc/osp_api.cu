@@ -144,6 +144,12 @@ int split_kv_enabled() {
   return (e && e[0] == '0') ? 0 : 1;
 }
 
+int persist_mode() {
+  const char* e = getenv("OSP_PERSIST");
+  if (!e || !e[0]) return 1;
+  return e[0] == '0' ? 0 : (e[0] == '2' ? 2 : 1);
+}
+
 int debug_withhold_q() {
   const char* e = getenv("OSP_DEBUG_WITHHOLD_Q");
   return (e && e[0] == '1') ? 1 : 0;

@@ -41,6 +41,10 @@ cudaMemPool_t workspace_pool();
 // Split-KV of the last partial wave of attention CTAs (OSP_SPLIT_KV=0 disables; read per launch).
 int split_kv_enabled();
 
+// Attention CTAs running several work items in turn (OSP_PERSIST, read per launch): 1 (default)
+// for short KV ranges, 0 never, 2 always (where the launch allows it).
+int persist_mode();
+
 int rope3d_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_shape& s,
                   const osp_rope& rope, cudaStream_t stream);
 int skiparse_gather_launch(const void* const src[3], void* const dst[3], int n_tensors, const osp_shape& s,
