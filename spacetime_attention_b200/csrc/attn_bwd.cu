@@ -572,18 +572,13 @@ int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const C
                  const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, long long rows, long long ctas,
                  cudaStream_t stream) {
   constexpr int smem = BwdCfg<D>::kSmemBytes;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attention backward, d=%d) failed", D);
-    attr_done = true;
-  }
+  int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_bwd_dkdv_kernel<D>), smem, "attn_bwd_dkdv_kernel");
+  if (rc || (rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_bwd_dq_kernel<D>), smem, "attn_bwd_dq_kernel")))
+    return rc;
   const long long dblocks = std::min<long long>((rows + 255) / 256, (long long)device_sm_count() * 16);
   attn_bwd_dvec_kernel<D><<<(unsigned)dblocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                                  static_cast<const __nv_bfloat16*>(dout), p, rows);
-  int rc = check_launch("attn_bwd_dvec_kernel");
+  rc = check_launch("attn_bwd_dvec_kernel");
   if (rc) return rc;
   attn_bwd_dkdv_kernel<D><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
   if ((rc = check_launch("attn_bwd_dkdv_kernel"))) return rc;

@@ -937,20 +937,18 @@ template <int D, int kMode, bool kLoop = false>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
              const SegParam<kMode>& seg, dim3 grid, cudaStream_t stream) {
   constexpr int smem = Cfg<D>::kSmemBytes;
-  static bool attr_done = false;  // per process; the attribute is per function, not per device
-  if (!attr_done) {
-    // The warpgroup register split only adds up if the kernel is launched with exactly
-    // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
+  // The warpgroup register split only adds up if the kernel is launched with exactly
+  // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
+  static const int regs = [] {
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode, kLoop>) != cudaSuccess)
-      return set_error(OSP_ERR_CUDA, "cudaFuncGetAttributes(attn_fwd_kernel<%d>) failed", D);
-    if ((uint32_t)fa.numRegs != kRegsLaunch)
-      return set_error(OSP_ERR_CUDA, "attn_fwd_kernel<%d> compiled to %d registers per thread, expected %u", D,
-                       fa.numRegs, kRegsLaunch);
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kMode, kLoop>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_fwd_kernel<%d>) failed", D);
-    attr_done = true;
-  }
+    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMode, kLoop>) == cudaSuccess ? fa.numRegs : -1;
+  }();
+  if (regs < 0) return set_error(OSP_ERR_CUDA, "cudaFuncGetAttributes(attn_fwd_kernel<%d>) failed", D);
+  if ((uint32_t)regs != kRegsLaunch)
+    return set_error(OSP_ERR_CUDA, "attn_fwd_kernel<%d> compiled to %d registers per thread, expected %u", D, regs,
+                     kRegsLaunch);
+  int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_fwd_kernel<D, kMode, kLoop>), smem, "attn_fwd_kernel");
+  if (rc) return rc;
   attn_fwd_kernel<D, kMode, kLoop><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
   return check_launch("attn_fwd_kernel");
 }

@@ -244,13 +244,9 @@ int launch_temporal_t(TemporalParams& p, cudaStream_t stream) {
   // as many warps per CTA (<= 8) as fit the shared-memory budget
   p.warps = std::max(1, std::min(8, (OSP_TEMPORAL_SMEM_KB * 1024) / C::kWarpBytes));
   const int smem = p.warps * C::kWarpBytes;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(attn_temporal_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(attn_temporal_kernel) failed");
-    attr_done = true;
-  }
+  const int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_temporal_kernel<D, MT>), smem,
+                                  "attn_temporal_kernel");
+  if (rc) return rc;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_temporal_kernel<D, MT>, p.warps * 32, smem) !=
           cudaSuccess ||

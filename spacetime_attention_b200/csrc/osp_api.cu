@@ -6,6 +6,10 @@
 #include <cstdlib>
 #include <mutex>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "osp_internal.h"
 
 namespace osp {
@@ -142,6 +146,20 @@ uint64_t wait_timeout_ns() {
 int split_kv_enabled() {
   const char* e = getenv("OSP_SPLIT_KV");
   return (e && e[0] == '0') ? 0 : 1;
+}
+
+int ensure_smem_attr(const void* func, int bytes, const char* name) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({dev, func})) return OSP_OK;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess)
+    return set_error(OSP_ERR_CUDA, "cudaFuncSetAttribute(%s, %d bytes of shared memory) failed: %s", name, bytes,
+                     cudaGetErrorString(e));
+  done.insert({dev, func});
+  return OSP_OK;
 }
 
 int persist_mode() {

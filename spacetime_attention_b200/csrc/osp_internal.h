@@ -41,6 +41,10 @@ cudaMemPool_t workspace_pool();
 // Split-KV of the last partial wave of attention CTAs (OSP_SPLIT_KV=0 disables; read per launch).
 int split_kv_enabled();
 
+// Sets the dynamic shared-memory limit of kernel `func` to `bytes` on the current device, once per
+// (device, kernel), from any host thread.  OSP_ERR_CUDA naming `name` on failure.
+int ensure_smem_attr(const void* func, int bytes, const char* name);
+
 // Attention CTAs running several work items in turn (OSP_PERSIST, read per launch): 1 (default)
 // for short KV ranges, 0 never, 2 always (where the launch allows it).
 int persist_mode();

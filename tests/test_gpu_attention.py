@@ -204,3 +204,30 @@ def test_maximum_sequence_length_sampled(gpu):
     rows = _sample_rows(N, 8, 3)
     ref = O.attn_ref(to_f64(q), to_f64(k), to_f64(v), rows=rows)
     assert_attn_close(o[:, rows], ref, "2^20 tokens")
+
+
+@pytest.mark.parametrize("kind", ["dense", "skiparse", "cross", "frame_causal", "skiparse_text", "spatial"])
+def test_items_in_turn_equal_one_item_per_cta(gpu, monkeypatch, kind):
+    """CTAs that run several work items in turn (OSP_PERSIST=2, one CTA per SM) compute every item
+    exactly as a CTA that runs one (OSP_PERSIST=0): bit-identical outputs, on shapes with more
+    items than SMs and several KV tiles per item."""
+    grid = (4, 16, 24)                    # 1,536 video tokens
+    q, k, v, qg, kg, vg = _qkv(gpu, 2, 6, 64, grid, 40 if kind in ("dense", "frame_causal") else 0, seed=29)
+    kt, vt = syn.randn_bf16((2, 300, 6, 64), 31).to(gpu), syn.randn_bf16((2, 300, 6, 64), 32).to(gpu)
+    if kind in ("skiparse_text",):
+        q, k, v, qg, kg, vg = _qkv(gpu, 2, 6, 64, grid, 77, seed=29)
+    calls = {
+        "dense": lambda: ops.attn_full(qg, kg, vg, grid, 40),
+        "skiparse": lambda: ops.skiparse_attn(qg, kg, vg, grid, 2, 1),
+        "cross": lambda: ops.attn_cross(qg, kt, vt, grid),
+        "frame_causal": lambda: ops.attn_frame_causal(qg, kg, vg, grid, 40),
+        "skiparse_text": lambda: ops.skiparse_attn(qg, kg, vg, grid, 2, 0, text_len=77),
+        "spatial": lambda: ops.attn_spatial(qg, kg, vg, grid),
+    }
+    monkeypatch.setenv("OSP_SPLIT_KV", "0")
+    monkeypatch.setenv("OSP_PERSIST", "0")
+    one = calls[kind]()
+    monkeypatch.setenv("OSP_PERSIST", "2")
+    turns = calls[kind]()
+    ops.check_status()
+    assert torch.equal(one, turns)
