@@ -211,11 +211,11 @@ def test_items_in_turn_equal_one_item_per_cta(gpu, monkeypatch, kind):
     """CTAs that run several work items in turn (OSP_PERSIST=2, one CTA per SM) compute every item
     exactly as a CTA that runs one (OSP_PERSIST=0): bit-identical outputs, on shapes with more
     items than SMs and several KV tiles per item."""
-    grid = (4, 16, 24)                    # 1,536 video tokens
-    q, k, v, qg, kg, vg = _qkv(gpu, 2, 6, 64, grid, 40 if kind in ("dense", "frame_causal") else 0, seed=29)
-    kt, vt = syn.randn_bf16((2, 300, 6, 64), 31).to(gpu), syn.randn_bf16((2, 300, 6, 64), 32).to(gpu)
+    grid = (4, 16, 24)                    # 1,536 video tokens; 24 heads x 2 samples: 288+ items
+    q, k, v, qg, kg, vg = _qkv(gpu, 2, 24, 64, grid, 40 if kind in ("dense", "frame_causal") else 0, seed=29)
+    kt, vt = syn.randn_bf16((2, 300, 24, 64), 31).to(gpu), syn.randn_bf16((2, 300, 24, 64), 32).to(gpu)
     if kind in ("skiparse_text",):
-        q, k, v, qg, kg, vg = _qkv(gpu, 2, 6, 64, grid, 77, seed=29)
+        q, k, v, qg, kg, vg = _qkv(gpu, 2, 24, 64, grid, 77, seed=29)
     calls = {
         "dense": lambda: ops.attn_full(qg, kg, vg, grid, 40),
         "skiparse": lambda: ops.skiparse_attn(qg, kg, vg, grid, 2, 1),
