@@ -28,11 +28,14 @@ namespace {
 constexpr int kBT = 128;                 // rows per tile (queries or keys)
 constexpr int kChunkBytes = 128 * 128;   // 128 rows x 64 bf16 channels, one SW128 atom wide
 // warps 0-7 compute (warp w: tensor-memory lane quarter w % 4, column half w / 4; two warps per
-// SM sub-partition keep its MUFU busy), 8 TMA producer, 9 MMA issuer
-constexpr int kBwdThreads = 320;
+// SM sub-partition keep its MUFU busy), 8 TMA producer, 9 issues the score products (S, dP),
+// 10 the accumulating products (dV, dK or dQ): the sub-tile products are short, and one issuing
+// thread for all of them left the tensor pipe waiting on issue.
+constexpr int kBwdThreads = 352;
 constexpr int kComputeThreads = 256;
 constexpr int kProdWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kAccWarp = 10;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 // The streamed 128-row tiles are processed as two 64-row sub-tiles, and the score buffers are
@@ -56,7 +59,7 @@ struct BwdCfg {
   static constexpr int kVecOff = kStageOff + kStages * 2 * kTileBytes;
   static constexpr int kVecBytes = 2 * kBT * 4;                     // lse + Dv of one query tile
   static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
-  static constexpr int kNumBars = 12;
+  static constexpr int kNumBars = 16;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t bar0 = sbase + C::kBarOff;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 2,
-            B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1;
+            B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1, B_BUFFREE = B_FIN + 1, B_FIN2 = B_BUFFREE + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -231,6 +234,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
+    mbar_init(bar(B_BUFFREE + 0), 1);
+    mbar_init(bar(B_BUFFREE + 1), 1);
+    mbar_init(bar(B_FIN2), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -285,8 +291,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
       mbar_drain(bar(B_FULL + t % kStages), (t / kStages) & 1, p.timeout_ns);
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kAccWarp) {
+    // ------------------------------------------------------------------ MMA issuers
     const bool leader = elect_one_sync();
     constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kSub, false);  // M = 128 keys, N = 64 queries, K-major
     constexpr uint32_t idesc_ts = idesc_bf16_f32(kBT, D, true);      // M = 128, N = D, B MN-major
@@ -313,35 +319,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
-    // Sub-tile t = 2i + hh is rows 64hh .. 64hh+63 of query tile i, in score buffer t & 1.  The
-    // products of sub-tile t are issued before waiting for the compute warps on sub-tile t-1:
-    // buffer t & 1 was last read by sub-tile t-2, whose P^T / dS^T products were issued (and so
-    // execute) before these.
+    // Sub-tile t = 2i + hh is rows 64hh .. 64hh+63 of query tile i, in score buffer t & 1.
+    // Warp 9 issues S^T / dP^T of sub-tile t once warp 10's products of sub-tile t-2 (the last
+    // readers of buffer t & 1) have completed; warp 10 issues dV / dK of sub-tile t once the
+    // compute warps have written P^T / dS^T.
     const int n_sub = 2 * nq;
-    bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
-    for (int t = 0; ok && t <= n_sub; ++t) {
-      if (t < n_sub) {
+    if (warp == kMmaWarp) {
+      bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      for (int t = 0; ok && t < n_sub; ++t) {
         const int i = t >> 1, hh = t & 1, s = i % kStages;
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
+        if (t >= 2 && !bwd_warp_wait(bar(B_BUFFREE + (t & 1)), ((t - 2) >> 1) & 1, wc)) break;
         tc_fence_after();
         const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
         issue_ss(col_s(t & 1), dK, dQk + sub);    // S^T = K Q_sub^T
         issue_ss(col_dp(t & 1), dV, dOk + sub);   // dP^T = V dO_sub^T
         if (leader) tc_commit(bar(B_SFULL + (t & 1)));
       }
-      if (t > 0) {
-        const int tp = t - 1, ip = tp >> 1, hp = tp & 1, sp = ip % kStages;
-        if (!bwd_warp_wait(bar(B_PREADY + (tp & 1)), (tp >> 1) & 1, wc)) break;
+      if (leader) tc_commit(bar(B_FIN));
+      mbar_drain(bar(B_FIN), 0, p.timeout_ns);
+    } else {
+      for (int t = 0; t < n_sub; ++t) {
+        const int i = t >> 1, hh = t & 1, s = i % kStages;
+        if (!bwd_warp_wait(bar(B_PREADY + (t & 1)), (t >> 1) & 1, wc)) break;
         tc_fence_after();
-        const uint64_t sub = stage_off(sp) + (hp ? kSubDescOff : 0);
-        issue_ts(kColAcc0, col_s(tp & 1), dOmn + sub, tp > 0);    // dV += P^T dO_sub
-        issue_ts(kColAcc1, col_dp(tp & 1), dQmn + sub, tp > 0);   // dK += dS^T Q_sub
-        if (hp == 1 && leader) tc_commit(bar(B_EMPTY + sp));    // both halves of tile ip consumed
+        const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
+        issue_ts(kColAcc0, col_s(t & 1), dOmn + sub, t > 0);    // dV += P^T dO_sub
+        issue_ts(kColAcc1, col_dp(t & 1), dQmn + sub, t > 0);   // dK += dS^T Q_sub
+        if (leader) tc_commit(bar(B_BUFFREE + (t & 1)));      // buffer t & 1 may be overwritten
+        if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));   // both halves of tile i consumed
+        if (t == n_sub - 1 && leader) tc_commit(bar(B_DONE));
       }
-      if (t == n_sub && leader) tc_commit(bar(B_DONE));
+      if (leader) tc_commit(bar(B_FIN2));
+      mbar_drain(bar(B_FIN2), 0, p.timeout_ns);
     }
-    if (leader) tc_commit(bar(B_FIN));
-    mbar_drain(bar(B_FIN), 0, p.timeout_ns);
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ compute warps 0-7
@@ -403,7 +414,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t bar0 = sbase + C::kBarOff;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 2,
-            B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1;
+            B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1, B_BUFFREE = B_FIN + 1, B_FIN2 = B_BUFFREE + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -428,6 +439,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
+    mbar_init(bar(B_BUFFREE + 0), 1);
+    mbar_init(bar(B_BUFFREE + 1), 1);
+    mbar_init(bar(B_FIN2), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -477,7 +491,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
       mbar_drain(bar(B_FULL + t % kStages), (t / kStages) & 1, p.timeout_ns);
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kAccWarp) {
     const bool leader = elect_one_sync();
     constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kSub, false);  // M = 128 queries, N = 64 keys
     constexpr uint32_t idesc_ts = idesc_bf16_f32(kBT, D, true);
@@ -500,30 +514,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
-    // sub-tile t = 2j + hh: keys 64hh .. 64hh+63 of key tile j, score buffer t & 1 (as dK/dV)
+    // sub-tile t = 2j + hh: keys 64hh .. 64hh+63 of key tile j, score buffer t & 1; the two
+    // issuing warps split as in the dK/dV kernel
     const int n_sub = 2 * nk;
-    bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
-    for (int t = 0; ok && t <= n_sub; ++t) {
-      if (t < n_sub) {
+    if (warp == kMmaWarp) {
+      bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      for (int t = 0; ok && t < n_sub; ++t) {
         const int j = t >> 1, hh = t & 1, s = j % kStages;
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (j / kStages) & 1, wc)) break;
+        if (t >= 2 && !bwd_warp_wait(bar(B_BUFFREE + (t & 1)), ((t - 2) >> 1) & 1, wc)) break;
         tc_fence_after();
         const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
         issue_ss(col_s(t & 1), dQ, dKk + sub);    // S = Q K_sub^T
         issue_ss(col_dp(t & 1), dO, dVk + sub);   // dP = dO V_sub^T
         if (leader) tc_commit(bar(B_SFULL + (t & 1)));
       }
-      if (t > 0) {
-        const int tp = t - 1, jp = tp >> 1, hp = tp & 1, sp = jp % kStages;
-        if (!bwd_warp_wait(bar(B_PREADY + (tp & 1)), (tp >> 1) & 1, wc)) break;
+      if (leader) tc_commit(bar(B_FIN));
+      mbar_drain(bar(B_FIN), 0, p.timeout_ns);
+    } else {
+      for (int t = 0; t < n_sub; ++t) {
+        const int j = t >> 1, hh = t & 1, s = j % kStages;
+        if (!bwd_warp_wait(bar(B_PREADY + (t & 1)), (t >> 1) & 1, wc)) break;
         tc_fence_after();
-        issue_ts(kColAcc0, col_dp(tp & 1), dKmn + stage_off(sp) + (hp ? kSubDescOff : 0), tp > 0);   // dQ += dS K_sub
-        if (hp == 1 && leader) tc_commit(bar(B_EMPTY + sp));
+        issue_ts(kColAcc0, col_dp(t & 1), dKmn + stage_off(s) + (hh ? kSubDescOff : 0), t > 0);   // dQ += dS K_sub
+        if (leader) tc_commit(bar(B_BUFFREE + (t & 1)));
+        if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));
+        if (t == n_sub - 1 && leader) tc_commit(bar(B_DONE));
       }
-      if (t == n_sub && leader) tc_commit(bar(B_DONE));
+      if (leader) tc_commit(bar(B_FIN2));
+      mbar_drain(bar(B_FIN2), 0, p.timeout_ns);
     }
-    if (leader) tc_commit(bar(B_FIN));
-    mbar_drain(bar(B_FIN), 0, p.timeout_ns);
     __syncwarp();
   } else {
     const int quarter = warp & 3, half = warp >> 2;
