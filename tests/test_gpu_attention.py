@@ -1,6 +1,6 @@
 """GPU parity of the tcgen05 attention kernels against the fp64 oracle.
 
-Tolerance (the benchmark spec): max-abs <= 2e-2 and relative-L2 <= 5e-3 for bf16 inputs.  Small cases
+Tolerance: max-abs <= 2e-2 and relative-L2 <= 5e-3 for bf16 inputs.  Small cases
 are compared element by element over the whole output; full-size workloads on sampled query
 rows (every head) that the oracle computes one by one."""
 
