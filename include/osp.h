@@ -142,10 +142,10 @@ int osp_attn_spatial(const void* q, const void* k, const void* v, void* o, const
  *   every t' (causal = 0) or t' <= t (causal = 1).
  *   T <= 64: a shared-memory-staged kernel with mma.sync tiles (the sets are too small for
  *   128-row tensor-memory tiles; the work is bound by HBM traffic), P rounded to bf16, fp32
- *   accumulation.  T > 64 (causal = 0 only): the osp_skiparse_attn kernel with the position's
- *   tokens as Single Skip set pos, k = H*W.
- *   Errors: OSP_ERR_INVALID_ARG (causal not 0/1, ...), OSP_ERR_UNSUPPORTED (text, causal with
- *   T > 64, head_dim), OSP_ERR_CUDA. */
+ *   accumulation.  T > 64: the osp_skiparse_attn kernel with the position's tokens as Single
+ *   Skip set pos, k = H*W (causal: with the osp_attn_frame_causal mask on one-token blocks).
+ *   Errors: OSP_ERR_INVALID_ARG (causal not 0/1, ...), OSP_ERR_UNSUPPORTED (text, head_dim),
+ *   OSP_ERR_CUDA. */
 int osp_attn_temporal(const void* q, const void* k, const void* v, void* o, const osp_shape* shape, int32_t causal,
                       float softmax_scale, void* stream);
 

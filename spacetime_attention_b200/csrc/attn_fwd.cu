@@ -1053,7 +1053,7 @@ AttnParams base_params(const osp_shape& s, int layout, int sparse_k, float scale
 // frame_causal: dense layout only; the frame-causal mask over s's text block and frames.
 int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
                        int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
-                       int N_kv = -1, bool frame_causal = false, float* lse = nullptr) {
+                       int N_kv = -1, bool frame_causal = false, float* lse = nullptr, int causal_block = 0) {
   const int N = (N_kv < 0) ? s.text_len + s.T * s.H * s.W : s.T * s.H * s.W;   // q / o tokens per sample
   if (N_kv < 0) N_kv = N;
   AttnParams p = base_params(s, layout, sparse_k, scale, o, status);
@@ -1062,7 +1062,8 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.n_q = n;
   p.n_kv = N_kv / G;
   p.N_q = N;
-  p.frame_hw = frame_causal ? s.H * s.W : 0;
+  // rows per causal block: a frame (H*W) by default; 1 makes the mask token-causal within a set
+  p.frame_hw = frame_causal ? (causal_block > 0 ? causal_block : s.H * s.W) : 0;
   p.text_len = s.text_len;
   p.lse = lse;
   p.lse_stride = (n + kBM - 1) / kBM * kBM;
@@ -1159,6 +1160,16 @@ int frame_causal_attention_launch(const void* q, const void* k, const void* v, v
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   return launch_with_status(q, k, v, o, s, 0, 1, scale, stream, status, false, -1, true);
+}
+
+int causal_temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
+                                     float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  // spatial position pos is Single Skip set pos with k = H*W (slot t = frame t); the frame-causal
+  // mask with one-row blocks lets slot t see slots 0..t
+  return launch_with_status(q, k, v, o, s, OSP_SKIP_SINGLE + 1, s.H * s.W, scale, stream, status, false, -1, true,
+                            nullptr, 1);
 }
 
 int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,

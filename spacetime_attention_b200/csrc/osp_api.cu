@@ -256,8 +256,6 @@ int osp_attn_temporal(const void* q, const void* k, const void* v, void* o, cons
   if (shape->text_len != 0)
     return set_error(OSP_ERR_UNSUPPORTED, "temporal attention takes video tokens only (text_len 0)");
   if (causal != 0 && causal != 1) return set_error(OSP_ERR_INVALID_ARG, "causal must be 0 or 1 (got %d)", causal);
-  if (causal && shape->T > 64)
-    return set_error(OSP_ERR_UNSUPPORTED, "causal temporal attention supports T <= 64 (got %d)", shape->T);
   if (!q || !k || !v || !o) return set_error(OSP_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return set_error(OSP_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
@@ -265,6 +263,7 @@ int osp_attn_temporal(const void* q, const void* k, const void* v, void* o, cons
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (shape->T <= 64) return temporal_attention_launch(q, k, v, o, *shape, causal, softmax_scale, st);
   // longer sets: the position's tokens t*H*W + pos are Single Skip set pos with k = H*W
+  if (causal) return causal_temporal_attention_launch(q, k, v, o, *shape, softmax_scale, st);
   return attention_launch(q, k, v, o, *shape, OSP_SKIP_SINGLE + 1, shape->H * shape->W, softmax_scale, st);
 }
 

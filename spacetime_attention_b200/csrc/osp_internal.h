@@ -76,6 +76,10 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
                                   float scale, cudaStream_t stream);
 
+// Causal temporal attention for any T: Single Skip sets (k = H*W) with a token-causal mask.
+int causal_temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
+                                     float scale, cudaStream_t stream);
+
 // Temporal attention of 2D + 1D (T <= 64): sets of T tokens at stride H*W, optionally causal in t.
 int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
                               float scale, cudaStream_t stream);

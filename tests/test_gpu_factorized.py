@@ -61,16 +61,17 @@ def test_causal_temporal_first_frame_returns_v(gpu):
     assert torch.equal(o[:, :16].cpu(), v[:, :16])
 
 
-def test_long_temporal_uses_single_skip_path(gpu):
-    # T > 64: the position's tokens form Single Skip set pos with k = H*W
-    grid = (80, 2, 3)
-    q, k, v = _qkv(1, 2, 64, grid, seed=55)
-    o = ops.attn_temporal(q.to(gpu), k.to(gpu), v.to(gpu), grid)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("T,d", [(80, 64), (300, 96), (129, 128)])
+def test_long_temporal_uses_single_skip_path(gpu, T, d, causal):
+    # T > 64: the position's tokens form Single Skip set pos with k = H*W (causal: the frame-causal
+    # mask with one-row blocks); 129 and 300 frames leave ragged query and key tiles
+    grid = (T, 2, 3)
+    q, k, v = _qkv(1, 2, d, grid, seed=55)
+    o = ops.attn_temporal(q.to(gpu), k.to(gpu), v.to(gpu), grid, causal=causal)
     ops.check_status()
-    assert_attn_close(o, O.temporal_attn_ref(to_f64(q), to_f64(k), to_f64(v), grid), "T80")
-    with pytest.raises(ops.OspError) as e:
-        ops.attn_temporal(q.to(gpu), k.to(gpu), v.to(gpu), grid, causal=True)
-    assert e.value.code == 2
+    assert_attn_close(o, O.temporal_attn_ref(to_f64(q), to_f64(k), to_f64(v), grid, causal=causal),
+                      f"T{T} causal={causal}")
 
 
 FRAME_CAUSAL = [
