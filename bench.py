@@ -52,7 +52,7 @@ def load_peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "osp_device.cuh"):
+    for f in ("attn_fwd_kernel.cuh", "osp_device.cuh"):
         with open(os.path.join(ROOT, "spacetime_attention_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
