@@ -22,6 +22,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libosp.so")
+# Debug build: every computed global index is checked on the device (a failed check records
+# OSP_ERR_BOUNDS in the status word and skips the access); objects in _build/debug.
+DEBUG_LIB = os.path.join(PKG, "libosp_debug.so")
 
 SOURCES = ["osp_api.cu", "rope_permute.cu", "attn_fwd.cu", "attn_temporal.cu", "attn_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -48,18 +51,21 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug_bounds: bool = False) -> str:
+    out_dir = os.path.join(BUILD, "debug") if debug_bounds else BUILD
+    lib = DEBUG_LIB if debug_bounds else LIB
+    flags = NVCC_FLAGS + (["-DOSP_BOUNDS_CHECK=1"] if debug_bounds else [])
+    os.makedirs(out_dir, exist_ok=True)
     cc = nvcc()
     headers = _headers()
     jobs = []
     objs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD, src.replace(".cu", ".o"))
+        o = os.path.join(out_dir, src.replace(".cu", ".o"))
         objs.append(o)
         if force or _stale(o, [s] + headers):
-            cmd = [cc] + ARCH + NVCC_FLAGS + (["-Xptxas", "-v"] if ptxas_info else []) + ["-c", s, "-o", o]
+            cmd = [cc] + ARCH + flags + (["-Xptxas", "-v"] if ptxas_info else []) + ["-c", s, "-o", o]
             jobs.append(cmd)
 
     def run(cmd):
@@ -74,14 +80,14 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
                 sys.stdout.write(r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed ({r.returncode}):\n{' '.join(cmd)}\n{r.stdout}{r.stderr}")
-    if force or _stale(LIB, objs):
-        cmd = [cc] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart_static", "-ldl", "-lpthread", "-lrt"]
+    if force or _stale(lib, objs):
+        cmd = [cc] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart_static", "-ldl", "-lpthread", "-lrt"]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}{r.stderr}")
-    return LIB
+    return lib
 
 
 def main():
@@ -89,8 +95,9 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers / spills / smem per kernel")
+    ap.add_argument("--debug-bounds", action="store_true", help="build libosp_debug.so with device index checks")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_info))
+    print(build(a.force, a.verbose, a.ptxas_info, a.debug_bounds))
 
 
 if __name__ == "__main__":

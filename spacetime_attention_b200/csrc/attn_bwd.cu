@@ -78,6 +78,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   unsigned* status;
   unsigned long long timeout_ns;
+  unsigned long long elems, vec_elems;   // elements of each BSHD tensor / of lse and Dv (debug checks)
 };
 
 __device__ __forceinline__ int bwd_slot_token(int layout, int s, int g, int k) {
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16*
     const long long bt = r / p.heads;
     const int token = (int)(bt % p.N);
     const int b = (int)(bt / p.N);
+    if (!index_ok(r * D + D - 1, p.elems, p.status)) continue;
     const uint4* a = reinterpret_cast<const uint4*>(o + r * D);
     const uint4* c = reinterpret_cast<const uint4*>(dout + r * D);
     float acc = 0.f;
@@ -140,7 +142,8 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16*
       g = rem / p.k;
       slot = ob * p.k + (rem - g * p.k);
     }
-    p.dvec[((size_t)(b * p.G + g) * p.heads + h) * p.vec_stride + slot] = acc;
+    const size_t vi = ((size_t)(b * p.G + g) * p.heads + h) * p.vec_stride + slot;
+    if (index_ok(vi, p.vec_elems, p.status)) p.dvec[vi] = acc;
   }
 }
 
@@ -274,15 +277,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int s = i % kStages;
       if (i >= kStages && !bwd_warp_wait(bar(B_EMPTY + s), ((i / kStages) - 1) & 1, wc)) break;
       if (leader) {
-        mbar_arrive_expect_tx(bar(B_FULL + s), 2 * C::kTileBytes + C::kVecBytes);
+        // the tile's lse / Dv slices (skipped, with their bytes, if a debug index check fails)
+        const bool vec_ok = index_ok(vec_row + (size_t)i * kBT + kBT - 1, p.vec_elems, p.status);
+        mbar_arrive_expect_tx(bar(B_FULL + s), 2 * C::kTileBytes + (vec_ok ? C::kVecBytes : 0));
         for (int c = 0; c < C::kChunks; ++c) {
           bwd_load_tile(&tm_q, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, i * kBT, g,
                         b, p.k);
           bwd_load_tile(&tm_do, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, i * kBT, g,
                         b, p.k);
         }
-        bulk_load(sVec(s), p.lse + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
-        bulk_load(sVec(s) + kBT * 4, p.dvec + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
+        if (vec_ok) {
+          bulk_load(sVec(s), p.lse + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
+          bulk_load(sVec(s) + kBT * 4, p.dvec + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
+        }
       }
       issued = i + 1;
     }
@@ -386,8 +393,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool live = j < p.n;
       const int token = bwd_slot_token(p.layout, live ? j : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
-      if (half == 0) bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, live);
-      else bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, live);
+      const bool store = live && index_ok(off + D - 1, p.elems, p.status);
+      if (half == 0) bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store);
+      else bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, store);
     }
   }
   tc_fence_before();
@@ -552,8 +560,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int qs = q0 + row;
     const bool live = qs < p.n;
     const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
-    const float lse_r = live ? p.lse[vec_row + qs] : 0.f;
-    const float dv_r = live ? p.dvec[vec_row + qs] : 0.f;
+    const bool vin = live && index_ok(vec_row + qs, p.vec_elems, p.status);
+    const float lse_r = vin ? p.lse[vec_row + qs] : 0.f;
+    const float dv_r = vin ? p.dvec[vec_row + qs] : 0.f;
     bool ok = true;
     for (int t = 0; t < 2 * nk; ++t) {
       const int j = t >> 1, hh = t & 1, bb = t & 1;
@@ -576,7 +585,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int token = bwd_slot_token(p.layout, live ? qs : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
-      bwd_store_row<D>(tmem + lane_base + kColAcc0, p.scale, p.dq + off, live, half);
+      const bool store = live && index_ok(off + D - 1, p.elems, p.status);
+      bwd_store_row<D>(tmem + lane_base + kColAcc0, p.scale, p.dq + off, store, half);
     }
   }
   tc_fence_before();
@@ -633,6 +643,8 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
+  p.elems = (unsigned long long)s.B * N * s.heads * s.head_dim / bounds_check_divisor();
+  p.vec_elems = (unsigned long long)s.B * G * s.heads * p.vec_stride / bounds_check_divisor();
   const long long ctas = (long long)p.n_tiles * s.heads * s.B * G;
   if (ctas > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld backward work units is too many", ctas);
   CUtensorMap tq, tk, tv, tdo;

@@ -132,7 +132,13 @@ int run_units(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& t
       return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", bytes);
     p.ws_o = static_cast<float*>(ws);
     p.ws_ml = reinterpret_cast<float2*>(p.ws_o + rows * (size_t)head_dim);
+    p.ws_rows = rows;
   }
+  // debug builds: the index checks' limits (a test divisor shrinks them to exercise the checks)
+  const unsigned long long div = (unsigned long long)bounds_check_divisor();
+  p.o_elems /= div;
+  p.lse_elems /= div;
+  p.ws_rows /= div;
   const long long ctas = p.n_full + (units - p.n_full) * p.n_split;
   p.n_items = (int)ctas;
   // Short KV ranges: one CTA per SM runs items in turn, so an item's Q load and first QK^T
@@ -206,6 +212,8 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   p.text_len = s.text_len;
   p.lse = lse;
   p.lse_stride = (n + kBM - 1) / kBM * kBM;
+  p.o_elems = (unsigned long long)s.B * N * s.heads * s.head_dim;
+  p.lse_elems = lse ? (unsigned long long)s.B * G * s.heads * p.lse_stride : 0;
   if (frame_causal) allow_split = false;   // a KV range could hold no visible key for some rows
   CUtensorMap tq, tk, tv;
   int rc;
@@ -254,6 +262,7 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
     p.N_q = N;
     p.text_len = L;
     p.q_row_base = L;
+    p.o_elems = (unsigned long long)s.B * N * s.heads * s.head_dim;
     CUtensorMap tq, tk, tv;
     TextMaps tm{};
     const char* qv = static_cast<const char*>(q) + L * row;
@@ -277,6 +286,7 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
   p.n_q = L;
   p.n_kv = N;
   p.N_q = N;
+  p.o_elems = (unsigned long long)s.B * N * s.heads * s.head_dim;
   CUtensorMap tq, tk, tv;
   if ((rc = make_tmap(&tq, q, s, L, 0, 1, N)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tk, k, s, N, 0, 1)) != OSP_OK) return rc;
@@ -344,6 +354,7 @@ int packed_attention_launch(const void* q, const void* k, const void* v, void* o
   p.n_full = (int)units;
   p.n_split = 1;
   p.n_items = (int)units;
+  p.o_elems = (unsigned long long)n_q_total * heads * head_dim / (unsigned long long)bounds_check_divisor();
   // the packed tensors are one sample of n_q_total (q, o) / n_kv_total (k, v) rows
   const osp_shape sh{1, 0, 1, 1, 1, heads, head_dim};
   CUtensorMap tq, tk, tv;

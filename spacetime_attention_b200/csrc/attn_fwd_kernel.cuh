@@ -135,6 +135,8 @@ struct AttnParams {
   // = m + log2(l) in the log2 domain of the scaled scores, rows lse_stride apart.
   float* lse;
   int lse_stride;
+  // element counts of the buffers written, for the debug build's index checks
+  unsigned long long o_elems, lse_elems, ws_rows;
   // Work items (1-D grid): units are (sample*set, head, query block) with the query block fastest.
   // CTAs [0, n_full) process whole units; every later unit is split into n_split KV ranges whose
   // CTAs write fp32 partials (unnormalised O, running max m, row sum l) to ws_o / ws_ml, merged
@@ -788,28 +790,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = 1.f / l;
       const int slot = w.q0 + i * kBM + row;
       const bool live = slot < w.nq;
-      if (!kPacked && part < 0 && p.lse && live)
-        p.lse[((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot] = m + __log2f(l);
+      if (!kPacked && part < 0 && p.lse && live) {
+        const size_t li = ((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot;
+        if (index_ok(li, p.lse_elems, p.status)) p.lse[li] = m + __log2f(l);
+      }
       if (part >= 0) {
         // split unit: unnormalised fp32 O (relative to m) and (m, l) for the combine kernel
         const size_t prow = ((size_t)(unit - p.n_full) * p.n_split + part) * (2 * kBM) + i * kBM + row;
+        const bool in = live && index_ok(prow, p.ws_rows, p.status);
         float4* wo = reinterpret_cast<float4*>(p.ws_o + prow * D);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + 32 * cc, o);
           tmem_wait_ld();
-          if (live) {
+          if (in) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               wo[8 * cc + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
                                            __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
           }
         }
-        if (live) p.ws_ml[prow] = make_float2(m, l);
+        if (in) p.ws_ml[prow] = make_float2(m, l);
       } else {
       const int token = w.q_out0 + slot_token(p.layout, live ? slot : 0, g, p.k);
-      uint4* dst = reinterpret_cast<uint4*>(p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D);
+      const size_t ooff = (((size_t)b * p.N_q + token) * p.heads + h) * D;
+      const bool store = live && index_ok(ooff + D - 1, p.o_elems, p.status);
+      uint4* dst = reinterpret_cast<uint4*>(p.o + ooff);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -819,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        if (live) {
+        if (store) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) dst[4 * cc + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         }
@@ -855,6 +862,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, i
   const int b = bg / p.G, g = bg % p.G;
   const int slot = qb * 2 * kBM + r;
   if (slot >= p.n_q) return;
+  if (!index_ok(((size_t)su * p.n_split + p.n_split - 1) * (2 * kBM) + r, p.ws_rows, p.status)) return;
   float mmax = -INFINITY;
   for (int s = 0; s < p.n_split; ++s)
     mmax = fmaxf(mmax, p.ws_ml[((size_t)su * p.n_split + s) * (2 * kBM) + r].x);
@@ -871,9 +879,14 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p, i
     for (int e = 0; e < kPer; ++e) acc[e] += wgt * p.ws_o[prow * D + e * 32 + lane];
   }
   const float inv = 1.f / lsum;
-  if (p.lse && lane == 0) p.lse[((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot] = mmax + __log2f(lsum);
+  if (p.lse && lane == 0) {
+    const size_t li = ((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot;
+    if (index_ok(li, p.lse_elems, p.status)) p.lse[li] = mmax + __log2f(lsum);
+  }
   const int token = p.q_row_base + slot_token(p.layout, slot, g, p.k);
-  __nv_bfloat16* dst = p.o + (((size_t)b * p.N_q + token) * p.heads + h) * D;
+  const size_t ooff = (((size_t)b * p.N_q + token) * p.heads + h) * D;
+  if (!index_ok(ooff + D - 1, p.o_elems, p.status)) return;
+  __nv_bfloat16* dst = p.o + ooff;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) dst[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
 }

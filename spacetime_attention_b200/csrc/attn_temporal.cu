@@ -44,6 +44,8 @@ struct TemporalParams {
   float scale_log2;
   int causal;
   int warps;            // warps per CTA (each with its own staging buffers)
+  unsigned long long elems;   // elements of each tensor (debug index checks)
+  unsigned* status;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool fill) {
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(256) attn_temporal_kernel(const TemporalParams
     const long long sb = set_base(s);
     for (int ch = lane; ch < C::kRows * kChunks; ch += 32) {
       const int r = ch / kChunks, cc = ch - r * kChunks;
-      const bool live = r < p.T;
+      const bool live = r < p.T && index_ok(sb + r * tstride + cc * 8 + 7, p.elems, p.status);
       const long long off = live ? sb + r * tstride + cc * 8 : 0;
       const uint32_t dst = base + (uint32_t)(r * C::kRowBytes + cc * 16);
       cp_async16(dst, p.q + off, live);
@@ -232,7 +234,8 @@ __global__ void __launch_bounds__(256) attn_temporal_kernel(const TemporalParams
       asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                    : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
                    : "r"(sq + (uint32_t)(r * C::kRowBytes + cc * 16)));
-      *reinterpret_cast<uint4*>(p.o + ob + r * tstride + cc * 8) = val;
+      if (index_ok(ob + r * tstride + cc * 8 + 7, p.elems, p.status))
+        *reinterpret_cast<uint4*>(p.o + ob + r * tstride + cc * 8) = val;
     }
     __syncwarp();   // this buffer is refilled by the prefetch two sets later
   }
@@ -284,6 +287,9 @@ int temporal_attention_launch(const void* q, const void* k, const void* v, void*
   if (p.n_sets > 0x7fffffffLL) return set_error(OSP_ERR_UNSUPPORTED, "%lld temporal sets is too many", p.n_sets);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
+  p.elems = (unsigned long long)s.B * s.T * p.HW * s.heads * s.head_dim / bounds_check_divisor();
+  p.status = device_status_word();
+  if (!p.status) return OSP_ERR_CUDA;
   switch (s.head_dim) {
     case 64: return launch_temporal_d<64>(p, stream);
     case 96: return launch_temporal_d<96>(p, stream);

@@ -162,6 +162,12 @@ int ensure_smem_attr(const void* func, int bytes, const char* name) {
   return OSP_OK;
 }
 
+unsigned bounds_check_divisor() {
+  const char* e = getenv("OSP_DEBUG_BOUNDS_DIV");
+  const long v = e ? strtol(e, nullptr, 10) : 1;
+  return v >= 1 ? (unsigned)v : 1u;
+}
+
 int persist_mode() {
   const char* e = getenv("OSP_PERSIST");
   if (!e || !e[0]) return 1;

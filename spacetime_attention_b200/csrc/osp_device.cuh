@@ -15,6 +15,25 @@ enum : unsigned {
   kDevBounds = 2u,    // a debug index check failed
 };
 
+// Debug builds (compiled with OSP_BOUNDS_CHECK=1) check every computed global index before the
+// access it guards: an index past its buffer records kDevBounds in the status word and the access
+// is skipped (no trap, no fault).  Release builds compile the checks away.
+#ifndef OSP_BOUNDS_CHECK
+#define OSP_BOUNDS_CHECK 0
+#endif
+__device__ __forceinline__ bool index_ok(unsigned long long idx, unsigned long long n, unsigned* status) {
+#if OSP_BOUNDS_CHECK
+  if (idx < n) return true;
+  atomicOr(status, 2u);   // kDevBounds
+  return false;
+#else
+  (void)idx;
+  (void)n;
+  (void)status;
+  return true;
+#endif
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -45,6 +45,11 @@ int split_kv_enabled();
 // (device, kernel), from any host thread.  OSP_ERR_CUDA naming `name` on failure.
 int ensure_smem_attr(const void* func, int bytes, const char* name);
 
+// Debug builds only (kernels compiled with OSP_BOUNDS_CHECK=1): the kernels' index-check limits
+// are divided by OSP_DEBUG_BOUNDS_DIV (default 1), so a test can make the checks fire without
+// any out-of-range access (the checked access is skipped).  Read per launch.
+unsigned bounds_check_divisor();
+
 // Attention CTAs running several work items in turn (OSP_PERSIST, read per launch): 1 (default)
 // for short KV ranges, 0 never, 2 always (where the launch allows it).
 int persist_mode();

@@ -42,6 +42,10 @@ struct PermuteParams {
   double log2_theta;
   int rows_per_tile;
   long long n_tiles;
+  // 16-byte vectors in each source / destination tensor and the status word, for the debug
+  // build's index checks
+  unsigned long long src_vecs, dst_vecs;
+  unsigned* status;
 };
 
 // Samples of a packed batch: sample i owns rows [start[i], start[i+1]), its first text[i] rows
@@ -177,6 +181,8 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
           rowi[u] = row;
           coli[u] = col;
           live[u] = base + u * kThreads < total && !(inplace && vid[row] < 0);  // text row in place: skip
+          live[u] = live[u] && index_ok(src_row[row] * p.vpr + col, p.src_vecs, p.status) &&
+                    index_ok(dst_row[row] * p.vpr + col, p.dst_vecs, p.status);
           if (live[u]) val[u] = src[src_row[row] * p.vpr + col];
           col += dcol;
           row += drow;
@@ -216,6 +222,11 @@ __global__ void index_map_kernel(int n_video, int k, int mode, int* out) {
 }
 
 int launch_permute(int map, PermuteParams& p, cudaStream_t stream, const PackTable* tab = nullptr) {
+  // every tensor of a call has the natural-order row count on one side and `rows` on the other
+  const unsigned long long nat = (unsigned long long)p.rows * p.vpr;
+  p.src_vecs = p.dst_vecs = nat / bounds_check_divisor();
+  p.status = device_status_word();
+  if (!p.status) return OSP_ERR_CUDA;
   const int npairs = p.head_dim / 2;
   // ~4096 vectors (64 KB of one tensor) per tile, at most 64 rows, and the cos/sin table within
   // 40 KB of shared memory

@@ -15,7 +15,12 @@ from typing import Optional, Sequence
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libosp.so")
+# OSP_LIBRARY=debug selects the debug build (libosp_debug.so: device-side index checks that report
+# OSP_ERR_BOUNDS); any other value is taken as a path.
+_LIB_DIR = os.path.dirname(os.path.abspath(__file__))
+_LIB_SEL = os.environ.get("OSP_LIBRARY", "")
+LIB_PATH = (os.path.join(_LIB_DIR, "libosp_debug.so") if _LIB_SEL == "debug"
+            else (_LIB_SEL or os.path.join(_LIB_DIR, "libosp.so")))
 
 OSP_SKIP_SINGLE = 0
 OSP_SKIP_GROUP = 1

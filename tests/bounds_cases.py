@@ -1,0 +1,63 @@
+"""Small calls of every kernel family, run in a child process against the debug build
+(OSP_LIBRARY=debug, device-side index checks) by tests/test_gpu_bounds.py.
+
+    python -m tests.bounds_cases <out.pt> [expect_bounds]
+
+Writes the outputs (CPU tensors) to <out.pt>.  With `expect_bounds`, every call must instead end
+in OSP_ERR_BOUNDS from osp_check_status (the caller shrinks the checks' limits)."""
+
+import sys
+
+import torch
+
+from spacetime_attention_b200 import ops, synthetic as syn
+
+
+def calls(dev):
+    w = syn.custom("b", 1, 2, 64, (4, 8, 8), 0, (16, 24, 24), skiparse_k=2)
+    q, k, v = (t.to(dev) for t in syn.make_qkv(w, 77))
+    do = syn.randn_bf16(tuple(q.shape), 81).to(dev)
+    kt, vt = syn.randn_bf16((1, 40, 2, 64), 82).to(dev), syn.randn_bf16((1, 40, 2, 64), 83).to(dev)
+
+    def backward():
+        o, lse = ops.attn_forward_train(q, k, v, w.grid, 0)
+        return ops.attn_backward(q, k, v, o, do, lse, w.grid, 0)
+
+    return {
+        "rope": lambda: ops.rope3d(q, k, w.grid, 0, w.split),
+        "gather": lambda: ops.skiparse_gather(q, k, v, w.grid, 2, 1, split=w.split),
+        "scatter": lambda: ops.skiparse_scatter(q.view(2, 128, 2, 64), w.grid, 2, 0),
+        "dense": lambda: ops.attn_full(q, k, v, w.grid, 0),
+        "skiparse": lambda: ops.skiparse_attn(q, k, v, w.grid, 2, 1),
+        "cross": lambda: ops.attn_cross(q, kt, vt, w.grid),
+        "temporal": lambda: ops.attn_temporal(q, k, v, w.grid, causal=True),
+        "packed": lambda: ops.attn_packed(q, k, v, [0, 100, 256]),
+        "backward": backward,
+    }
+
+
+def main():
+    out_path = sys.argv[1]
+    expect_bounds = len(sys.argv) > 2 and sys.argv[2] == "expect_bounds"
+    assert ops.LIB_PATH.endswith("libosp_debug.so"), ops.LIB_PATH
+    dev = torch.device("cuda:0")
+    results = {}
+    for name, fn in calls(dev).items():
+        r = fn()
+        try:
+            ops.check_status(dev)
+            status = 0
+        except ops.OspError as e:
+            status = e.code
+        if expect_bounds:
+            assert status == 6, f"{name}: status {status}, expected OSP_ERR_BOUNDS (6)"
+        else:
+            assert status == 0, f"{name}: status {status}"
+            rs = r if isinstance(r, tuple) else (r,)
+            results[name] = [t.cpu() for t in rs if t is not None]
+    torch.save(results, out_path)
+    print("ok", sorted(results) if results else "bounds")
+
+
+if __name__ == "__main__":
+    main()
