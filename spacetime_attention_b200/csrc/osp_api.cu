@@ -4,8 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
-#include <mutex>
-
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -21,7 +20,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned* g_status[kMaxDevices] = {};
 cudaMemPool_t g_pool[kMaxDevices] = {};
-int g_sms[kMaxDevices] = {};
+std::atomic<int> g_sms[kMaxDevices] = {};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -91,12 +90,13 @@ int check_launch(const char* what) {
 int device_sm_count() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 148;
-  if (!g_sms[dev]) {
-    int n = 0;
+  int n = g_sms[dev].load(std::memory_order_relaxed);
+  if (!n) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    g_sms[dev] = n > 0 ? n : 148;
+    n = n > 0 ? n : 148;
+    g_sms[dev].store(n, std::memory_order_relaxed);
   }
-  return g_sms[dev];
+  return n;
 }
 
 unsigned* device_status_word() {
