@@ -16,6 +16,7 @@ from .spacetime_oracle import (  # noqa: F401
     cross_attn_ref,
     default_scale,
     frame_causal_attn_ref,
+    frame_causal_backward_ref,
     frame_causal_limit,
     packed_attn_ref,
     rope3d_packed_ref,

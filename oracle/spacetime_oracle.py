@@ -618,3 +618,25 @@ def attention_head_backward_rows_ref(q, k, v, do, scale: float, q_rows, k_rows, 
     dk = dst.T @ q * scale
     dv = pt.T @ do
     return dq, dk, dv
+
+
+def frame_causal_backward_ref(q, k, v, do, grid: Sequence[int], text_len: int, scale: float | None = None):
+    """Gradients of frame-causal attention (frame_causal_attn_ref): the backward chain rule above
+    with P zero outside the mask (query token r sees the first frame_causal_limit(r) keys)."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    lim = np.array([frame_causal_limit(r, text_len, H * W) for r in range(N)])
+    allowed = np.arange(N)[None, :] < lim[:, None]
+    out = [np.empty((B, N, nh, d)) for _ in range(3)]
+    for b in range(B):
+        for h in range(nh):
+            qh, kh, vh, dh = (np.asarray(a[b, :, h], np.float64) for a in (q, k, v, do))
+            s = np.where(allowed, (qh @ kh.T) * scale, -np.inf)
+            p = softmax_rows(s)
+            o = p @ vh
+            ds = p * (dh @ vh.T - (dh * o).sum(axis=1, keepdims=True))
+            out[0][b, :, h] = ds @ kh * scale
+            out[1][b, :, h] = ds.T @ qh * scale
+            out[2][b, :, h] = p.T @ dh
+    return tuple(out)

@@ -633,3 +633,17 @@ def test_backward_rows_agree_with_full_backward():
     np.testing.assert_allclose(sq, dq[rq], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(sk, dk[rk], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(sv, dv[rk], rtol=1e-12, atol=1e-13)
+
+
+def test_frame_causal_backward_matches_finite_differences():
+    rng = np.random.default_rng(84)
+    grid, L = (3, 1, 2), 1                       # 7 tokens: text, then three frames of two
+    q, k, v = (rng.standard_normal((1, 7, 1, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 7, 1, 3))
+    loss = lambda q_, k_, v_: float((O.frame_causal_attn_ref(q_, k_, v_, grid, L) * G).sum())
+    dq, dk, dv = O.frame_causal_backward_ref(q, k, v, G, grid, L)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+    # keys of the last frame are seen only by the last frame's queries: their dV is P^T dO of those
+    assert not np.allclose(dv[0, 5:], 0)
