@@ -163,8 +163,8 @@ ATTN_MODE = {"value": "auto"}
 
 
 def sparse(w) -> bool:
-    """Skiparse pair (Single + Group) for workloads that define k, unless --attn dense."""
-    return bool(w.skiparse_k) and ATTN_MODE["value"] != "dense"
+    """Skiparse pair (Single + Group) for workloads that define k, unless --attn dense / frame_causal."""
+    return bool(w.skiparse_k) and ATTN_MODE["value"] not in ("dense", "frame_causal")
 
 
 def attention_launches(w, sms: int) -> int:
@@ -472,14 +472,21 @@ def run_backward_op(args, rank, world, local_rank):
     w = syn.WORKLOADS[args.workload]
     q, k, v = (t.to(dev) for t in syn.make_qkv(w, w.seed + 17 * rank))
     do = syn.randn_bf16(tuple(q.shape), w.seed + 99 + 17 * rank).to(dev)
+    causal = ATTN_MODE["value"] == "frame_causal"
     modes = [(w.skiparse_k, ops.OSP_SKIP_SINGLE), (w.skiparse_k, ops.OSP_SKIP_GROUP)] if sparse(w) else [(1, 0)]
     L = 0 if sparse(w) else w.text_len
-    saved = [ops.attn_forward_train(q, k, v, w.grid, L, sparse_k=kk, mode=m) for kk, m in modes]
+    if causal:
+        saved = [ops.attn_frame_causal_train(q, k, v, w.grid, L)]
+    else:
+        saved = [ops.attn_forward_train(q, k, v, w.grid, L, sparse_k=kk, mode=m) for kk, m in modes]
     grads = [tuple(torch.empty_like(q) for _ in range(3)) for _ in modes]
 
     def step():
         for (kk, m), (o, lse), (dq, dk, dv) in zip(modes, saved, grads):
-            ops.attn_backward(q, k, v, o, do, lse, w.grid, L, sparse_k=kk, mode=m, dq=dq, dk=dk, dv=dv)
+            if causal:
+                ops.attn_frame_causal_backward(q, k, v, o, do, lse, w.grid, L, dq=dq, dk=dk, dv=dv)
+            else:
+                ops.attn_backward(q, k, v, o, do, lse, w.grid, L, sparse_k=kk, mode=m, dq=dq, dk=dk, dv=dv)
 
     for _ in range(args.warmup):
         step()
@@ -499,14 +506,21 @@ def run_backward_op(args, rank, world, local_rank):
     ops.check_status(dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
     peaks, src = load_peaks()
-    flops = 2.5 * step_flops(w)
+    if causal:   # unmasked (query, key) pairs only
+        T, H, W = w.grid
+        HW = H * W
+        pairs = w.B * (L * L + sum(HW * (L + (t + 1) * HW) for t in range(T)))
+        flops = 2.5 * 4.0 * w.heads * w.head_dim * pairs
+    else:
+        flops = 2.5 * step_flops(w)
     tflops = flops / (ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops_sustained"])
     return {"metric": "attention backward TFLOP/s (2.5x forward flops)", "value": round(world * tflops, 1),
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": dict(w.describe(), op="backward", attn="skiparse pair" if sparse(w) else "dense",
+            "config": dict(w.describe(), op="backward",
+                           attn="frame-causal" if causal else ("skiparse pair" if sparse(w) else "dense"),
                            flops_per_step=flops, l2="inputs > L2, no flush"),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tflops / peak, 4), "traffic": None,
@@ -747,8 +761,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="cogvideox_2b", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse"],
-                    help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention")
+    ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse", "frame_causal"],
+                    help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention; "
+                         "frame_causal: the frame-causal backward (--op backward)")
     ap.add_argument("--op", default="step",
                     choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
                              "frame_causal", "skiparse_text", "backward"],
@@ -763,6 +778,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.attn == "frame_causal" and args.op != "backward":
+        ap.error("--attn frame_causal applies to --op backward (use --op frame_causal for the forward)")
     ATTN_MODE["value"] = args.attn
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

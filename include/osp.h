@@ -187,6 +187,18 @@ int osp_attn_backward(const void* q, const void* k, const void* v, const void* o
                       void* dq, void* dk, void* dv, const osp_shape* shape, int32_t sparse_k, int32_t mode,
                       float softmax_scale, void* stream);
 
+/* Training with the frame-causal mask (osp_attn_frame_causal): the forward with its saved lse
+ * (dense layout, G = 1: lse[(b*heads + h)*n_pad + token], n_pad = ceil(N / 128) * 128) and the
+ * backward, with the same arithmetic as osp_attn_forward_train / osp_attn_backward and P zero
+ * outside the mask.  The dK/dV kernel skips query tiles that cannot see its keys and the dQ kernel
+ * key tiles past its queries' limit.
+ *  Errors: as osp_attn_frame_causal, OSP_ERR_CUDA. */
+int osp_attn_frame_causal_train(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const osp_shape* shape, float softmax_scale, void* stream);
+int osp_attn_frame_causal_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                   const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape,
+                                   float softmax_scale, void* stream);
+
 /* 3D RoPE of a packed batch (CogVideoX section 3.1: every video keeps its own position grid,
  * starting at (0, 0, 0); extrapolation, never rescaled).
  *  samples:       HOST array of n_samples (1 .. OSP_MAX_SEGMENTS) sample grids, read during the call.

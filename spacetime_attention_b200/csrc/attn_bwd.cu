@@ -79,7 +79,34 @@ struct BwdParams {
   unsigned* status;
   unsigned long long timeout_ns;
   unsigned long long elems, vec_elems;   // elements of each BSHD tensor / of lse and Dv (debug checks)
+  // Frame-causal mask (dense layout; 0 = off): blocks are [text], [frame 0], [frame 1], ...
+  // (frame_hw tokens each after text_len text tokens); query r sees keys of blocks <= its own.
+  int frame_hw;
+  int text_len;
 };
+
+__device__ __forceinline__ int causal_block(int x, int text_len, int hw) {
+  return x < text_len ? 0 : 1 + (x - text_len) / hw;
+}
+// Keys visible to query r: the tokens of blocks 0 .. block(r).
+__device__ __forceinline__ int causal_limit(int r, int text_len, int hw) {
+  return r < text_len ? text_len : text_len + ((r - text_len) / hw + 1) * hw;
+}
+// Bit e set when query column q0 + e (e < 32) may see a key of block bk.
+__device__ __forceinline__ uint32_t causal_columns(int q0, int bk, int text_len, int hw) {
+  int bq = causal_block(q0, text_len, hw);
+  int next = q0 < text_len ? text_len : text_len + bq * hw;   // first token of block bq + 1
+  uint32_t vis = 0;
+#pragma unroll 4
+  for (int e = 0; e < 32; ++e) {
+    while (q0 + e >= next) {
+      ++bq;
+      next += hw;
+    }
+    vis |= (uint32_t)(bq >= bk) << e;
+  }
+  return vis;
+}
 
 __device__ __forceinline__ int bwd_slot_token(int layout, int s, int g, int k) {
   if (layout == 0) return s;
@@ -149,11 +176,12 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16*
 
 // P and dS of one 32-column chunk for one TMEM lane (the thread's row).
 //   s, dp: raw scores / dP of the chunk; lse, dv: per-column (kCols) or per-row values.
-//   valid: columns [0, valid) of the chunk are real.
+//   valid: columns [0, valid) of the chunk are real; vis: bit e clear masks column e out.
 template <bool kPerColumn>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
                                           const float* lse_col, const float* dv_col, float lse_row, float dv_row,
-                                          int valid, uint32_t (&pk)[16], uint32_t (&dk)[16]) {
+                                          int valid, uint32_t (&pk)[16], uint32_t (&dk)[16],
+                                          uint32_t vis = 0xffffffffu) {
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float pv[2], dsv[2];
@@ -163,7 +191,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_
       const float dd = kPerColumn ? dv_col[e + u] : dv_row;
       const float pe = ex2_approx(fmaf(__uint_as_float(s[e + u]), sl2, -l));
       const float de = pe * (__uint_as_float(dp[e + u]) - dd);
-      const bool ok = e + u < valid;
+      const bool ok = e + u < valid && ((vis >> (e + u)) & 1u);
       pv[u] = ok ? pe : 0.f;
       dsv[u] = ok ? de : 0.f;
     }
@@ -221,7 +249,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int h = hb % p.heads, bg = hb / p.heads;
   const int b = bg / p.G, g = bg % p.G;
   const int kv0 = tile * kBT;
-  const int nq = p.n_tiles;   // query tiles of the set
+  // query tiles i0 .. n_tiles-1 (frame-causal: the first query that may see key kv0 opens the range)
+  const int i0 = (p.frame_hw && kv0 >= p.text_len)
+                     ? (p.text_len + (kv0 - p.text_len) / p.frame_hw * p.frame_hw) / kBT
+                     : 0;
+  const int nq = p.n_tiles - i0;
   const int chan0 = h * D;
   const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
 
@@ -273,9 +305,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bwd_load_tile(&tm_v, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, kv0, g, b, p.k);
       }
     }
-    for (int i = 0; i < nq; ++i) {
-      const int s = i % kStages;
-      if (i >= kStages && !bwd_warp_wait(bar(B_EMPTY + s), ((i / kStages) - 1) & 1, wc)) break;
+    for (int il = 0; il < nq; ++il) {
+      const int s = il % kStages, i = i0 + il;
+      if (il >= kStages && !bwd_warp_wait(bar(B_EMPTY + s), ((il / kStages) - 1) & 1, wc)) break;
       if (leader) {
         // the tile's lse / Dv slices (skipped, with their bytes, if a debug index check fails)
         const bool vec_ok = index_ok(vec_row + (size_t)i * kBT + kBT - 1, p.vec_elems, p.status);
@@ -291,7 +323,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           bulk_load(sVec(s) + kBT * 4, p.dvec + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
         }
       }
-      issued = i + 1;
+      issued = il + 1;
     }
     // every load issued lands before the CTA may exit
     mbar_drain(bar(B_RES), 0, p.timeout_ns);
@@ -367,20 +399,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quarter * 32 + lane;                    // key row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
+    const int bk = p.frame_hw ? causal_block(kv0 + row, p.text_len, p.frame_hw) : 0;   // this key's block
     for (int t = 0; t < 2 * nq; ++t) {
-      const int i = t >> 1, hh = t & 1, bb = t & 1;
+      const int il = t >> 1, i = i0 + il, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (i % kStages) * C::kVecBytes) +
+      const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (il % kStages) * C::kVecBytes) +
                          kSub * hh + 32 * half;
-      const int valid_q = p.n - (i * kBT + kSub * hh + 32 * half);   // of this warp's 32 query columns
+      const int qa = i * kBT + kSub * hh + 32 * half;   // this warp's first query column
+      const int valid_q = p.n - qa;
+      const uint32_t vis = p.frame_hw ? causal_columns(qa, bk, p.text_len, p.frame_hw) : 0xffffffffu;
       const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
       uint32_t s[32], dp[32];
       tmem_ld32(tS, s);
       tmem_ld32(tP, dp);
       tmem_wait_ld();
       uint32_t pk[16], dk[16];
-      bwd_chunk<true>(s, dp, p.scale_log2, vec, vec + kBT, 0.f, 0.f, valid_q, pk, dk);
+      bwd_chunk<true>(s, dp, p.scale_log2, vec, vec + kBT, 0.f, 0.f, valid_q, pk, dk, vis);
       tmem_st16(tS, pk);    // P^T over this warp's consumed S^T columns
       tmem_st16(tP, dk);    // dS^T over this warp's consumed dP^T columns
       tmem_wait_st();
@@ -432,7 +467,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int h = hb % p.heads, bg = hb / p.heads;
   const int b = bg / p.G, g = bg % p.G;
   const int q0 = tile * kBT;
-  const int nk = p.n_tiles;   // key tiles of the set
+  // key tiles 0 .. nk-1 (frame-causal: up to the last key the tile's last query may see)
+  const int nk = p.frame_hw
+                     ? (min(p.n, causal_limit(min(q0 + kBT, p.n) - 1, p.text_len, p.frame_hw)) + kBT - 1) / kBT
+                     : p.n_tiles;
   const int chan0 = h * D;
 
   if (threadIdx.x == 0) {
@@ -564,11 +602,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float lse_r = vin ? p.lse[vec_row + qs] : 0.f;
     const float dv_r = vin ? p.dvec[vec_row + qs] : 0.f;
     bool ok = true;
+    const int klim = p.frame_hw ? min(p.n, causal_limit(qs, p.text_len, p.frame_hw)) : p.n;   // keys this row sees
     for (int t = 0; t < 2 * nk; ++t) {
       const int j = t >> 1, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      const int valid_k = p.n - (j * kBT + kSub * hh + 32 * half);   // of this warp's 32 key columns
+      const int valid_k = klim - (j * kBT + kSub * hh + 32 * half);   // of this warp's 32 key columns
       const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
       uint32_t s[32], dp[32];
       tmem_ld32(tS, s);
@@ -620,7 +659,7 @@ int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const C
 
 int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
-                              int sparse_k, float scale, cudaStream_t stream) {
+                              int sparse_k, float scale, cudaStream_t stream, bool frame_causal) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   const int N = s.text_len + s.T * s.H * s.W;
@@ -644,6 +683,8 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
   p.elems = (unsigned long long)s.B * N * s.heads * s.head_dim / bounds_check_divisor();
+  p.frame_hw = frame_causal ? s.H * s.W : 0;
+  p.text_len = s.text_len;
   p.vec_elems = (unsigned long long)s.B * G * s.heads * p.vec_stride / bounds_check_divisor();
   const long long ctas = (long long)p.n_tiles * s.heads * s.B * G;
   if (ctas > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld backward work units is too many", ctas);

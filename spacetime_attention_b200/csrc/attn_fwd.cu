@@ -298,10 +298,11 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
 }
 
 int attention_forward_lse_launch(const void* q, const void* k, const void* v, void* o, float* lse,
-                                 const osp_shape& s, int layout, int sparse_k, float scale, cudaStream_t stream) {
+                                 const osp_shape& s, int layout, int sparse_k, float scale, cudaStream_t stream,
+                                 bool frame_causal) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
-  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true, -1, false, lse);
+  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true, -1, frame_causal, lse);
 }
 
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,

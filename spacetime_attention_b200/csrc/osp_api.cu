@@ -331,6 +331,34 @@ int osp_attn_backward(const void* q, const void* k, const void* v, const void* o
                                    static_cast<cudaStream_t>(stream));
 }
 
+int osp_attn_frame_causal_train(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const osp_shape* shape, float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse) return set_error(OSP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_forward_lse_launch(q, k, v, o, lse, *shape, 0, 1, softmax_scale, static_cast<cudaStream_t>(stream),
+                                      true);
+}
+
+int osp_attn_frame_causal_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                   const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape,
+                                   float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return set_error(OSP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, 0, 1, softmax_scale,
+                                   static_cast<cudaStream_t>(stream), true);
+}
+
 int osp_rope3d_packed(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
                       int32_t n_samples, int32_t heads, int32_t head_dim, const osp_rope* rope, void* stream) {
   g_last_error[0] = 0;

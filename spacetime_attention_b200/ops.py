@@ -33,7 +33,7 @@ EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_
             "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version",
             "osp_attn_full_noalloc", "osp_attn_cross", "osp_rope3d_packed", "osp_attn_packed",
             "osp_attn_spatial", "osp_attn_temporal", "osp_attn_frame_causal", "osp_attn_forward_train",
-            "osp_attn_backward")
+            "osp_attn_backward", "osp_attn_frame_causal_train", "osp_attn_frame_causal_backward")
 
 MAX_SEGMENTS = 256   # OSP_MAX_SEGMENTS
 
@@ -78,6 +78,8 @@ def library() -> ctypes.CDLL:
             "osp_attn_spatial": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_forward_train": [vp, vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
             "osp_attn_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
+            "osp_attn_frame_causal_train": [vp, vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_frame_causal_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_temporal": [vp, vp, vp, vp, sp, i32, ctypes.c_float, vp],
             "osp_attn_frame_causal": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_rope3d_packed": [vp, vp, vp, vp, ctypes.POINTER(OspSampleGrid), i32, i32, i32, rp, vp],
@@ -235,6 +237,35 @@ def attn_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, sparse_k: int 
            library().osp_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                        _ptr(dv), ctypes.byref(shp), int(sparse_k), int(mode), ctypes.c_float(scale),
                                        _stream_handle(q)))
+    return dq, dk, dv
+
+
+def attn_frame_causal_train(q, k, v, grid, text_len: int = 0, scale: float = 0.0, o=None, lse=None):
+    """osp_attn_frame_causal_train: returns (o, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(lse_shape(q, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    shp = _shape_of(q, grid, text_len)
+    _check("osp_attn_frame_causal_train",
+           library().osp_attn_frame_causal_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
+                                                 ctypes.c_float(scale), _stream_handle(q)))
+    return o, lse
+
+
+def attn_frame_causal_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, scale: float = 0.0, dq=None, dk=None,
+                               dv=None):
+    """osp_attn_frame_causal_backward: returns (dq, dk, dv)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _bshd(t, n)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    shp = _shape_of(q, grid, text_len)
+    _check("osp_attn_frame_causal_backward",
+           library().osp_attn_frame_causal_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                                    _ptr(dq), _ptr(dk), _ptr(dv), ctypes.byref(shp),
+                                                    ctypes.c_float(scale), _stream_handle(q)))
     return dq, dk, dv
 
 

@@ -148,3 +148,10 @@ def test_training_validation(lib):
     assert lib.osp_attn_forward_train(p, p, p, p, p, shp(), 3, 0, 0.0, None) == 3             # 256 % 3
     assert lib.osp_attn_backward(p, p, p, p, p, p, p, p, None, shp(), 1, 0, 0.0, None) == 1   # no dv
     assert lib.osp_attn_backward(p, p, p, p, p, p, p, p, p, shp(d=80), 1, 0, 0.0, None) == 2
+
+
+def test_frame_causal_training_validation(lib):
+    p = ctypes.c_void_p(256)
+    assert lib.osp_attn_frame_causal_train(p, p, p, p, None, shp(), 0.0, None) == 1
+    assert lib.osp_attn_frame_causal_backward(p, p, p, p, p, p, p, p, None, shp(), 0.0, None) == 1
+    assert lib.osp_attn_frame_causal_backward(p, p, p, p, p, p, p, p, p, shp(d=80), 0.0, None) == 2

@@ -127,3 +127,28 @@ def test_full_size_backward_sampled(gpu):
         assert_grad_close(dq[0, rows, h], rq, f"dq head {h}")
         assert_grad_close(dk[0, rows, h], rk, f"dk head {h}")
         assert_grad_close(dv[0, rows, h], rv, f"dv head {h}")
+
+
+FRAME_CAUSAL = [
+    # B, heads, d, grid, text_len
+    (1, 2, 64, (3, 5, 7), 0),          # 35-token frames: block boundaries inside every tile
+    (1, 2, 96, (4, 6, 8), 13),
+    (2, 1, 128, (3, 9, 15), 5),
+    (1, 2, 64, (2, 16, 16), 200),      # text spanning a tile boundary
+    (1, 2, 64, (6, 8, 32), 0),         # 256-token frames: later key tiles skip early query tiles
+]
+
+
+@pytest.mark.parametrize("case", FRAME_CAUSAL, ids=[f"{c[3]}_L{c[4]}_d{c[2]}" for c in FRAME_CAUSAL])
+def test_frame_causal_backward_matches_oracle(gpu, case):
+    B, heads, d, grid, L = case
+    q, k, v, do = _inputs(B, heads, d, grid, L, 94)
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    o, lse = ops.attn_frame_causal_train(qg, kg, vg, grid, L)
+    dq, dk, dv = ops.attn_frame_causal_backward(qg, kg, vg, o, dog, lse, grid, L)
+    ops.check_status()
+    assert torch.equal(o, ops.attn_frame_causal(qg, kg, vg, grid, L))
+    rq, rk, rv = O.frame_causal_backward_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), grid, L)
+    assert_grad_close(dq, rq, "dq")
+    assert_grad_close(dk, rk, "dk")
+    assert_grad_close(dv, rv, "dv")
