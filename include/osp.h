@@ -11,9 +11,13 @@
  *     "3D Full Attention");
  *   - Skiparse sparse attention, Single Skip and Group Skip with sparse ratio k
  *     ("Open-Sora Plan: Open-Source Large Video Generation Model", section 2.2.2);
- *   - video -> text cross-attention (Open-Sora Plan section 2.2.1);
+ *   - video -> text cross-attention (Open-Sora Plan section 2.2.1), and Skiparse with a text
+ *     prefix joined to every set;
+ *   - the factorized 2D + 1D attention CogVideoX compares against (section 2.2, Table 8) and
+ *     frame-causal attention (the Sora page);
  *   - packed batches of videos of different shapes, with per-sample RoPE grids and
- *     block-diagonal attention (CogVideoX section 3.1 "Multi-Resolution Frame Pack").
+ *     block-diagonal attention (CogVideoX section 3.1 "Multi-Resolution Frame Pack");
+ *   - the backward pass of dense, Skiparse and frame-causal attention (training).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
