@@ -85,27 +85,19 @@ struct BwdParams {
   int text_len;
 };
 
-__device__ __forceinline__ int causal_block(int x, int text_len, int hw) {
-  return x < text_len ? 0 : 1 + (x - text_len) / hw;
+// First token of the block that token x belongs to (block 0: the text prefix; block 1 + f: frame f).
+__device__ __forceinline__ int causal_block_start(int x, int text_len, int hw) {
+  return x < text_len ? 0 : text_len + (x - text_len) / hw * hw;
 }
 // Keys visible to query r: the tokens of blocks 0 .. block(r).
 __device__ __forceinline__ int causal_limit(int r, int text_len, int hw) {
   return r < text_len ? text_len : text_len + ((r - text_len) / hw + 1) * hw;
 }
-// Bit e set when query column q0 + e (e < 32) may see a key of block bk.
-__device__ __forceinline__ uint32_t causal_columns(int q0, int bk, int text_len, int hw) {
-  int bq = causal_block(q0, text_len, hw);
-  int next = q0 < text_len ? text_len : text_len + bq * hw;   // first token of block bq + 1
-  uint32_t vis = 0;
-#pragma unroll 4
-  for (int e = 0; e < 32; ++e) {
-    while (q0 + e >= next) {
-      ++bq;
-      next += hw;
-    }
-    vis |= (uint32_t)(bq >= bk) << e;
-  }
-  return vis;
+// Bit e set when query q0 + e (e < 32) may see a key whose block starts at token kstart.  Block
+// indices never decrease along the sequence, so block(q) >= block(key) exactly when q >= kstart.
+__device__ __forceinline__ uint32_t causal_columns(int q0, int kstart) {
+  const int sh = kstart - q0;
+  return sh <= 0 ? 0xffffffffu : (sh >= 32 ? 0u : (0xffffffffu << sh));
 }
 
 __device__ __forceinline__ int bwd_slot_token(int layout, int s, int g, int k) {
@@ -250,9 +242,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int b = bg / p.G, g = bg % p.G;
   const int kv0 = tile * kBT;
   // query tiles i0 .. n_tiles-1 (frame-causal: the first query that may see key kv0 opens the range)
-  const int i0 = (p.frame_hw && kv0 >= p.text_len)
-                     ? (p.text_len + (kv0 - p.text_len) / p.frame_hw * p.frame_hw) / kBT
-                     : 0;
+  const int i0 = p.frame_hw ? causal_block_start(kv0, p.text_len, p.frame_hw) / kBT : 0;
   const int nq = p.n_tiles - i0;
   const int chan0 = h * D;
   const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
@@ -399,7 +389,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quarter * 32 + lane;                    // key row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
-    const int bk = p.frame_hw ? causal_block(kv0 + row, p.text_len, p.frame_hw) : 0;   // this key's block
+    const int kstart = p.frame_hw ? causal_block_start(kv0 + row, p.text_len, p.frame_hw) : 0;   // its block's start
     for (int t = 0; t < 2 * nq; ++t) {
       const int il = t >> 1, i = i0 + il, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
@@ -408,7 +398,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          kSub * hh + 32 * half;
       const int qa = i * kBT + kSub * hh + 32 * half;   // this warp's first query column
       const int valid_q = p.n - qa;
-      const uint32_t vis = p.frame_hw ? causal_columns(qa, bk, p.text_len, p.frame_hw) : 0xffffffffu;
+      const uint32_t vis = p.frame_hw ? causal_columns(qa, kstart) : 0xffffffffu;
       const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
       uint32_t s[32], dp[32];
       tmem_ld32(tS, s);
@@ -462,7 +452,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int tile = blockIdx.x % p.n_tiles;
+  // frame-causal: a head's query tiles in reverse, so that those seeing the most keys start first
+  const int tile = p.frame_hw ? p.n_tiles - 1 - (int)(blockIdx.x % p.n_tiles) : (int)(blockIdx.x % p.n_tiles);
   const int hb = blockIdx.x / p.n_tiles;
   const int h = hb % p.heads, bg = hb / p.heads;
   const int b = bg / p.G, g = bg % p.G;
