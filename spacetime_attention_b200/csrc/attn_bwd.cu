@@ -174,6 +174,22 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_
                                           const float* lse_col, const float* dv_col, float lse_row, float dv_row,
                                           int valid, uint32_t (&pk)[16], uint32_t (&dk)[16],
                                           uint32_t vis = 0xffffffffu) {
+  if (valid >= 32 && vis == 0xffffffffu) {   // every column real and visible: no per-element mask
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float pv[2], dsv[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float l = kPerColumn ? lse_col[e + u] : lse_row;
+        const float dd = kPerColumn ? dv_col[e + u] : dv_row;
+        pv[u] = ex2_approx(fmaf(__uint_as_float(s[e + u]), sl2, -l));
+        dsv[u] = pv[u] * (__uint_as_float(dp[e + u]) - dd);
+      }
+      pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+      dk[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+    }
+    return;
+  }
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float pv[2], dsv[2];
