@@ -34,6 +34,8 @@ from .spacetime_oracle import (  # noqa: F401
     skiparse_text_attn_ref,
     softmax_rows,
     spatial_attn_ref,
+    spatial_backward_ref,
     temporal_attn_ref,
+    temporal_backward_ref,
     video_positions,
 )

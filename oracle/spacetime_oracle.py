@@ -640,3 +640,49 @@ def frame_causal_backward_ref(q, k, v, do, grid: Sequence[int], text_len: int, s
             out[1][b, :, h] = ds.T @ qh * scale
             out[2][b, :, h] = p.T @ dh
     return tuple(out)
+
+
+def spatial_backward_ref(q, k, v, do, grid: Sequence[int], scale: float | None = None):
+    """Gradients of per-frame attention (spatial_attn_ref): every frame's own backward by the
+    chain rule above.  q, k, v, do: [B, T*H*W, n_h, d] video tokens."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    if N != T * H * W:
+        raise ValueError("spatial attention takes the T*H*W video tokens only")
+    scale = default_scale(d) if scale is None else scale
+    HW = H * W
+    out = [np.empty((B, N, nh, d)) for _ in range(3)]
+    for b in range(B):
+        for t in range(T):
+            f = slice(t * HW, (t + 1) * HW)
+            for h in range(nh):
+                g = attention_head_backward_ref(q[b, f, h], k[b, f, h], v[b, f, h], do[b, f, h], scale)
+                for o_, g_ in zip(out, g):
+                    o_[b, f, h] = g_
+    return tuple(out)
+
+
+def temporal_backward_ref(q, k, v, do, grid: Sequence[int], causal: bool = False, scale: float | None = None):
+    """Gradients of per-position attention over time (temporal_attn_ref): for each spatial
+    position, the chain rule above over its T tokens, with P zero where t' > t when causal."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    if N != T * H * W:
+        raise ValueError("temporal attention takes the T*H*W video tokens only")
+    scale = default_scale(d) if scale is None else scale
+    HW = H * W
+    allowed = np.tril(np.ones((T, T), dtype=bool)) if causal else np.ones((T, T), dtype=bool)
+    out = [np.empty((B, N, nh, d)) for _ in range(3)]
+    for b in range(B):
+        for pos in range(HW):
+            idx = pos + HW * np.arange(T)
+            for h in range(nh):
+                qh, kh, vh, dh = (np.asarray(a[b, idx, h], np.float64) for a in (q, k, v, do))
+                p = softmax_rows(np.where(allowed, (qh @ kh.T) * scale, -np.inf))
+                o = p @ vh
+                ds = p * (dh @ vh.T - (dh * o).sum(axis=1, keepdims=True))
+                out[0][b, idx, h] = ds @ kh * scale
+                out[1][b, idx, h] = ds.T @ qh * scale
+                out[2][b, idx, h] = p.T @ dh
+    return tuple(out)
+

@@ -647,3 +647,51 @@ def test_frame_causal_backward_matches_finite_differences():
     np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
     # keys of the last frame are seen only by the last frame's queries: their dV is P^T dO of those
     assert not np.allclose(dv[0, 5:], 0)
+
+
+def test_spatial_backward_matches_finite_differences_and_reduces_to_dense():
+    rng = np.random.default_rng(85)
+    grid = (2, 1, 3)                             # two frames of three tokens
+    q, k, v = (rng.standard_normal((1, 6, 2, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 6, 2, 3))
+    loss = lambda q_, k_, v_: float((O.spatial_attn_ref(q_, k_, v_, grid, scale=0.6) * G).sum())
+    dq, dk, dv = O.spatial_backward_ref(q, k, v, G, grid, scale=0.6)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+    # one frame: spatial attention is full attention over the frame
+    for a, b in zip(O.spatial_backward_ref(q, k, v, G, (1, 2, 3), scale=0.6),
+                    O.attn_backward_ref(q, k, v, G, scale=0.6)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_temporal_backward_matches_finite_differences(causal):
+    rng = np.random.default_rng(86 + causal)
+    grid = (3, 1, 2)                             # three frames, two positions
+    q, k, v = (rng.standard_normal((1, 6, 1, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 6, 1, 3))
+    loss = lambda q_, k_, v_: float((O.temporal_attn_ref(q_, k_, v_, grid, causal=causal) * G).sum())
+    dq, dk, dv = O.temporal_backward_ref(q, k, v, G, grid, causal=causal)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+    if causal:   # a first-frame query sees its own key only: softmax over one key, dQ = 0
+        np.testing.assert_allclose(dq[0, :2], 0, atol=1e-14)
+        assert np.abs(dq[0, 2:]).max() > 1e-3
+
+
+def test_temporal_backward_special_cases():
+    rng = np.random.default_rng(88)
+    q, k, v, G = (rng.standard_normal((2, 5, 2, 4)) for _ in range(4))
+    # one position: attention over the T tokens (full), frame-causal with one-token frames (causal)
+    for a, b in zip(O.temporal_backward_ref(q, k, v, G, (5, 1, 1)), O.attn_backward_ref(q, k, v, G)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    for a, b in zip(O.temporal_backward_ref(q, k, v, G, (5, 1, 1), causal=True),
+                    O.frame_causal_backward_ref(q, k, v, G, (5, 1, 1), 0)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    # a position's tokens t*H*W + pos are the Single Skip set pos with k = H*W
+    q, k, v, G = (rng.standard_normal((1, 12, 1, 4)) for _ in range(4))
+    for a, b in zip(O.temporal_backward_ref(q, k, v, G, (3, 2, 2)),
+                    O.skiparse_backward_ref(q, k, v, G, 4, O.SKIP_SINGLE)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
