@@ -163,8 +163,9 @@ ATTN_MODE = {"value": "auto"}
 
 
 def sparse(w) -> bool:
-    """Skiparse pair (Single + Group) for workloads that define k, unless --attn dense / frame_causal."""
-    return bool(w.skiparse_k) and ATTN_MODE["value"] not in ("dense", "frame_causal")
+    """Skiparse pair (Single + Group) for workloads that define k, unless --attn names another form."""
+    return bool(w.skiparse_k) and ATTN_MODE["value"] not in ("dense", "frame_causal", "spatial", "temporal",
+                                                             "temporal_causal")
 
 
 def attention_launches(w, sms: int) -> int:
@@ -472,11 +473,22 @@ def run_backward_op(args, rank, world, local_rank):
     w = syn.WORKLOADS[args.workload]
     q, k, v = (t.to(dev) for t in syn.make_qkv(w, w.seed + 17 * rank))
     do = syn.randn_bf16(tuple(q.shape), w.seed + 99 + 17 * rank).to(dev)
-    causal = ATTN_MODE["value"] == "frame_causal"
+    attn = ATTN_MODE["value"]
+    causal = attn == "frame_causal"
+    factor = attn in ("spatial", "temporal", "temporal_causal")
     modes = [(w.skiparse_k, ops.OSP_SKIP_SINGLE), (w.skiparse_k, ops.OSP_SKIP_GROUP)] if sparse(w) else [(1, 0)]
     L = 0 if sparse(w) else w.text_len
+    if factor:   # the factorized attention runs over the video tokens only
+        q, k, v, do = (t[:, L:].contiguous() for t in (q, k, v, do))
+        L = 0
+        modes = [(1, 0)]
+    t_causal = attn == "temporal_causal"
     if causal:
         saved = [ops.attn_frame_causal_train(q, k, v, w.grid, L)]
+    elif attn == "spatial":
+        saved = [ops.attn_spatial_train(q, k, v, w.grid)]
+    elif factor:
+        saved = [ops.attn_temporal_train(q, k, v, w.grid, causal=t_causal)]
     else:
         saved = [ops.attn_forward_train(q, k, v, w.grid, L, sparse_k=kk, mode=m) for kk, m in modes]
     grads = [tuple(torch.empty_like(q) for _ in range(3)) for _ in modes]
@@ -485,6 +497,10 @@ def run_backward_op(args, rank, world, local_rank):
         for (kk, m), (o, lse), (dq, dk, dv) in zip(modes, saved, grads):
             if causal:
                 ops.attn_frame_causal_backward(q, k, v, o, do, lse, w.grid, L, dq=dq, dk=dk, dv=dv)
+            elif attn == "spatial":
+                ops.attn_spatial_backward(q, k, v, o, do, lse, w.grid, dq=dq, dk=dk, dv=dv)
+            elif factor:
+                ops.attn_temporal_backward(q, k, v, o, do, lse, w.grid, causal=t_causal, dq=dq, dk=dk, dv=dv)
             else:
                 ops.attn_backward(q, k, v, o, do, lse, w.grid, L, sparse_k=kk, mode=m, dq=dq, dk=dk, dv=dv)
 
@@ -506,27 +522,42 @@ def run_backward_op(args, rank, world, local_rank):
     ops.check_status(dev)
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
     peaks, src = load_peaks()
+    T, H, W = w.grid
+    HW = H * W
     if causal:   # unmasked (query, key) pairs only
-        T, H, W = w.grid
-        HW = H * W
         pairs = w.B * (L * L + sum(HW * (L + (t + 1) * HW) for t in range(T)))
-        flops = 2.5 * 4.0 * w.heads * w.head_dim * pairs
+    elif attn == "spatial":
+        pairs = w.B * T * HW * HW
+    elif factor:
+        pairs = w.B * HW * (T * (T + 1) // 2 if t_causal else T * T)
     else:
-        flops = 2.5 * step_flops(w)
+        pairs = None
+    flops = 2.5 * 4.0 * w.heads * w.head_dim * pairs if pairs is not None else 2.5 * step_flops(w)
     tflops = flops / (ms * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops_sustained"])
+    # algorithmic bytes: q, k, v, o, dO read and dQ, dK, dV written once (bf16), lse read (fp32)
+    rows = q.shape[0] * q.shape[1] * w.heads
+    nbytes = len(modes) * (8 * 2 * rows * w.head_dim + 4 * rows)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    t_tensor = flops / (float(peaks["bf16_tflops_sustained"]) * 1e12)
+    t_hbm = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": float(peaks["bf16_tflops_sustained"]),
+                "unit": "TFLOP/s", "frac": round(tflops / float(peaks["bf16_tflops_sustained"]), 4),
+                "peak_source": f"{src} (sustained bf16 GEMM)"}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": f"{src} (copy bandwidth)"}
+    roof.update(traffic=None, kernel="attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel",
+                bytes_per_step=nbytes)
+    label = {"frame_causal": "frame-causal", "spatial": "spatial (per frame)", "temporal": "temporal (per position)",
+             "temporal_causal": "causal temporal (per position)"}.get(attn, "skiparse pair" if sparse(w) else "dense")
     return {"metric": "attention backward TFLOP/s (2.5x forward flops)", "value": round(world * tflops, 1),
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": dict(w.describe(), op="backward",
-                           attn="frame-causal" if causal else ("skiparse pair" if sparse(w) else "dense"),
-                           flops_per_step=flops, l2="inputs > L2, no flush"),
-            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(tflops / peak, 4), "traffic": None,
-                         "kernel": "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel",
-                         "peak_source": f"{src} (sustained bf16 GEMM)"},
-            "clocks": clocks, "gpu_launches": 3 * len(modes) * args.steps}
+            "config": dict(w.describe(), op="backward", attn=label, flops_per_step=flops,
+                           l2="inputs > L2, no flush"),
+            "roofline": roof, "clocks": clocks, "gpu_launches": 3 * len(modes) * args.steps}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -761,9 +792,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="cogvideox_2b", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--attn", default="auto", choices=["auto", "dense", "skiparse", "frame_causal"],
+    ap.add_argument("--attn", default="auto",
+                    choices=["auto", "dense", "skiparse", "frame_causal", "spatial", "temporal", "temporal_causal"],
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention; "
-                         "frame_causal: the frame-causal backward (--op backward)")
+                         "frame_causal / spatial / temporal / temporal_causal: that backward (--op backward)")
     ap.add_argument("--op", default="step",
                     choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
                              "frame_causal", "skiparse_text", "backward"],
@@ -778,8 +810,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.attn == "frame_causal" and args.op != "backward":
-        ap.error("--attn frame_causal applies to --op backward (use --op frame_causal for the forward)")
+    if args.attn in ("frame_causal", "spatial", "temporal", "temporal_causal") and args.op != "backward":
+        ap.error(f"--attn {args.attn} applies to --op backward (use --op {args.attn.split('_')[0]} for the forward)")
     ATTN_MODE["value"] = args.attn
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

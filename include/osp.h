@@ -17,7 +17,7 @@
  *     frame-causal attention (the Sora page);
  *   - packed batches of videos of different shapes, with per-sample RoPE grids and
  *     block-diagonal attention (CogVideoX section 3.1 "Multi-Resolution Frame Pack");
- *   - the backward pass of dense, Skiparse and frame-causal attention (training).
+ *   - the backward pass of dense, Skiparse, frame-causal and factorized attention (training).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -202,6 +202,31 @@ int osp_attn_frame_causal_train(const void* q, const void* k, const void* v, voi
 int osp_attn_frame_causal_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
                                    const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape,
                                    float softmax_scale, void* stream);
+
+/* Training of the factorized (2D + 1D) attention (osp_attn_spatial, osp_attn_temporal): the
+ * forward with its saved lse and the backward, with the arithmetic of osp_attn_forward_train /
+ * osp_attn_backward.  Video tokens only (text_len 0); q, k, v, o, dout, dq, dk, dv as
+ * osp_attn_backward (written completely, no overlap with the inputs).
+ *
+ * osp_attn_spatial_train / _backward: the dense kernels on the B*T frames, each of H*W tokens;
+ *   lse[((b*T + t)*heads + h)*n_pad + (h'*W + w)], n_pad = ceil(H*W / 128) * 128.
+ * osp_attn_temporal_train / _backward: the Skiparse kernels with spatial position pos = h*W + w
+ *   as Single Skip set pos, k = H*W (slot t = frame t; causal = 1: P zero where t' > t, through
+ *   the block-causal mask with one-slot blocks); lse[((b*H*W + pos)*heads + h)*n_pad + t],
+ *   n_pad = ceil(T / 128) * 128.  Every set is one 128-row tile (T <= 128) or a few; for short
+ *   clips most of each tile is padding.
+ *  Errors: OSP_ERR_INVALID_ARG (null or unaligned pointer, causal not 0/1), OSP_ERR_UNSUPPORTED
+ *  (text, head_dim, too many frames or positions), OSP_ERR_CUDA. */
+int osp_attn_spatial_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
+                           float softmax_scale, void* stream);
+int osp_attn_spatial_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape,
+                              float softmax_scale, void* stream);
+int osp_attn_temporal_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
+                            int32_t causal, float softmax_scale, void* stream);
+int osp_attn_temporal_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                               const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape, int32_t causal,
+                               float softmax_scale, void* stream);
 
 /* 3D RoPE of a packed batch (CogVideoX section 3.1: every video keeps its own position grid,
  * starting at (0, 0, 0); extrapolation, never rescaled).

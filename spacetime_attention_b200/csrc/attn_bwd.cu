@@ -666,7 +666,8 @@ int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const C
 
 int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
-                              int sparse_k, float scale, cudaStream_t stream, bool frame_causal) {
+                              int sparse_k, float scale, cudaStream_t stream, bool frame_causal,
+                              int causal_block) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   const int N = s.text_len + s.T * s.H * s.W;
@@ -690,7 +691,7 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
   p.elems = (unsigned long long)s.B * N * s.heads * s.head_dim / bounds_check_divisor();
-  p.frame_hw = frame_causal ? s.H * s.W : 0;
+  p.frame_hw = frame_causal ? (causal_block > 0 ? causal_block : s.H * s.W) : 0;
   p.text_len = s.text_len;
   p.vec_elems = (unsigned long long)s.B * G * s.heads * p.vec_stride / bounds_check_divisor();
   const long long ctas = (long long)p.n_tiles * s.heads * s.B * G;

@@ -195,7 +195,8 @@ AttnParams base_params(const osp_shape& s, int layout, int sparse_k, float scale
   return p;
 }
 
-// frame_causal: dense layout only; the frame-causal mask over s's text block and frames.
+// frame_causal: the block-causal mask over a set's slots: s's text block, then blocks of
+// causal_block slots (a frame, H*W, when 0).
 int launch_with_status(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int layout,
                        int sparse_k, float scale, cudaStream_t stream, unsigned* status, bool allow_split,
                        int N_kv = -1, bool frame_causal = false, float* lse = nullptr, int causal_block = 0) {
@@ -299,10 +300,11 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
 
 int attention_forward_lse_launch(const void* q, const void* k, const void* v, void* o, float* lse,
                                  const osp_shape& s, int layout, int sparse_k, float scale, cudaStream_t stream,
-                                 bool frame_causal) {
+                                 bool frame_causal, int causal_block) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
-  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true, -1, frame_causal, lse);
+  return launch_with_status(q, k, v, o, s, layout, sparse_k, scale, stream, status, true, -1, frame_causal, lse,
+                            causal_block);
 }
 
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,

@@ -359,6 +359,99 @@ int osp_attn_frame_causal_backward(const void* q, const void* k, const void* v, 
                                    static_cast<cudaStream_t>(stream), true);
 }
 
+// Factorized (2D + 1D) training: per-frame attention is dense attention over the frames
+// [B*T][H*W]; the temporal set of spatial position pos is Single Skip set pos with k = H*W
+// (slot t = frame t), causal through the block-causal mask with one-slot blocks.
+static int check_factorized(const osp_shape* shape, const char* what) {
+  int rc = check_shape(shape, true);
+  if (rc) return rc;
+  if (shape->text_len != 0)
+    return set_error(OSP_ERR_UNSUPPORTED, "%s attention takes video tokens only (text_len 0)", what);
+  if ((long long)shape->B * shape->T > (1LL << 30) || (long long)shape->B * shape->H * shape->W > (1LL << 30))
+    return set_error(OSP_ERR_UNSUPPORTED, "too many frames or positions");
+  return OSP_OK;
+}
+
+static bool fwd_ptrs_ok(const void* q, const void* k, const void* v, const void* o, const void* lse) {
+  if (!q || !k || !v || !o || !lse) {
+    set_error(OSP_ERR_INVALID_ARG, "null pointer");
+    return false;
+  }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) {
+    set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    return false;
+  }
+  return true;
+}
+
+static bool bwd_ptrs_ok(const void* q, const void* k, const void* v, const void* o, const void* dout, const void* lse,
+                        const void* dq, const void* dk, const void* dv) {
+  if (!fwd_ptrs_ok(q, k, v, o, lse)) return false;
+  if (!dout || !dq || !dk || !dv) {
+    set_error(OSP_ERR_INVALID_ARG, "null pointer");
+    return false;
+  }
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) {
+    set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    return false;
+  }
+  return true;
+}
+
+static osp_shape frames_of(const osp_shape& s) {
+  return osp_shape{s.B * s.T, 0, 1, 1, s.H * s.W, s.heads, s.head_dim};
+}
+
+int osp_attn_spatial_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
+                           float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_factorized(shape, "spatial");
+  if (rc) return rc;
+  if (!fwd_ptrs_ok(q, k, v, o, lse)) return OSP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_forward_lse_launch(q, k, v, o, lse, frames_of(*shape), 0, 1, softmax_scale,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+int osp_attn_spatial_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape,
+                              float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_factorized(shape, "spatial");
+  if (rc) return rc;
+  if (!bwd_ptrs_ok(q, k, v, o, dout, lse, dq, dk, dv)) return OSP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  return attention_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, frames_of(*shape), 0, 1, softmax_scale,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int osp_attn_temporal_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
+                            int32_t causal, float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_factorized(shape, "temporal");
+  if (rc) return rc;
+  if (causal != 0 && causal != 1) return set_error(OSP_ERR_INVALID_ARG, "causal must be 0 or 1 (got %d)", causal);
+  if (!fwd_ptrs_ok(q, k, v, o, lse)) return OSP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  const int HW = shape->H * shape->W;
+  return attention_forward_lse_launch(q, k, v, o, lse, *shape, HW > 1 ? OSP_SKIP_SINGLE + 1 : 0, HW, softmax_scale,
+                                      static_cast<cudaStream_t>(stream), causal != 0, 1);
+}
+
+int osp_attn_temporal_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                               const float* lse, void* dq, void* dk, void* dv, const osp_shape* shape, int32_t causal,
+                               float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_factorized(shape, "temporal");
+  if (rc) return rc;
+  if (causal != 0 && causal != 1) return set_error(OSP_ERR_INVALID_ARG, "causal must be 0 or 1 (got %d)", causal);
+  if (!bwd_ptrs_ok(q, k, v, o, dout, lse, dq, dk, dv)) return OSP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  const int HW = shape->H * shape->W;
+  return attention_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, HW > 1 ? OSP_SKIP_SINGLE + 1 : 0, HW,
+                                   softmax_scale, static_cast<cudaStream_t>(stream), causal != 0, 1);
+}
+
 int osp_rope3d_packed(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,
                       int32_t n_samples, int32_t heads, int32_t head_dim, const osp_rope* rope, void* stream) {
   g_last_error[0] = 0;

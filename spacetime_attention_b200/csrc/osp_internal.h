@@ -98,12 +98,13 @@ int make_attn_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, 
 // the row log-sum-exp (log2 domain of the scaled scores) to lse, [B*G][heads][ceil(n/128)*128].
 int attention_forward_lse_launch(const void* q, const void* k, const void* v, void* o, float* lse,
                                  const osp_shape& s, int layout, int sparse_k, float scale, cudaStream_t stream,
-                                 bool frame_causal = false);
+                                 bool frame_causal = false, int causal_block = 0);
 
 // Backward pass of attention_forward_lse_launch: dq, dk, dv from q, k, v, o, dout and lse.
 int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
-                              int sparse_k, float scale, cudaStream_t stream, bool frame_causal = false);
+                              int sparse_k, float scale, cudaStream_t stream, bool frame_causal = false,
+                              int causal_block = 0);
 
 // Packed batch (block-diagonal attention): segment i owns q/o rows [q_bounds[i], q_bounds[i+1])
 // and k/v rows [kv_bounds[i], kv_bounds[i+1]); host arrays of n_seg + 1 validated offsets.

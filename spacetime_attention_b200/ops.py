@@ -10,6 +10,7 @@ every call raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional, Sequence
 
@@ -33,7 +34,9 @@ EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_
             "osp_skiparse_index_map", "osp_check_status", "osp_get_last_error", "osp_version",
             "osp_attn_full_noalloc", "osp_attn_cross", "osp_rope3d_packed", "osp_attn_packed",
             "osp_attn_spatial", "osp_attn_temporal", "osp_attn_frame_causal", "osp_attn_forward_train",
-            "osp_attn_backward", "osp_attn_frame_causal_train", "osp_attn_frame_causal_backward")
+            "osp_attn_backward", "osp_attn_frame_causal_train", "osp_attn_frame_causal_backward",
+            "osp_attn_spatial_train", "osp_attn_spatial_backward", "osp_attn_temporal_train",
+            "osp_attn_temporal_backward")
 
 MAX_SEGMENTS = 256   # OSP_MAX_SEGMENTS
 
@@ -81,6 +84,10 @@ def library() -> ctypes.CDLL:
             "osp_attn_frame_causal_train": [vp, vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_frame_causal_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_attn_temporal": [vp, vp, vp, vp, sp, i32, ctypes.c_float, vp],
+            "osp_attn_spatial_train": [vp, vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_spatial_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, ctypes.c_float, vp],
+            "osp_attn_temporal_train": [vp, vp, vp, vp, vp, sp, i32, ctypes.c_float, vp],
+            "osp_attn_temporal_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, sp, i32, ctypes.c_float, vp],
             "osp_attn_frame_causal": [vp, vp, vp, vp, sp, ctypes.c_float, vp],
             "osp_rope3d_packed": [vp, vp, vp, vp, ctypes.POINTER(OspSampleGrid), i32, i32, i32, rp, vp],
             "osp_attn_packed": [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
@@ -210,13 +217,24 @@ def lse_shape(q: torch.Tensor, sparse_k: int = 1):
     return (B * G, heads, (n + 127) // 128 * 128)
 
 
+def _lse_buffer(lse, shape, q: torch.Tensor) -> torch.Tensor:
+    """The caller's lse buffer, checked against the shape the call writes, or a new one."""
+    if lse is None:
+        return torch.empty(shape, dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or lse.device != q.device or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor on q's device")
+    if lse.numel() < math.prod(shape):
+        raise ValueError(f"lse holds {lse.numel()} values, the call writes {shape}")
+    return lse
+
+
 def attn_forward_train(q, k, v, grid, text_len: int = 0, sparse_k: int = 1, mode: int = 0, scale: float = 0.0,
                        o=None, lse=None):
     """osp_attn_forward_train: returns (o, lse)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _bshd(t, n)
     o = torch.empty_like(q) if o is None else o
-    lse = torch.empty(lse_shape(q, sparse_k), dtype=torch.float32, device=q.device) if lse is None else lse
+    lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_forward_train",
            library().osp_attn_forward_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
@@ -232,6 +250,7 @@ def attn_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, sparse_k: int 
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_backward",
            library().osp_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
@@ -245,7 +264,7 @@ def attn_frame_causal_train(q, k, v, grid, text_len: int = 0, scale: float = 0.0
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _bshd(t, n)
     o = torch.empty_like(q) if o is None else o
-    lse = torch.empty(lse_shape(q, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    lse = _lse_buffer(lse, lse_shape(q, 1), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_frame_causal_train",
            library().osp_attn_frame_causal_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
@@ -261,12 +280,69 @@ def attn_frame_causal_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, s
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    lse = _lse_buffer(lse, lse_shape(q, 1), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_frame_causal_backward",
            library().osp_attn_frame_causal_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                                                     _ptr(dq), _ptr(dk), _ptr(dv), ctypes.byref(shp),
                                                     ctypes.c_float(scale), _stream_handle(q)))
     return dq, dk, dv
+
+
+def factorized_lse_shape(q: torch.Tensor, grid, temporal: bool):
+    """Shape of the lse buffer of the factorized training calls: [B*T, heads, ceil(H*W/128)*128]
+    (spatial, one set per frame) or [B*H*W, heads, ceil(T/128)*128] (temporal, one per position)."""
+    B, _, heads, _ = q.shape
+    T, H, W = (int(a) for a in grid)
+    sets, n = (B * H * W, T) if temporal else (B * T, H * W)
+    return (sets, heads, (n + 127) // 128 * 128)
+
+
+def _factorized_train(fn: str, q, k, v, grid, temporal: bool, extra, scale, o, lse):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    o = torch.empty_like(q) if o is None else o
+    lse = _lse_buffer(lse, factorized_lse_shape(q, grid, temporal), q)
+    shp = _shape_of(q, grid, 0)
+    _check(fn, getattr(library(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp), *extra,
+                                      ctypes.c_float(scale), _stream_handle(q)))
+    return o, lse
+
+
+def _factorized_backward(fn: str, q, k, v, o, dout, lse, grid, temporal: bool, extra, scale, dq, dk, dv):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _bshd(t, n)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    lse = _lse_buffer(lse, factorized_lse_shape(q, grid, temporal), q)
+    shp = _shape_of(q, grid, 0)
+    _check(fn, getattr(library(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), ctypes.byref(shp), *extra, ctypes.c_float(scale), _stream_handle(q)))
+    return dq, dk, dv
+
+
+def attn_spatial_train(q, k, v, grid, scale: float = 0.0, o=None, lse=None):
+    """osp_attn_spatial_train: per-frame attention with its saved lse; returns (o, lse)."""
+    return _factorized_train("osp_attn_spatial_train", q, k, v, grid, False, (), scale, o, lse)
+
+
+def attn_spatial_backward(q, k, v, o, dout, lse, grid, scale: float = 0.0, dq=None, dk=None, dv=None):
+    """osp_attn_spatial_backward: returns (dq, dk, dv)."""
+    return _factorized_backward("osp_attn_spatial_backward", q, k, v, o, dout, lse, grid, False, (), scale,
+                                dq, dk, dv)
+
+
+def attn_temporal_train(q, k, v, grid, causal: bool = False, scale: float = 0.0, o=None, lse=None):
+    """osp_attn_temporal_train: per-position attention over time with its saved lse; returns (o, lse)."""
+    return _factorized_train("osp_attn_temporal_train", q, k, v, grid, True, (int(bool(causal)),), scale, o, lse)
+
+
+def attn_temporal_backward(q, k, v, o, dout, lse, grid, causal: bool = False, scale: float = 0.0, dq=None, dk=None,
+                           dv=None):
+    """osp_attn_temporal_backward: returns (dq, dk, dv)."""
+    return _factorized_backward("osp_attn_temporal_backward", q, k, v, o, dout, lse, grid, True,
+                                (int(bool(causal)),), scale, dq, dk, dv)
 
 
 def _bounds(b) -> ctypes.Array:

@@ -155,3 +155,30 @@ def test_frame_causal_training_validation(lib):
     assert lib.osp_attn_frame_causal_train(p, p, p, p, None, shp(), 0.0, None) == 1
     assert lib.osp_attn_frame_causal_backward(p, p, p, p, p, p, p, p, None, shp(), 0.0, None) == 1
     assert lib.osp_attn_frame_causal_backward(p, p, p, p, p, p, p, p, p, shp(d=80), 0.0, None) == 2
+
+
+def test_factorized_training_validation(lib):
+    p, bad = ctypes.c_void_p(256), ctypes.c_void_p(264)
+    assert lib.osp_attn_spatial_train(p, p, p, p, None, shp(), 0.0, None) == 1               # no lse
+    assert lib.osp_attn_spatial_train(p, p, p, p, bad, shp(), 0.0, None) == 1                # misaligned lse
+    assert lib.osp_attn_spatial_train(p, p, p, p, p, shp(L=2), 0.0, None) == 2               # text not allowed
+    assert lib.osp_attn_spatial_backward(p, p, p, p, p, p, p, None, p, shp(), 0.0, None) == 1
+    assert lib.osp_attn_spatial_backward(p, p, p, p, p, p, p, p, p, shp(d=80), 0.0, None) == 2
+    assert lib.osp_attn_temporal_train(p, p, p, p, p, shp(), 2, 0.0, None) == 1             # causal must be 0/1
+    assert lib.osp_attn_temporal_train(p, p, p, p, p, shp(L=1), 0, 0.0, None) == 2
+    assert lib.osp_attn_temporal_backward(p, p, p, p, p, p, p, p, p, shp(), -1, 0.0, None) == 1
+    assert lib.osp_attn_temporal_backward(p, p, p, p, p, p, p, p, bad, shp(), 1, 0.0, None) == 1
+    assert lib.osp_attn_temporal_backward(p, p, p, p, p, p, p, p, p, shp(d=60), 0, 0.0, None) == 2
+
+
+def test_binding_checks_the_lse_buffer():
+    import torch
+    q = torch.zeros((1, 32, 2, 64), dtype=torch.bfloat16)
+    assert ops.factorized_lse_shape(q, (4, 2, 4), temporal=False) == (4, 2, 128)
+    assert ops.factorized_lse_shape(q, (4, 2, 4), temporal=True) == (8, 2, 128)
+    with pytest.raises(ValueError):
+        ops._lse_buffer(torch.zeros(10), (4, 2, 128), q)                  # too small
+    with pytest.raises(ValueError):
+        ops._lse_buffer(torch.zeros((4, 2, 128), dtype=torch.float64), (4, 2, 128), q)
+    buf = torch.zeros((4, 2, 128))
+    assert ops._lse_buffer(buf, (4, 2, 128), q) is buf

@@ -1,0 +1,108 @@
+"""GPU parity of the factorized (2D + 1D) training calls: per-frame spatial and per-position
+temporal attention, forward with saved log-sum-exp and backward, against the fp64 oracle
+(spatial_backward_ref / temporal_backward_ref, pinned by finite differences and by reduction to
+the dense, frame-causal and Single Skip backward).  Tolerances as the other backward tests: P and
+dS rounded to bf16 before the tensor-core products, fp32 accumulation, bf16 outputs."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from spacetime_attention_b200 import ops, synthetic as syn
+from tests.gpu_common import gpu  # noqa: F401
+from tests.helpers import assert_attn_close, to_f64
+from tests.test_gpu_backward import assert_grad_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, heads, d, grid, seed):
+    N = grid[0] * grid[1] * grid[2]
+    return tuple(syn.randn_bf16((B, N, heads, d), seed + i) for i in range(4))
+
+
+SPATIAL = [
+    # B, heads, d, grid
+    (1, 2, 64, (3, 8, 16)),       # 128-token frames: one tile each
+    (2, 2, 96, (2, 9, 15)),       # 135-token frames: ragged second tile
+    (1, 1, 128, (4, 5, 7)),       # 35-token frames
+]
+
+
+@pytest.mark.parametrize("case", SPATIAL, ids=[f"{c[3]}_d{c[2]}_B{c[0]}" for c in SPATIAL])
+def test_spatial_backward_matches_oracle(gpu, case):
+    B, heads, d, grid = case
+    q, k, v, do = _inputs(B, heads, d, grid, 120)
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    o, lse = ops.attn_spatial_train(qg, kg, vg, grid)
+    dq, dk, dv = ops.attn_spatial_backward(qg, kg, vg, o, dog, lse, grid)
+    ops.check_status()
+    # the training forward is the inference forward, bit for bit
+    assert torch.equal(o, ops.attn_spatial(qg, kg, vg, grid))
+    rq, rk, rv = O.spatial_backward_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), grid)
+    assert_grad_close(dq, rq, "dq")
+    assert_grad_close(dk, rk, "dk")
+    assert_grad_close(dv, rv, "dv")
+    # lse of frame t, head h, slot = the token's index within the frame (log2 domain)
+    T, H, W = grid
+    HW = H * W
+    scale = 1 / math.sqrt(d)
+    for b, t, h in ((0, 0, 0), (B - 1, T - 1, heads - 1)):
+        f = slice(t * HW, (t + 1) * HW)
+        ref = O.attention_head_lse_ref(to_f64(q)[b, f, h], to_f64(k)[b, f, h], scale) / math.log(2.0)
+        np.testing.assert_allclose(lse[b * T + t, h, :HW].double().cpu().numpy(), ref, rtol=0, atol=2e-3)
+
+
+TEMPORAL = [
+    # B, heads, d, grid
+    (1, 2, 64, (13, 3, 4)),       # 13 frames, one partial tile per position
+    (2, 1, 96, (80, 2, 3)),       # longer than the inference kernel's shared-memory limit
+    (1, 2, 128, (130, 1, 2)),     # two tiles per position, ragged
+    (1, 1, 64, (7, 1, 1)),        # one position: the dense layout
+    (1, 1, 64, (13, 16, 20)),     # 320 one-tile work units: the forward runs them in turn
+]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", TEMPORAL, ids=[f"{c[3]}_d{c[2]}_B{c[0]}" for c in TEMPORAL])
+def test_temporal_backward_matches_oracle(gpu, case, causal):
+    B, heads, d, grid = case
+    q, k, v, do = _inputs(B, heads, d, grid, 130 + causal)
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    o, lse = ops.attn_temporal_train(qg, kg, vg, grid, causal=causal)
+    dq, dk, dv = ops.attn_temporal_backward(qg, kg, vg, o, dog, lse, grid, causal=causal)
+    ops.check_status()
+    qd, kd, vd = to_f64(q), to_f64(k), to_f64(v)
+    assert_attn_close(o, O.temporal_attn_ref(qd, kd, vd, grid, causal=causal), f"temporal train {grid}")
+    rq, rk, rv = O.temporal_backward_ref(qd, kd, vd, to_f64(do), grid, causal=causal)
+    assert_grad_close(dq, rq, "dq")
+    assert_grad_close(dk, rk, "dk")
+    assert_grad_close(dv, rv, "dv")
+    # lse of position pos, head h, slot t: over keys t' (all, or t' <= t when causal)
+    T, H, W = grid
+    HW = H * W
+    scale = 1 / math.sqrt(d)
+    for b, pos, h in ((0, 0, 0), (B - 1, HW - 1, heads - 1)):
+        idx = pos + HW * np.arange(T)
+        got = lse[b * HW + pos, h, :T].double().cpu().numpy()
+        if causal:
+            ref = np.array([O.attention_head_lse_ref(qd[b, idx[t:t + 1], h], kd[b, idx[:t + 1], h], scale)[0]
+                            for t in range(T)])
+        else:
+            ref = O.attention_head_lse_ref(qd[b, idx, h], kd[b, idx, h], scale)
+        np.testing.assert_allclose(got, ref / math.log(2.0), rtol=0, atol=2e-3)
+
+
+def test_causal_temporal_first_frame_has_no_query_gradient(gpu):
+    # a first-frame query sees only its own key: softmax over one key, so dQ = 0 up to the fp32
+    # rounding of dP - rowsum(dO * O) (two sums of the same products in different orders)
+    q, k, v, do = _inputs(1, 2, 64, (6, 4, 4), 140)
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    o, lse = ops.attn_temporal_train(qg, kg, vg, (6, 4, 4), causal=True)
+    dq, _, _ = ops.attn_temporal_backward(qg, kg, vg, o, dog, lse, (6, 4, 4), causal=True)
+    ops.check_status()
+    first, rest = dq[:, :16].float().abs().max().item(), dq[:, 16:].float().abs().max().item()
+    assert rest > 0 and first <= 1e-2 * rest
