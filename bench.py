@@ -547,8 +547,10 @@ def run_backward_op(args, rank, world, local_rank):
     else:
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                 "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": f"{src} (copy bandwidth)"}
-    roof.update(traffic=None, kernel="attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel",
-                bytes_per_step=nbytes)
+    per_set = attn in ("temporal", "temporal_causal") and T <= 64 and os.environ.get("OSP_TEMPORAL_BWD", "0") != "0"
+    roof.update(traffic=None, bytes_per_step=nbytes,
+                kernel="attn_temporal_bwd_kernel" if per_set
+                else "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel")
     label = {"frame_causal": "frame-causal", "spatial": "spatial (per frame)", "temporal": "temporal (per position)",
              "temporal_causal": "causal temporal (per position)"}.get(attn, "skiparse pair" if sparse(w) else "dense")
     return {"metric": "attention backward TFLOP/s (2.5x forward flops)", "value": round(world * tflops, 1),
@@ -557,7 +559,7 @@ def run_backward_op(args, rank, world, local_rank):
             "dtype": "bf16", "data": "synthetic",
             "config": dict(w.describe(), op="backward", attn=label, flops_per_step=flops,
                            l2="inputs > L2, no flush"),
-            "roofline": roof, "clocks": clocks, "gpu_launches": 3 * len(modes) * args.steps}
+            "roofline": roof, "clocks": clocks, "gpu_launches": (1 if per_set else 3) * len(modes) * args.steps}
 
 
 def run_ours(args, rank, world, local_rank):

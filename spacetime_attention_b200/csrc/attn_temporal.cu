@@ -271,6 +271,291 @@ int launch_temporal_d(TemporalParams& p, cudaStream_t stream) {
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Backward of the temporal attention for T <= 64: one warp per set, as the forward.
+//
+// Per set the warp stages q, k, v, o and dO (T rows each) and the set's saved lse, forms
+// Dv_i = rowsum(dO_i * O_i), then runs two passes over the same mma.sync fragment patterns as
+// the forward (C = X Y^T from rows of X and Y; C = A Z with A the packed bf16 fragments of a
+// score tile and Z rows read transposed):
+//   keys major   (16 keys at a time):  S^T = K Q^T, dP^T = V dO^T, P^T = exp2(S^T * c - lse),
+//                                      dS^T = P^T * (dP^T - Dv); dV = P^T dO, dK = dS^T Q * scale;
+//   queries major (16 queries at a time): S, dP, P, dS as above; dQ = dS K * scale.
+// The second pass recomputes S and dP instead of transposing P / dS through shared memory:
+// the set's products are tiny next to its 16 rows of HBM traffic per token and head.
+// ------------------------------------------------------------------------------------------
+#ifndef OSP_TEMPORAL_BWD_SMEM_KB
+#define OSP_TEMPORAL_BWD_SMEM_KB 100
+#endif
+
+struct TemporalBwdParams {
+  const __nv_bfloat16 *q, *k, *v, *o, *dout;
+  const float* lse;
+  __nv_bfloat16 *dq, *dk, *dv;
+  int T, HW, heads;
+  long long n_sets;     // B * HW * heads, set s = (b * HW + pos) * heads + h
+  int lse_stride;       // floats between the lse rows of consecutive sets
+  float scale, scale_log2;
+  int causal;
+  int warps;
+  unsigned long long elems, lse_elems;
+  unsigned* status;
+};
+
+template <int D, int MT>
+struct TemporalBwdCfg {
+  static constexpr int kRows = 16 * MT;
+  static constexpr int kRowBytes = D * 2 + 16;
+  static constexpr int kTensorBytes = kRows * kRowBytes;
+  static constexpr int kOutOff = 5 * kTensorBytes;             // q, k, v, o, dO, then 16 output rows
+  static constexpr int kVecOff = kOutOff + 16 * kRowBytes;      // lse[kRows], Dv[kRows] (fp32)
+  static constexpr int kWarpBytes = kVecOff + 2 * kRows * 4;
+};
+
+// acc[2*MT] (16 x kRows, C layout) = rows x0 .. x0+15 of X times the kRows rows of Y, transposed
+template <int D, int MT>
+__device__ __forceinline__ void tb_rows_by_rows(uint32_t X, int x0, uint32_t Y, int lane, float (&acc)[2 * MT][4]) {
+  using C = TemporalBwdCfg<D, MT>;
+#pragma unroll
+  for (int nt = 0; nt < 2 * MT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a[4];
+    ldsm_x4(X + (uint32_t)((x0 + (lane & 15)) * C::kRowBytes + (kk * 16 + (lane >> 4) * 8) * 2), a[0], a[1], a[2],
+            a[3]);
+#pragma unroll
+    for (int n2 = 0; n2 < MT; ++n2) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(Y + (uint32_t)((n2 * 16 + (lane & 7) + ((lane >> 4) << 3)) * C::kRowBytes +
+                             (kk * 16 + ((lane >> 3) & 1) * 8) * 2),
+              b0, b1, b2, b3);
+      mma_bf16_16816(acc[2 * n2], a, b0, b1);
+      mma_bf16_16816(acc[2 * n2 + 1], a, b2, b3);
+    }
+  }
+}
+
+// out (16 x D, C layout) = A (16 x kRows, packed bf16 fragments) times the kRows rows of Z
+template <int D, int MT>
+__device__ __forceinline__ void tb_frag_by_rows(const uint32_t (&a)[MT][4], uint32_t Z, int lane,
+                                                float (&out)[D / 8][4]) {
+  using C = TemporalBwdCfg<D, MT>;
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt) out[nt][0] = out[nt][1] = out[nt][2] = out[nt][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < MT; ++kk) {
+#pragma unroll
+    for (int n2 = 0; n2 < D / 16; ++n2) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(Z + (uint32_t)((kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * C::kRowBytes +
+                               (n2 * 16 + (lane >> 4) * 8) * 2),
+                b0, b1, b2, b3);
+      mma_bf16_16816(out[2 * n2], a[kk], b0, b1);
+      mma_bf16_16816(out[2 * n2 + 1], a[kk], b2, b3);
+    }
+  }
+}
+
+// Writes a 16 x D fp32 C-layout tile, times mul, as bf16 rows r0 .. r0+15 (< T) of dst.
+template <int D, int MT>
+__device__ __forceinline__ void tb_store_rows(const float (&acc)[D / 8][4], float mul, uint32_t so, int lane, int r0,
+                                              int T, long long base, long long tstride, __nv_bfloat16* dst,
+                                              const TemporalBwdParams& p) {
+  using C = TemporalBwdCfg<D, MT>;
+  constexpr int kChunks = D / 8;
+  const int g = lane >> 2, c = lane & 3;
+  __syncwarp();
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt) {
+    const uint32_t col = (uint32_t)((nt * 8 + 2 * c) * 2);
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(so + (uint32_t)(g * C::kRowBytes) + col),
+                 "r"(pack_bf16x2(acc[nt][0] * mul, acc[nt][1] * mul))
+                 : "memory");
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(so + (uint32_t)((g + 8) * C::kRowBytes) + col),
+                 "r"(pack_bf16x2(acc[nt][2] * mul, acc[nt][3] * mul))
+                 : "memory");
+  }
+  __syncwarp();
+  const int rows = min(16, T - r0);
+  for (int ch = lane; ch < rows * kChunks; ch += 32) {
+    const int r = ch / kChunks, cc = ch - r * kChunks;
+    uint4 val;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                 : "r"(so + (uint32_t)(r * C::kRowBytes + cc * 16)));
+    const long long off = base + (long long)(r0 + r) * tstride + cc * 8;
+    if (index_ok(off + 7, p.elems, p.status)) *reinterpret_cast<uint4*>(dst + off) = val;
+  }
+}
+
+template <int D, int MT>
+__global__ void __launch_bounds__(256) attn_temporal_bwd_kernel(const TemporalBwdParams p) {
+  using C = TemporalBwdCfg<D, MT>;
+  constexpr int kChunks = D / 8;
+  extern __shared__ __align__(128) unsigned char smem_tb[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sq = smem_u32(smem_tb) + (uint32_t)(warp * C::kWarpBytes);
+  const uint32_t sk = sq + C::kTensorBytes, sv = sq + 2 * C::kTensorBytes, so_in = sq + 3 * C::kTensorBytes,
+                 sdo = sq + 4 * C::kTensorBytes, sout = sq + C::kOutOff;
+  float* vec = reinterpret_cast<float*>(smem_tb + warp * C::kWarpBytes + C::kVecOff);
+  float* s_lse = vec;
+  float* s_dv = vec + C::kRows;
+  const int g = lane >> 2, c = lane & 3;
+  const long long tstride = (long long)p.HW * p.heads * D;
+  const long long step = (long long)gridDim.x * p.warps;
+
+  for (long long set = (long long)blockIdx.x * p.warps + warp; set < p.n_sets; set += step) {
+    const int si = (int)set;
+    const int h = si % p.heads, bp = si / p.heads;
+    const int pos = bp % p.HW, b = bp / p.HW;
+    const long long base = ((long long)b * p.T * p.HW + pos) * p.heads * D + (long long)h * D;
+    // ---- stage the set's q, k, v, o, dO rows (zero past T) and its lse
+    for (int ch = lane; ch < C::kRows * kChunks; ch += 32) {
+      const int r = ch / kChunks, cc = ch - r * kChunks;
+      const bool live = r < p.T && index_ok(base + r * tstride + cc * 8 + 7, p.elems, p.status);
+      const long long off = live ? base + r * tstride + cc * 8 : 0;
+      const uint32_t dst = sq + (uint32_t)(r * C::kRowBytes + cc * 16);
+      cp_async16(dst, p.q + off, live);
+      cp_async16(dst + C::kTensorBytes, p.k + off, live);
+      cp_async16(dst + 2 * C::kTensorBytes, p.v + off, live);
+      cp_async16(dst + 3 * C::kTensorBytes, p.o + off, live);
+      cp_async16(dst + 4 * C::kTensorBytes, p.dout + off, live);
+    }
+    cp_async_commit();
+    for (int t = lane; t < C::kRows; t += 32) {
+      const unsigned long long li = (unsigned long long)set * p.lse_stride + t;
+      s_lse[t] = (t < p.T && index_ok(li, p.lse_elems, p.status)) ? p.lse[li] : 0.f;
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+    // ---- Dv = rowsum(dO * O): four lanes per row, D / 4 channels each (zero rows past T)
+#pragma unroll
+    for (int i = 0; i < C::kRows / 8; ++i) {
+      const int r = i * 8 + g;
+      float acc = 0.f;
+#pragma unroll
+      for (int v4 = 0; v4 < D / 32; ++v4) {
+        const uint32_t off = (uint32_t)(r * C::kRowBytes + (c * (D / 4) + v4 * 8) * 2);
+        uint4 a, d;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w)
+                     : "r"(so_in + off));
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(d.x), "=r"(d.y), "=r"(d.z), "=r"(d.w)
+                     : "r"(sdo + off));
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[e]));
+          const float2 df = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dw[e]));
+          acc = fmaf(af.x, df.x, acc);
+          acc = fmaf(af.y, df.y, acc);
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (c == 0) s_dv[r] = acc;
+    }
+    __syncwarp();
+
+    // ---- keys major: dV and dK of keys kt*16 .. kt*16+15
+#pragma unroll 1
+    for (int kt = 0; kt < MT; ++kt) {
+      if (kt * 16 >= p.T) break;
+      uint32_t pa[MT][4], da[MT][4];
+      {
+        float st[2 * MT][4], dpt[2 * MT][4];
+        tb_rows_by_rows<D, MT>(sk, kt * 16, sq, lane, st);
+        tb_rows_by_rows<D, MT>(sv, kt * 16, sdo, lane, dpt);
+        const int j0 = kt * 16 + g, j1 = j0 + 8;
+#pragma unroll
+        for (int nt = 0; nt < 2 * MT; ++nt) {
+          float pe[4], de[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = nt * 8 + 2 * c + (e & 1);   // query (column)
+            const int j = (e < 2) ? j0 : j1;          // key (row)
+            const bool ok = i < p.T && j < p.T && (!p.causal || j <= i);
+            const float pv = ok ? ex2_approx(st[nt][e] * p.scale_log2 - s_lse[i]) : 0.f;
+            pe[e] = pv;
+            de[e] = pv * (dpt[nt][e] - s_dv[i]);
+          }
+          pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(pe[0], pe[1]);
+          pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+          da[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(de[0], de[1]);
+          da[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(de[2], de[3]);
+        }
+      }
+      {
+        float acc[D / 8][4];
+        tb_frag_by_rows<D, MT>(pa, sdo, lane, acc);
+        tb_store_rows<D, MT>(acc, 1.f, sout, lane, kt * 16, p.T, base, tstride, p.dv, p);
+        tb_frag_by_rows<D, MT>(da, sq, lane, acc);
+        tb_store_rows<D, MT>(acc, p.scale, sout, lane, kt * 16, p.T, base, tstride, p.dk, p);
+      }
+    }
+    // ---- queries major: dQ of queries mt*16 .. mt*16+15
+#pragma unroll 1
+    for (int mt = 0; mt < MT; ++mt) {
+      if (mt * 16 >= p.T) break;
+      uint32_t da[MT][4];
+      {
+        float s[2 * MT][4], dp[2 * MT][4];
+        tb_rows_by_rows<D, MT>(sq, mt * 16, sk, lane, s);
+        tb_rows_by_rows<D, MT>(sdo, mt * 16, sv, lane, dp);
+        const int i0 = mt * 16 + g, i1 = i0 + 8;
+#pragma unroll
+        for (int nt = 0; nt < 2 * MT; ++nt) {
+          float de[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = nt * 8 + 2 * c + (e & 1);   // key (column)
+            const int i = (e < 2) ? i0 : i1;          // query (row)
+            const bool ok = i < p.T && j < p.T && (!p.causal || j <= i);
+            const float pv = ok ? ex2_approx(s[nt][e] * p.scale_log2 - s_lse[i]) : 0.f;
+            de[e] = pv * (dp[nt][e] - s_dv[i]);
+          }
+          da[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(de[0], de[1]);
+          da[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(de[2], de[3]);
+        }
+      }
+      float acc[D / 8][4];
+      tb_frag_by_rows<D, MT>(da, sk, lane, acc);
+      tb_store_rows<D, MT>(acc, p.scale, sout, lane, mt * 16, p.T, base, tstride, p.dq, p);
+    }
+    __syncwarp();   // the staging area is refilled for the next set
+  }
+}
+
+template <int D, int MT>
+int launch_temporal_bwd_t(TemporalBwdParams& p, cudaStream_t stream) {
+  using C = TemporalBwdCfg<D, MT>;
+  p.warps = std::max(1, std::min(8, (OSP_TEMPORAL_BWD_SMEM_KB * 1024) / C::kWarpBytes));
+  const int smem = p.warps * C::kWarpBytes;
+  const int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_temporal_bwd_kernel<D, MT>), smem,
+                                  "attn_temporal_bwd_kernel");
+  if (rc) return rc;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_temporal_bwd_kernel<D, MT>, p.warps * 32, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const long long ctas_needed = (p.n_sets + p.warps - 1) / p.warps;
+  const long long grid = std::min<long long>(ctas_needed, (long long)device_sm_count() * per_sm);
+  attn_temporal_bwd_kernel<D, MT><<<(unsigned)grid, p.warps * 32, smem, stream>>>(p);
+  return check_launch("attn_temporal_bwd_kernel");
+}
+
+template <int D>
+int launch_temporal_bwd_d(TemporalBwdParams& p, cudaStream_t stream) {
+  switch ((p.T + 15) / 16) {
+    case 1: return launch_temporal_bwd_t<D, 1>(p, stream);
+    case 2: return launch_temporal_bwd_t<D, 2>(p, stream);
+    case 3: return launch_temporal_bwd_t<D, 3>(p, stream);
+    default: return launch_temporal_bwd_t<D, 4>(p, stream);
+  }
+}
+
 }  // namespace
 
 int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
@@ -294,6 +579,42 @@ int temporal_attention_launch(const void* q, const void* k, const void* v, void*
     case 64: return launch_temporal_d<64>(p, stream);
     case 96: return launch_temporal_d<96>(p, stream);
     case 128: return launch_temporal_d<128>(p, stream);
+    default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  }
+}
+
+int temporal_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int causal,
+                             float scale, cudaStream_t stream) {
+  if (s.T > 64) return set_error(OSP_ERR_UNSUPPORTED, "the per-set temporal backward takes T <= 64 (got %d)", s.T);
+  TemporalBwdParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.T = s.T;
+  p.HW = s.H * s.W;
+  p.heads = s.heads;
+  p.n_sets = (long long)s.B * p.HW * s.heads;
+  if (p.n_sets > 0x7fffffffLL) return set_error(OSP_ERR_UNSUPPORTED, "%lld temporal sets is too many", p.n_sets);
+  p.lse_stride = (s.T + 127) / 128 * 128;   // the training forward's lse rows (one per set and head)
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  const unsigned long long div = (unsigned long long)bounds_check_divisor();
+  p.elems = (unsigned long long)s.B * s.T * p.HW * s.heads * s.head_dim / div;
+  p.lse_elems = (unsigned long long)p.n_sets * p.lse_stride / div;
+  p.status = device_status_word();
+  if (!p.status) return OSP_ERR_CUDA;
+  switch (s.head_dim) {
+    case 64: return launch_temporal_bwd_d<64>(p, stream);
+    case 96: return launch_temporal_bwd_d<96>(p, stream);
+    case 128: return launch_temporal_bwd_d<128>(p, stream);
     default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
   }
 }

@@ -398,6 +398,13 @@ static bool bwd_ptrs_ok(const void* q, const void* k, const void* v, const void*
   return true;
 }
 
+// T <= 64: the per-set temporal backward kernel (OSP_TEMPORAL_BWD=1) instead of the Skiparse
+// backward kernels on one 128-row tile per set.  Read on every call.
+static bool temporal_bwd_kernel() {
+  const char* e = std::getenv("OSP_TEMPORAL_BWD");
+  return e != nullptr && std::atoi(e) != 0;
+}
+
 static osp_shape frames_of(const osp_shape& s) {
   return osp_shape{s.B * s.T, 0, 1, 1, s.H * s.W, s.heads, s.head_dim};
 }
@@ -448,6 +455,9 @@ int osp_attn_temporal_backward(const void* q, const void* k, const void* v, cons
   if (!bwd_ptrs_ok(q, k, v, o, dout, lse, dq, dk, dv)) return OSP_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
   const int HW = shape->H * shape->W;
+  if (shape->T <= 64 && temporal_bwd_kernel())
+    return temporal_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, causal, softmax_scale,
+                                    static_cast<cudaStream_t>(stream));
   return attention_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, HW > 1 ? OSP_SKIP_SINGLE + 1 : 0, HW,
                                    softmax_scale, static_cast<cudaStream_t>(stream), causal != 0, 1);
 }

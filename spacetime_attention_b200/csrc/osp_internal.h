@@ -89,6 +89,12 @@ int causal_temporal_attention_launch(const void* q, const void* k, const void* v
 int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
                               float scale, cudaStream_t stream);
 
+// Backward of temporal attention for T <= 64 (one warp per set): dq, dk, dv from q, k, v, o,
+// dout and the training forward's lse ([B*H*W][heads][ceil(T/128)*128], log2 domain).
+int temporal_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int causal,
+                             float scale, cudaStream_t stream);
+
 // TMA map over a BSHD tensor for the attention kernels' 128-row x 64-channel SW128 tiles, viewed
 // per layout (0 dense, 1 Single Skip, 2 Group Skip); batch_rows = rows between samples (< 0: N).
 int make_attn_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k,

@@ -59,6 +59,8 @@ def test_spatial_backward_matches_oracle(gpu, case):
 TEMPORAL = [
     # B, heads, d, grid
     (1, 2, 64, (13, 3, 4)),       # 13 frames, one partial tile per position
+    (1, 2, 96, (33, 2, 5)),       # three 16-row tiles per set (per-set kernel), ragged
+    (2, 1, 128, (64, 3, 1)),      # the per-set kernel's largest sets
     (2, 1, 96, (80, 2, 3)),       # longer than the inference kernel's shared-memory limit
     (1, 2, 128, (130, 1, 2)),     # two tiles per position, ragged
     (1, 1, 64, (7, 1, 1)),        # one position: the dense layout
@@ -66,9 +68,17 @@ TEMPORAL = [
 ]
 
 
+@pytest.fixture(params=["per_set", "tiles"])
+def temporal_path(request, monkeypatch):
+    """T <= 64: the per-set temporal backward kernel, or the Skiparse backward kernels on one
+    128-row tile per set (T > 64 always takes the latter)."""
+    monkeypatch.setenv("OSP_TEMPORAL_BWD", "1" if request.param == "per_set" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("case", TEMPORAL, ids=[f"{c[3]}_d{c[2]}_B{c[0]}" for c in TEMPORAL])
-def test_temporal_backward_matches_oracle(gpu, case, causal):
+def test_temporal_backward_matches_oracle(gpu, case, causal, temporal_path):
     B, heads, d, grid = case
     q, k, v, do = _inputs(B, heads, d, grid, 130 + causal)
     qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
@@ -96,7 +106,7 @@ def test_temporal_backward_matches_oracle(gpu, case, causal):
         np.testing.assert_allclose(got, ref / math.log(2.0), rtol=0, atol=2e-3)
 
 
-def test_causal_temporal_first_frame_has_no_query_gradient(gpu):
+def test_causal_temporal_first_frame_has_no_query_gradient(gpu, temporal_path):
     # a first-frame query sees only its own key: softmax over one key, so dQ = 0 up to the fp32
     # rounding of dP - rowsum(dO * O) (two sums of the same products in different orders)
     q, k, v, do = _inputs(1, 2, 64, (6, 4, 4), 140)
