@@ -547,7 +547,7 @@ def run_backward_op(args, rank, world, local_rank):
     else:
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                 "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": f"{src} (copy bandwidth)"}
-    per_set = attn in ("temporal", "temporal_causal") and T <= 64 and os.environ.get("OSP_TEMPORAL_BWD", "0") != "0"
+    per_set = attn in ("temporal", "temporal_causal") and T <= 64 and os.environ.get("OSP_TEMPORAL_BWD", "1") != "0"
     roof.update(traffic=None, bytes_per_step=nbytes,
                 kernel="attn_temporal_bwd_kernel" if per_set
                 else "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel")

@@ -398,11 +398,11 @@ static bool bwd_ptrs_ok(const void* q, const void* k, const void* v, const void*
   return true;
 }
 
-// T <= 64: the per-set temporal backward kernel (OSP_TEMPORAL_BWD=1) instead of the Skiparse
+// T <= 64: the per-set temporal backward kernel, unless OSP_TEMPORAL_BWD=0 selects the Skiparse
 // backward kernels on one 128-row tile per set.  Read on every call.
 static bool temporal_bwd_kernel() {
   const char* e = std::getenv("OSP_TEMPORAL_BWD");
-  return e != nullptr && std::atoi(e) != 0;
+  return e == nullptr || std::atoi(e) != 0;
 }
 
 static osp_shape frames_of(const osp_shape& s) {
