@@ -141,17 +141,51 @@ def make_rope(split: Sequence[int], theta: float = 10000.0) -> OspRope:
 
 
 def _shape_of(t: torch.Tensor, grid, text_len: int) -> OspShape:
+    """The call's shape from q's [B, N, heads, d]; N must be text_len + T*H*W, since the library
+    sizes every access from the shape alone."""
     B, N, heads, d = t.shape
+    T, H, W = (int(x) for x in grid)
+    if N != int(text_len) + T * H * W:
+        raise ValueError(f"q has {N} tokens per sample, but text_len + T*H*W = {int(text_len)} + "
+                         f"{T}*{H}*{W} = {int(text_len) + T * H * W}")
     return make_shape(B, text_len, grid, heads, d)
+
+
+def _same(t: torch.Tensor, ref: torch.Tensor, name: str) -> torch.Tensor:
+    """t, checked to have ref's shape and device (the library reads or writes it with ref's
+    layout), and to be a contiguous bf16 CUDA tensor."""
+    if tuple(t.shape) != tuple(ref.shape) or t.device != ref.device:
+        raise ValueError(f"{name} must have shape {tuple(ref.shape)} on {ref.device} "
+                         f"(got {tuple(t.shape)} on {t.device})")
+    _bshd(t, name)
+    return t
+
+
+def _out(t: Optional[torch.Tensor], ref: torch.Tensor, name: str) -> torch.Tensor:
+    """A caller's output tensor, checked like ref, or a new one."""
+    return torch.empty_like(ref) if t is None else _same(t, ref, name)
+
+
+def _heads_match(t: torch.Tensor, ref: torch.Tensor, name: str) -> None:
+    """t has ref's batch, heads and head_dim (its token count may differ)."""
+    if t.dim() != 4 or t.shape[0] != ref.shape[0] or tuple(t.shape[2:]) != tuple(ref.shape[2:]) \
+            or t.device != ref.device:
+        raise ValueError(f"{name} must be [{ref.shape[0]}, n, {ref.shape[2]}, {ref.shape[3]}] on {ref.device} "
+                         f"(got {tuple(t.shape)} on {t.device})")
+    _bshd(t, name)
+
+
+def _packed_rows(samples) -> int:
+    """Rows of a packed batch: the sum of text_len + T*H*W over its samples."""
+    return sum(int(L) + int(T) * int(H) * int(W) for L, T, H, W in samples)
 
 
 def rope3d(q: torch.Tensor, k: torch.Tensor, grid, text_len: int, split, theta: float = 10000.0,
            q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None):
     """osp_rope3d: 3D RoPE of q and k; returns (q_out, k_out) (new tensors unless given)."""
-    _bshd(q, "q"); _bshd(k, "k")
-    q_out = torch.empty_like(q) if q_out is None else q_out
-    k_out = torch.empty_like(k) if k_out is None else k_out
+    _bshd(q, "q"); _same(k, q, "k")
     shp, rp = _shape_of(q, grid, text_len), make_rope(split, theta)
+    q_out, k_out = _out(q_out, q, "q_out"), _out(k_out, k, "k_out")
     _check("osp_rope3d", library().osp_rope3d(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), ctypes.byref(shp),
                                               ctypes.byref(rp), _stream_handle(q)))
     return q_out, k_out
@@ -160,10 +194,9 @@ def rope3d(q: torch.Tensor, k: torch.Tensor, grid, text_len: int, split, theta: 
 def attn_full(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, scale: float = 0.0,
               o: Optional[torch.Tensor] = None) -> torch.Tensor:
     """osp_attn_full: dense 3D full attention over text_len + T*H*W tokens."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
+    o = _out(o, q, "o")
     _check("osp_attn_full", library().osp_attn_full(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                     ctypes.c_float(scale), _stream_handle(q)))
     return o
@@ -173,21 +206,22 @@ def attn_cross(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, scale: f
                o: Optional[torch.Tensor] = None) -> torch.Tensor:
     """osp_attn_cross: video queries q [B, T*H*W, heads, d] attend to text keys/values
     k, v [B, text_len, heads, d]."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
-    B, _, heads, d = q.shape
+    _bshd(q, "q"); _heads_match(k, q, "k"); _same(v, k, "v")
+    B, N, heads, d = q.shape
+    T, H, W = (int(x) for x in grid)
+    if N != T * H * W:
+        raise ValueError(f"q has {N} tokens per sample, the grid {T}x{H}x{W} has {T * H * W}")
     shp = make_shape(B, k.shape[1], grid, heads, d)
+    o = _out(o, q, "o")
     _check("osp_attn_cross", library().osp_attn_cross(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                       ctypes.c_float(scale), _stream_handle(q)))
     return o
 
 
 def _attn3(fn: str, q, k, v, grid, text_len, scale, o, *extra):
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
+    o = _out(o, q, "o")
     f = getattr(library(), fn)
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp), *extra, ctypes.c_float(scale), _stream_handle(q)]
     _check(fn, f(*args))
@@ -231,11 +265,10 @@ def _lse_buffer(lse, shape, q: torch.Tensor) -> torch.Tensor:
 def attn_forward_train(q, k, v, grid, text_len: int = 0, sparse_k: int = 1, mode: int = 0, scale: float = 0.0,
                        o=None, lse=None):
     """osp_attn_forward_train: returns (o, lse)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
-    lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
+    o = _out(o, q, "o")
+    lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
     _check("osp_attn_forward_train",
            library().osp_attn_forward_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
                                             int(sparse_k), int(mode), ctypes.c_float(scale), _stream_handle(q)))
@@ -245,11 +278,10 @@ def attn_forward_train(q, k, v, grid, text_len: int = 0, sparse_k: int = 1, mode
 def attn_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, sparse_k: int = 1, mode: int = 0,
                   scale: float = 0.0, dq=None, dk=None, dv=None):
     """osp_attn_backward: returns (dq, dk, dv)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
-        _bshd(t, n)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    _bshd(q, "q")
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _same(t, q, n)
+    dq, dk, dv = _out(dq, q, "dq"), _out(dk, q, "dk"), _out(dv, q, "dv")
     lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_backward",
@@ -261,11 +293,10 @@ def attn_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, sparse_k: int 
 
 def attn_frame_causal_train(q, k, v, grid, text_len: int = 0, scale: float = 0.0, o=None, lse=None):
     """osp_attn_frame_causal_train: returns (o, lse)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
-    lse = _lse_buffer(lse, lse_shape(q, 1), q)
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
+    o = _out(o, q, "o")
+    lse = _lse_buffer(lse, lse_shape(q, 1), q)
     _check("osp_attn_frame_causal_train",
            library().osp_attn_frame_causal_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
                                                  ctypes.c_float(scale), _stream_handle(q)))
@@ -275,11 +306,10 @@ def attn_frame_causal_train(q, k, v, grid, text_len: int = 0, scale: float = 0.0
 def attn_frame_causal_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, scale: float = 0.0, dq=None, dk=None,
                                dv=None):
     """osp_attn_frame_causal_backward: returns (dq, dk, dv)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
-        _bshd(t, n)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    _bshd(q, "q")
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _same(t, q, n)
+    dq, dk, dv = _out(dq, q, "dq"), _out(dk, q, "dk"), _out(dv, q, "dv")
     lse = _lse_buffer(lse, lse_shape(q, 1), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_frame_causal_backward",
@@ -299,24 +329,22 @@ def factorized_lse_shape(q: torch.Tensor, grid, temporal: bool):
 
 
 def _factorized_train(fn: str, q, k, v, grid, temporal: bool, extra, scale, o, lse):
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
-    lse = _lse_buffer(lse, factorized_lse_shape(q, grid, temporal), q)
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, 0)
+    o = _out(o, q, "o")
+    lse = _lse_buffer(lse, factorized_lse_shape(q, grid, temporal), q)
     _check(fn, getattr(library(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp), *extra,
                                       ctypes.c_float(scale), _stream_handle(q)))
     return o, lse
 
 
 def _factorized_backward(fn: str, q, k, v, o, dout, lse, grid, temporal: bool, extra, scale, dq, dk, dv):
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
-        _bshd(t, n)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    lse = _lse_buffer(lse, factorized_lse_shape(q, grid, temporal), q)
+    _bshd(q, "q")
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _same(t, q, n)
+    dq, dk, dv = _out(dq, q, "dq"), _out(dk, q, "dk"), _out(dv, q, "dv")
     shp = _shape_of(q, grid, 0)
+    lse = _lse_buffer(lse, factorized_lse_shape(q, grid, temporal), q)
     _check(fn, getattr(library(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                       _ptr(dv), ctypes.byref(shp), *extra, ctypes.c_float(scale), _stream_handle(q)))
     return dq, dk, dv
@@ -354,9 +382,11 @@ def rope3d_packed(q: torch.Tensor, k: torch.Tensor, samples, split, theta: float
                   q_out: Optional[torch.Tensor] = None, k_out: Optional[torch.Tensor] = None):
     """osp_rope3d_packed: 3D RoPE of a packed batch [1, total, heads, d]; ``samples`` lists
     (text_len, T, H, W) per sample.  Returns (q_out, k_out)."""
-    _bshd(q, "q"); _bshd(k, "k")
-    q_out = torch.empty_like(q) if q_out is None else q_out
-    k_out = torch.empty_like(k) if k_out is None else k_out
+    _bshd(q, "q"); _same(k, q, "k")
+    if q.shape[0] != 1 or q.shape[1] != _packed_rows(samples):
+        raise ValueError(f"a packed batch is [1, {_packed_rows(samples)}, heads, d] for these samples "
+                         f"(got {tuple(q.shape)})")
+    q_out, k_out = _out(q_out, q, "q_out"), _out(k_out, k, "k_out")
     arr = (OspSampleGrid * max(1, len(samples)))(*[OspSampleGrid(*(int(x) for x in s)) for s in samples])
     rp = make_rope(split, theta)
     _, _, heads, d = q.shape
@@ -370,12 +400,18 @@ def attn_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_bounds, kv_
                 o: Optional[torch.Tensor] = None) -> torch.Tensor:
     """osp_attn_packed: block-diagonal attention over a packed batch q [1, total_q, heads, d],
     k, v [1, total_kv, heads, d]; sample i owns rows [bounds[i], bounds[i+1])."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
+    _bshd(q, "q"); _heads_match(k, q, "k"); _same(v, k, "v")
+    if q.shape[0] != 1:
+        raise ValueError(f"a packed batch has B = 1 (got {q.shape[0]})")
     _, _, heads, d = q.shape
     qb = _bounds(q_bounds)
     kb = _bounds(kv_bounds) if kv_bounds is not None else None
+    if len(qb) < 1 or qb[len(qb) - 1] != q.shape[1]:
+        raise ValueError(f"the last query bound must be q's {q.shape[1]} rows")
+    kv_end = kb[len(kb) - 1] if kb is not None and len(kb) else (qb[len(qb) - 1] if len(qb) else -1)
+    if kv_end != k.shape[1]:
+        raise ValueError(f"the last key bound must be k's {k.shape[1]} rows (got {kv_end})")
+    o = _out(o, q, "o")
     _check("osp_attn_packed", library().osp_attn_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(o), qb, kb, len(qb) - 1,
                                                         heads, d, ctypes.c_float(scale), _stream_handle(q)))
     return o
@@ -385,10 +421,9 @@ def attn_full_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, t
                       o: Optional[torch.Tensor] = None) -> torch.Tensor:
     """osp_attn_full_noalloc: dense attention whose call allocates no device memory (the
     library's scratch is a static device array).  `o` should be preallocated by such callers."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
+    o = _out(o, q, "o")
     _check("osp_attn_full_noalloc",
            library().osp_attn_full_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                            ctypes.c_float(scale), _stream_handle(q)))
@@ -399,10 +434,9 @@ def skiparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, spars
                   scale: float = 0.0, o: Optional[torch.Tensor] = None, text_len: int = 0) -> torch.Tensor:
     """osp_skiparse_attn: fused Skiparse attention in natural token order (text_len > 0: the text
     prefix is joined to every set as global tokens)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _bshd(t, n)
-    o = torch.empty_like(q) if o is None else o
+    _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
+    o = _out(o, q, "o")
     _check("osp_skiparse_attn", library().osp_skiparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), ctypes.byref(shp),
                                                             int(sparse_k), int(mode), ctypes.c_float(scale),
                                                             _stream_handle(q)))
@@ -414,12 +448,17 @@ def skiparse_gather(q: torch.Tensor, k: Optional[torch.Tensor], v: Optional[torc
     """osp_skiparse_gather: returns (q_out, k_out, v_out) in the k-fold batch layout; RoPE on q, k
     with the tokens' own positions when ``split`` is given."""
     _bshd(q, "q")
+    for t, n in ((k, "k"), (v, "v")):
+        if t is not None:
+            _same(t, q, n)
+    shp = _shape_of(q, grid, 0)
+    if sparse_k < 1 or q.shape[1] % sparse_k:
+        raise ValueError(f"sparse_k {sparse_k} must divide the {q.shape[1]} video tokens")
     B, N, heads, d = q.shape
     outs = []
     for t in (q, k, v):
         outs.append(None if t is None else torch.empty((B * sparse_k, N // sparse_k, heads, d), dtype=t.dtype,
                                                           device=t.device))
-    shp = _shape_of(q, grid, 0)
     rp = make_rope(split, theta) if split is not None else None
     _check("osp_skiparse_gather",
            library().osp_skiparse_gather(_ptr(q), _ptr(k), _ptr(v), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]),
@@ -433,8 +472,16 @@ def skiparse_scatter(o_perm: torch.Tensor, grid, sparse_k: int, mode: int,
     """osp_skiparse_scatter: inverse of the gather for one tensor."""
     _bshd(o_perm, "o_perm")
     Bk, n_set, heads, d = o_perm.shape
+    T, H, W = (int(x) for x in grid)
+    if sparse_k < 1 or Bk % sparse_k or n_set * sparse_k != T * H * W:
+        raise ValueError(f"o_perm {tuple(o_perm.shape)} is not the k-fold batch of a {T}x{H}x{W} grid "
+                         f"with sparse_k {sparse_k}")
     B, N = Bk // sparse_k, n_set * sparse_k
-    o = torch.empty((B, N, heads, d), dtype=o_perm.dtype, device=o_perm.device) if o is None else o
+    if o is None:
+        o = torch.empty((B, N, heads, d), dtype=o_perm.dtype, device=o_perm.device)
+    elif tuple(o.shape) != (B, N, heads, d) or o.device != o_perm.device:
+        raise ValueError(f"o must have shape {(B, N, heads, d)} on {o_perm.device} (got {tuple(o.shape)})")
+    _bshd(o, "o")
     shp = make_shape(B, 0, grid, heads, d)
     _check("osp_skiparse_scatter", library().osp_skiparse_scatter(_ptr(o_perm), _ptr(o), ctypes.byref(shp),
                                                                   int(sparse_k), int(mode), _stream_handle(o)))

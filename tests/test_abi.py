@@ -182,3 +182,29 @@ def test_binding_checks_the_lse_buffer():
         ops._lse_buffer(torch.zeros((4, 2, 128), dtype=torch.float64), (4, 2, 128), q)
     buf = torch.zeros((4, 2, 128))
     assert ops._lse_buffer(buf, (4, 2, 128), q) is buf
+
+
+def test_binding_shape_checks():
+    # the library sizes every access from the shape struct alone, so the bindings compare the
+    # tensors with it before any call
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros((2, 3 + 4 * 2 * 2, 2, 64), dtype=bf)
+    assert ops._shape_of(q, (4, 2, 2), 3).T == 4
+    with pytest.raises(ValueError, match="text_len"):
+        ops._shape_of(q, (4, 2, 2), 0)                 # 16 video tokens + 0 != 19
+    with pytest.raises(ValueError, match="text_len"):
+        ops._shape_of(q, (5, 2, 2), 3)
+    with pytest.raises(ValueError, match="shape"):
+        ops._same(torch.zeros((2, 18, 2, 64), dtype=bf), q, "k")     # one token short
+    with pytest.raises(ValueError, match="shape"):
+        ops._same(torch.zeros((2, 19, 1, 64), dtype=bf), q, "v")     # other head count
+    with pytest.raises(ValueError, match="shape"):
+        ops._out(torch.zeros((1, 19, 2, 64), dtype=bf), q, "o")
+    with pytest.raises(ValueError, match="CUDA"):
+        ops._same(torch.zeros_like(q), q, "k")        # right shape, but on the host
+    with pytest.raises(ValueError):
+        ops._heads_match(torch.zeros((2, 7, 2, 32), dtype=bf), q, "k")
+    with pytest.raises(ValueError, match="CUDA"):
+        ops._heads_match(torch.zeros((2, 7, 2, 64), dtype=bf), q, "k")   # any token count
+    assert ops._packed_rows([(13, 2, 5, 7), (0, 3, 8, 8), (77, 1, 4, 4)]) == 83 + 192 + 93
