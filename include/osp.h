@@ -26,6 +26,11 @@
  *    (row-major over the grid, w fastest).
  *  Pointers. All tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned.
  *    The library never frees or retains them beyond the call's stream work.
+ *  Sizes. The library sizes every access from the shape arguments alone and cannot see the
+ *    allocations behind the pointers: each buffer must hold at least the elements its entry
+ *    point documents for that shape.  A smaller buffer is out-of-bounds device access (the
+ *    index-checked debug build skips such accesses and reports OSP_ERR_BOUNDS through
+ *    osp_check_status; the release build does not check).
  *  Streams. `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
  *    enqueues work on that stream and returns; results are ready when the stream is.
  *  Errors. Every entry point returns an osp_status. On a non-zero return nothing has been
