@@ -281,8 +281,9 @@ int launch_temporal_d(TemporalParams& p, cudaStream_t stream) {
 //   keys major   (16 keys at a time):  S^T = K Q^T, dP^T = V dO^T, P^T = exp2(S^T * c - lse),
 //                                      dS^T = P^T * (dP^T - Dv); dV = P^T dO, dK = dS^T Q * scale;
 //   queries major (16 queries at a time): S, dP, P, dS as above; dQ = dS K * scale.
-// The second pass recomputes S and dP instead of transposing P / dS through shared memory:
-// the set's products are tiny next to its 16 rows of HBM traffic per token and head.
+// The second pass recomputes S and dP instead of transposing P / dS through shared memory: the
+// products are small next to the 16 * head_dim bytes that every token and head moves through HBM
+// (q, k, v, o, dO read; dQ, dK, dV written).
 // ------------------------------------------------------------------------------------------
 #ifndef OSP_TEMPORAL_BWD_SMEM_KB
 #define OSP_TEMPORAL_BWD_SMEM_KB 100
