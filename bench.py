@@ -5,11 +5,19 @@
 A step is one pass of the hot path over one batch of synthetic input: 3D RoPE of q and k
 (osp_rope3d) followed by attention (osp_attn_full for dense workloads; for Skiparse workloads
 osp_skiparse_attn, Single then Group Skip as an alternating pair).  The default workload is the
-CogVideoX-2B-shaped joint attention: B=1, 30 heads, head_dim 64, 13x30x45 video tokens after
-226 text tokens.  `value` counts attention flops (4*B*heads*Nq*Nkv*d, summed over sets) per
-second of the whole step (RoPE included), with q/k/v resident in HBM.
+largest one-GPU configuration, the Open-Sora Plan v1.5-shaped long video: B=1, 32 heads,
+head_dim 128, 16x36x64 video tokens, RoPE split 32/48/48, Skiparse k=4 Single + Group.  `value`
+counts attention flops (4*B*heads*Nq*Nkv*d, summed over sets) per second of the whole step (RoPE
+included), with q/k/v resident in HBM.  The same JSON line carries a per_config block: every
+measured configuration (tiny, CogVideoX-2B, Open-Sora Plan dense and Skiparse, CogVideoX-5B,
+long video dense and Skiparse), each timed as its own region.
 
-N > 1 (one process per GPU, launched by torch.distributed.run): every rank runs its own
+Roofline denominators: the burst bf16 GEMM peak, unless the timed region lasted a second or
+more under the power cap with the SM clock held below its maximum, where the sustained GEMM
+peak is the like-for-like figure; the line names the one it used.
+
+N > 1 (one process per GPU, launched by torch.distributed.run, or spawned by this script when
+no launcher set WORLD_SIZE): every rank runs its own
 independent copy of the workload (the (sample, head) units of attention share nothing), so
 per-GPU work is fixed ("weak" scaling) and the only collectives are the timing barrier and the
 max-over-ranks reduction.
@@ -50,6 +58,46 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# A timed region counts as sustained (power-capped) only when it lasted at least this long AND
+# the sampled SM clock sat below this fraction of its maximum with sw_power_cap active; every
+# shorter or full-clock region is compared with the burst GEMM figure.
+SUSTAINED_MIN_S = 1.0
+SUSTAINED_CLOCK_FRAC = 0.95
+
+
+def tensor_peak(peaks: dict, src: str, clocks: dict | None, region_s: float):
+    """(peak TFLOP/s, description) for a tensor-bound kernel timed over `region_s` seconds with
+    the sampled `clocks`: the burst bf16 GEMM figure unless the region was long and power-capped,
+    where the GEMM's own sustained figure is the like-for-like denominator."""
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    sm, mx = (clocks or {}).get("sm_mhz"), (clocks or {}).get("sm_max_mhz")
+    capped = ("sw_power_cap" in (clocks or {}).get("reasons", []) and sm is not None and mx
+              and sm < SUSTAINED_CLOCK_FRAC * mx)
+    if region_s >= SUSTAINED_MIN_S and capped:
+        return sustained, (f"{src} sustained bf16 GEMM: timed region {region_s:.2f} s, power-capped at "
+                           f"median {sm:.0f} of {mx:.0f} MHz")
+    clk = f"median SM {sm:.0f} of {mx:.0f} MHz" if sm is not None and mx else "clocks not sampled"
+    return burst, f"{src} burst bf16 GEMM: timed region {region_s:.2f} s, {clk}"
+
+
+def tensor_or_hbm_roofline(flops: float, nbytes: float, ms: float, peaks: dict, src: str, clocks, region_s: float):
+    """Roofline of a launch that may be bound by either unit: the bound is the unit whose time at
+    its peak is the longer one; frac = achieved / that unit's peak."""
+    pt, pt_src = tensor_peak(peaks, src, clocks, region_s)
+    pb = float(peaks["hbm_gbs"])
+    tflops, gbs = flops / (ms * 1e-3) / 1e12, nbytes / (ms * 1e-3) / 1e9
+    t_tensor, t_hbm = flops / (pt * 1e12), nbytes / (pb * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": pt, "unit": "TFLOP/s",
+                "frac": round(tflops / pt, 4), "peak_source": pt_src}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pb, "unit": "GB/s",
+                "frac": round(gbs / pb, 4), "peak_source": f"{src} (copy bandwidth)"}
+    roof["time_bound_frac"] = round(max(t_tensor, t_hbm) / (ms * 1e-3), 4)
+    return roof, tflops, gbs
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for f in ("attn_fwd_kernel.cuh", "osp_device.cuh"):
@@ -58,10 +106,10 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.txt")
+def profiled_traffic(workload: str, kind: str = "dense"):
+    """DRAM bytes per step's attention launches from the committed ncu summary of that workload
+    and attention form, if it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}" + ("_skiparse" if kind == "skiparse" else "") + ".txt")
     if not os.path.exists(p):
         return None
     kv = {}
@@ -73,7 +121,7 @@ def profiled_traffic(workload: str):
     if kv.get("kernel_source_sha") != kernel_source_sha():
         return None
     try:
-        return float(kv["dram_bytes_per_launch"])
+        return float(kv["dram_bytes_per_step"] if "dram_bytes_per_step" in kv else kv["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
 
@@ -137,10 +185,14 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def step_fns(w, q, k, v, qr, kr, o, launch_events=None):
-    """Returns step() running one pass of the hot path (all launches on torch's current stream)."""
+def step_fns(w, q, k, v, qr, kr, o, launch_events=None, kind=None):
+    """Returns step() running one pass of the hot path (all launches on torch's current stream):
+    3D RoPE of q and k, then dense attention or the Skiparse Single + Group pair (`kind`, default
+    from the workload and --attn)."""
+    sp = sparse(w, kind)
+
     def attn():
-        if sparse(w):
+        if sp:
             ops.skiparse_attn(qr, kr, v, w.grid, w.skiparse_k, ops.OSP_SKIP_SINGLE, o=o)
             ops.skiparse_attn(qr, kr, v, w.grid, w.skiparse_k, ops.OSP_SKIP_GROUP, o=o)
         else:
@@ -162,18 +214,22 @@ def step_fns(w, q, k, v, qr, kr, o, launch_events=None):
 ATTN_MODE = {"value": "auto"}
 
 
-def sparse(w) -> bool:
-    """Skiparse pair (Single + Group) for workloads that define k, unless --attn names another form."""
+def sparse(w, kind=None) -> bool:
+    """Skiparse pair (Single + Group) for workloads that define k, unless `kind` ("dense" /
+    "skiparse") or --attn names another form."""
+    if kind is not None:
+        return kind == "skiparse"
     return bool(w.skiparse_k) and ATTN_MODE["value"] not in ("dense", "frame_causal", "spatial", "temporal",
                                                              "temporal_causal")
 
 
-def attention_launches(w, sms: int) -> int:
+def attention_launches(w, sms: int, kind=None) -> int:
     """Kernel launches of one attention call: the attention kernel, plus the combine kernel when
     the library splits the last partial wave of (sample*set, head, 256-row block) units over KV
     ranges (the rule of osp_attn_full: units mod SMs = R > 0 and min(SMs / R, KV tiles / 2, 8) >= 2)."""
-    k = w.skiparse_k if sparse(w) else 1
-    n = (w.seq_len if not sparse(w) else w.n_video // k)
+    sp = sparse(w, kind)
+    k = w.skiparse_k if sp else 1
+    n = (w.seq_len if not sp else w.n_video // k)
     units = -(-n // 256) * w.heads * w.B * k
     rem = units % sms
     if rem == 0:
@@ -182,12 +238,13 @@ def attention_launches(w, sms: int) -> int:
     return 2 if ns >= 2 else 1
 
 
-def launches_per_step(w, sms: int = 148) -> int:
-    return 1 + (2 * attention_launches(w, sms) if sparse(w) else attention_launches(w, sms))
+def launches_per_step(w, sms: int = 148, kind=None) -> int:
+    n = attention_launches(w, sms, kind)
+    return 1 + (2 * n if sparse(w, kind) else n)
 
 
-def step_flops(w) -> float:
-    return 2 * w.skiparse_flops() if sparse(w) else w.dense_flops()
+def step_flops(w, kind=None) -> float:
+    return 2 * w.skiparse_flops() if sparse(w, kind) else w.dense_flops()
 
 
 def run_hbm_op(args, rank, world, local_rank):
@@ -299,19 +356,8 @@ def run_cross_op(args, rank, world, local_rank):
     peaks, src = load_peaks()
     flops = 4.0 * w.B * w.heads * w.n_video * L * w.head_dim
     nbytes = 2 * 2 * w.B * w.heads * w.head_dim * (w.n_video + L)      # q read + o written, k and v read
-    tflops = flops / (ms * 1e-3) / 1e12
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    t_tensor = flops / (float(peaks["bf16_tflops_sustained"]) * 1e12)
-    t_hbm = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
-    if t_tensor >= t_hbm:
-        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": float(peaks["bf16_tflops_sustained"]),
-                "unit": "TFLOP/s", "frac": round(tflops / float(peaks["bf16_tflops_sustained"]), 4),
-                "peak_source": f"{src} (cuBLAS bf16, sustained)"}
-    else:
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": f"{src} (copy bandwidth)"}
-    roof.update(traffic=None, time_bound_frac=round(max(t_tensor, t_hbm) / (ms * 1e-3), 4),
-                hbm_gb_s=round(gbs, 1), bytes_per_launch=nbytes)
+    roof, tflops, gbs = tensor_or_hbm_roofline(flops, nbytes, ms, peaks, src, clocks, ms * args.steps * 1e-3)
+    roof.update(traffic=None, hbm_gb_s=round(gbs, 1), bytes_per_launch=nbytes)
     n_launch = cross_launches(w, L)
     return {"metric": "cross-attention TFLOP/s (video queries, text keys)", "value": round(world * tflops, 1),
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -366,7 +412,7 @@ def run_packed_op(args, rank, world, local_rank):
     flops = w.flops()
     tflops = flops / (ms * 1e-3) / 1e12
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops_sustained"])
+    peak, peak_src = tensor_peak(peaks, src, clocks, ms * args.steps * 1e-3)
     nbytes = 2 * w.total * w.heads * w.head_dim
     return {"metric": "packed-batch attention TFLOP/s (Multi-Resolution Frame Pack, 1 GPU)",
             "value": round(world * tflops, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -377,7 +423,7 @@ def run_packed_op(args, rank, world, local_rank):
             "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(attn_tflops / peak, 4), "traffic": None,
                          "kernel": "attn_fwd_kernel (packed segment table)",
-                         "peak_source": f"{src} (sustained bf16 GEMM)", "avg_launch_ms": round(attn_ms, 4)},
+                         "peak_source": peak_src, "avg_launch_ms": round(attn_ms, 4)},
             "clocks": clocks, "gpu_launches": 2 * args.steps}
 
 
@@ -437,7 +483,8 @@ def run_variant_op(args, rank, world, local_rank):
     peaks, src = load_peaks()
     tflops = flops / (ms * 1e-3) / 1e12
     gbs = nbytes / (ms * 1e-3) / 1e9
-    peak_t, peak_b = float(peaks["bf16_tflops_sustained"]), float(peaks["hbm_gbs"])
+    peak_t, peak_t_src = tensor_peak(peaks, src, clocks, ms * args.steps * 1e-3)
+    peak_b = float(peaks["hbm_gbs"])
     if args.op == "temporal":
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_b, "unit": "GB/s",
                 "frac": round(gbs / peak_b, 4), "peak_source": f"{src} (copy bandwidth)",
@@ -445,7 +492,7 @@ def run_variant_op(args, rank, world, local_rank):
         metric, value, unit = "temporal attention GB/s (2D+1D, 1D part)", gbs, "GB/s"
     else:
         roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_t, "unit": "TFLOP/s",
-                "frac": round(tflops / peak_t, 4), "peak_source": f"{src} (sustained bf16 GEMM)",
+                "frac": round(tflops / peak_t, 4), "peak_source": peak_t_src,
                 "kernel": "attn_fwd_kernel"}
         metric = {"spatial": "spatial attention TFLOP/s (2D+1D, 2D part)",
                   "frame_causal": "frame-causal attention TFLOP/s (unmasked pairs)",
@@ -537,16 +584,7 @@ def run_backward_op(args, rank, world, local_rank):
     # algorithmic bytes: q, k, v, o, dO read and dQ, dK, dV written once (bf16), lse read (fp32)
     rows = q.shape[0] * q.shape[1] * w.heads
     nbytes = len(modes) * (8 * 2 * rows * w.head_dim + 4 * rows)
-    gbs = nbytes / (ms * 1e-3) / 1e9
-    t_tensor = flops / (float(peaks["bf16_tflops_sustained"]) * 1e12)
-    t_hbm = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
-    if t_tensor >= t_hbm:
-        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": float(peaks["bf16_tflops_sustained"]),
-                "unit": "TFLOP/s", "frac": round(tflops / float(peaks["bf16_tflops_sustained"]), 4),
-                "peak_source": f"{src} (sustained bf16 GEMM)"}
-    else:
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                "frac": round(gbs / float(peaks["hbm_gbs"]), 4), "peak_source": f"{src} (copy bandwidth)"}
+    roof, tflops, gbs = tensor_or_hbm_roofline(flops, nbytes, ms, peaks, src, clocks, ms * args.steps * 1e-3)
     per_set = attn in ("temporal", "temporal_causal") and T <= 64 and os.environ.get("OSP_TEMPORAL_BWD", "1") != "0"
     roof.update(traffic=None, bytes_per_step=nbytes,
                 kernel="attn_temporal_bwd_kernel" if per_set
@@ -562,41 +600,105 @@ def run_backward_op(args, rank, world, local_rank):
             "roofline": roof, "clocks": clocks, "gpu_launches": (1 if per_set else 3) * len(modes) * args.steps}
 
 
-def run_ours(args, rank, world, local_rank):
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = syn.WORKLOADS[args.workload]
-    q_h, k_h, v_h = syn.make_qkv(w, w.seed + 17 * rank)
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+# Every configuration of the measured workloads, each timed as its own step in the default run:
+# (workload, attention form).  Tiny is launch-latency bound and reported in microseconds.
+PER_CONFIG = [("tiny", "dense"), ("tiny", "skiparse"), ("cogvideox_2b", "dense"), ("open_sora_plan", "dense"),
+              ("open_sora_plan", "skiparse"), ("cogvideox_5b", "dense"), ("long_video", "dense"),
+              ("long_video", "skiparse")]
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def time_steps(w, kind, q, k, v, steps: int, warmup: int, dev, world: int, local_rank: int, flush_l2: bool):
+    """Times `steps` steps of the hot path on resident q, k, v (after `warmup` untimed ones):
+    barrier + synchronize on both sides, CUDA events on the launching stream, clocks sampled
+    during the region.  With flush_l2 every step is preceded by a write larger than L2 and timed
+    by its own events (the flush is outside them).  Returns the timings and the output tensors."""
     qr, kr, o = torch.empty_like(q), torch.empty_like(k), torch.empty_like(q)
-    step = step_fns(w, q, k, v, qr, kr, o)
-    for _ in range(args.warmup):
+    step = step_fns(w, q, k, v, qr, kr, o, kind=kind)
+    for _ in range(warmup):
         step()
     ops.check_status(dev)
-
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
-    # ---- device-timed region: K steps, inputs resident in HBM
     events = []
-    step_timed = step_fns(w, q, k, v, qr, kr, o, launch_events=events)
+    step_timed = step_fns(w, q, k, v, qr, kr, o, launch_events=events, kind=kind)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush_l2 else None
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.3)
-    barrier()
+    _barrier(world)
     torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(args.steps):
-        step_timed()
-    t1.record()
-    torch.cuda.synchronize()
-    barrier()
+    if flush_l2:
+        pairs = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            step_timed()
+            b.record()
+            pairs.append((a, b))
+        torch.cuda.synchronize()
+        ms_total = float(sum(a.elapsed_time(b) for a, b in pairs))
+    else:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            step_timed()
+        t1.record()
+        torch.cuda.synchronize()
+        ms_total = t0.elapsed_time(t1)
+    _barrier(world)
     clocks = sampler.stop()
     ops.check_status(dev)
-    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    ms_total = max_over_ranks(ms_total, world, dev)
     attn_ms = float(np.mean([a.elapsed_time(b) for a, b in events]))
+    return {"ms_total": ms_total, "attn_ms": attn_ms, "clocks": clocks}, (qr, kr, o)
+
+
+def attn_kernel_name(w, kind, sms: int) -> str:
+    return "attn_fwd_kernel" + (" + attn_combine_kernel (split tail)" if attention_launches(w, sms, kind) > 1 else "")
+
+
+def per_config_entry(w, kind, t: dict, steps: int, sms: int, flushed: bool) -> dict:
+    """One entry of the per-config block: step time, step and attention-kernel TFLOP/s, and the
+    attention kernel's fraction of the tensor peak chosen for this region's length and clocks."""
+    flops = step_flops(w, kind)
+    ms = t["ms_total"] / steps
+    peaks, src = load_peaks()
+    peak, peak_src = tensor_peak(peaks, src, t["clocks"], t["ms_total"] * 1e-3)
+    attn_tf = flops / (t["attn_ms"] * 1e-3) / 1e12
+    e = {"workload": w.name,
+         "attn": f"skiparse k={w.skiparse_k} single+group" if sparse(w, kind) else "dense",
+         "grid": "x".join(str(x) for x in w.grid), "B": w.B, "heads": w.heads, "head_dim": w.head_dim,
+         "text_len": w.text_len, "seq_len": w.seq_len, "flops_per_step": flops, "steps": steps,
+         "ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+         "attn_ms": round(t["attn_ms"], 4), "attn_tflops": round(attn_tf, 2), "kernel": attn_kernel_name(w, kind, sms),
+         "frac": round(attn_tf / peak, 4), "peak": peak, "peak_source": peak_src,
+         "l2": "L2 flushed (256 MiB write) before every step, outside its events" if flushed
+               else "inputs larger than L2, no flush",
+         "clocks": t["clocks"], "gpu_launches": launches_per_step(w, sms, kind) * steps}
+    if w.seq_len < 4096:
+        e["us_per_step"] = round(ms * 1e3, 2)
+        e["note"] = "launch-latency bound; its roofline fraction is not meaningful"
+    return e
+
+
+def run_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    w = syn.WORKLOADS[args.workload]
+    kind = "skiparse" if sparse(w) else "dense"
+    q_h, k_h, v_h = syn.make_qkv(w, w.seed + 17 * rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    in_bytes = 3 * q.numel() * q.element_size()
+    flush = in_bytes < 2 * L2_BYTES
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    t, (qr, kr, o) = time_steps(w, kind, q, k, v, args.steps, args.warmup, dev, world, local_rank, flush)
+    ms_total, attn_ms, clocks = t["ms_total"], t["attn_ms"], t["clocks"]
 
     # ---- end to end through the public API: pinned host inputs -> device -> hot path -> host.
     # Every step copies its q, k, v from pinned host memory and its o back; the copies run on
@@ -604,9 +706,9 @@ def run_ours(args, rank, world, local_rank):
     # upload of step i+1 and the download of step i-1 (what a host-fed caller would do).
     qp, kp, vp = (x.pin_memory() for x in (q_h, k_h, v_h))
     ops_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for _ in range(2)]
-    dev_in = [(q, k, v), tuple(torch.empty_like(t) for t in (q, k, v))]
+    dev_in = [(q, k, v), tuple(torch.empty_like(x) for x in (q, k, v))]
     dev_out = [o, torch.empty_like(o)]
-    steps_pipe = [step_fns(w, *dev_in[r], qr, kr, dev_out[r]) for r in range(2)]
+    steps_pipe = [step_fns(w, *dev_in[r], qr, kr, dev_out[r], kind=kind) for r in range(2)]
     e2e_steps = max(4, min(40, args.steps))
     compute = torch.cuda.current_stream(dev)
     h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -634,7 +736,7 @@ def run_ours(args, rank, world, local_rank):
     for i in range(2):
         e2e_step(i)
     torch.cuda.synchronize()
-    barrier()
+    _barrier(world)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(compute)
@@ -644,19 +746,18 @@ def run_ours(args, rank, world, local_rank):
     compute.wait_event(down_done[(e2e_steps - 2) & 1])
     b.record(compute)
     torch.cuda.synchronize()
-    barrier()
+    _barrier(world)
     e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dev)
     ops.check_status(dev)
+    del qp, kp, vp, ops_h, dev_in, dev_out, steps_pipe
 
-    flops = step_flops(w)
+    flops = step_flops(w, kind)
     ms_step = ms_total / args.steps
     value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
     peaks, peaks_src = load_peaks()
-    # the attention kernels run back to back for the whole timed region: sustained peak
-    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    peak, peak_src = tensor_peak(peaks, peaks_src, clocks, ms_total * 1e-3)
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    traffic = profiled_traffic(w.name)
-    in_bytes = 3 * q.numel() * q.element_size()
+    traffic = profiled_traffic(w.name, kind)
     out_bytes = o.numel() * o.element_size()
     line = {
         "metric": METRIC,
@@ -671,25 +772,47 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(w.describe(), ops=("rope3d+skiparse_single+skiparse_group" if sparse(w)
+        "config": dict(w.describe(), ops=("rope3d+skiparse_single+skiparse_group" if kind == "skiparse"
                                           else "rope3d+attn_full"),
-                       skiparse_k=w.skiparse_k if sparse(w) else None, parallelism=f"replicas x{world} (independent samples)",
-                       l2=f"inputs {in_bytes / 1e6:.0f} MB > L2 126 MiB, no flush",
+                       skiparse_k=w.skiparse_k if kind == "skiparse" else None,
+                       parallelism=f"replicas x{world} (independent samples)",
+                       l2=(f"L2 flushed (256 MiB write) before every step, outside its events" if flush
+                           else f"inputs {in_bytes / 1e6:.0f} MB > L2 126 MiB, no flush"),
                        flops_per_step=flops),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "attn_fwd_kernel" + (" + attn_combine_kernel (split tail)" if attention_launches(
-                         w, torch.cuda.get_device_properties(dev).multi_processor_count) > 1 else ""),
-                     "peak_source": f"{peaks_src} (sustained bf16 GEMM)",
+                     "kernel": attn_kernel_name(w, kind, sms), "peak_source": peak_src,
                      "frac_of_burst_peak": round(achieved / float(peaks["bf16_tflops"]), 4),
-                     "avg_launch_ms": round(attn_ms, 4)},
+                     "frac_of_sustained_peak": round(achieved / float(peaks.get("bf16_tflops_sustained",
+                                                                                 peaks["bf16_tflops"])), 4),
+                     "avg_launch_ms": round(attn_ms, 4),
+                     "flops_per_launch": flops},
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "ms_per_step": round(e2e_ms, 4),
                 "steps": e2e_steps, "copies": "pinned host <-> device on two copy streams, double-buffered, "
                                               "overlapping the previous/next step's kernels"},
-        "gpu_launches": launches_per_step(w, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
+        "gpu_launches": launches_per_step(w, sms, kind) * args.steps,
         "clocks": clocks,
     }
+    del q, k, v, qr, kr, o
+    torch.cuda.empty_cache()
+
+    # ---- every other configuration, each its own timed region (1 GPU runs only)
+    if world == 1 and not args.no_per_config:
+        block = []
+        for name, kd in PER_CONFIG:
+            wc = syn.WORKLOADS[name]
+            if name == w.name and kd == kind:
+                block.append(per_config_entry(wc, kd, t, args.steps, sms, flush))
+                continue
+            qc, kc, vc = (x.to(dev) for x in syn.make_qkv(wc))
+            fl = 3 * qc.numel() * qc.element_size() < 2 * L2_BYTES
+            steps = max(args.steps, 50) if fl else args.steps
+            tc, outs = time_steps(wc, kd, qc, kc, vc, steps, args.warmup, dev, world, local_rank, fl)
+            block.append(per_config_entry(wc, kd, tc, steps, sms, fl))
+            del qc, kc, vc, outs
+            torch.cuda.empty_cache()
+        line["per_config"] = block
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
     return line
@@ -738,25 +861,32 @@ def _threads():
         return os.cpu_count()
 
 
-def _fit_rows(w, q, k, v, nheads: int, budget_s: float):
+def _fit_rows(w, q, k, v, nheads: int, budget_s: float, probe=None):
     """Query rows per head such that RoPE of `nheads` heads plus their attention rows take about
     `budget_s` seconds, from a 32-row probe on one head."""
-    _, tr, ta = oracle_sample(w, [0], 32, q, k, v)
+    _, tr, ta = probe or oracle_sample(w, [0], 32, q, k, v)
     per_row = ta / 32
     rows = (budget_s - nheads * tr) / max(nheads * per_row, 1e-9)
     return int(max(8, min(w.seq_len, rows)))
 
 
 def cpu_baseline(w, budget_s: float = 15.0):
+    """The oracle on a bounded sample of the workload: as many heads as keep their RoPE within a
+    third of the budget, and as many query rows of those heads as fill the rest."""
     q, k, v = syn.make_qkv(w)
-    heads = range(w.heads)
-    rows = _fit_rows(w, q, k, v, w.heads, budget_s)
+    probe = oracle_sample(w, [0], 32, q, k, v)
+    nh = int(max(1, min(w.heads, (budget_s / 3) / max(probe[1], 1e-9))))
+    heads = range(nh)
+    rows = _fit_rows(w, q, k, v, nh, budget_s, probe)
     fl, tr, ta = oracle_sample(w, heads, rows, q, k, v)
+    if tr + ta < 0.5 * budget_s and rows < w.seq_len:   # the small probe overestimated the per-row cost
+        rows = int(min(w.seq_len, rows * max(1.0, (budget_s - tr) / max(ta, 1e-9))))
+        fl, tr, ta = oracle_sample(w, heads, rows, q, k, v)
     return {"value": round(fl / (tr + ta) / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"{w.name}: RoPE of all q/k tokens of all {w.heads} heads + fp64 attention of "
+            "sample": f"{w.name}: RoPE of all q/k tokens of {nh} of {w.heads} heads + fp64 attention of "
                       + (f"the first {rows // w.skiparse_k} slots of every set (Single and Group Skip)"
                          if sparse(w) else f"the first {rows} query tokens")
-                      + f" of every head; {tr + ta:.1f} s ({tr:.1f} s RoPE)"}
+                      + f" of those heads; {tr + ta:.1f} s ({tr:.1f} s RoPE)"}
 
 
 def run_reference(args, rank, world):
@@ -787,12 +917,23 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def spawn_ranks(n: int, argv) -> int:
+    """Runs this script under torch.distributed.run with n local ranks; returns its exit status."""
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="cogvideox_2b", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_video", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--attn", default="auto",
                     choices=["auto", "dense", "skiparse", "frame_causal", "spatial", "temporal", "temporal_causal"],
@@ -809,6 +950,7 @@ def main():
     ap.add_argument("--causal", action="store_true", help="--op temporal: causal in time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="step: skip the per-config block")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -816,11 +958,15 @@ def main():
         ap.error(f"--attn {args.attn} applies to --op backward (use --op {args.attn.split('_')[0]} for the forward)")
     ATTN_MODE["value"] = args.attn
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # no launcher: start one process per GPU here (127.0.0.1 rendezvous) and pass on its status
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
-        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}; using WORLD_SIZE", file=sys.stderr)
+        ap.error(f"WORLD_SIZE={world} but --gpus={args.gpus}: launch one process per GPU (torch.distributed.run "
+                 f"--nproc-per-node {args.gpus}) or pass --gpus {world}")
 
     if args.impl == "reference":
         line = run_reference(args, rank, world)

@@ -1,6 +1,6 @@
 """Derive the polynomial the attention kernel uses to evaluate part of its exp2 calls on the FMA pipe.
 
-    python spacetime_attention_b200/csrc/exp2_poly.py
+    python docs/exp2_poly.py
 
 exp2(x) = 2^n * 2^f with n = round(x) and f = x - n in [-1/2, 1/2] (Cody & Waite style
 reduction; the kernel rounds with the 1.5 * 2^23 addition trick and adds n to the exponent

@@ -316,20 +316,26 @@ int osp_skiparse_index_map(int32_t n_video, int32_t sparse_k, int32_t mode, int3
  *    a call whose scratch would exceed the array is rejected with OSP_ERR_UNSUPPORTED). Every
  *    GPU that loads the library holds the array until the process exits.
  *  First call per device: looks up the array's device address (cudaGetSymbolAddress) with that
- *    device current and caches it; make that first call before any stream capture.
+ *    device current and caches it; make that first call before any stream capture (a first
+ *    call on a capturing stream returns OSP_ERR_CUDA and says so). Device ordinals 0..63 only
+ *    (a higher ordinal returns OSP_ERR_UNSUPPORTED).
  *  Sharing: all calls on a device share the array, and each call clears the status word on
  *    `stream` before its kernel. Calls that overlap on the GPU (different streams) race on it.
- *  Errors: as osp_attn_full. A bounded-wait timeout inside this call is recorded in the static
- *    word, which osp_check_status does not read: the kernel still ends, its output is invalid.
+ *  Errors: as osp_attn_full (OSP_ERR_INVALID_ARG, OSP_ERR_UNSUPPORTED, OSP_ERR_CUDA). A
+ *    bounded-wait timeout inside the kernel is recorded in the static word; osp_check_status
+ *    reports it (OSP_ERR_TIMEOUT, output invalid) and clears it, allocating nothing.
  *  Arguments, layout and arithmetic are those of osp_attn_full, without its split of the last
  *    wave (which needs a workspace): results are bit-identical whenever osp_attn_full does not
  *    split, and otherwise differ only in fp32 summation order. */
 int osp_attn_full_noalloc(const void* q, const void* k, const void* v, void* o, const osp_shape* shape,
                           float softmax_scale, void* stream);
 
-/* Synchronises `stream`, then reads and clears this device's status word.
+/* Synchronises `stream`, then reads and clears this device's status words: the library's own
+ * word and, once osp_attn_full_noalloc has run on the device, that entry point's static word.
+ * A word that does not exist yet has never been written and is skipped, so this call allocates
+ * nothing.
  * Returns OSP_OK, OSP_ERR_TIMEOUT (a kernel's bounded wait gave up; its output is invalid),
- * OSP_ERR_BOUNDS, or OSP_ERR_CUDA (the synchronisation itself failed). */
+ * OSP_ERR_BOUNDS, or OSP_ERR_CUDA (the synchronisation or the read failed). */
 int osp_check_status(void* stream);
 
 /* Message for the last non-zero return on the calling thread ("" if none). The pointer stays

@@ -396,13 +396,21 @@ void* g_noalloc_addr[kNoAllocMaxDevices] = {};
 size_t noalloc_scratch_bytes(const osp_shape&) { return sizeof(unsigned); }
 
 // Device address of g_noalloc_scratch on the current device; looked up on the first call per
-// device (with that device current) and cached.
-int noalloc_scratch_address(void** out) {
+// device (with that device current) and cached.  The lookup is refused while `stream` is being
+// captured, so that a first call inside a capture fails with a message saying so.
+int noalloc_scratch_address(void** out, cudaStream_t stream) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
     return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: no usable current CUDA device");
+  if (dev >= kNoAllocMaxDevices)
+    return set_error(OSP_ERR_UNSUPPORTED, "osp_attn_full_noalloc: device ordinal %d is beyond its limit of %d devices",
+                     dev, kNoAllocMaxDevices);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
   if (!g_noalloc_addr[dev]) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+      return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: the first call on device %d must come before any "
+                       "stream capture (it looks up the static scratch's address)", dev);
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
@@ -415,6 +423,13 @@ int noalloc_scratch_address(void** out) {
 }
 
 }  // namespace
+
+unsigned* noalloc_status_word_if_present() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  return static_cast<unsigned*>(g_noalloc_addr[dev]);
+}
 
 }  // namespace osp
 
@@ -440,9 +455,9 @@ extern "C" int osp_attn_full_noalloc(const void* q, const void* k, const void* v
     return set_error(OSP_ERR_UNSUPPORTED, "osp_attn_full_noalloc needs %zu bytes of scratch, more than its %zu-byte "
                      "static array", need, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  int rc = noalloc_scratch_address(&scratch);
-  if (rc) return rc;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = noalloc_scratch_address(&scratch, st);
+  if (rc) return rc;
   // the array keeps the previous call's contents: the status word must start at zero
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess)
     return set_error(OSP_ERR_CUDA, "osp_attn_full_noalloc: clearing the scratch word failed");

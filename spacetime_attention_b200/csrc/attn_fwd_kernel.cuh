@@ -195,7 +195,7 @@ __device__ __forceinline__ int slot_token(int layout, int s, int g, int k) {
 
 // exp2 of two values on the FMA and ALU pipes: 2^x = 2^n * 2^f with n = round(x) (added to the
 // exponent field) and f = x - n in [-1/2, 1/2]; 2^f is the degree-3 minimax polynomial derived
-// by csrc/exp2_poly.py (Remez, relative error 7.5e-5, far below the bf16 step of P).  Inputs
+// by docs/exp2_poly.py (Remez, relative error 7.5e-5, far below the bf16 step of P).  Inputs
 // are clamped at -125 so that the exponent field cannot underflow (2^-125 is negligible next to
 // the row maximum's 1).
 __device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {

@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <atomic>
+#include <initializer_list>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -114,6 +115,13 @@ unsigned* device_status_word() {
     }
     g_status[dev] = static_cast<unsigned*>(p);
   }
+  return g_status[dev];
+}
+
+unsigned* device_status_word_if_present() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
   return g_status[dev];
 }
 
@@ -592,12 +600,17 @@ int osp_check_status(void* stream) {
   g_last_error[0] = 0;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return set_error(OSP_ERR_CUDA, "stream synchronize failed: %s", cudaGetErrorString(e));
-  unsigned* w = device_status_word();
-  if (!w) return OSP_ERR_CUDA;
+  // Both words of this device, where they exist: a word that was never created was never
+  // written, and creating one here would allocate (which allocation-free callers cannot have).
   unsigned h = 0;
-  if (cudaMemcpy(&h, w, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess ||
-      cudaMemset(w, 0, sizeof(unsigned)) != cudaSuccess)
-    return set_error(OSP_ERR_CUDA, "status word read failed");
+  for (unsigned* w : {device_status_word_if_present(), noalloc_status_word_if_present()}) {
+    if (!w) continue;
+    unsigned x = 0;
+    if (cudaMemcpy(&x, w, sizeof(x), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(w, 0, sizeof(unsigned)) != cudaSuccess)
+      return set_error(OSP_ERR_CUDA, "status word read failed");
+    h |= x;
+  }
   if (h & kDevTimeout) return set_error(OSP_ERR_TIMEOUT, "a device-side bounded wait timed out");
   if (h & kDevBounds) return set_error(OSP_ERR_BOUNDS, "a device-side index check failed");
   return OSP_OK;

@@ -25,6 +25,11 @@ int device_sm_count();
 
 // Per-device status word (allocated on first use, kept until exit).
 unsigned* device_status_word();
+// The status words of the current device that exist, without creating any: the library's
+// (nullptr before its first use) and osp_attn_full_noalloc's static word (nullptr before that
+// entry point's first call on this device).
+unsigned* device_status_word_if_present();
+unsigned* noalloc_status_word_if_present();
 
 // Bounded-wait limit for the attention kernels, in nanoseconds (OSP_WAIT_TIMEOUT_MS, default
 // 2000 ms; read on every launch).

@@ -1,19 +1,23 @@
 """osp_attn_full_noalloc: the attention entry point for callers that cannot allocate device
 memory (their memory belongs to another allocator's pool, or cudaMalloc's device-wide
 synchronisation is not acceptable on their path).  Its scratch is a static device array, so it
-must give the same output as osp_attn_full, call after call, with no allocation of its own.
+must give the same output as osp_attn_full, call after call, with no allocation of its own, and
+a timeout recorded in that array must reach the caller through osp_check_status, which must not
+allocate either.
 
 This file is named to be collected last: if it fails, a run that stops at the first failure has
 already run every other test.  It passes on its own in a fresh process and after the others."""
 
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from spacetime_attention_b200 import ops, synthetic as syn
 from tests.gpu_common import gpu  # noqa: F401
-from tests.helpers import ATTN_MAX_ABS, ATTN_REL_L2, attn_errors, to_f64
+from tests.helpers import ATTN_MAX_ABS, ATTN_REL_L2, assert_attn_close, attn_errors, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -64,3 +68,59 @@ def test_noalloc_allocates_no_torch_memory_and_rejects_bad_args(gpu):
     p = ctypes.c_void_p(q.data_ptr())
     assert lib.osp_attn_full_noalloc(p, p, p, p, ctypes.byref(bad), ctypes.c_float(0.0), None) == 2
     assert lib.osp_attn_full_noalloc(None, p, p, p, ctypes.byref(shape), ctypes.c_float(0.0), None) == 1
+
+
+def test_noalloc_against_the_oracle_where_osp_attn_full_splits(gpu):
+    # 20 heads x 16 query blocks = 320 units on 148 SMs: osp_attn_full splits the last 24 units
+    # over KV ranges (workspace + combine kernel); the allocation-free call cannot, and runs its
+    # 320 items in turn on one CTA per SM instead.  Both are compared with the fp64 oracle.
+    grid, heads = (4, 32, 32), 20
+    w = syn.custom("na", 1, heads, 64, grid, 0, (16, 24, 24))
+    q, k, v = syn.make_qkv(w, 23)
+    qg, kg, vg = (t.to(gpu) for t in (q, k, v))
+    lib = ops.library()
+    shape = ops.make_shape(1, 0, grid, heads, 64)
+    stream = torch.cuda.current_stream(gpu).cuda_stream
+    full = torch.empty_like(qg)
+    _call(lib, "osp_attn_full", qg, kg, vg, full, shape, stream)
+    outs = []
+    for _ in range(2):
+        o = torch.full_like(qg, float("nan"))
+        _call(lib, "osp_attn_full_noalloc", qg, kg, vg, o, shape, stream)
+        outs.append(o)
+    assert lib.osp_check_status(ctypes.c_void_p(stream)) == 0
+    rows = np.arange(0, w.seq_len, 7)
+    ref = O.attn_ref(to_f64(q), to_f64(k), to_f64(v), rows=rows)
+    for o in (full, *outs):
+        assert_attn_close(o[:, rows], ref, "sampled rows")
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_noalloc_timeout_reaches_osp_check_status(gpu, monkeypatch):
+    # the kernel's bounded waits run out (Q is never loaded); the static word records it,
+    # osp_check_status reports it once and clears it, and the next call is correct
+    lib = ops.library()
+    grid = (4, 8, 8)
+    w = syn.custom("na", 1, 2, 64, grid, 0, (16, 24, 24))
+    q, k, v = syn.make_qkv(w, 24)
+    qg, kg, vg = (t.to(gpu) for t in (q, k, v))
+    shape = ops.make_shape(1, 0, grid, 2, 64)
+    stream = torch.cuda.current_stream(gpu).cuda_stream
+    st = ctypes.c_void_p(stream)
+    o = torch.empty_like(qg)
+    _call(lib, "osp_attn_full_noalloc", qg, kg, vg, o, shape, stream)   # looks up the array first
+    assert lib.osp_check_status(st) == 0
+    # osp_check_status allocates nothing: the device's free memory is unchanged across it
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(gpu)[0]
+    assert lib.osp_check_status(st) == 0
+    assert torch.cuda.mem_get_info(gpu)[0] == free0
+    monkeypatch.setenv("OSP_WAIT_TIMEOUT_MS", "100")
+    monkeypatch.setenv("OSP_DEBUG_WITHHOLD_Q", "1")
+    _call(lib, "osp_attn_full_noalloc", qg, kg, vg, o, shape, stream)
+    assert lib.osp_check_status(st) == 5                  # OSP_ERR_TIMEOUT
+    assert lib.osp_check_status(st) == 0                  # cleared by the read
+    monkeypatch.delenv("OSP_DEBUG_WITHHOLD_Q")
+    _call(lib, "osp_attn_full_noalloc", qg, kg, vg, o, shape, stream)
+    assert lib.osp_check_status(st) == 0
+    assert_attn_close(o, O.attn_ref(to_f64(q), to_f64(k), to_f64(v)), "after the timeout")
