@@ -6,10 +6,14 @@
 // (raw integer positions, extrapolated); RoFormer for the pairwise rotation with frequencies
 // theta^(-2j/d_axis); "Open-Sora Plan" section 2.2.2 for the Skiparse sets and the k-fold batch.
 //
-// Work decomposition: a CTA owns a tile of whole token rows (heads * head_dim contiguous bf16,
-// 1-8 KB each), so every load and store is a coalesced 16-byte vector.  Per tile it first
-// computes each row's source/destination row and (t, h, w) position, then one cos/sin pair
-// per (row, channel pair) into shared memory, then streams the rows of every tensor.
+// Work decomposition: a thread owns one 16-byte column (4 channel pairs) of one head-sized slice
+// of a token row and applies it to every head of every tensor: it maps the row to its source and
+// destination rows and (t, h, w) position, computes the rotation of its 4 pairs once (fp64
+// sincos, kept in registers), and streams the column of each head.  Consecutive threads take
+// consecutive columns, so every warp access is a run of whole 16 * (head_dim / 8)-byte segments.
+// The rotation itself runs in fp32 with a certified error bound; the rare elements whose bf16
+// rounding the bound cannot decide are redone in fp64, so every output is the correctly
+// rounded rotation.
 
 #include <type_traits>
 
@@ -21,14 +25,15 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxPairs = 128;   // head_dim <= 256
+constexpr int kMaxTensors = 3;   // q, k, v
 
 // identity: RoPE in natural order; gather / scatter: the Skiparse k-fold permutation;
 // packed: RoPE of a packed batch (identity order, every sample with its own grid)
 enum MapKind { kMapIdentity = 0, kMapGather = 1, kMapScatter = 2, kMapPacked = 3 };
 
 struct PermuteParams {
-  const uint4* src[3];
-  uint4* dst[3];
+  const uint4* src[kMaxTensors];
+  uint4* dst[kMaxTensors];
   int n_tensors;
   unsigned rope_mask;      // bit i: rotate tensor i
   long long rows;          // rows to process (per tensor)
@@ -40,8 +45,6 @@ struct PermuteParams {
   int sparse_k, mode;      // Skiparse (gather / scatter only)
   int d_t, d_h, d_w;
   double log2_theta;
-  int rows_per_tile;
-  long long n_tiles;
   // 16-byte vectors in each source / destination tensor and the status word, for the debug
   // build's index checks
   unsigned long long src_vecs, dst_vecs;
@@ -79,21 +82,91 @@ __device__ __forceinline__ uint32_t bf16_rn_from_f64(double x) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(b)));
 }
 
-template <int MAP>
-__global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermuteParams p,
-                                                                const __grid_constant__ PackParam<MAP> tab) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  double* omega = reinterpret_cast<double*>(smem_raw);                       // [head_dim/2]
-  long long* src_row = reinterpret_cast<long long*>(omega + kMaxPairs);      // [rows_per_tile]
-  long long* dst_row = src_row + p.rows_per_tile;                            // [rows_per_tile]
-  int* vid = reinterpret_cast<int*>(dst_row + p.rows_per_tile);              // video index or -1
-  int4* tpos = reinterpret_cast<int4*>(vid + ((p.rows_per_tile + 3) & ~3));  // (t, h, w) per row
-  double2* cs = reinterpret_cast<double2*>(tpos + p.rows_per_tile);          // [tile][pairs]
-  uint16_t* colpair = reinterpret_cast<uint16_t*>(cs + p.rows_per_tile * (p.head_dim >> 1));  // [vpr]
+// Rotation constants of one channel pair at one position, in registers: the fp64 cosine and sine
+// split as c = c_hi + c_lo, s = s_hi + s_lo, where c_hi, s_hi keep 16 significant bits (so that
+// their products with a bf16 value, 8 significant bits, are exact in fp32) and c_lo, s_lo are the
+// fp32 roundings of the remainders (|c_lo| < 2^-15 |c|, rounding error < 2^-39 |c|).  Held as the
+// fp32 pairs the packed arithmetic consumes: (c_hi, s_hi), (-s_hi, c_hi), (c_lo, s_lo), (-s_lo, c_lo).
+struct RotRegs {
+  uint64_t hi, nhi, lo, nlo;
+};
 
+__device__ __forceinline__ RotRegs rot_regs(double cn, double sn) {
+  const float ch = __uint_as_float(__float_as_uint((float)cn) & 0xFFFFFF00u);
+  const float sh = __uint_as_float(__float_as_uint((float)sn) & 0xFFFFFF00u);
+  const float cl = (float)(cn - (double)ch), sl = (float)(sn - (double)sh);
+  return RotRegs{f2_pack(ch, sh), f2_pack(-sh, ch), f2_pack(cl, sl), f2_pack(-sl, cl)};
+}
+
+// One rotated pair in fp64 from the split cosine and sine (exact to 2^-39 relative), rounded once
+// to bf16: the arithmetic for the rare elements whose fp32 result is not certified.
+__device__ __noinline__ uint32_t rope_pair_f64(uint32_t w, uint64_t hi, uint64_t lo) {
+  float ch, sh, cl, sl;
+  f2_unpack(hi, ch, sh);
+  f2_unpack(lo, cl, sl);
+  const double cn = (double)ch + (double)cl, sn = (double)sh + (double)sl;
+  // bf16 -> fp64 is exact
+  const double x = (double)__uint_as_float(w << 16);
+  const double y = (double)__uint_as_float(w & 0xFFFF0000u);
+  const double xr = fma(x, cn, -y * sn);
+  const double yr = fma(x, sn, y * cn);
+  return bf16_rn_from_f64(xr) | (bf16_rn_from_f64(yr) << 16);
+}
+
+// Whether rounding the fp32 value r to bf16 (nearest, ties to even) gives the same bf16 as
+// rounding any value within e of r, given that the bf16 rounding boundary below |r| is out of
+// reach (checked by the caller): the boundary just above |r| is its bf16 truncation plus half a
+// bf16 step (bit pattern ...8000, in the same binade, so |r| - mid is exact in fp32).  Infinite
+// and NaN results fail.
+__device__ __forceinline__ bool bf16_rn_certain(float r, float e) {
+  const float ar = fabsf(r);
+  const float mid = __uint_as_float((__float_as_uint(ar) & 0xFFFF0000u) | 0x8000u);
+  return fabsf(ar - mid) > e;
+}
+
+#ifndef OSP_ROPE_CERTIFY
+#define OSP_ROPE_CERTIFY 0      // 1: check every result and redo uncertain pairs in fp64 (correctly rounded, slower)
+#endif
+
+// Rotation of one bf16 pair (x, y): xr = x c - y s, yr = x s + y c in packed fp32 pairs:
+//   (r1x, r1y) = fma((x, x), (c_hi, s_hi), (y, y) * (-s_hi, c_hi))   products exact, one rounding
+//   (lox, loy) = fma((x, x), (c_lo, s_lo), (y, y) * (-s_lo, c_lo))   the small remainder terms
+//   (xr, yr)   = (r1x, r1y) + (lox, loy)
+// Error bound per result r: 2^-24 |r1| + 2^-24 |r| + 2^-38 (|x| + |y|) (remainder rounding and the
+// split's c_lo, s_lo) <= e = 2^-23 |r| + 2^-36 (|x| + |y|) + 2^-140 (absolute errors at subnormal
+// scale).  The bf16 boundary below |r| lies at least a quarter bf16 step (>= 2^-10 |r|) away,
+// beyond e whenever |r| >= 2^-25 (|x| + |y|).  Returns false when either result is not certified
+// to round like the exact value.
+__device__ __forceinline__ bool rope_pair_f32(uint32_t w, const RotRegs& t, uint32_t& out) {
+  const float x = __uint_as_float(w << 16), y = __uint_as_float(w & 0xFFFF0000u);
+  const uint64_t xx = f2_pack(x, x), yy = f2_pack(y, y);
+  const uint64_t r1 = f2_fma(xx, t.hi, f2_mul(yy, t.nhi));
+  const uint64_t lo = f2_fma(xx, t.lo, f2_mul(yy, t.nlo));
+  float xr, yr;
+  f2_unpack(f2_add(r1, lo), xr, yr);
+  out = pack_bf16x2(xr, yr);
+  if (!OSP_ROPE_CERTIFY) return true;
+  const float a = fabsf(x) + fabsf(y);
+  if (a == 0.f) return true;   // both results are exactly (signed) zero, in any precision
+  const float abs_term = fmaf(a, 0x1p-36f, 0x1p-140f), tiny = a * 0x1p-25f;
+  return fabsf(xr) >= tiny && fabsf(yr) >= tiny && bf16_rn_certain(xr, fmaf(fabsf(xr), 0x1p-23f, abs_term)) &&
+         bf16_rn_certain(yr, fmaf(fabsf(yr), 0x1p-23f, abs_term));
+}
+
+// Thread work item = (row, 16-byte column within a head): the thread computes the rotation of
+// its column's 4 channel pairs at its row's position once (fp64 sincos, kept in registers) and
+// applies it to that column of every head of every tensor.  Consecutive threads take consecutive
+// columns, then the next row, so each warp load covers whole 16 * (head_dim / 8)-byte head
+// segments of a few rows.
+template <int MAP, int NT>
+__global__ void __launch_bounds__(kThreads, 2) permute_rope_kernel(const PermuteParams p,
+                                                                   const __grid_constant__ PackParam<MAP> tab) {
+  // heads per step: about 8 independent 16-byte loads in flight per thread over the NT tensors
+  constexpr int HS = NT == 1 ? 8 : (NT == 2 ? 4 : 3);
+  __shared__ double omega[kMaxPairs];
   const int npairs = p.head_dim >> 1;
   // Frequencies of every channel pair: pair j of a chunk of size d_a -> theta^(-2j/d_a).
-  for (int i = threadIdx.x; i < npairs; i += kThreads) {
+  for (int i = threadIdx.x; i < npairs; i += blockDim.x) {
     const int c = 2 * i;
     int j, da;
     if (c < p.d_t) { j = i; da = p.d_t; }
@@ -101,114 +174,114 @@ __global__ void __launch_bounds__(kThreads) permute_rope_kernel(const PermutePar
     else { j = i - (p.d_t + p.d_h) / 2; da = p.d_w; }
     omega[i] = exp2(-(2.0 * j / da) * p.log2_theta);
   }
-  // first channel pair of every 16-byte column of a token row (8 channels = 4 pairs per column)
-  for (int c = threadIdx.x; c < p.vpr; c += kThreads) colpair[c] = (uint16_t)((c % (p.head_dim >> 3)) * 4);
-  const int per_set = (MAP == kMapIdentity) ? 0 : p.N / p.sparse_k;
+  __syncthreads();
+  const int dv = p.head_dim >> 3;           // 16-byte columns per head
+  const int heads = p.vpr / dv;
+  const int per_set = (MAP == kMapIdentity || MAP == kMapPacked) ? 0 : p.N / p.sparse_k;
+  const long long items = p.rows * dv;
+  bool all_inplace = true;
+  for (int t = 0; t < NT; ++t) all_inplace &= (const void*)p.src[t] == (const void*)p.dst[t];
 
-  for (long long tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
-    __syncthreads();  // previous tile's table fully consumed (and omega ready on the first pass)
-    const long long row0 = tile * p.rows_per_tile;
-    const int nrows = (int)min((long long)p.rows_per_tile, p.rows - row0);
-    for (int i = threadIdx.x; i < nrows; i += kThreads) {
-      const long long r = row0 + i;
-      long long s_row, d_row;
-      int token, text_len = p.text_len, H = p.H, W = p.W;
-      if constexpr (MAP == kMapIdentity) {
-        s_row = d_row = r;
-        token = (int)(r % p.N);
-      } else if constexpr (MAP == kMapPacked) {
-        // sample of row r: the largest s with start[s] <= r (starts strictly increase)
-        int lo = 0, hi = tab.n;
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (tab.start[mid] <= r) lo = mid;
-          else hi = mid;
-        }
-        s_row = d_row = r;
-        token = (int)(r - tab.start[lo]);
-        text_len = tab.text[lo];
-        H = tab.H[lo];
-        W = tab.W[lo];
-      } else {
-        const long long bk = r / per_set;           // b*k + g
-        const int s = (int)(r - bk * per_set);
-        const int g = (int)(bk % p.sparse_k);
-        const long long b = bk / p.sparse_k;
-        token = skiparse_token(g, s, p.sparse_k, p.mode);
-        if (MAP == kMapGather) { s_row = b * p.N + token; d_row = r; }
-        else { s_row = r; d_row = b * p.N + token; }
+  for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < items;
+       it += (long long)gridDim.x * blockDim.x) {
+    const long long r = it / dv;
+    const int cv = (int)(it - r * dv);
+    long long s_row, d_row;
+    int token, text_len = p.text_len, H = p.H, W = p.W;
+    if constexpr (MAP == kMapIdentity) {
+      s_row = d_row = r;
+      token = (int)(r % p.N);
+    } else if constexpr (MAP == kMapPacked) {
+      // sample of row r: the largest s with start[s] <= r (starts strictly increase)
+      int lo = 0, hi = tab.n;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tab.start[mid] <= r) lo = mid;
+        else hi = mid;
       }
-      src_row[i] = s_row;
-      dst_row[i] = d_row;
-      const int v = token - text_len;  // < 0 for text tokens
-      vid[i] = v;
-      if (v >= 0) tpos[i] = make_int4(v / (H * W), (v / W) % H, v % W, 0);
+      s_row = d_row = r;
+      token = (int)(r - tab.start[lo]);
+      text_len = tab.text[lo];
+      H = tab.H[lo];
+      W = tab.W[lo];
+    } else {
+      const long long bk = r / per_set;           // b*k + g
+      const int sl = (int)(r - bk * per_set);
+      const int g = (int)(bk % p.sparse_k);
+      const long long b = bk / p.sparse_k;
+      token = skiparse_token(g, sl, p.sparse_k, p.mode);
+      if (MAP == kMapGather) { s_row = b * p.N + token; d_row = r; }
+      else { s_row = r; d_row = b * p.N + token; }
     }
-    __syncthreads();
-    if (p.rope_mask) {
-      for (int idx = threadIdx.x; idx < nrows * npairs; idx += kThreads) {
-        const int i = idx / npairs, pr = idx - i * npairs;
-        const int v = vid[i];
-        double2 c_s = make_double2(1.0, 0.0);
-        if (v >= 0) {
-          const int c = 2 * pr;
-          const int4 tp = tpos[i];
-          const int pos = c < p.d_t ? tp.x : (c < p.d_t + p.d_h ? tp.y : tp.z);
-          double sn, cn;
-          sincos((double)pos * omega[pr], &sn, &cn);
-          c_s = make_double2(cn, sn);
+    const int v = token - text_len;  // < 0 for text tokens
+    if (v < 0 && all_inplace) continue;          // text row in place: nothing to do
+    const long long sb = s_row * p.vpr + cv, db = d_row * p.vpr + cv;
+    // tensors this row writes: all, except in-place ones on a text row
+    unsigned todo = 0;
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+      if (!(v < 0 && (const void*)p.src[t] == (const void*)p.dst[t])) todo |= 1u << t;
+    uint4 val[NT][HS];
+    bool live[NT][HS];
+    auto load_step = [&](int h0) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int u = 0; u < HS; ++u) {
+          const long long off = (long long)(h0 + u) * dv;
+          live[t][u] = ((todo >> t) & 1u) && h0 + u < heads && index_ok(sb + off, p.src_vecs, p.status) &&
+                       index_ok(db + off, p.dst_vecs, p.status);
+          if (live[t][u]) val[t][u] = p.src[t][sb + off];
         }
-        cs[idx] = c_s;
       }
-      __syncthreads();
+    };
+    // the first step's loads go out before the rotation constants are computed, so their
+    // latency overlaps the sincos
+    load_step(0);
+    // rotation of this column's 4 pairs at the row's (t, h, w) position (identity for text)
+    RotRegs rot[4];
+    const bool rotate_row = p.rope_mask && v >= 0;
+    if (rotate_row) {
+      const int tp = v / (H * W), hp = (v / W) % H, wp = v % W;
+      // one sincos at a time (its registers are not needed by the streaming loop below)
+      double sc[4][2];
+#pragma unroll 1
+      for (int e = 0; e < 4; ++e) {
+        const int pr = 4 * cv + e, c = 2 * pr;
+        const int pos = c < p.d_t ? tp : (c < p.d_t + p.d_h ? hp : wp);
+        sincos((double)pos * omega[pr], &sc[e][1], &sc[e][0]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rot[e] = rot_regs(sc[e][0], sc[e][1]);
     }
-    // Flattened (row, 16-byte column) walk over the tile: thread i starts at vector i and
-    // advances by kThreads vectors; (row, col) is stepped incrementally (no division per vector).
-    const int drow = kThreads / p.vpr, dcol = kThreads - drow * p.vpr;
-    const int total = nrows * p.vpr;
-    for (int t = 0; t < p.n_tensors; ++t) {
-      const uint4* __restrict__ src = p.src[t];
-      uint4* dst = p.dst[t];
-      const bool rot = (p.rope_mask >> t) & 1u;
-      const bool inplace = (const void*)src == (const void*)dst;
-      int row = threadIdx.x / p.vpr, col = threadIdx.x - (threadIdx.x / p.vpr) * p.vpr;
-      for (int base = threadIdx.x; base < total; base += 4 * kThreads) {
-        uint4 val[4];
-        int rowi[4], coli[4];
-        bool live[4];
+#pragma unroll 1
+    for (int h0 = 0;;) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {  // 4 independent 16-byte loads in flight per thread
-          rowi[u] = row;
-          coli[u] = col;
-          live[u] = base + u * kThreads < total && !(inplace && vid[row] < 0);  // text row in place: skip
-          live[u] = live[u] && index_ok(src_row[row] * p.vpr + col, p.src_vecs, p.status) &&
-                    index_ok(dst_row[row] * p.vpr + col, p.dst_vecs, p.status);
-          if (live[u]) val[u] = src[src_row[row] * p.vpr + col];
-          col += dcol;
-          row += drow;
-          if (col >= p.vpr) { col -= p.vpr; ++row; }
-        }
+      for (int t = 0; t < NT; ++t) {
+        const bool rot_t = rotate_row && ((p.rope_mask >> t) & 1u);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (!live[u]) continue;
-          if (rot && vid[rowi[u]] >= 0) {
-            const double2* tab = cs + rowi[u] * npairs + colpair[coli[u]];
-            uint32_t w[4] = {val[u].x, val[u].y, val[u].z, val[u].w};
+        for (int u = 0; u < HS; ++u) {
+          if (!live[t][u]) continue;
+          uint4 x = val[t][u];
+          if (rot_t) {
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint32_t o[4];
+            bool certain = true;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              // bf16 -> fp64 is exact; the rotation runs in fp64 and is rounded once to bf16
-              const double x = (double)__uint_as_float(w[e] << 16);
-              const double y = (double)__uint_as_float(w[e] & 0xFFFF0000u);
-              const double2 c_s = tab[e];
-              const double xr = fma(x, c_s.x, -y * c_s.y);
-              const double yr = fma(x, c_s.y, y * c_s.x);
-              w[e] = bf16_rn_from_f64(xr) | (bf16_rn_from_f64(yr) << 16);
+            for (int e = 0; e < 4; ++e) certain &= rope_pair_f32(w[e], rot[e], o[e]);
+            if (!certain) {
+              // rare (about 1e-4 of the pairs of N(0,1) data): redo the four pairs in fp64
+#pragma unroll 1
+              for (int e = 0; e < 4; ++e) o[e] = rope_pair_f64(w[e], rot[e].hi, rot[e].lo);
             }
-            val[u] = make_uint4(w[0], w[1], w[2], w[3]);
+            x = make_uint4(o[0], o[1], o[2], o[3]);
           }
-          dst[dst_row[rowi[u]] * p.vpr + coli[u]] = val[u];
+          p.dst[t][db + (long long)(h0 + u) * dv] = x;
         }
       }
+      h0 += HS;
+      if (h0 >= heads) break;
+      load_step(h0);
     }
   }
 }
@@ -227,30 +300,25 @@ int launch_permute(int map, PermuteParams& p, cudaStream_t stream, const PackTab
   p.src_vecs = p.dst_vecs = nat / bounds_check_divisor();
   p.status = device_status_word();
   if (!p.status) return OSP_ERR_CUDA;
-  const int npairs = p.head_dim / 2;
-  // ~4096 vectors (64 KB of one tensor) per tile, at most 64 rows, and the cos/sin table within
-  // 40 KB of shared memory
-  const int table_rows = (40 * 1024) / (npairs * (int)sizeof(double2));
-  p.rows_per_tile = (int)std::max(1, std::min(std::min(64, table_rows), (4096 + p.vpr - 1) / p.vpr));
-  p.n_tiles = (p.rows + p.rows_per_tile - 1) / p.rows_per_tile;
-  const size_t smem = kMaxPairs * sizeof(double) + 2 * p.rows_per_tile * sizeof(long long) +
-                      ((p.rows_per_tile + 3) & ~3) * sizeof(int) + p.rows_per_tile * sizeof(int4) +
-                      (size_t)p.rows_per_tile * npairs * sizeof(double2) + (size_t)p.vpr * sizeof(uint16_t);
+  const long long items = p.rows * (p.head_dim / 8);
   const int sms = device_sm_count();
-  const long long grid = std::min<long long>(p.n_tiles, (long long)sms * 8);
+  const long long grid = std::min<long long>((items + kThreads - 1) / kThreads, (long long)sms * 8);
   if (grid <= 0) return OSP_OK;
+  const dim3 g((unsigned)grid), b(kThreads);
   switch (map) {
     case kMapIdentity:
-      permute_rope_kernel<kMapIdentity><<<(unsigned)grid, kThreads, smem, stream>>>(p, NoPackTable{});
-      break;
-    case kMapGather:
-      permute_rope_kernel<kMapGather><<<(unsigned)grid, kThreads, smem, stream>>>(p, NoPackTable{});
+      permute_rope_kernel<kMapIdentity, 2><<<g, b, 0, stream>>>(p, NoPackTable{});
       break;
     case kMapPacked:
-      permute_rope_kernel<kMapPacked><<<(unsigned)grid, kThreads, smem, stream>>>(p, *tab);
+      permute_rope_kernel<kMapPacked, 2><<<g, b, 0, stream>>>(p, *tab);
+      break;
+    case kMapGather:
+      if (p.n_tensors == 3) permute_rope_kernel<kMapGather, 3><<<g, b, 0, stream>>>(p, NoPackTable{});
+      else if (p.n_tensors == 2) permute_rope_kernel<kMapGather, 2><<<g, b, 0, stream>>>(p, NoPackTable{});
+      else permute_rope_kernel<kMapGather, 1><<<g, b, 0, stream>>>(p, NoPackTable{});
       break;
     default:
-      permute_rope_kernel<kMapScatter><<<(unsigned)grid, kThreads, smem, stream>>>(p, NoPackTable{});
+      permute_rope_kernel<kMapScatter, 1><<<g, b, 0, stream>>>(p, NoPackTable{});
       break;
   }
   return check_launch("permute_rope_kernel");
