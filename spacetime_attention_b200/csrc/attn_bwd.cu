@@ -36,6 +36,10 @@ constexpr int kComputeThreads = 256;
 constexpr int kProdWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kAccWarp = 10;
+constexpr int kRedWarp = 11;             // fused dQ: issues the bulk reduce-adds of dQ
+#ifndef OSP_BWD_FUSE_DQ
+#define OSP_BWD_FUSE_DQ 1                // d = 64: dQ accumulated by the dK/dV kernel (no dQ kernel)
+#endif
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 // The streamed 128-row tiles are processed as two 64-row sub-tiles, and the score buffers are
@@ -54,12 +58,24 @@ template <int D>
 struct BwdCfg {
   static constexpr int kChunks = (D + 63) / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;
+  // Fused dQ (d = 64, where two 64-column tensor-memory buffers are free next to dV and dK): the
+  // dK/dV kernel also computes dQ_i = dS_i K for every query tile it streams, from dS^T written to
+  // shared memory by the compute warps, and adds it into an fp32 accumulator with one bulk
+  // reduce-add per tile; the dQ kernel (which recomputes S, dP and P) is not launched.
+  static constexpr bool kFuseDq = (D == 64) && OSP_BWD_FUSE_DQ;
+  static constexpr int kThreads = kFuseDq ? kBwdThreads + 32 : kBwdThreads;
   static constexpr int kResOff = 0;                                 // two resident tiles
   static constexpr int kStageOff = 2 * kTileBytes;                  // stages of two tiles each
   static constexpr int kVecOff = kStageOff + kStages * 2 * kTileBytes;
   static constexpr int kVecBytes = 2 * kBT * 4;                     // lse + Dv of one query tile
-  static constexpr int kBarOff = kVecOff + kStages * kVecBytes;
-  static constexpr int kNumBars = 16;
+  // fused dQ: dS^T of a query tile (bf16, two 64-query SW128 chunks) double-buffered, and the
+  // fp32 staging tile of dQ (row-major [128][D]) read by the bulk reduce
+  static constexpr int kDsOff = (kVecOff + kStages * kVecBytes + 1023) / 1024 * 1024;
+  static constexpr int kDsBytes = kFuseDq ? 2 * 2 * kChunkBytes : 0;
+  static constexpr int kStgOff = kDsOff + kDsBytes;
+  static constexpr int kStgBytes = kFuseDq ? kBT * D * 4 : 0;
+  static constexpr int kBarOff = kStgOff + kStgBytes;
+  static constexpr int kNumBars = 24;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -76,6 +92,8 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dq_acc;    // fused dQ: fp32 [B*G][heads][vec_stride][D], zeroed before the dK/dV kernel
+  unsigned long long dq_acc_elems;
   unsigned* status;
   unsigned long long timeout_ns;
   unsigned long long elems, vec_elems;   // elements of each BSHD tensor / of lse and Dv (debug checks)
@@ -235,7 +253,7 @@ __device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_
 // ------------------------------------------------------------------------------------------
 // kKeysMajor = true: the kernel's "resident" tiles are K, V and the streamed ones Q, dO.
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                          const BwdParams p) {
@@ -248,9 +266,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 2,
             B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1, B_BUFFREE = B_FIN + 1, B_FIN2 = B_BUFFREE + 2;
+  // fused dQ: dS buffer free (dQ product of the tile two back done) [2], dQ product done [2], dQ
+  // tensor-memory buffer read out [2], staging tile written, staging tile read by the reduce
+  const int B_DSFREE = B_FIN2 + 1, B_DQFULL = B_DSFREE + 2, B_DQTFREE = B_DQFULL + 2, B_STGFULL = B_DQTFREE + 2,
+            B_STGFREE = B_STGFULL + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // fused dQ tensor-memory buffers (64 columns each, next to dV at 256 and dK at 384)
+  auto col_dq = [](int b) { return b ? 448u : 320u; };
 
   const int tile = blockIdx.x % p.n_tiles;
   const int hb = blockIdx.x / p.n_tiles;
@@ -278,6 +302,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(B_BUFFREE + 0), 1);
     mbar_init(bar(B_BUFFREE + 1), 1);
     mbar_init(bar(B_FIN2), 1);
+    if constexpr (C::kFuseDq) {
+      for (int u = 0; u < 2; ++u) {
+        mbar_init(bar(B_DSFREE + u), 1);
+        mbar_init(bar(B_DQFULL + u), 1);
+        mbar_init(bar(B_DQTFREE + u), kComputeThreads);
+      }
+      mbar_init(bar(B_STGFULL), kComputeThreads);
+      mbar_init(bar(B_STGFREE), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -296,6 +329,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+  auto sDs = [&](int b) { return sbase + C::kDsOff + (uint32_t)(b * 2 * kChunkBytes); };   // fused dQ: dS^T
+  const uint32_t sStg = sbase + C::kStgOff;                                              // fused dQ: staging
   auto sRes = [&](int i) { return sbase + C::kResOff + (uint32_t)(i * C::kTileBytes); };           // K, V
   auto sStr = [&](int s, int i) { return sbase + C::kStageOff + (uint32_t)((2 * s + i) * C::kTileBytes); };  // Q, dO
   auto sVec = [&](int s) { return sbase + C::kVecOff + (uint32_t)(s * C::kVecBytes); };
@@ -384,6 +419,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (leader) tc_commit(bar(B_FIN));
       mbar_drain(bar(B_FIN), 0, p.timeout_ns);
     } else {
+      // fused dQ: dQ_i = dS_i K, A = dS_i^T from shared memory (MN-major: rows = keys, queries
+      // contiguous in two 64-query SW128 chunks 16 KB apart), B = the resident K (MN-major, N = D)
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(kBT, D, true, true);
+      const uint64_t dKres_mn = sdesc_sw128(sRes(0), kChunkBytes, 1024);
       for (int t = 0; t < n_sub; ++t) {
         const int i = t >> 1, hh = t & 1, s = i % kStages;
         if (!bwd_warp_wait(bar(B_PREADY + (t & 1)), (t >> 1) & 1, wc)) break;
@@ -393,12 +432,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_ts(kColAcc1, col_dp(t & 1), dQmn + sub, t > 0);   // dK += dS^T Q_sub
         if (leader) tc_commit(bar(B_BUFFREE + (t & 1)));      // buffer t & 1 may be overwritten
         if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));   // both halves of tile i consumed
+        if constexpr (C::kFuseDq) {
+          if (hh == 1) {
+            const int b = i & 1;
+            // the tensor-memory buffer's previous tile (i - 2) has been read out
+            if (i >= 2 && !bwd_warp_wait(bar(B_DQTFREE + b), ((i >> 1) - 1) & 1, wc)) break;
+            tc_fence_after();
+            const uint64_t da = sdesc_sw128(sDs(b), kChunkBytes, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kBT / 16; ++kk)   // 16 keys (two 8-row groups, 2 KB) per step
+              if (leader) mma_ss(tmem + col_dq(b), da + (uint64_t)(128 * kk), dKres_mn + (uint64_t)(128 * kk),
+                                 idesc_dq, kk > 0 ? 1u : 0u);
+            if (leader) tc_commit(bar(B_DQFULL + b));
+            if (leader) tc_commit(bar(B_DSFREE + b));
+          }
+        }
         if (t == n_sub - 1 && leader) tc_commit(bar(B_DONE));
       }
       if (leader) tc_commit(bar(B_FIN2));
       mbar_drain(bar(B_FIN2), 0, p.timeout_ns);
     }
     __syncwarp();
+  } else if (warp == kRedWarp) {
+    // ------------------------------------------------------------------ fused dQ: bulk reduce-add
+    // of each query tile's fp32 dQ (staged in shared memory by the compute warps) into the
+    // accumulator rows of this (sample*set, head); the staging tile is released once read
+    if constexpr (C::kFuseDq) {
+      const bool leader = elect_one_sync();
+      for (int il = 0; il < nq; ++il) {
+        if (!bwd_warp_wait(bar(B_STGFULL), il & 1, wc)) break;
+        const size_t row0 = ((size_t)bg * p.heads + h) * p.vec_stride + (size_t)(i0 + il) * kBT;
+        if (leader && index_ok((row0 + kBT) * D - 1, p.dq_acc_elems, p.status)) {
+          bulk_reduce_add_f32(p.dq_acc + row0 * D, sStg, kBT * D * 4);
+          bulk_wait_read();
+        }
+        __syncwarp();
+        if (leader) mbar_arrive(bar(B_STGFREE));
+      }
+      if (leader) bulk_wait_all();
+      __syncwarp();
+    }
   } else {
     // ------------------------------------------------------------------ compute warps 0-7
     const int quarter = warp & 3, half = warp >> 2;
@@ -406,6 +479,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
     const int kstart = p.frame_hw ? causal_block_start(kv0 + row, p.text_len, p.frame_hw) : 0;   // its block's start
+    // fused dQ: reads this warp's 32 x 32 block (query rows of its lane quarter, columns 32 half)
+    // of dQ of local tile ix out of tensor memory and writes it into the staging tile: row-major
+    // fp32, with the eight 16-byte chunks of each 32-float half row permuted by XOR (row & 7) so
+    // that a warp's stores spread over all banks.  The accumulator rows keep that permutation
+    // (it depends on the row alone, so every key tile's contribution lands on the same element);
+    // the finalize kernel undoes it.
+    auto drain_dq = [&](int ix) -> bool {
+      const int b = ix & 1;
+      if (!bwd_warp_wait(bar(B_DQFULL + b), (ix >> 1) & 1, wc)) return false;
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + col_dq(b) + 32u * half, r);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_DQTFREE + b));
+      if (ix >= 1 && !bwd_warp_wait(bar(B_STGFREE), (ix - 1) & 1, wc)) return false;
+      const uint32_t rowb = sStg + (uint32_t)(row * D * 4 + half * 128);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t pc = (uint32_t)(c ^ (row & 7));
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + 16u * pc), "r"(r[4 * c]),
+                     "r"(r[4 * c + 1]), "r"(r[4 * c + 2]), "r"(r[4 * c + 3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();   // visible to the bulk reduce issued after STGFULL
+      mbar_arrive(bar(B_STGFULL));
+      return true;
+    };
     for (int t = 0; t < 2 * nq; ++t) {
       const int il = t >> 1, i = i0 + il, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
@@ -424,9 +525,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bwd_chunk<true>(s, dp, p.scale_log2, vec, vec + kBT, 0.f, 0.f, valid_q, pk, dk, vis);
       tmem_st16(tS, pk);    // P^T over this warp's consumed S^T columns
       tmem_st16(tP, dk);    // dS^T over this warp's consumed dP^T columns
+      if constexpr (C::kFuseDq) {
+        // dS^T row (this key) for queries 64hh + 32half .. +31 into the dS buffer of tile il:
+        // SW128 chunk hh, 16-byte column c = 4 half + v XOR (row & 7), 8-row groups 1 KB apart
+        const int b = il & 1;
+        if (hh == 0 && il >= 2 && !bwd_warp_wait(bar(B_DSFREE + b), ((il >> 1) - 1) & 1, wc)) { ok = false; break; }
+        const uint32_t base = sDs(b) + (uint32_t)(hh * kChunkBytes) + (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t c = (uint32_t)((4 * half + v) ^ (row & 7));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + 16u * c), "r"(dk[4 * v]),
+                       "r"(dk[4 * v + 1]), "r"(dk[4 * v + 2]), "r"(dk[4 * v + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();   // visible to the dQ product issued after P_ready
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PREADY + bb));
+      if constexpr (C::kFuseDq) {
+        if (hh == 1 && il >= 1 && !drain_dq(il - 1)) { ok = false; break; }
+      }
+    }
+    if constexpr (C::kFuseDq) {
+      if (ok && nq > 0) ok = drain_dq(nq - 1);
     }
     if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
       tc_fence_after();
@@ -643,6 +765,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// fused dQ: dq = bf16(scale * dq_acc), from the accumulator's set-slot rows to natural token order
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_dq_finalize_kernel(const BwdParams p, long long rows) {
+  constexpr int V = D / 8;   // 16-byte output vectors (8 channels) per row
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < rows * V;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long r = idx / V;
+    const int v = (int)(idx - r * V);
+    const int slot = (int)(r % p.n);
+    const long long bh = r / p.n;
+    const int h = (int)(bh % p.heads), bg = (int)(bh / p.heads);
+    const int b = bg / p.G, g = bg % p.G;
+    // logical 16-byte chunks 2v, 2v + 1 of the row; within each 32-float half (8 chunks) the
+    // dK/dV kernel stored chunk c at c ^ (slot & 7)
+    const int c0 = 2 * v, hc = c0 & ~7;
+    const size_t rbase = (((size_t)bg * p.heads + h) * p.vec_stride + slot) * D;
+    const size_t src = rbase + 4 * (hc + ((c0 & 7) ^ (slot & 7)));
+    const size_t src1 = rbase + 4 * (hc + (((c0 + 1) & 7) ^ (slot & 7)));
+    const int token = bwd_slot_token(p.layout, slot, g, p.k);
+    const size_t dst = (((size_t)b * p.N + token) * p.heads + h) * D + 8 * v;
+    if (!index_ok(rbase + D - 1, p.dq_acc_elems, p.status) || !index_ok(dst + 7, p.elems, p.status)) continue;
+    const float4 x = *reinterpret_cast<const float4*>(p.dq_acc + src);
+    const float4 y = *reinterpret_cast<const float4*>(p.dq_acc + src1);
+    const float sc = p.scale;
+    *reinterpret_cast<uint4*>(p.dq + dst) =
+        make_uint4(pack_bf16x2(x.x * sc, x.y * sc), pack_bf16x2(x.z * sc, x.w * sc), pack_bf16x2(y.x * sc, y.y * sc),
+                   pack_bf16x2(y.z * sc, y.w * sc));
+  }
+}
+
 template <int D>
 int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const CUtensorMap& tk,
                  const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, long long rows, long long ctas,
@@ -656,8 +810,15 @@ int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const C
                                                                  static_cast<const __nv_bfloat16*>(dout), p, rows);
   rc = check_launch("attn_bwd_dvec_kernel");
   if (rc) return rc;
-  attn_bwd_dkdv_kernel<D><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  attn_bwd_dkdv_kernel<D><<<(unsigned)ctas, BwdCfg<D>::kThreads, smem, stream>>>(tq, tk, tv, tdo, p);
   if ((rc = check_launch("attn_bwd_dkdv_kernel"))) return rc;
+  if constexpr (BwdCfg<D>::kFuseDq) {
+    const long long qrows = rows;   // (sample*set, head, slot) rows: B * G * heads * n = B * N * heads
+    const long long fblocks = std::min<long long>((qrows * (D / 8) + 255) / 256, (long long)device_sm_count() * 16);
+    if (fblocks > 0)
+      attn_bwd_dq_finalize_kernel<D><<<(unsigned)fblocks, 256, 0, stream>>>(p, qrows);
+    return check_launch("attn_bwd_dq_finalize_kernel");
+  }
   attn_bwd_dq_kernel<D><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
   return check_launch("attn_bwd_dq_kernel");
 }
@@ -714,6 +875,22 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
     return set_error(OSP_ERR_CUDA, "clearing the backward workspace failed");
   }
   p.dvec = static_cast<float*>(ws);
+  // fused dQ (d = 64): the fp32 dQ accumulator [B*G][heads][vec_stride][D], zeroed
+  void* acc = nullptr;
+  if (s.head_dim == 64 && BwdCfg<64>::kFuseDq) {
+    const size_t acc_bytes = (size_t)s.B * G * s.heads * p.vec_stride * s.head_dim * sizeof(float);
+    if (cudaMallocFromPoolAsync(&acc, acc_bytes, pool, stream) != cudaSuccess) {
+      cudaFreeAsync(ws, stream);
+      return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", acc_bytes);
+    }
+    if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) {
+      cudaFreeAsync(acc, stream);
+      cudaFreeAsync(ws, stream);
+      return set_error(OSP_ERR_CUDA, "clearing the backward workspace failed");
+    }
+    p.dq_acc = static_cast<float*>(acc);
+    p.dq_acc_elems = (unsigned long long)(acc_bytes / sizeof(float)) / bounds_check_divisor();
+  }
   const long long rows = (long long)s.B * N * s.heads;
   switch (s.head_dim) {
     case 64: rc = launch_bwd_d<64>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
@@ -721,6 +898,7 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
     case 128: rc = launch_bwd_d<128>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
     default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
   }
+  if (acc) cudaFreeAsync(acc, stream);
   cudaFreeAsync(ws, stream);
   return rc;
 }
