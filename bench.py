@@ -448,6 +448,12 @@ def run_variant_op(args, rank, world, local_rank):
     elif args.op == "temporal":
         launch = lambda i: ops.attn_temporal(*sets[i % nset], w.grid, causal=args.causal, o=outs[i % nset])
         pairs = w.B * HW * (T * (T + 1) // 2 if args.causal else T * T)
+    elif args.op == "temporal_train":   # the training forward: o and the saved lse
+        lses = [torch.empty((w.B * HW, w.heads, -(-T // 128) * 128), dtype=torch.float32, device=dev)
+                for _ in range(nset)]
+        launch = lambda i: ops.attn_temporal_train(*sets[i % nset], w.grid, causal=args.causal, o=outs[i % nset],
+                                                   lse=lses[i % nset])
+        pairs = w.B * HW * (T * (T + 1) // 2 if args.causal else T * T)
     elif args.op == "skiparse_text":
         kk = w.skiparse_k
         if not kk:
@@ -463,6 +469,8 @@ def run_variant_op(args, rank, world, local_rank):
         pairs = w.B * (L * L + sum(HW * (L + (t + 1) * HW) for t in range(T)))
     flops = 4.0 * w.heads * w.head_dim * pairs            # unmasked (query, key) pairs only
     nbytes = 4 * w.B * N * w.heads * w.head_dim * 2       # q, k, v read once, o written once
+    if args.op == "temporal_train":
+        nbytes += 4 * w.B * w.n_video * w.heads           # the lse, one fp32 per token and head
     for i in range(args.warmup):
         launch(i)
     torch.cuda.synchronize()
@@ -485,11 +493,14 @@ def run_variant_op(args, rank, world, local_rank):
     gbs = nbytes / (ms * 1e-3) / 1e9
     peak_t, peak_t_src = tensor_peak(peaks, src, clocks, ms * args.steps * 1e-3)
     peak_b = float(peaks["hbm_gbs"])
-    if args.op == "temporal":
+    if args.op in ("temporal", "temporal_train"):
+        per_set = T <= 64 and (args.op == "temporal" or os.environ.get("OSP_TEMPORAL_BWD", "1") != "0")
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_b, "unit": "GB/s",
                 "frac": round(gbs / peak_b, 4), "peak_source": f"{src} (copy bandwidth)",
-                "kernel": "attn_temporal_kernel" if T <= 64 else "attn_fwd_kernel (Single Skip, k = H*W)"}
-        metric, value, unit = "temporal attention GB/s (2D+1D, 1D part)", gbs, "GB/s"
+                "kernel": "attn_temporal_kernel" if per_set else "attn_fwd_kernel (Single Skip, k = H*W)"}
+        metric = ("temporal attention training forward GB/s (o and lse)" if args.op == "temporal_train"
+                  else "temporal attention GB/s (2D+1D, 1D part)")
+        value, unit = gbs, "GB/s"
     else:
         roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak_t, "unit": "TFLOP/s",
                 "frac": round(tflops / peak_t, 4), "peak_source": peak_t_src,
@@ -500,7 +511,7 @@ def run_variant_op(args, rank, world, local_rank):
         value, unit = tflops, "TFLOP/s"
     roof.update(traffic=None, bytes_per_launch=nbytes, flops_per_launch=flops)
     cfg = dict(w.describe(), op=args.op, text_len=L, l2=f"{nset} input sets rotated ({nset * nbytes / 1e6:.0f} MB)")
-    if args.op == "temporal":
+    if args.op in ("temporal", "temporal_train"):
         cfg["causal"] = bool(args.causal)
     return {"metric": metric, "value": round(world * value, 1), "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -941,13 +952,13 @@ def main():
                          "frame_causal / spatial / temporal / temporal_causal: that backward (--op backward)")
     ap.add_argument("--op", default="step",
                     choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
-                             "frame_causal", "skiparse_text", "backward"],
+                             "temporal_train", "frame_causal", "skiparse_text", "backward"],
                     help="step: the whole hot path (default); rope/gather/scatter: one HBM-bound row alone; "
                          "cross: video -> text cross-attention alone; packed: a packed batch of mixed shapes")
     ap.add_argument("--packed", default="frame_pack_cog2b", choices=sorted(syn.PACKED_WORKLOADS),
                     help="--op packed: the packed batch")
     ap.add_argument("--text-len", type=int, default=226, help="--op cross / skiparse_text: text tokens")
-    ap.add_argument("--causal", action="store_true", help="--op temporal: causal in time")
+    ap.add_argument("--causal", action="store_true", help="--op temporal / temporal_train: causal in time")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="step: skip the per-config block")
@@ -981,7 +992,7 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     try:
         runner = {"step": run_ours, "cross": run_cross_op, "packed": run_packed_op, "spatial": run_variant_op,
-                  "temporal": run_variant_op, "frame_causal": run_variant_op,
+                  "temporal": run_variant_op, "temporal_train": run_variant_op, "frame_causal": run_variant_op,
                   "skiparse_text": run_variant_op, "backward": run_backward_op}.get(args.op, run_hbm_op)
         line = runner(args, rank, world, local_rank)
         if rank == 0:

@@ -218,10 +218,11 @@ int osp_attn_frame_causal_backward(const void* q, const void* k, const void* v, 
  * osp_attn_temporal_train / _backward: the Skiparse kernels with spatial position pos = h*W + w
  *   as Single Skip set pos, k = H*W (slot t = frame t; causal = 1: P zero where t' > t, through
  *   the block-causal mask with one-slot blocks); lse[((b*H*W + pos)*heads + h)*n_pad + t],
- *   n_pad = ceil(T / 128) * 128.  The backward with T <= 64 runs a per-set kernel instead (one
- *   warp per (sample, position, head) set, mma.sync tiles of 16 rows, bound by HBM traffic; the
- *   environment variable OSP_TEMPORAL_BWD=0 selects the tile kernels), with the same rounding
- *   points: P and dS in bf16 before their products, fp32 accumulation, bf16 outputs.
+ *   n_pad = ceil(T / 128) * 128.  With T <= 64 the training forward and the backward run per-set
+ *   kernels instead (one warp per (sample, position, head) set, mma.sync tiles of 16 rows, bound
+ *   by HBM traffic; the environment variable OSP_TEMPORAL_BWD=0 selects the tile kernels), with
+ *   the same rounding points: P and dS in bf16 before their products, fp32 accumulation, bf16
+ *   outputs; the forward writes the lse slots t < T of each set's row.
  *  Errors: OSP_ERR_INVALID_ARG (null or unaligned pointer, causal not 0/1), OSP_ERR_UNSUPPORTED
  *  (text, head_dim, too many frames or positions), OSP_ERR_CUDA. */
 int osp_attn_spatial_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,

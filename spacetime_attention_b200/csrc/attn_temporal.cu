@@ -46,6 +46,11 @@ struct TemporalParams {
   int warps;            // warps per CTA (each with its own staging buffers)
   unsigned long long elems;   // elements of each tensor (debug index checks)
   unsigned* status;
+  // training forward (optional): row log-sum-exp lse[set * lse_stride + t] = m + log2(l) in the
+  // log2 domain of the scaled scores, the layout the backward kernels read
+  float* lse;
+  int lse_stride;
+  unsigned long long lse_elems;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool fill) {
@@ -194,6 +199,11 @@ __global__ void __launch_bounds__(256) attn_temporal_kernel(const TemporalParams
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      if (p.lse && c == 0) {   // one lane of the four holding each row
+        const unsigned long long lb = (unsigned long long)set * p.lse_stride;
+        if (r0 < p.T && index_ok(lb + r0, p.lse_elems, p.status)) p.lse[lb + r0] = m0 + __log2f(l0);
+        if (r1 < p.T && index_ok(lb + r1, p.lse_elems, p.status)) p.lse[lb + r1] = m1 + __log2f(l1);
+      }
       // ---- O = P V
       float o[D / 8][4];
 #pragma unroll
@@ -560,7 +570,8 @@ int launch_temporal_bwd_d(TemporalBwdParams& p, cudaStream_t stream) {
 }  // namespace
 
 int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
-                              float scale, cudaStream_t stream) {
+                              float scale, cudaStream_t stream, float* lse) {
+  if (s.T > 64) return set_error(OSP_ERR_UNSUPPORTED, "the per-set temporal kernel takes T <= 64 (got %d)", s.T);
   TemporalParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
@@ -574,6 +585,9 @@ int temporal_attention_launch(const void* q, const void* k, const void* v, void*
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.elems = (unsigned long long)s.B * s.T * p.HW * s.heads * s.head_dim / bounds_check_divisor();
+  p.lse = lse;
+  p.lse_stride = (s.T + 127) / 128 * 128;   // the layout of the tile kernels' lse (one row per set)
+  p.lse_elems = (unsigned long long)p.n_sets * p.lse_stride / bounds_check_divisor();
   p.status = device_status_word();
   if (!p.status) return OSP_ERR_CUDA;
   switch (s.head_dim) {

@@ -406,8 +406,8 @@ static bool bwd_ptrs_ok(const void* q, const void* k, const void* v, const void*
   return true;
 }
 
-// T <= 64: the per-set temporal backward kernel, unless OSP_TEMPORAL_BWD=0 selects the Skiparse
-// backward kernels on one 128-row tile per set.  Read on every call.
+// T <= 64: the per-set temporal kernels for the training forward and the backward, unless
+// OSP_TEMPORAL_BWD=0 selects the Skiparse kernels on one 128-row tile per set.  Read on every call.
 static bool temporal_bwd_kernel() {
   const char* e = std::getenv("OSP_TEMPORAL_BWD");
   return e == nullptr || std::atoi(e) != 0;
@@ -449,6 +449,9 @@ int osp_attn_temporal_train(const void* q, const void* k, const void* v, void* o
   if (!fwd_ptrs_ok(q, k, v, o, lse)) return OSP_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
   const int HW = shape->H * shape->W;
+  if (shape->T <= 64 && temporal_bwd_kernel())
+    return temporal_attention_launch(q, k, v, o, *shape, causal, softmax_scale, static_cast<cudaStream_t>(stream),
+                                     lse);
   return attention_forward_lse_launch(q, k, v, o, lse, *shape, HW > 1 ? OSP_SKIP_SINGLE + 1 : 0, HW, softmax_scale,
                                       static_cast<cudaStream_t>(stream), causal != 0, 1);
 }

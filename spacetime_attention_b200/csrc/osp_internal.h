@@ -91,8 +91,10 @@ int causal_temporal_attention_launch(const void* q, const void* k, const void* v
                                      float scale, cudaStream_t stream);
 
 // Temporal attention of 2D + 1D (T <= 64): sets of T tokens at stride H*W, optionally causal in t.
+// T <= 64: one warp per (sample, position, head) set; lse (optional, training forward): the row
+// log-sum-exp in the layout of the tile kernels' lse.
 int temporal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s, int causal,
-                              float scale, cudaStream_t stream);
+                              float scale, cudaStream_t stream, float* lse = nullptr);
 
 // Backward of temporal attention for T <= 64 (one warp per set): dq, dk, dv from q, k, v, o,
 // dout and the training forward's lse ([B*H*W][heads][ceil(T/128)*128], log2 domain).

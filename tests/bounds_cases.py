@@ -23,6 +23,10 @@ def calls(dev):
         o, lse = ops.attn_forward_train(q, k, v, w.grid, 0)
         return ops.attn_backward(q, k, v, o, do, lse, w.grid, 0)
 
+    def temporal_training():   # the per-set temporal kernels (T <= 64): forward with lse, backward
+        o, lse = ops.attn_temporal_train(q, k, v, w.grid, causal=True)
+        return ops.attn_temporal_backward(q, k, v, o, do, lse, w.grid, causal=True)
+
     return {
         "rope": lambda: ops.rope3d(q, k, w.grid, 0, w.split),
         "gather": lambda: ops.skiparse_gather(q, k, v, w.grid, 2, 1, split=w.split),
@@ -33,6 +37,7 @@ def calls(dev):
         "temporal": lambda: ops.attn_temporal(q, k, v, w.grid, causal=True),
         "packed": lambda: ops.attn_packed(q, k, v, [0, 100, 256]),
         "backward": backward,
+        "temporal_training": temporal_training,
     }
 
 

@@ -116,3 +116,16 @@ def test_causal_temporal_first_frame_has_no_query_gradient(gpu, temporal_path):
     ops.check_status()
     first, rest = dq[:, :16].float().abs().max().item(), dq[:, 16:].float().abs().max().item()
     assert rest > 0 and first <= 1e-2 * rest
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_per_set_temporal_training_forward_equals_inference(gpu, monkeypatch, causal):
+    # T <= 64: the training forward runs the inference kernel with its lse output switched on
+    monkeypatch.setenv("OSP_TEMPORAL_BWD", "1")
+    grid = (13, 6, 10)
+    q, k, v, _ = _inputs(2, 3, 64, grid, 150 + causal)
+    qg, kg, vg = (t.to(gpu) for t in (q, k, v))
+    o_train, _ = ops.attn_temporal_train(qg, kg, vg, grid, causal=causal)
+    o_inf = ops.attn_temporal(qg, kg, vg, grid, causal=causal)
+    ops.check_status()
+    assert torch.equal(o_train, o_inf)
