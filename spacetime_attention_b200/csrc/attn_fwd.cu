@@ -39,7 +39,8 @@ EncodeTiledFn encode_fn() {
 // batch_rows: rows between samples (default N); a view of part of each sample (the text rows,
 // or the video rows from an offset pointer) keeps the full sample stride.
 int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int layout, int k,
-              long long batch_rows = -1) {
+              long long batch_rows = -1, int box_ch = 64,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return set_error(OSP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t HD = (cuuint64_t)s.heads * s.head_dim;
@@ -52,29 +53,45 @@ int make_tmap(CUtensorMap* tm, const void* ptr, const osp_shape& s, int N, int l
     rank = 3;
     dims[0] = HD; dims[1] = (cuuint64_t)N; dims[2] = (cuuint64_t)s.B;
     strides[0] = row; strides[1] = bstride;
-    box[0] = 64; box[1] = kBM; box[2] = 1;
+    box[0] = (cuuint32_t)box_ch; box[1] = kBM; box[2] = 1;
   } else if (layout == 1) {
     rank = 4;
     dims[0] = HD; dims[1] = (cuuint64_t)k; dims[2] = (cuuint64_t)(N / k); dims[3] = (cuuint64_t)s.B;
     strides[0] = row; strides[1] = row * k; strides[2] = bstride;
-    box[0] = 64; box[1] = 1; box[2] = kBM; box[3] = 1;
+    box[0] = (cuuint32_t)box_ch; box[1] = 1; box[2] = kBM; box[3] = 1;
   } else {
     rank = 5;
     dims[0] = HD; dims[1] = (cuuint64_t)k; dims[2] = (cuuint64_t)k; dims[3] = (cuuint64_t)(N / (k * k));
     dims[4] = (cuuint64_t)s.B;
     strides[0] = row; strides[1] = row * k; strides[2] = row * k * k; strides[3] = bstride;
-    box[0] = 64; box[1] = (cuuint32_t)k; box[2] = 1; box[3] = (cuuint32_t)(kBM / k); box[4] = 1;
+    box[0] = (cuuint32_t)box_ch; box[1] = (cuuint32_t)k; box[2] = 1; box[3] = (cuuint32_t)(kBM / k); box[4] = 1;
   }
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(OSP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return OSP_OK;
 }
 
+// Output maps of the TMA-store epilogue: the same view of o as make_tmap gives of q, plus at
+// d = 96 a 32-channel box (64-byte swizzle) for each head's channels 64 .. 95.  Used at d >= 96,
+// where a thread's row is 192-256 bytes of strided stores; at d = 64 (softmax-bound, 128-byte
+// rows) the per-row stores measured faster (CogVideoX-2B grid: dense -1.5 %, spatial -8 % and
+// cross-attention -5 % through the staging tile).
+int make_out_maps(OutMaps* om, const void* o, const osp_shape& s, int N, int layout, int k,
+                  long long batch_rows = -1) {
+  *om = OutMaps{};
+  if (s.head_dim < 96) return OSP_OK;
+  int rc = make_tmap(&om->o, o, s, N, layout, k, batch_rows);
+  if (rc == OSP_OK && s.head_dim == 96)
+    rc = make_tmap(&om->tail, o, s, N, layout, k, batch_rows, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  om->use = rc == OSP_OK ? 1 : 0;
+  return rc;
+}
+
 template <int D, int kMode, bool kLoop = false>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
-             const SegParam<kMode>& seg, dim3 grid, cudaStream_t stream) {
+             const SegParam<kMode>& seg, const OutMaps& om, dim3 grid, cudaStream_t stream) {
   constexpr int smem = Cfg<D>::kSmemBytes;
   // The warpgroup register split only adds up if the kernel is launched with exactly
   // kRegsLaunch registers per thread; otherwise setmaxnreg.inc could never be satisfied.
@@ -88,7 +105,7 @@ int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
                      kRegsLaunch);
   int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_fwd_kernel<D, kMode, kLoop>), smem, "attn_fwd_kernel");
   if (rc) return rc;
-  attn_fwd_kernel<D, kMode, kLoop><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg);
+  attn_fwd_kernel<D, kMode, kLoop><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p, seg, om);
   return check_launch("attn_fwd_kernel");
 }
 
@@ -107,8 +124,8 @@ namespace {
 // the last partial wave over KV ranges (when allowed), its workspace and the combine kernel.
 template <int kMode>
 int run_units(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, AttnParams& p,
-              const SegParam<kMode>& extra, long long units, int n_kv_tiles, bool allow_split, int head_dim,
-              cudaStream_t stream) {
+              const SegParam<kMode>& extra, const OutMaps& om, long long units, int n_kv_tiles, bool allow_split,
+              int head_dim, cudaStream_t stream) {
   if (units > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld attention work units is too many", units);
   p.n_full = (int)units;
   p.n_split = 1;
@@ -154,16 +171,16 @@ int run_units(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& t
   int rc;
   switch (head_dim) {
     case 64:
-      rc = loop ? launch_d<64, kMode, true>(tq, tk, tv, p, extra, grid, stream)
-                : launch_d<64, kMode, false>(tq, tk, tv, p, extra, grid, stream);
+      rc = loop ? launch_d<64, kMode, true>(tq, tk, tv, p, extra, om, grid, stream)
+                : launch_d<64, kMode, false>(tq, tk, tv, p, extra, om, grid, stream);
       break;
     case 96:
-      rc = loop ? launch_d<96, kMode, true>(tq, tk, tv, p, extra, grid, stream)
-                : launch_d<96, kMode, false>(tq, tk, tv, p, extra, grid, stream);
+      rc = loop ? launch_d<96, kMode, true>(tq, tk, tv, p, extra, om, grid, stream)
+                : launch_d<96, kMode, false>(tq, tk, tv, p, extra, om, grid, stream);
       break;
     case 128:
-      rc = loop ? launch_d<128, kMode, true>(tq, tk, tv, p, extra, grid, stream)
-                : launch_d<128, kMode, false>(tq, tk, tv, p, extra, grid, stream);
+      rc = loop ? launch_d<128, kMode, true>(tq, tk, tv, p, extra, om, grid, stream)
+                : launch_d<128, kMode, false>(tq, tk, tv, p, extra, om, grid, stream);
       break;
     default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
   }
@@ -221,13 +238,15 @@ int launch_with_status(const void* q, const void* k, const void* v, void* o, con
   if ((rc = make_tmap(&tq, q, s, N, layout, p.k)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tk, k, s, N_kv, layout, p.k)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tv, v, s, N_kv, layout, p.k)) != OSP_OK) return rc;
+  OutMaps om;
+  if ((rc = make_out_maps(&om, o, s, N, layout, p.k)) != OSP_OK) return rc;
   const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
   p.qblocks = (int)qblocks;
   const long long units = qblocks * s.heads * (long long)s.B * G;
   const int n_kv_tiles = (p.n_kv + kBN - 1) / kBN;
   if (frame_causal)
-    return run_units<kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, units, n_kv_tiles, false, s.head_dim, stream);
-  return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, units, n_kv_tiles, allow_split, s.head_dim, stream);
+    return run_units<kModeFrameCausal>(tq, tk, tv, p, NoSegTable{}, om, units, n_kv_tiles, false, s.head_dim, stream);
+  return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, om, units, n_kv_tiles, allow_split, s.head_dim, stream);
 }
 
 }  // namespace
@@ -274,11 +293,13 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
     if ((rc = make_tmap(&tv, vv, sv, Nv, layout, sparse_k, N)) != OSP_OK) return rc;
     if ((rc = make_tmap(&tm.k, k, s, L, 0, 1, N)) != OSP_OK) return rc;
     if ((rc = make_tmap(&tm.v, v, s, L, 0, 1, N)) != OSP_OK) return rc;
+    OutMaps om;
+    if ((rc = make_out_maps(&om, static_cast<char*>(o) + L * row, sv, Nv, layout, sparse_k, N)) != OSP_OK) return rc;
     const long long qblocks = (n + 2 * kBM - 1) / (2 * kBM);
     p.qblocks = (int)qblocks;
     const long long units = qblocks * s.heads * (long long)s.B * sparse_k;
     const int n_kv_tiles = (n + kBN - 1) / kBN + (L + kBN - 1) / kBN;
-    rc = run_units<kModeSkipText>(tq, tk, tv, p, tm, units, n_kv_tiles, true, s.head_dim, stream);
+    rc = run_units<kModeSkipText>(tq, tk, tv, p, tm, om, units, n_kv_tiles, true, s.head_dim, stream);
     if (rc) return rc;
   }
   if (L == 0) return OSP_OK;
@@ -292,10 +313,13 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
   if ((rc = make_tmap(&tq, q, s, L, 0, 1, N)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tk, k, s, N, 0, 1)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tv, v, s, N, 0, 1)) != OSP_OK) return rc;
+  OutMaps om;
+  if ((rc = make_out_maps(&om, o, s, L, 0, 1, N)) != OSP_OK) return rc;
   const long long qblocks = (L + 2 * kBM - 1) / (2 * kBM);
   p.qblocks = (int)qblocks;
   const long long units = qblocks * s.heads * (long long)s.B;
-  return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, units, (N + kBN - 1) / kBN, true, s.head_dim, stream);
+  return run_units<kModePlain>(tq, tk, tv, p, NoSegTable{}, om, units, (N + kBN - 1) / kBN, true, s.head_dim,
+                               stream);
 }
 
 int attention_forward_lse_launch(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -367,9 +391,9 @@ int packed_attention_launch(const void* q, const void* k, const void* v, void* o
   if ((rc = make_tmap(&tv, v, sh, n_kv_total, 0, 1)) != OSP_OK) return rc;
   const dim3 grid((unsigned)units);
   switch (head_dim) {
-    case 64: return launch_d<64, kModePacked>(tq, tk, tv, p, seg, grid, stream);
-    case 96: return launch_d<96, kModePacked>(tq, tk, tv, p, seg, grid, stream);
-    case 128: return launch_d<128, kModePacked>(tq, tk, tv, p, seg, grid, stream);
+    case 64: return launch_d<64, kModePacked>(tq, tk, tv, p, seg, OutMaps{}, grid, stream);
+    case 96: return launch_d<96, kModePacked>(tq, tk, tv, p, seg, OutMaps{}, grid, stream);
+    case 128: return launch_d<128, kModePacked>(tq, tk, tv, p, seg, OutMaps{}, grid, stream);
     default: return set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
   }
 }

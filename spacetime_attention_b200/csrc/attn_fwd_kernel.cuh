@@ -102,11 +102,27 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // Output staging for the TMA-store epilogue, per query tile: one 64-channel SW128 chunk (16 KB),
+  // through which a row's 64-channel parts go in turn (rounds); at d = 96 the second round holds
+  // the last 32 channels as a 64-byte-swizzled 128 x 64-byte tile, stored with a 32-channel box
+  // so that no box reaches into the next head's channels.
+  static constexpr int kStgTileBytes = (D >= 96) ? kChunkBytes : 0;   // d = 64 keeps per-row stores
+  static constexpr int kStgOff = kVOff + kStages * kTileBytes;
+  static constexpr int kStgRounds = kChunks;
+  static constexpr int kBarOff = kStgOff + 2 * kStgTileBytes;
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_ready[2],
-  // o_full[2], mma_done, s_free[2], turn[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 16;
-  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+  // o_full[2], mma_done, s_free[2], turn[2], ..., stg_full[2], stg_free[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 16 + 4;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 32 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
+
+// Output tensor maps for the TMA-store epilogue (the same view of o as the query map's of q);
+// use = 0 keeps per-thread row stores (packed batches).  tail: d = 96's channels 64 .. 95.
+struct OutMaps {
+  CUtensorMap o;
+  CUtensorMap tail;
+  int use;
 };
 
 struct AttnParams {
@@ -272,7 +288,7 @@ template <int D, int kMode, bool kLoop>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p,
-                    const __grid_constant__ SegParam<kMode> seg) {
+                    const __grid_constant__ SegParam<kMode> seg, const __grid_constant__ OutMaps om) {
   constexpr bool kPacked = kMode == kModePacked;
   constexpr bool kFrameCausal = kMode == kModeFrameCausal;
   constexpr bool kSkipText = kMode == kModeSkipText;
@@ -293,6 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // A CTA may run several work items in turn (grid smaller than the item count):
   const int B_QEMPTY = B_PV1DONE + 1; // Q may be overwritten: every QK^T of the item has completed
   const int B_OFREE = B_QEMPTY + 1;   // [2] the softmax has read O_i out (the next item may overwrite it)
+  const int B_STGFULL = B_OFREE + 2;  // [2] tile i's rows are in its output staging tile
+  const int B_STGFREE = B_STGFULL + 2; // [2] the TMA store has read tile i's staging tile
   constexpr bool kSplitMma = C::kSepP && OSP_SPLIT_MMA > 0;
   constexpr bool kSplitPv = C::kSepP && OSP_SPLIT_MMA > 1;
   // per-tile issuers (9 and 11) pay at d = 96 (+2 %); at d = 128 the tensor pipe is the bottleneck
@@ -301,6 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* seg_slot = reinterpret_cast<int*>(tmem_slot + 2);   // packed batches: this CTA's segment
+  // debug builds: a row of tile i failed its output index check (its staged store is skipped)
+  volatile int* stg_bad = reinterpret_cast<volatile int*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // work item -> unit (sample*set, head, query block) and KV tile range [kv_lo, kv_lo + n_kv).
@@ -379,7 +399,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_OFREE + 1), 128);
     mbar_init(bar(B_TURN + 0), 128);
     mbar_init(bar(B_TURN + 1), 128);
+    if constexpr (D >= 96)
+      for (int t = 0; t < 2; ++t) {
+        mbar_init(bar(B_STGFULL + t), 128);
+        mbar_init(bar(B_STGFREE + t), 1);
+      }
     *abort_flag = 0;
+    stg_bad[0] = stg_bad[1] = 0;
     fence_mbar_init();
   }
   if constexpr (kPacked) {
@@ -403,6 +429,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (kSkipText) {
       prefetch_tmap(&seg.k);
       prefetch_tmap(&seg.v);
+    }
+    if (D >= 96 && om.use) {
+      prefetch_tmap(&om.o);
+      if (D == 96) prefetch_tmap(&om.tail);
     }
   }
   if (warp == kMmaWarp) {
@@ -689,7 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tP = tmem + lane_base + colP(i);
     const float sl2 = p.scale_log2;
     bool ok = true;
-    int jb = 0;   // KV tiles of this CTA's earlier items
+    int jb = 0;            // KV tiles of this CTA's earlier items
+    int stg_rounds = 0;    // output staging rounds of this tile so far (TMA-store epilogue)
     for (int item = blockIdx.x, ub = 0; ok && (kLoop ? item < p.n_items : ub == 0); item += gridDim.x, ++ub) {
     const Work wk = decode(item);
     const int n_kv = wk.n_kv;
@@ -812,6 +843,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (in) p.ws_ml[prow] = make_float2(m, l);
+      } else if (D >= 96 && !kPacked && om.use) {
+        // TMA-store epilogue: the tile's rows go through a shared staging tile in the box layout
+        // of the output map (the query map's view of o), and one thread stores the box; rows past
+        // the set's end lie outside the map's extent and are not written.  Compiled for d >= 96
+        // only (at d = 64 its presence alone slowed the softmax loop).
+        if constexpr (D >= 96) {
+        const uint32_t stg = sbase + C::kStgOff + (uint32_t)(i * C::kStgTileBytes);
+        const uint32_t rb = stg + (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
+        const bool issuer = (warp & 3) == 0 && lane == 0;
+        for (int rd = 0; rd < C::kStgRounds; ++rd) {
+          // the previous store from this staging tile has been read out
+          if (stg_rounds > 0 && !warp_wait(bar(B_STGFREE + i), (uint32_t)((stg_rounds - 1) & 1), wc)) {
+            ok = false;
+            break;
+          }
+          const bool tail = D == 96 && rd == 1;   // channels 64 .. 95: 64-byte rows, SW64
+          for (int cx = 0; cx < (tail ? 1 : 2); ++cx) {
+            uint32_t o[32];
+            tmem_ld32(tO + 64 * rd + 32 * cx, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t pw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                pw[e] = pack_bf16x2(__uint_as_float(o[8 * v + 2 * e]) * inv_l, __uint_as_float(o[8 * v + 2 * e + 1]) * inv_l);
+              // 16-byte chunk: SW128 chunk (4 cx + v) ^ (row & 7) of a 128-byte row, or SW64 chunk
+              // v ^ ((row >> 1) & 3) of a 64-byte row
+              const uint32_t addr = tail ? stg + (uint32_t)(row * 64) + 16u * (uint32_t)(v ^ ((row >> 1) & 3))
+                                         : rb + 16u * (uint32_t)((4 * cx + v) ^ (row & 7));
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pw[0]), "r"(pw[1]),
+                           "r"(pw[2]), "r"(pw[3])
+                           : "memory");
+            }
+          }
+#if OSP_BOUNDS_CHECK
+          if (rd == 0 && live) {   // the row's natural-order output elements, as the per-row stores check them
+            const int token = w.q_out0 + slot_token(p.layout, slot, g, p.k);
+            const size_t ooff = (((size_t)b * p.N_q + token) * p.heads + h) * D;
+            if (!index_ok(ooff + D - 1, p.o_elems, p.status)) stg_bad[i] = 1;
+          }
+#endif
+          fence_proxy_async_smem();
+          mbar_arrive(bar(B_STGFULL + i));
+          if (issuer) {
+            if (!mbar_wait(bar(B_STGFULL + i), (uint32_t)(stg_rounds & 1), wc)) {
+              ok = false;
+            } else {
+              if (!stg_bad[i]) {
+                const int row0 = w.q0 + i * kBM, chan = h * D + 64 * rd;
+                const CUtensorMap* m = (D == 96 && rd == 1) ? &om.tail : &om.o;
+                if (p.layout == 0) tma_store_3d(m, stg, chan, row0, b);
+                else if (p.layout == 1) tma_store_4d(m, stg, chan, g, row0, b);
+                else tma_store_5d(m, stg, chan, 0, g, row0 / p.k, b);
+                bulk_commit();
+                bulk_wait_read();
+              }
+              if (rd == C::kStgRounds - 1) stg_bad[i] = 0;
+              mbar_arrive(bar(B_STGFREE + i));
+            }
+          }
+          ++stg_rounds;
+          if (!__all_sync(0xffffffffu, ok)) break;
+        }
+        if (!ok) break;
+        }
       } else {
       const int token = w.q_out0 + slot_token(p.layout, live ? slot : 0, g, p.k);
       const size_t ooff = (((size_t)b * p.N_q + token) * p.heads + h) * D;
@@ -837,6 +934,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive(bar(B_OFREE + i));   // O_i is read out: the next item's first PV may overwrite it
     jb += n_kv;
     }   // items
+    if constexpr (D >= 96)
+      if ((warp & 3) == 0 && lane == 0) bulk_wait_all();   // this tile's output stores are complete
   }
   tc_fence_before();
   __syncthreads();

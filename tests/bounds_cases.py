@@ -18,6 +18,9 @@ def calls(dev):
     q, k, v = (t.to(dev) for t in syn.make_qkv(w, 77))
     do = syn.randn_bf16(tuple(q.shape), 81).to(dev)
     kt, vt = syn.randn_bf16((1, 40, 2, 64), 82).to(dev), syn.randn_bf16((1, 40, 2, 64), 83).to(dev)
+    # d = 128: outputs leave through the staging tile and TMA stores (d >= 96)
+    w2 = syn.custom("b2", 1, 2, 128, (2, 8, 10), 0, (32, 48, 48), skiparse_k=2)
+    q2, k2, v2 = (t.to(dev) for t in syn.make_qkv(w2, 78))
 
     def backward():
         o, lse = ops.attn_forward_train(q, k, v, w.grid, 0)
@@ -32,6 +35,8 @@ def calls(dev):
         "gather": lambda: ops.skiparse_gather(q, k, v, w.grid, 2, 1, split=w.split),
         "scatter": lambda: ops.skiparse_scatter(q.view(2, 128, 2, 64), w.grid, 2, 0),
         "dense": lambda: ops.attn_full(q, k, v, w.grid, 0),
+        "dense_d128": lambda: ops.attn_full(q2, k2, v2, w2.grid, 0),
+        "skiparse_d128": lambda: ops.skiparse_attn(q2, k2, v2, w2.grid, 2, 1),
         "skiparse": lambda: ops.skiparse_attn(q, k, v, w.grid, 2, 1),
         "cross": lambda: ops.attn_cross(q, kt, vt, w.grid),
         "temporal": lambda: ops.attn_temporal(q, k, v, w.grid, causal=True),
