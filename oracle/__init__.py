@@ -19,6 +19,7 @@ from .spacetime_oracle import (  # noqa: F401
     frame_causal_backward_ref,
     frame_causal_limit,
     packed_attn_ref,
+    packed_backward_ref,
     rope3d_packed_ref,
     rope3d_positions_ref,
     rope3d_ref,

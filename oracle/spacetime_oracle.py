@@ -686,3 +686,24 @@ def temporal_backward_ref(q, k, v, do, grid: Sequence[int], causal: bool = False
                 out[2][b, idx, h] = p.T @ dh
     return tuple(out)
 
+
+
+def packed_backward_ref(q, k, v, do, q_bounds: Sequence[int], scale: float | None = None):
+    """Gradients of block-diagonal self-attention over a packed batch (packed_attn_ref with
+    kv_bounds = q_bounds; CogVideoX section 3.1, Multi-Resolution Frame Pack): each sample's own
+    backward by the chain rule above, per head, written at the sample's rows.
+
+    q, k, v, do: [1, N, n_h, d] packed tensors; sample i owns rows [q_bounds[i], q_bounds[i+1])."""
+    qb = np.asarray(q_bounds, dtype=np.int64)
+    _, N, nh, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    out = [np.zeros((1, N, nh, d)) for _ in range(3)]
+    for i in range(len(qb) - 1):
+        r = slice(qb[i], qb[i + 1])
+        if qb[i + 1] <= qb[i]:
+            continue
+        for h in range(nh):
+            g = attention_head_backward_ref(q[0, r, h], k[0, r, h], v[0, r, h], do[0, r, h], scale)
+            for o_, g_ in zip(out, g):
+                o_[0, r, h] = g_
+    return tuple(out)

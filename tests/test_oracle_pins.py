@@ -695,3 +695,24 @@ def test_temporal_backward_special_cases():
     for a, b in zip(O.temporal_backward_ref(q, k, v, G, (3, 2, 2)),
                     O.skiparse_backward_ref(q, k, v, G, 4, O.SKIP_SINGLE)):
         np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+def test_packed_backward_matches_finite_differences_and_reduces_to_dense():
+    # three samples of 4, 0 and 1 tokens, then 3: the empty and one-token samples included
+    rng = np.random.default_rng(83)
+    bounds = [0, 4, 4, 5, 8]
+    q, k, v = (rng.standard_normal((1, 8, 2, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 8, 2, 3))
+    loss = lambda q_, k_, v_: float((O.packed_attn_ref(q_, k_, v_, bounds, scale=0.6) * G).sum())
+    dq, dk, dv = O.packed_backward_ref(q, k, v, G, bounds, scale=0.6)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+    # a one-token sample sees only itself (P = 1): its dq and dk vanish, its dv is its dO
+    assert np.abs(dq[0, 4]).max() <= 1e-15 and np.abs(dk[0, 4]).max() <= 1e-15   # zero up to fp64 rounding
+    np.testing.assert_array_equal(dv[0, 4], G[0, 4])
+    # one sample spanning the batch is the dense backward
+    one = O.packed_backward_ref(q, k, v, G, [0, 8], scale=0.6)
+    dense = O.attn_backward_ref(q, k, v, G, scale=0.6)
+    for a, b in zip(one, dense):
+        np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-14)
