@@ -267,6 +267,31 @@ int osp_attn_packed(const void* q, const void* k, const void* v, void* o, const 
                     const int32_t* kv_bounds, int32_t n_seg, int32_t heads, int32_t head_dim,
                     float softmax_scale, void* stream);
 
+/* Training a model on packed batches (CogVideoX section 3.1: Multi-Resolution Frame Pack trains on
+ * mixed-shape batches): osp_attn_packed's self-attention (each sample attends to its own rows)
+ * with the row log-sum-exp saved, and its backward pass.
+ *  bounds:  HOST, n_seg + 1 offsets of the samples' rows in every tensor (as q_bounds above).
+ *  lse:     fp32, device, 16-byte aligned, [heads][osp_attn_packed_lse_rows(bounds, n_seg)];
+ *           sample i's rows start at the start of its 256-row blocks (the sum of
+ *           ceil(len_j / 256) * 256 over j < i); row r of sample i holds m + log2(l) of its scaled
+ *           scores (log2 domain); padding slots are not written.
+ *  osp_attn_packed_train: o = osp_attn_packed(q, k, v, bounds, NULL) bit for bit, plus lse.
+ *  osp_attn_packed_backward: dq, dk, dv [bounds[n_seg]][heads][head_dim] bf16, device (not
+ *    overlapping the inputs), from q, k, v, o, dout and the lse of osp_attn_packed_train: each
+ *    sample's own attention backward, the arithmetic of osp_attn_backward (P and dS rounded to
+ *    bf16, fp32 accumulation); the call takes a stream-ordered workspace from the library's pool
+ *    (row sums, and at head_dim 64 an fp32 dQ accumulator of heads * lse_rows * 64 floats).
+ *  osp_attn_packed_lse_rows: the lse row count per head (>= 0), or -OSP_ERR_INVALID_ARG for bad
+ *    bounds.
+ *  Errors: OSP_ERR_INVALID_ARG (null or unaligned pointer, bad bounds), OSP_ERR_UNSUPPORTED
+ *  (head_dim, n_seg > OSP_MAX_SEGMENTS), OSP_ERR_CUDA. */
+int osp_attn_packed_lse_rows(const int32_t* bounds, int32_t n_seg);
+int osp_attn_packed_train(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* bounds,
+                          int32_t n_seg, int32_t heads, int32_t head_dim, float softmax_scale, void* stream);
+int osp_attn_packed_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, const int32_t* bounds, int32_t n_seg,
+                             int32_t heads, int32_t head_dim, float softmax_scale, void* stream);
+
 /* Skiparse gather ("Open-Sora Plan" section 2.2.2: sequence cut to 1/k, batch grown k-fold):
  *   x_out[b*k + g][s] = RoPE(x[b][token(g, s)])   for q and k (RoPE skipped if rope == NULL),
  *   v_out[b*k + g][s] = v[b][token(g, s)]         (exact copy).

@@ -19,6 +19,8 @@
 // Rows are addressed through the same TMA maps as the forward kernel, so Skiparse sets are
 // never gathered.  Every wait is bounded (status word + abort flag, as in the forward kernel).
 
+#include <type_traits>
+
 #include "osp_internal.h"
 
 namespace osp {
@@ -103,6 +105,63 @@ struct BwdParams {
   int text_len;
 };
 
+// Packed batch (block-diagonal self-attention, every sample its own set): sample i owns packed
+// rows [row[i], row[i+1]), its lse / Dv / dQ-accumulator rows start at vrow[i] (the training
+// forward's 256-row blocks), and tile[i] counts the 128-row tiles of the samples before it (a
+// kernel's CTAs are heads * tile[n_seg]).  Passed by value as a kernel parameter.
+struct BwdSegTable {
+  int n_seg;
+  int row[kMaxSegments + 1];
+  int vrow[kMaxSegments + 1];
+  int tile[kMaxSegments + 1];
+};
+struct NoBwdSeg {};
+template <bool kPk>
+using BwdSegParam = typename std::conditional<kPk, BwdSegTable, NoBwdSeg>::type;
+
+// The (sample*set, head, 128-row tile) a CTA works on, the set's rows n (tiles n_tiles), the
+// packed row its rows start at, and the first lse / Dv row of the (set, head).
+struct BwdUnit {
+  int tile, h, bg, b, g, n, n_tiles, row_base;
+  size_t vec_row;
+};
+template <bool kPk>
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, const BwdSegParam<kPk>& seg, int cta, bool reverse) {
+  BwdUnit u;
+  if constexpr (kPk) {
+    // sample: the largest i < n_seg with heads * tile[i] <= cta (empty samples own no CTA)
+    int lo = 0, hi = seg.n_seg;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.heads * seg.tile[mid] <= cta) lo = mid;
+      else hi = mid;
+    }
+    const int nt = seg.tile[lo + 1] - seg.tile[lo];
+    const int local = cta - p.heads * seg.tile[lo];
+    u.h = local / nt;
+    const int t = local - u.h * nt;
+    u.tile = reverse ? nt - 1 - t : t;
+    u.bg = u.b = u.g = 0;
+    u.n = seg.row[lo + 1] - seg.row[lo];
+    u.n_tiles = nt;
+    u.row_base = seg.row[lo];
+    u.vec_row = (size_t)u.h * p.vec_stride + seg.vrow[lo];
+  } else {
+    const int t = cta % p.n_tiles;
+    u.tile = reverse ? p.n_tiles - 1 - t : t;
+    const int hb = cta / p.n_tiles;
+    u.h = hb % p.heads;
+    u.bg = hb / p.heads;
+    u.b = u.bg / p.G;
+    u.g = u.bg % p.G;
+    u.n = p.n;
+    u.n_tiles = p.n_tiles;
+    u.row_base = 0;
+    u.vec_row = ((size_t)u.bg * p.heads + u.h) * p.vec_stride;
+  }
+  return u;
+}
+
 // First token of the block that token x belongs to (block 0: the text prefix; block 1 + f: frame f).
 __device__ __forceinline__ int causal_block_start(int x, int text_len, int hw) {
   return x < text_len ? 0 : text_len + (x - text_len) / hw * hw;
@@ -146,10 +205,11 @@ __device__ __forceinline__ bool bwd_warp_wait(uint32_t bar, uint32_t parity, con
 // ------------------------------------------------------------------------------------------
 // Dv = rowsum(dO * O), one thread per (sample, token, head) row, stored at the row's set slot
 // ------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool kPk = false>
 __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16* __restrict__ o,
                                                             const __nv_bfloat16* __restrict__ dout,
-                                                            const BwdParams p, long long rows) {
+                                                            const BwdParams p, long long rows,
+                                                            const __grid_constant__ BwdSegParam<kPk> seg) {
   for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < rows;
        r += (long long)gridDim.x * blockDim.x) {
     const int h = (int)(r % p.heads);
@@ -169,6 +229,17 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16*
         acc = fmaf(__uint_as_float(xs[e] << 16), __uint_as_float(ys[e] << 16), acc);
         acc = fmaf(__uint_as_float(xs[e] & 0xFFFF0000u), __uint_as_float(ys[e] & 0xFFFF0000u), acc);
       }
+    }
+    if constexpr (kPk) {   // packed row -> its sample's lse / Dv row
+      int lo = 0, hi = seg.n_seg;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (seg.row[mid] <= token) lo = mid;
+        else hi = mid;
+      }
+      const size_t vi = (size_t)h * p.vec_stride + seg.vrow[lo] + (token - seg.row[lo]);
+      if (index_ok(vi, p.vec_elems, p.status)) p.dvec[vi] = acc;
+      continue;
     }
     int g = 0, slot = token;
     if (p.layout == 1) {
@@ -252,11 +323,11 @@ __device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_
 // dK, dV: one CTA per (sample*set, head, 128-key tile)
 // ------------------------------------------------------------------------------------------
 // kKeysMajor = true: the kernel's "resident" tiles are K, V and the streamed ones Q, dO.
-template <int D>
+template <int D, bool kPk = false>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                         const BwdParams p) {
+                         const BwdParams p, const __grid_constant__ BwdSegParam<kPk> seg) {
   using C = BwdCfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -276,16 +347,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   // fused dQ tensor-memory buffers (64 columns each, next to dV at 256 and dK at 384)
   auto col_dq = [](int b) { return b ? 448u : 320u; };
 
-  const int tile = blockIdx.x % p.n_tiles;
-  const int hb = blockIdx.x / p.n_tiles;
-  const int h = hb % p.heads, bg = hb / p.heads;
-  const int b = bg / p.G, g = bg % p.G;
+  const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, false);
+  const int tile = un.tile, h = un.h, bg = un.bg, b = un.b, g = un.g;
+  const int n_rows = un.n, rb = un.row_base;   // the set's rows; its first packed row (packed batches)
   const int kv0 = tile * kBT;
   // query tiles i0 .. n_tiles-1 (frame-causal: the first query that may see key kv0 opens the range)
   const int i0 = p.frame_hw ? causal_block_start(kv0, p.text_len, p.frame_hw) / kBT : 0;
-  const int nq = p.n_tiles - i0;
+  const int nq = un.n_tiles - i0;
   const int chan0 = h * D;
-  const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
+  const size_t vec_row = un.vec_row;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(B_RES), 1);
@@ -342,8 +412,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     if (leader) {
       mbar_arrive_expect_tx(bar(B_RES), 2 * C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c) {
-        bwd_load_tile(&tm_k, sRes(0) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, kv0, g, b, p.k);
-        bwd_load_tile(&tm_v, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, kv0, g, b, p.k);
+        bwd_load_tile(&tm_k, sRes(0) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, rb + kv0, g, b, p.k);
+        bwd_load_tile(&tm_v, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, rb + kv0, g, b, p.k);
       }
     }
     for (int il = 0; il < nq; ++il) {
@@ -354,10 +424,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         const bool vec_ok = index_ok(vec_row + (size_t)i * kBT + kBT - 1, p.vec_elems, p.status);
         mbar_arrive_expect_tx(bar(B_FULL + s), 2 * C::kTileBytes + (vec_ok ? C::kVecBytes : 0));
         for (int c = 0; c < C::kChunks; ++c) {
-          bwd_load_tile(&tm_q, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, i * kBT, g,
-                        b, p.k);
-          bwd_load_tile(&tm_do, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, i * kBT, g,
-                        b, p.k);
+          bwd_load_tile(&tm_q, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c,
+                        rb + i * kBT, g, b, p.k);
+          bwd_load_tile(&tm_do, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c,
+                        rb + i * kBT, g, b, p.k);
         }
         if (vec_ok) {
           bulk_load(sVec(s), p.lse + vec_row + (size_t)i * kBT, kBT * 4, bar(B_FULL + s));
@@ -461,7 +531,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const bool leader = elect_one_sync();
       for (int il = 0; il < nq; ++il) {
         if (!bwd_warp_wait(bar(B_STGFULL), il & 1, wc)) break;
-        const size_t row0 = ((size_t)bg * p.heads + h) * p.vec_stride + (size_t)(i0 + il) * kBT;
+        const size_t row0 = vec_row + (size_t)(i0 + il) * kBT;
         if (leader && index_ok((row0 + kBT) * D - 1, p.dq_acc_elems, p.status)) {
           bulk_reduce_add_f32(p.dq_acc + row0 * D, sStg, kBT * D * 4);
           bulk_wait_read();
@@ -514,7 +584,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (il % kStages) * C::kVecBytes) +
                          kSub * hh + 32 * half;
       const int qa = i * kBT + kSub * hh + 32 * half;   // this warp's first query column
-      const int valid_q = p.n - qa;
+      // a key row past the set's end (zero-fill, or in a packed batch the next sample's keys) gets
+      // no valid column: its P and dS are zero, so the fused dQ product sums real keys only
+      const int valid_q = (kv0 + row < n_rows) ? n_rows - qa : 0;
       const uint32_t vis = p.frame_hw ? causal_columns(qa, kstart) : 0xffffffffu;
       const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
       uint32_t s[32], dp[32];
@@ -553,8 +625,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
       tc_fence_after();
       const int j = kv0 + row;
-      const bool live = j < p.n;
-      const int token = bwd_slot_token(p.layout, live ? j : 0, g, p.k);
+      const bool live = j < n_rows;
+      const int token = rb + bwd_slot_token(p.layout, live ? j : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
       const bool store = live && index_ok(off + D - 1, p.elems, p.status);
       if (half == 0) bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store);
@@ -572,11 +644,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
 // ------------------------------------------------------------------------------------------
 // dQ: one CTA per (sample*set, head, 128-query tile)
 // ------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool kPk = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const BwdParams p) {
+                       const BwdParams p, const __grid_constant__ BwdSegParam<kPk> seg) {
   using C = BwdCfg<D>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -591,15 +663,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // frame-causal: a head's query tiles in reverse, so that those seeing the most keys start first
-  const int tile = p.frame_hw ? p.n_tiles - 1 - (int)(blockIdx.x % p.n_tiles) : (int)(blockIdx.x % p.n_tiles);
-  const int hb = blockIdx.x / p.n_tiles;
-  const int h = hb % p.heads, bg = hb / p.heads;
-  const int b = bg / p.G, g = bg % p.G;
+  const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, p.frame_hw != 0);
+  const int tile = un.tile, h = un.h, bg = un.bg, b = un.b, g = un.g;
+  const int n_rows = un.n, rb = un.row_base;   // the set's rows; its first packed row (packed batches)
   const int q0 = tile * kBT;
   // key tiles 0 .. nk-1 (frame-causal: up to the last key the tile's last query may see)
   const int nk = p.frame_hw
-                     ? (min(p.n, causal_limit(min(q0 + kBT, p.n) - 1, p.text_len, p.frame_hw)) + kBT - 1) / kBT
-                     : p.n_tiles;
+                     ? (min(n_rows, causal_limit(min(q0 + kBT, n_rows) - 1, p.text_len, p.frame_hw)) + kBT - 1) / kBT
+                     : un.n_tiles;
   const int chan0 = h * D;
 
   if (threadIdx.x == 0) {
@@ -644,8 +715,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (leader) {
       mbar_arrive_expect_tx(bar(B_RES), 2 * C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c) {
-        bwd_load_tile(&tm_q, sRes(0) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, q0, g, b, p.k);
-        bwd_load_tile(&tm_do, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, q0, g, b, p.k);
+        bwd_load_tile(&tm_q, sRes(0) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, rb + q0, g, b, p.k);
+        bwd_load_tile(&tm_do, sRes(1) + c * kChunkBytes, bar(B_RES), p.layout, chan0 + 64 * c, rb + q0, g, b, p.k);
       }
     }
     for (int j = 0; j < nk; ++j) {
@@ -654,10 +725,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (leader) {
         mbar_arrive_expect_tx(bar(B_FULL + s), 2 * C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c) {
-          bwd_load_tile(&tm_k, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, j * kBT, g, b,
-                        p.k);
-          bwd_load_tile(&tm_v, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c, j * kBT, g, b,
-                        p.k);
+          bwd_load_tile(&tm_k, sStr(s, 0) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c,
+                        rb + j * kBT, g, b, p.k);
+          bwd_load_tile(&tm_v, sStr(s, 1) + c * kChunkBytes, bar(B_FULL + s), p.layout, chan0 + 64 * c,
+                        rb + j * kBT, g, b, p.k);
         }
       }
       issued = j + 1;
@@ -725,13 +796,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quarter * 32 + lane;                    // query row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int qs = q0 + row;
-    const bool live = qs < p.n;
-    const size_t vec_row = ((size_t)bg * p.heads + h) * p.vec_stride;
+    const bool live = qs < n_rows;
+    const size_t vec_row = un.vec_row;
     const bool vin = live && index_ok(vec_row + qs, p.vec_elems, p.status);
     const float lse_r = vin ? p.lse[vec_row + qs] : 0.f;
     const float dv_r = vin ? p.dvec[vec_row + qs] : 0.f;
     bool ok = true;
-    const int klim = p.frame_hw ? min(p.n, causal_limit(qs, p.text_len, p.frame_hw)) : p.n;   // keys this row sees
+    const int klim = p.frame_hw ? min(n_rows, causal_limit(qs, p.text_len, p.frame_hw)) : n_rows;   // keys it sees
     for (int t = 0; t < 2 * nk; ++t) {
       const int j = t >> 1, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
@@ -751,7 +822,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (ok && bwd_warp_wait(bar(B_DONE), 0, wc)) {
       tc_fence_after();
-      const int token = bwd_slot_token(p.layout, live ? qs : 0, g, p.k);
+      const int token = rb + bwd_slot_token(p.layout, live ? qs : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
       const bool store = live && index_ok(off + D - 1, p.elems, p.status);
       bwd_store_row<D>(tmem + lane_base + kColAcc0, p.scale, p.dq + off, store, half);
@@ -768,24 +839,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ------------------------------------------------------------------------------------------
 // fused dQ: dq = bf16(scale * dq_acc), from the accumulator's set-slot rows to natural token order
 // ------------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_dq_finalize_kernel(const BwdParams p, long long rows) {
+template <int D, bool kPk = false>
+__global__ void __launch_bounds__(256) attn_bwd_dq_finalize_kernel(const BwdParams p, long long rows,
+                                                                   const __grid_constant__ BwdSegParam<kPk> seg) {
   constexpr int V = D / 8;   // 16-byte output vectors (8 channels) per row
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < rows * V;
        idx += (long long)gridDim.x * blockDim.x) {
     const long long r = idx / V;
     const int v = (int)(idx - r * V);
-    const int slot = (int)(r % p.n);
-    const long long bh = r / p.n;
-    const int h = (int)(bh % p.heads), bg = (int)(bh / p.heads);
-    const int b = bg / p.G, g = bg % p.G;
+    int slot, h, token, b = 0;
+    size_t vrow;   // the (set, head)'s first accumulator row
+    if constexpr (kPk) {   // r = packed row * heads + h
+      h = (int)(r % p.heads);
+      token = (int)(r / p.heads);
+      int lo = 0, hi = seg.n_seg;
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (seg.row[mid] <= token) lo = mid;
+        else hi = mid;
+      }
+      slot = token - seg.row[lo];
+      vrow = (size_t)h * p.vec_stride + seg.vrow[lo];
+    } else {
+      slot = (int)(r % p.n);
+      const long long bh = r / p.n;
+      h = (int)(bh % p.heads);
+      const int bg = (int)(bh / p.heads);
+      b = bg / p.G;
+      vrow = ((size_t)bg * p.heads + h) * p.vec_stride;
+      token = bwd_slot_token(p.layout, slot, bg % p.G, p.k);
+    }
     // logical 16-byte chunks 2v, 2v + 1 of the row; within each 32-float half (8 chunks) the
     // dK/dV kernel stored chunk c at c ^ (slot & 7)
     const int c0 = 2 * v, hc = c0 & ~7;
-    const size_t rbase = (((size_t)bg * p.heads + h) * p.vec_stride + slot) * D;
+    const size_t rbase = (vrow + slot) * D;
     const size_t src = rbase + 4 * (hc + ((c0 & 7) ^ (slot & 7)));
     const size_t src1 = rbase + 4 * (hc + (((c0 + 1) & 7) ^ (slot & 7)));
-    const int token = bwd_slot_token(p.layout, slot, g, p.k);
     const size_t dst = (((size_t)b * p.N + token) * p.heads + h) * D + 8 * v;
     if (!index_ok(rbase + D - 1, p.dq_acc_elems, p.status) || !index_ok(dst + 7, p.elems, p.status)) continue;
     const float4 x = *reinterpret_cast<const float4*>(p.dq_acc + src);
@@ -797,29 +886,33 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_finalize_kernel(const BwdPara
   }
 }
 
-template <int D>
+template <int D, bool kPk = false>
 int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const CUtensorMap& tk,
                  const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, long long rows, long long ctas,
-                 cudaStream_t stream) {
+                 cudaStream_t stream, const BwdSegParam<kPk>& seg = BwdSegParam<kPk>{}) {
   constexpr int smem = BwdCfg<D>::kSmemBytes;
-  int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_bwd_dkdv_kernel<D>), smem, "attn_bwd_dkdv_kernel");
-  if (rc || (rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_bwd_dq_kernel<D>), smem, "attn_bwd_dq_kernel")))
+  int rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_bwd_dkdv_kernel<D, kPk>), smem,
+                            "attn_bwd_dkdv_kernel");
+  if (rc || (rc = ensure_smem_attr(reinterpret_cast<const void*>(attn_bwd_dq_kernel<D, kPk>), smem,
+                                   "attn_bwd_dq_kernel")))
     return rc;
   const long long dblocks = std::min<long long>((rows + 255) / 256, (long long)device_sm_count() * 16);
-  attn_bwd_dvec_kernel<D><<<(unsigned)dblocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                                 static_cast<const __nv_bfloat16*>(dout), p, rows);
+  attn_bwd_dvec_kernel<D, kPk><<<(unsigned)dblocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                                      static_cast<const __nv_bfloat16*>(dout), p, rows,
+                                                                      seg);
   rc = check_launch("attn_bwd_dvec_kernel");
   if (rc) return rc;
-  attn_bwd_dkdv_kernel<D><<<(unsigned)ctas, BwdCfg<D>::kThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  if (ctas <= 0) return OSP_OK;   // no rows at all
+  attn_bwd_dkdv_kernel<D, kPk><<<(unsigned)ctas, BwdCfg<D>::kThreads, smem, stream>>>(tq, tk, tv, tdo, p, seg);
   if ((rc = check_launch("attn_bwd_dkdv_kernel"))) return rc;
   if constexpr (BwdCfg<D>::kFuseDq) {
     const long long qrows = rows;   // (sample*set, head, slot) rows: B * G * heads * n = B * N * heads
     const long long fblocks = std::min<long long>((qrows * (D / 8) + 255) / 256, (long long)device_sm_count() * 16);
     if (fblocks > 0)
-      attn_bwd_dq_finalize_kernel<D><<<(unsigned)fblocks, 256, 0, stream>>>(p, qrows);
+      attn_bwd_dq_finalize_kernel<D, kPk><<<(unsigned)fblocks, 256, 0, stream>>>(p, qrows, seg);
     return check_launch("attn_bwd_dq_finalize_kernel");
   }
-  attn_bwd_dq_kernel<D><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  attn_bwd_dq_kernel<D, kPk><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p, seg);
   return check_launch("attn_bwd_dq_kernel");
 }
 
@@ -897,6 +990,97 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
     case 96: rc = launch_bwd_d<96>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
     case 128: rc = launch_bwd_d<128>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream); break;
     default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", s.head_dim);
+  }
+  if (acc) cudaFreeAsync(acc, stream);
+  cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+int packed_lse_rows(const int32_t* bounds, int n_seg) {
+  long long rows = 0;
+  for (int i = 0; i < n_seg; ++i) rows += (bounds[i + 1] - bounds[i] + 255) / 256 * 256;
+  return (int)rows;
+}
+
+int packed_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, const int32_t* bounds, int n_seg,
+                           int heads, int head_dim, float scale, cudaStream_t stream) {
+  unsigned* status = device_status_word();
+  if (!status) return OSP_ERR_CUDA;
+  const int N = bounds[n_seg];
+  BwdSegTable seg{};
+  seg.n_seg = n_seg;
+  long long tiles = 0, vrows = 0;
+  for (int i = 0; i <= n_seg; ++i) {
+    seg.row[i] = bounds[i];
+    seg.vrow[i] = (int)vrows;
+    seg.tile[i] = (int)tiles;
+    if (i < n_seg) {
+      const int len = bounds[i + 1] - bounds[i];
+      tiles += (len + kBT - 1) / kBT;
+      vrows += (len + 255) / 256 * 256;   // the training forward's 256-row blocks
+    }
+  }
+  BwdParams p{};
+  p.N = N;
+  p.heads = heads;
+  p.G = 1;
+  p.k = 1;
+  p.layout = 0;
+  p.n = N;                                // unused per CTA (each sample's own rows); for the host checks
+  p.n_tiles = (int)tiles;
+  p.vec_stride = (int)vrows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale = scale;
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.status = status;
+  p.timeout_ns = wait_timeout_ns();
+  p.elems = (unsigned long long)N * heads * head_dim / bounds_check_divisor();
+  p.vec_elems = (unsigned long long)heads * p.vec_stride / bounds_check_divisor();
+  const long long ctas = tiles * heads;
+  if (ctas > (1LL << 30)) return set_error(OSP_ERR_UNSUPPORTED, "%lld backward work units is too many", ctas);
+  if (N == 0) return OSP_OK;
+  const osp_shape sh{1, 0, 1, 1, 1, heads, head_dim};   // one sample of N packed rows
+  CUtensorMap tq, tk, tv, tdo;
+  int rc;
+  if ((rc = make_attn_tmap(&tq, q, sh, N, 0, 1)) != OSP_OK) return rc;
+  if ((rc = make_attn_tmap(&tk, k, sh, N, 0, 1)) != OSP_OK) return rc;
+  if ((rc = make_attn_tmap(&tv, v, sh, N, 0, 1)) != OSP_OK) return rc;
+  if ((rc = make_attn_tmap(&tdo, dout, sh, N, 0, 1)) != OSP_OK) return rc;
+  const size_t vec_bytes = (size_t)heads * p.vec_stride * sizeof(float);
+  void* ws = nullptr;
+  cudaMemPool_t pool = workspace_pool();
+  if (!pool || cudaMallocFromPoolAsync(&ws, vec_bytes, pool, stream) != cudaSuccess)
+    return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", vec_bytes);
+  if (cudaMemsetAsync(ws, 0, vec_bytes, stream) != cudaSuccess) {
+    cudaFreeAsync(ws, stream);
+    return set_error(OSP_ERR_CUDA, "clearing the backward workspace failed");
+  }
+  p.dvec = static_cast<float*>(ws);
+  void* acc = nullptr;
+  if (head_dim == 64 && BwdCfg<64>::kFuseDq) {
+    const size_t acc_bytes = (size_t)heads * p.vec_stride * head_dim * sizeof(float);
+    if (cudaMallocFromPoolAsync(&acc, acc_bytes, pool, stream) != cudaSuccess) {
+      cudaFreeAsync(ws, stream);
+      return set_error(OSP_ERR_CUDA, "stream-ordered workspace allocation (%zu bytes) failed", acc_bytes);
+    }
+    if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) {
+      cudaFreeAsync(acc, stream);
+      cudaFreeAsync(ws, stream);
+      return set_error(OSP_ERR_CUDA, "clearing the backward workspace failed");
+    }
+    p.dq_acc = static_cast<float*>(acc);
+    p.dq_acc_elems = (unsigned long long)(acc_bytes / sizeof(float)) / bounds_check_divisor();
+  }
+  const long long rows = (long long)N * heads;
+  switch (head_dim) {
+    case 64: rc = launch_bwd_d<64, true>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream, seg); break;
+    case 96: rc = launch_bwd_d<96, true>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream, seg); break;
+    case 128: rc = launch_bwd_d<128, true>(o, dout, tq, tk, tv, tdo, p, rows, ctas, stream, seg); break;
+    default: rc = set_error(OSP_ERR_UNSUPPORTED, "head_dim %d not in {64, 96, 128}", head_dim);
   }
   if (acc) cudaFreeAsync(acc, stream);
   cudaFreeAsync(ws, stream);

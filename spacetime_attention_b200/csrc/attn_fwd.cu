@@ -350,7 +350,7 @@ int causal_temporal_attention_launch(const void* q, const void* k, const void* v
 
 int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
                             const int32_t* kv_bounds, int n_seg, int heads, int head_dim, float scale,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, float* lse) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   SegTable seg{};
@@ -382,6 +382,10 @@ int packed_attention_launch(const void* q, const void* k, const void* v, void* o
   p.n_split = 1;
   p.n_items = (int)units;
   p.o_elems = (unsigned long long)n_q_total * heads * head_dim / (unsigned long long)bounds_check_divisor();
+  // training forward: lse [heads][blocks * 256], sample i's rows from blk[i] * 256
+  p.lse = lse;
+  p.lse_stride = (int)(blocks * 2 * kBM);
+  p.lse_elems = lse ? (unsigned long long)heads * p.lse_stride / (unsigned long long)bounds_check_divisor() : 0;
   // the packed tensors are one sample of n_q_total (q, o) / n_kv_total (k, v) rows
   const osp_shape sh{1, 0, 1, 1, 1, heads, head_dim};
   CUtensorMap tq, tk, tv;

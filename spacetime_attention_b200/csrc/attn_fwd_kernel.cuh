@@ -821,8 +821,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = 1.f / l;
       const int slot = w.q0 + i * kBM + row;
       const bool live = slot < w.nq;
-      if (!kPacked && part < 0 && p.lse && live) {
-        const size_t li = ((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot;
+      if (part < 0 && p.lse && live) {
+        // packed batches: [heads][sum of the samples' 256-row blocks], sample sg at row blk[sg] * 256
+        size_t li;
+        if constexpr (kPacked) li = (size_t)h * p.lse_stride + (size_t)seg.blk[*seg_slot] * (2 * kBM) + slot;
+        else li = ((size_t)(b * p.G + g) * p.heads + h) * p.lse_stride + slot;
         if (index_ok(li, p.lse_elems, p.status)) p.lse[li] = m + __log2f(l);
       }
       if (part >= 0) {

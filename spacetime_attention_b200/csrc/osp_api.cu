@@ -528,6 +528,52 @@ int osp_attn_packed(const void* q, const void* k, const void* v, void* o, const 
                                  static_cast<cudaStream_t>(stream));
 }
 
+static int check_packed_call(const int32_t* bounds, int32_t n_seg, int32_t heads, int32_t head_dim) {
+  if (n_seg < 1 || n_seg > OSP_MAX_SEGMENTS)
+    return set_error(n_seg < 1 ? OSP_ERR_INVALID_ARG : OSP_ERR_UNSUPPORTED, "n_seg = %d not in [1, %d]", n_seg,
+                     OSP_MAX_SEGMENTS);
+  if (heads < 1) return set_error(OSP_ERR_INVALID_ARG, "heads = %d", heads);
+  if (head_dim != 64 && head_dim != 96 && head_dim != 128)
+    return set_error(OSP_ERR_UNSUPPORTED, "attention head_dim %d not in {64, 96, 128}", head_dim);
+  return check_bounds(bounds, n_seg, "bounds");
+}
+
+int osp_attn_packed_lse_rows(const int32_t* bounds, int32_t n_seg) {
+  g_last_error[0] = 0;
+  if (n_seg < 1 || n_seg > OSP_MAX_SEGMENTS) return -set_error(OSP_ERR_INVALID_ARG, "n_seg = %d", n_seg);
+  const int rc = check_bounds(bounds, n_seg, "bounds");
+  if (rc) return -rc;
+  return packed_lse_rows(bounds, n_seg);
+}
+
+int osp_attn_packed_train(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* bounds,
+                          int32_t n_seg, int32_t heads, int32_t head_dim, float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_packed_call(bounds, n_seg, heads, head_dim);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse) return set_error(OSP_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)head_dim);
+  return packed_attention_launch(q, k, v, o, bounds, bounds, n_seg, heads, head_dim, softmax_scale,
+                                 static_cast<cudaStream_t>(stream), lse);
+}
+
+int osp_attn_packed_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, const int32_t* bounds, int32_t n_seg,
+                             int32_t heads, int32_t head_dim, float softmax_scale, void* stream) {
+  g_last_error[0] = 0;
+  int rc = check_packed_call(bounds, n_seg, heads, head_dim);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return set_error(OSP_ERR_INVALID_ARG, "null pointer");
+  for (const void* t : {q, k, v, o, dout, static_cast<const void*>(lse), static_cast<const void*>(dq),
+                        static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (!aligned16(t)) return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)head_dim);
+  return packed_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, bounds, n_seg, heads, head_dim, softmax_scale,
+                                static_cast<cudaStream_t>(stream));
+}
+
 int osp_skiparse_gather(const void* q, const void* k, const void* v, void* q_out, void* k_out, void* v_out,
                         const osp_shape* shape, int32_t sparse_k, int32_t mode, const osp_rope* rope, void* stream) {
   g_last_error[0] = 0;

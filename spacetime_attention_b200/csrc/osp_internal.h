@@ -121,9 +121,17 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
 
 // Packed batch (block-diagonal attention): segment i owns q/o rows [q_bounds[i], q_bounds[i+1])
 // and k/v rows [kv_bounds[i], kv_bounds[i+1]); host arrays of n_seg + 1 validated offsets.
+// lse (optional, training forward of self-attention): [heads][packed_lse_rows], sample i's rows
+// from the start of its 256-row blocks.
 int packed_attention_launch(const void* q, const void* k, const void* v, void* o, const int32_t* q_bounds,
                             const int32_t* kv_bounds, int n_seg, int heads, int head_dim, float scale,
-                            cudaStream_t stream);
+                            cudaStream_t stream, float* lse = nullptr);
+// Rows of a packed batch's lse per head: sum over samples of ceil(len / 256) * 256.
+int packed_lse_rows(const int32_t* bounds, int n_seg);
+// Backward of packed self-attention (each sample's own attention) from the training forward's lse.
+int packed_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, const int32_t* bounds, int n_seg,
+                           int heads, int head_dim, float scale, cudaStream_t stream);
 
 // 3D RoPE of a packed batch: sample i is text_len_i unrotated tokens then its own T_i x H_i x W_i grid.
 int rope3d_packed_launch(const void* q, const void* k, void* q_out, void* k_out, const osp_sample_grid* samples,

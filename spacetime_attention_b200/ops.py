@@ -36,7 +36,8 @@ EXPORTED = ("osp_rope3d", "osp_attn_full", "osp_skiparse_gather", "osp_skiparse_
             "osp_attn_spatial", "osp_attn_temporal", "osp_attn_frame_causal", "osp_attn_forward_train",
             "osp_attn_backward", "osp_attn_frame_causal_train", "osp_attn_frame_causal_backward",
             "osp_attn_spatial_train", "osp_attn_spatial_backward", "osp_attn_temporal_train",
-            "osp_attn_temporal_backward")
+            "osp_attn_temporal_backward", "osp_attn_packed_lse_rows", "osp_attn_packed_train",
+            "osp_attn_packed_backward")
 
 MAX_SEGMENTS = 256   # OSP_MAX_SEGMENTS
 
@@ -92,6 +93,11 @@ def library() -> ctypes.CDLL:
             "osp_rope3d_packed": [vp, vp, vp, vp, ctypes.POINTER(OspSampleGrid), i32, i32, i32, rp, vp],
             "osp_attn_packed": [vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
                                 i32, i32, ctypes.c_float, vp],
+            "osp_attn_packed_lse_rows": [ctypes.POINTER(ctypes.c_int32), i32],
+            "osp_attn_packed_train": [vp, vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), i32, i32, i32,
+                                      ctypes.c_float, vp],
+            "osp_attn_packed_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ctypes.c_int32), i32,
+                                         i32, i32, ctypes.c_float, vp],
             "osp_skiparse_gather": [vp, vp, vp, vp, vp, vp, sp, i32, i32, rp, vp],
             "osp_skiparse_scatter": [vp, vp, sp, i32, i32, vp],
             "osp_skiparse_attn": [vp, vp, vp, vp, sp, i32, i32, ctypes.c_float, vp],
@@ -415,6 +421,58 @@ def attn_packed(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_bounds, kv_
     _check("osp_attn_packed", library().osp_attn_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(o), qb, kb, len(qb) - 1,
                                                         heads, d, ctypes.c_float(scale), _stream_handle(q)))
     return o
+
+
+def packed_lse_rows(bounds) -> int:
+    """osp_attn_packed_lse_rows: lse rows per head of a packed batch (each sample's 256-row blocks)."""
+    b = _bounds(bounds)
+    n = library().osp_attn_packed_lse_rows(b, len(b) - 1)
+    if n < 0:
+        _check("osp_attn_packed_lse_rows", -n)
+    return n
+
+
+def _packed_self(q: torch.Tensor, bounds):
+    _bshd(q, "q")
+    if q.shape[0] != 1:
+        raise ValueError(f"a packed batch has B = 1 (got {q.shape[0]})")
+    b = _bounds(bounds)
+    if len(b) < 2 or b[len(b) - 1] != q.shape[1]:
+        raise ValueError(f"the last bound must be the batch's {q.shape[1]} rows")
+    return b
+
+
+def attn_packed_train(q, k, v, bounds, scale: float = 0.0, o=None, lse=None):
+    """osp_attn_packed_train: packed self-attention with the saved lse; returns (o, lse), lse
+    [heads, packed_lse_rows(bounds)] fp32."""
+    b = _packed_self(q, bounds); _same(k, q, "k"); _same(v, q, "v")
+    _, _, heads, d = q.shape
+    o = _out(o, q, "o")
+    rows = packed_lse_rows(bounds)
+    if lse is None:
+        lse = torch.empty((heads, rows), dtype=torch.float32, device=q.device)
+    elif lse.dtype != torch.float32 or not lse.is_contiguous() or lse.numel() != heads * rows:
+        raise ValueError(f"lse must be contiguous fp32 with {heads} x {rows} elements")
+    _check("osp_attn_packed_train", library().osp_attn_packed_train(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), b, len(b) - 1, heads, d, ctypes.c_float(scale),
+        _stream_handle(q)))
+    return o, lse
+
+
+def attn_packed_backward(q, k, v, o, dout, lse, bounds, scale: float = 0.0, dq=None, dk=None, dv=None):
+    """osp_attn_packed_backward: returns (dq, dk, dv)."""
+    b = _packed_self(q, bounds)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _same(t, q, n)
+    _, _, heads, d = q.shape
+    rows = packed_lse_rows(bounds)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.numel() != heads * rows:
+        raise ValueError(f"lse must be contiguous fp32 with {heads} x {rows} elements")
+    dq, dk, dv = _out(dq, q, "dq"), _out(dk, q, "dk"), _out(dv, q, "dv")
+    _check("osp_attn_packed_backward", library().osp_attn_packed_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), b, len(b) - 1,
+        heads, d, ctypes.c_float(scale), _stream_handle(q)))
+    return dq, dk, dv
 
 
 def attn_full_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, text_len: int, scale: float = 0.0,

@@ -26,6 +26,10 @@ def calls(dev):
         o, lse = ops.attn_forward_train(q, k, v, w.grid, 0)
         return ops.attn_backward(q, k, v, o, do, lse, w.grid, 0)
 
+    def packed_training():   # two samples of 100 and 156 rows: packed forward with lse, backward
+        o, lse = ops.attn_packed_train(q, k, v, [0, 100, 256])
+        return ops.attn_packed_backward(q, k, v, o, do, lse, [0, 100, 256])
+
     def temporal_training():   # the per-set temporal kernels (T <= 64): forward with lse, backward
         o, lse = ops.attn_temporal_train(q, k, v, w.grid, causal=True)
         return ops.attn_temporal_backward(q, k, v, o, do, lse, w.grid, causal=True)
@@ -43,6 +47,7 @@ def calls(dev):
         "packed": lambda: ops.attn_packed(q, k, v, [0, 100, 256]),
         "backward": backward,
         "temporal_training": temporal_training,
+        "packed_training": packed_training,
     }
 
 
