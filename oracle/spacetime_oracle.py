@@ -707,3 +707,29 @@ def packed_backward_ref(q, k, v, do, q_bounds: Sequence[int], scale: float | Non
             for o_, g_ in zip(out, g):
                 o_[0, r, h] = g_
     return tuple(out)
+
+
+def skiparse_text_backward_ref(q, k, v, do, text_len: int, k_ratio: int, mode: int, scale: float | None = None):
+    """Gradients of Skiparse attention with a joined text prefix (skiparse_text_attn_ref): per
+    sample and head, the chain rule above on the masked score matrix whose row for a text token
+    sees every token and whose row for a video token of set g sees the text tokens and set g."""
+    B, N, nh, d = q.shape
+    L = int(text_len)
+    scale = default_scale(d) if scale is None else scale
+    visible = np.zeros((N, N), dtype=bool)
+    visible[:L, :] = True
+    for st in skiparse_sets(N - L, k_ratio, mode):
+        rows = L + np.asarray(st)
+        visible[np.ix_(rows, np.arange(L))] = True
+        visible[np.ix_(rows, rows)] = True
+    out = [np.empty((B, N, nh, d)) for _ in range(3)]
+    for b in range(B):
+        for h in range(nh):
+            qh, kh, vh, dh = (np.asarray(a[b, :, h], np.float64) for a in (q, k, v, do))
+            p = softmax_rows(np.where(visible, (qh @ kh.T) * scale, -np.inf))
+            o = p @ vh
+            ds = p * (dh @ vh.T - (dh * o).sum(axis=1, keepdims=True))
+            out[0][b, :, h] = ds @ kh * scale
+            out[1][b, :, h] = ds.T @ qh * scale
+            out[2][b, :, h] = p.T @ dh
+    return tuple(out)

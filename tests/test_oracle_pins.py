@@ -716,3 +716,28 @@ def test_packed_backward_matches_finite_differences_and_reduces_to_dense():
     dense = O.attn_backward_ref(q, k, v, G, scale=0.6)
     for a, b in zip(one, dense):
         np.testing.assert_allclose(a, b, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("mode", [O.SKIP_SINGLE, O.SKIP_GROUP])
+def test_skiparse_text_backward_matches_finite_differences(mode):
+    # 3 text tokens + 8 video tokens in k = 2 sets
+    rng = np.random.default_rng(84 + mode)
+    q, k, v = (rng.standard_normal((1, 11, 2, 3)) for _ in range(3))
+    G = rng.standard_normal((1, 11, 2, 3))
+    loss = lambda q_, k_, v_: float((O.skiparse_text_attn_ref(q_, k_, v_, 3, 2, mode, scale=0.8) * G).sum())
+    dq, dk, dv = O.skiparse_text_backward_ref(q, k, v, G, 3, 2, mode, scale=0.8)
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v), rtol=1e-6, atol=1e-8)
+
+
+def test_skiparse_text_backward_reduces_to_skiparse_and_dense():
+    rng = np.random.default_rng(86)
+    q, k, v, G = (rng.standard_normal((2, 12, 2, 3)) for _ in range(4))
+    # no text: the Skiparse backward
+    for a, b in zip(O.skiparse_text_backward_ref(q, k, v, G, 0, 3, O.SKIP_SINGLE),
+                    O.skiparse_backward_ref(q, k, v, G, 3, O.SKIP_SINGLE)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    # one set: every token sees every token, the dense backward
+    for a, b in zip(O.skiparse_text_backward_ref(q, k, v, G, 4, 1, O.SKIP_GROUP), O.attn_backward_ref(q, k, v, G)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
