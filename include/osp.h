@@ -171,14 +171,18 @@ int osp_attn_frame_causal(const void* q, const void* k, const void* v, void* o, 
 /* Training: forward with saved statistics, and the backward pass (Open-Sora Plan section 2.2.2:
  * the model is trained with Skiparse attention).  sparse_k == 1: dense attention over
  * N = text_len + T*H*W tokens (as osp_attn_full); sparse_k > 1: Skiparse Single / Group Skip
- * (as osp_skiparse_attn, text_len must be 0, Group Skip needs k | 128).
+ * (as osp_skiparse_attn, Group Skip needs k | 128), text_len > 0 joining the text prefix to
+ * every set (a text query sees all N tokens, a video query of set g the text and set g).
  *
  * osp_attn_forward_train: o as the corresponding inference call (same kernel, arithmetic and work
  *   split), plus lse, the log2-domain log-sum-exp of every query row's scaled scores:
  *   lse[((b*G + g)*heads + h)*n_pad + s] = log2(sum_j exp2(score_sj * scale * log2(e))) for slot s
  *   of set g (G = 1 and slot = token for dense; G = k for Skiparse), n = N / G,
  *   n_pad = ceil(n / 128) * 128.  lse: device fp32 array of B * G * heads * n_pad values (the
- *   padding entries are not written), 16-byte aligned; it is an opaque input of the backward. */
+ *   padding entries are not written), 16-byte aligned; it is an opaque input of the backward.
+ *   Skiparse with text_len > 0: n = T*H*W / k for the video rows' block, which is followed by the
+ *   text rows' lse[B*k*heads*n_pad + (b*heads + h)*L_pad + t], L_pad = ceil(text_len / 128) * 128
+ *   (B * (k * heads * n_pad + heads * L_pad) values). */
 int osp_attn_forward_train(const void* q, const void* k, const void* v, void* o, float* lse, const osp_shape* shape,
                            int32_t sparse_k, int32_t mode, float softmax_scale, void* stream);
 
@@ -191,6 +195,12 @@ int osp_attn_forward_train(const void* q, const void* k, const void* v, void* o,
  *   accumulation in tensor memory, outputs rounded to bf16.  Scratch: rowsum(dO * O) in a
  *   stream-ordered block (B * G * heads * n_pad floats) from the library's memory pool.
  *   Three kernel launches (row sums, dK/dV, dQ).
+ *   Skiparse with text_len > 0: the video queries' part runs over B*k gathered samples of
+ *   [set g's n rows; the text rows] (queries: the first n), the text queries' part over the
+ *   natural samples (queries: the first text_len rows); dK and dV of a row sum their fp32
+ *   contributions (sets 0..k-1, then the text queries) before one rounding to bf16.  Scratch:
+ *   the gathered q, k, v, o, dout and dq (bf16) and dk, dv (fp32) of B*k*(n + text_len) rows,
+ *   and the text queries' fp32 dk, dv of B*N rows, from the same pool.
  *  Errors: as the forward, OSP_ERR_CUDA. */
 int osp_attn_backward(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                       void* dq, void* dk, void* dv, const osp_shape* shape, int32_t sparse_k, int32_t mode,

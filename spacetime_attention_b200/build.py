@@ -26,7 +26,7 @@ LIB = os.path.join(PKG, "libosp.so")
 # OSP_ERR_BOUNDS in the status word and skips the access); objects in _build/debug.
 DEBUG_LIB = os.path.join(PKG, "libosp_debug.so")
 
-SOURCES = ["osp_api.cu", "rope_permute.cu", "attn_fwd.cu", "attn_temporal.cu", "attn_bwd.cu"]
+SOURCES = ["osp_api.cu", "rope_permute.cu", "attn_fwd.cu", "attn_temporal.cu", "attn_bwd.cu", "attn_text_bwd.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
               "-I", CSRC, "-I", INCLUDE]

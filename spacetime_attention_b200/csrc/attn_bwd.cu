@@ -87,6 +87,9 @@ struct BwdParams {
   int heads, G, k, layout;
   int n_tiles;      // ceil(n / 128)
   int vec_stride;   // floats per (sample*set, head) row of lse / Dv (n rounded up to 128)
+  // Queries: the first q_rows rows of each set (q_tiles = ceil(q_rows / 128) tiles); n and
+  // n_tiles unless only a prefix of the rows are queries (the text queries of a joined-text call)
+  int q_rows, q_tiles;
   float scale_log2;
   float scale;
   const float* lse;
@@ -94,6 +97,8 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dk32;      // non-null: dK and dV are written unrounded, fp32, here and in dv32 (not dk, dv)
+  float* dv32;
   float* dq_acc;    // fused dQ: fp32 [B*G][heads][vec_stride][D], zeroed before the dK/dV kernel
   unsigned long long dq_acc_elems;
   unsigned* status;
@@ -126,7 +131,8 @@ struct BwdUnit {
   size_t vec_row;
 };
 template <bool kPk>
-__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, const BwdSegParam<kPk>& seg, int cta, bool reverse) {
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, const BwdSegParam<kPk>& seg, int cta, bool reverse,
+                                            int tiles_per_set = 0) {
   BwdUnit u;
   if constexpr (kPk) {
     // sample: the largest i < n_seg with heads * tile[i] <= cta (empty samples own no CTA)
@@ -147,9 +153,10 @@ __device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, const BwdSegPara
     u.row_base = seg.row[lo];
     u.vec_row = (size_t)u.h * p.vec_stride + seg.vrow[lo];
   } else {
-    const int t = cta % p.n_tiles;
-    u.tile = reverse ? p.n_tiles - 1 - t : t;
-    const int hb = cta / p.n_tiles;
+    const int tps = tiles_per_set > 0 ? tiles_per_set : p.n_tiles;   // CTAs per (set, head)
+    const int t = cta % tps;
+    u.tile = reverse ? tps - 1 - t : t;
+    const int hb = cta / tps;
     u.h = hb % p.heads;
     u.bg = hb / p.heads;
     u.b = u.bg / p.G;
@@ -242,6 +249,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16*
       continue;
     }
     int g = 0, slot = token;
+    if (p.layout == 0 && slot >= p.q_rows) continue;   // not a query row (joined-text's text queries)
     if (p.layout == 1) {
       g = token % p.k;
       slot = token / p.k;
@@ -319,6 +327,24 @@ __device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_
   }
 }
 
+// fp32 variant: the row's D accumulator columns times scale, unrounded
+template <int D>
+__device__ __forceinline__ void bwd_store_row_f32(uint32_t taddr, float scale, float* dst, bool live) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t r[32];
+    tmem_ld32(taddr + 32 * cc, r);
+    tmem_wait_ld();
+    if (live) {
+      float4* d4 = reinterpret_cast<float4*>(dst + 32 * cc);
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        d4[v] = make_float4(__uint_as_float(r[4 * v]) * scale, __uint_as_float(r[4 * v + 1]) * scale,
+                            __uint_as_float(r[4 * v + 2]) * scale, __uint_as_float(r[4 * v + 3]) * scale);
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // dK, dV: one CTA per (sample*set, head, 128-key tile)
 // ------------------------------------------------------------------------------------------
@@ -353,7 +379,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const int kv0 = tile * kBT;
   // query tiles i0 .. n_tiles-1 (frame-causal: the first query that may see key kv0 opens the range)
   const int i0 = p.frame_hw ? causal_block_start(kv0, p.text_len, p.frame_hw) / kBT : 0;
-  const int nq = un.n_tiles - i0;
+  const int nq = (kPk ? un.n_tiles : p.q_tiles) - i0;
+  const int q_rows = kPk ? n_rows : p.q_rows;   // query rows of the set (a prefix of its rows)
   const int chan0 = h * D;
   const size_t vec_row = un.vec_row;
 
@@ -586,7 +613,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const int qa = i * kBT + kSub * hh + 32 * half;   // this warp's first query column
       // a key row past the set's end (zero-fill, or in a packed batch the next sample's keys) gets
       // no valid column: its P and dS are zero, so the fused dQ product sums real keys only
-      const int valid_q = (kv0 + row < n_rows) ? n_rows - qa : 0;
+      const int valid_q = (kv0 + row < n_rows) ? q_rows - qa : 0;
       const uint32_t vis = p.frame_hw ? causal_columns(qa, kstart) : 0xffffffffu;
       const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
       uint32_t s[32], dp[32];
@@ -629,8 +656,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const int token = rb + bwd_slot_token(p.layout, live ? j : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
       const bool store = live && index_ok(off + D - 1, p.elems, p.status);
-      if (half == 0) bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store);
-      else bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, store);
+      if (p.dk32) {
+        if (half == 0) bwd_store_row_f32<D>(tmem + lane_base + kColAcc0, 1.f, p.dv32 + off, store);
+        else bwd_store_row_f32<D>(tmem + lane_base + kColAcc1, p.scale, p.dk32 + off, store);
+      } else if (half == 0) {
+        bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store);
+      } else {
+        bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, store);
+      }
     }
   }
   tc_fence_before();
@@ -663,9 +696,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // frame-causal: a head's query tiles in reverse, so that those seeing the most keys start first
-  const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, p.frame_hw != 0);
+  const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, p.frame_hw != 0, kPk ? 0 : p.q_tiles);
   const int tile = un.tile, h = un.h, bg = un.bg, b = un.b, g = un.g;
   const int n_rows = un.n, rb = un.row_base;   // the set's rows; its first packed row (packed batches)
+  const int q_rows = kPk ? n_rows : p.q_rows;  // its query rows
   const int q0 = tile * kBT;
   // key tiles 0 .. nk-1 (frame-causal: up to the last key the tile's last query may see)
   const int nk = p.frame_hw
@@ -796,7 +830,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = quarter * 32 + lane;                    // query row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int qs = q0 + row;
-    const bool live = qs < n_rows;
+    const bool live = qs < q_rows;
     const size_t vec_row = un.vec_row;
     const bool vin = live && index_ok(vec_row + qs, p.vec_elems, p.status);
     const float lse_r = vin ? p.lse[vec_row + qs] : 0.f;
@@ -861,8 +895,8 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_finalize_kernel(const BwdPara
       slot = token - seg.row[lo];
       vrow = (size_t)h * p.vec_stride + seg.vrow[lo];
     } else {
-      slot = (int)(r % p.n);
-      const long long bh = r / p.n;
+      slot = (int)(r % p.q_rows);
+      const long long bh = r / p.q_rows;
       h = (int)(bh % p.heads);
       const int bg = (int)(bh / p.heads);
       b = bg / p.G;
@@ -906,13 +940,15 @@ int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const C
   attn_bwd_dkdv_kernel<D, kPk><<<(unsigned)ctas, BwdCfg<D>::kThreads, smem, stream>>>(tq, tk, tv, tdo, p, seg);
   if ((rc = check_launch("attn_bwd_dkdv_kernel"))) return rc;
   if constexpr (BwdCfg<D>::kFuseDq) {
-    const long long qrows = rows;   // (sample*set, head, slot) rows: B * G * heads * n = B * N * heads
+    // (sample*set, head, query slot) rows: B * G * heads * q_rows (all rows unless a prefix)
+    const long long qrows = kPk ? rows : rows / p.n * p.q_rows;
     const long long fblocks = std::min<long long>((qrows * (D / 8) + 255) / 256, (long long)device_sm_count() * 16);
     if (fblocks > 0)
       attn_bwd_dq_finalize_kernel<D, kPk><<<(unsigned)fblocks, 256, 0, stream>>>(p, qrows, seg);
     return check_launch("attn_bwd_dq_finalize_kernel");
   }
-  attn_bwd_dq_kernel<D, kPk><<<(unsigned)ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p, seg);
+  const long long dq_ctas = kPk ? ctas : ctas / p.n_tiles * p.q_tiles;   // query tiles
+  attn_bwd_dq_kernel<D, kPk><<<(unsigned)dq_ctas, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p, seg);
   return check_launch("attn_bwd_dq_kernel");
 }
 
@@ -921,7 +957,7 @@ int launch_bwd_d(const void* o, const void* dout, const CUtensorMap& tq, const C
 int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
                               int sparse_k, float scale, cudaStream_t stream, bool frame_causal,
-                              int causal_block) {
+                              int causal_block, int q_limit, bool dkdv_f32) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   const int N = s.text_len + s.T * s.H * s.W;
@@ -935,13 +971,21 @@ int attention_backward_launch(const void* q, const void* k, const void* v, const
   p.k = (layout == 0) ? 1 : sparse_k;
   p.layout = layout;
   p.n_tiles = (n + kBT - 1) / kBT;
-  p.vec_stride = p.n_tiles * kBT;
+  // queries: all n rows of each set, or (dense layout) its first q_limit rows
+  p.q_rows = (layout == 0 && q_limit >= 0 && q_limit < n) ? q_limit : n;
+  p.q_tiles = (p.q_rows + kBT - 1) / kBT;
+  p.vec_stride = p.q_tiles * kBT;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;
   p.lse = lse;
   p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  if (dkdv_f32) {
+    p.dk32 = static_cast<float*>(dk);
+    p.dv32 = static_cast<float*>(dv);
+  } else {
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+  }
   p.status = status;
   p.timeout_ns = wait_timeout_ns();
   p.elems = (unsigned long long)s.B * N * s.heads * s.head_dim / bounds_check_divisor();
@@ -1029,6 +1073,8 @@ int packed_backward_launch(const void* q, const void* k, const void* v, const vo
   p.layout = 0;
   p.n = N;                                // unused per CTA (each sample's own rows); for the host checks
   p.n_tiles = (int)tiles;
+  p.q_rows = N;
+  p.q_tiles = (int)tiles;
   p.vec_stride = (int)vrows;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.scale = scale;

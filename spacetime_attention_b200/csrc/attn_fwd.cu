@@ -266,7 +266,7 @@ int cross_attention_launch(const void* q, const void* k, const void* v, void* o,
 }
 
 int skiparse_text_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
-                                   int sparse_k, int mode, float scale, cudaStream_t stream) {
+                                   int sparse_k, int mode, float scale, cudaStream_t stream, float* lse) {
   unsigned* status = device_status_word();
   if (!status) return OSP_ERR_CUDA;
   const int L = s.text_len, Nv = s.T * s.H * s.W, N = L + Nv;
@@ -283,6 +283,9 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
     p.text_len = L;
     p.q_row_base = L;
     p.o_elems = (unsigned long long)s.B * N * s.heads * s.head_dim;
+    p.lse = lse;
+    p.lse_stride = (n + kBM - 1) / kBM * kBM;
+    p.lse_elems = lse ? (unsigned long long)s.B * sparse_k * s.heads * p.lse_stride : 0;
     CUtensorMap tq, tk, tv;
     TextMaps tm{};
     const char* qv = static_cast<const char*>(q) + L * row;
@@ -309,6 +312,12 @@ int skiparse_text_attention_launch(const void* q, const void* k, const void* v, 
   p.n_kv = N;
   p.N_q = N;
   p.o_elems = (unsigned long long)s.B * N * s.heads * s.head_dim;
+  if (lse) {   // after the video rows' block
+    const long long n_pad = (Nv / sparse_k + kBM - 1) / kBM * kBM;
+    p.lse = lse + (size_t)s.B * sparse_k * s.heads * n_pad;
+    p.lse_stride = (L + kBM - 1) / kBM * kBM;
+    p.lse_elems = (unsigned long long)s.B * s.heads * p.lse_stride;
+  }
   CUtensorMap tq, tk, tv;
   if ((rc = make_tmap(&tq, q, s, L, 0, 1, N)) != OSP_OK) return rc;
   if ((rc = make_tmap(&tk, k, s, N, 0, 1)) != OSP_OK) return rc;

@@ -302,7 +302,7 @@ static int check_train(const osp_shape* shape, int32_t sparse_k, int32_t mode, i
     *layout = 0;
     return OSP_OK;
   }
-  if ((rc = check_skiparse(shape, sparse_k, mode, false))) return rc;
+  if ((rc = check_skiparse(shape, sparse_k, mode, true))) return rc;
   if (mode == OSP_SKIP_GROUP && (sparse_k > 128 || (128 % sparse_k) != 0))
     return set_error(OSP_ERR_UNSUPPORTED, "fused Group Skip needs k to divide 128 (got k=%d)", sparse_k);
   *layout = mode + 1;
@@ -319,6 +319,9 @@ int osp_attn_forward_train(const void* q, const void* k, const void* v, void* o,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  if (shape->text_len > 0 && layout != 0)
+    return skiparse_text_attention_launch(q, k, v, o, *shape, sparse_k, mode, softmax_scale,
+                                          static_cast<cudaStream_t>(stream), lse);
   return attention_forward_lse_launch(q, k, v, o, lse, *shape, layout, sparse_k, softmax_scale,
                                       static_cast<cudaStream_t>(stream));
 }
@@ -335,6 +338,9 @@ int osp_attn_backward(const void* q, const void* k, const void* v, const void* o
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return set_error(OSP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (!(softmax_scale > 0.f)) softmax_scale = 1.0f / std::sqrt((float)shape->head_dim);
+  if (shape->text_len > 0 && layout != 0)
+    return skiparse_text_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, sparse_k, mode, softmax_scale,
+                                         static_cast<cudaStream_t>(stream));
   return attention_backward_launch(q, k, v, o, dout, lse, dq, dk, dv, *shape, layout, sparse_k, softmax_scale,
                                    static_cast<cudaStream_t>(stream));
 }

@@ -79,8 +79,16 @@ int cross_attention_launch(const void* q, const void* k, const void* v, void* o,
 
 // Skiparse with a joined text prefix (text_len > 0, k > 1): video queries of set g attend to the
 // text rows and set g; text queries attend to every row.  Two launches of the attention kernel.
+// lse (training forward, may be null): the video queries' rows in set-slot order,
+// [B*G][heads][ceil(n/128)*128] (n = T*H*W / G), followed by the text queries' rows,
+// [B][heads][ceil(text_len/128)*128].
 int skiparse_text_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
-                                   int sparse_k, int mode, float scale, cudaStream_t stream);
+                                   int sparse_k, int mode, float scale, cudaStream_t stream, float* lse = nullptr);
+// Backward of the above from its o and lse: a per-set pass over [set rows; text rows] samples
+// (video queries) and a pass of the text queries over all tokens, summed in fp32.
+int skiparse_text_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                  const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int sparse_k,
+                                  int mode, float scale, cudaStream_t stream);
 
 // Frame-causal attention (dense layout): token r attends to the text block and the frames up to its own.
 int frame_causal_attention_launch(const void* q, const void* k, const void* v, void* o, const osp_shape& s,
@@ -114,10 +122,13 @@ int attention_forward_lse_launch(const void* q, const void* k, const void* v, vo
                                  bool frame_causal = false, int causal_block = 0);
 
 // Backward pass of attention_forward_lse_launch: dq, dk, dv from q, k, v, o, dout and lse.
+// q_limit >= 0 (dense layout): only the first q_limit rows of each sample are queries (their
+// lse in rows of ceil(q_limit / 128) * 128); dq is written for those rows only, dk and dv carry
+// their contributions.  dkdv_f32: dk and dv are fp32 arrays, written unrounded.
 int attention_backward_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                               const float* lse, void* dq, void* dk, void* dv, const osp_shape& s, int layout,
                               int sparse_k, float scale, cudaStream_t stream, bool frame_causal = false,
-                              int causal_block = 0);
+                              int causal_block = 0, int q_limit = -1, bool dkdv_f32 = false);
 
 // Packed batch (block-diagonal attention): segment i owns q/o rows [q_bounds[i], q_bounds[i+1])
 // and k/v rows [kv_bounds[i], kv_bounds[i+1]); host arrays of n_seg + 1 validated offsets.

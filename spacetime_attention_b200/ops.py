@@ -249,9 +249,14 @@ def attn_frame_causal(q, k, v, grid, text_len: int, scale: float = 0.0, o=None) 
     return _attn3("osp_attn_frame_causal", q, k, v, grid, text_len, scale, o)
 
 
-def lse_shape(q: torch.Tensor, sparse_k: int = 1):
-    """Shape of the lse buffer of osp_attn_forward_train: [B*G, heads, ceil(n/128)*128]."""
+def lse_shape(q: torch.Tensor, sparse_k: int = 1, text_len: int = 0):
+    """Shape of the lse buffer of osp_attn_forward_train: [B*G, heads, ceil(n/128)*128]; with a
+    joined text prefix (Skiparse, text_len > 0) one flat run: the video rows' block, then the
+    text rows' [B, heads, ceil(text_len/128)*128]."""
     B, N, heads, _ = q.shape
+    if sparse_k > 1 and text_len > 0:
+        n = (N - text_len) // sparse_k
+        return (B * sparse_k * heads * ((n + 127) // 128 * 128) + B * heads * ((text_len + 127) // 128 * 128),)
     G = 1 if sparse_k == 1 else sparse_k
     n = N // G
     return (B * G, heads, (n + 127) // 128 * 128)
@@ -274,7 +279,7 @@ def attn_forward_train(q, k, v, grid, text_len: int = 0, sparse_k: int = 1, mode
     _bshd(q, "q"); _same(k, q, "k"); _same(v, q, "v")
     shp = _shape_of(q, grid, text_len)
     o = _out(o, q, "o")
-    lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
+    lse = _lse_buffer(lse, lse_shape(q, sparse_k, text_len), q)
     _check("osp_attn_forward_train",
            library().osp_attn_forward_train(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), ctypes.byref(shp),
                                             int(sparse_k), int(mode), ctypes.c_float(scale), _stream_handle(q)))
@@ -288,7 +293,7 @@ def attn_backward(q, k, v, o, dout, lse, grid, text_len: int = 0, sparse_k: int 
     for t, n in ((k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _same(t, q, n)
     dq, dk, dv = _out(dq, q, "dq"), _out(dk, q, "dk"), _out(dv, q, "dv")
-    lse = _lse_buffer(lse, lse_shape(q, sparse_k), q)
+    lse = _lse_buffer(lse, lse_shape(q, sparse_k, text_len), q)
     shp = _shape_of(q, grid, text_len)
     _check("osp_attn_backward",
            library().osp_attn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),

@@ -30,6 +30,11 @@ def calls(dev):
         o, lse = ops.attn_packed_train(q, k, v, [0, 100, 256])
         return ops.attn_packed_backward(q, k, v, o, do, lse, [0, 100, 256])
 
+    def skiparse_text_training():   # 64 text rows joined to Group Skip k = 2 sets of 96: forward, backward
+        g = (4, 8, 6)
+        o, lse = ops.attn_forward_train(q, k, v, g, 64, sparse_k=2, mode=1)
+        return ops.attn_backward(q, k, v, o, do, lse, g, 64, sparse_k=2, mode=1)
+
     def temporal_training():   # the per-set temporal kernels (T <= 64): forward with lse, backward
         o, lse = ops.attn_temporal_train(q, k, v, w.grid, causal=True)
         return ops.attn_temporal_backward(q, k, v, o, do, lse, w.grid, causal=True)
@@ -48,6 +53,7 @@ def calls(dev):
         "backward": backward,
         "temporal_training": temporal_training,
         "packed_training": packed_training,
+        "skiparse_text_training": skiparse_text_training,
     }
 
 

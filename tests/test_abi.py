@@ -144,7 +144,7 @@ def test_training_validation(lib):
     p, bad = ctypes.c_void_p(256), ctypes.c_void_p(264)
     assert lib.osp_attn_forward_train(p, p, p, p, None, shp(), 1, 0, 0.0, None) == 1          # no lse
     assert lib.osp_attn_forward_train(p, p, p, p, bad, shp(), 1, 0, 0.0, None) == 1           # misaligned lse
-    assert lib.osp_attn_forward_train(p, p, p, p, p, shp(L=3), 2, 0, 0.0, None) == 2          # Skiparse + text
+    assert lib.osp_attn_forward_train(p, p, p, p, p, shp(L=3), 3, 0, 0.0, None) == 3          # Skiparse + text, 256 % 3
     assert lib.osp_attn_forward_train(p, p, p, p, p, shp(), 3, 0, 0.0, None) == 3             # 256 % 3
     assert lib.osp_attn_backward(p, p, p, p, p, p, p, p, None, shp(), 1, 0, 0.0, None) == 1   # no dv
     assert lib.osp_attn_backward(p, p, p, p, p, p, p, p, p, shp(d=80), 1, 0, 0.0, None) == 2

@@ -152,3 +152,50 @@ def test_frame_causal_backward_matches_oracle(gpu, case):
     assert_grad_close(dq, rq, "dq")
     assert_grad_close(dk, rk, "dk")
     assert_grad_close(dv, rv, "dv")
+
+
+SKIP_TEXT = [
+    # B, heads, d, grid, k, text_len
+    (1, 2, 64, (4, 8, 8), 2, 5),         # sets of 128 plus 5 text rows: the text opens a second key tile
+    (2, 1, 64, (2, 16, 16), 4, 140),     # text over a tile boundary; B = 2
+    (1, 2, 96, (4, 10, 15), 2, 17),      # sets of 300: ragged tiles
+    (1, 1, 128, (4, 16, 18), 4, 33),
+]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("case", SKIP_TEXT, ids=[f"{c[3]}_k{c[4]}_L{c[5]}_d{c[2]}" for c in SKIP_TEXT])
+def test_skiparse_text_backward_matches_oracle(gpu, case, mode):
+    """Skiparse with a joined text prefix: text queries see every token, a video query of set g
+    sees the text and set g.  Training forward = inference forward bit for bit; lse of the video
+    rows (set-slot order) and of the text rows against the oracle; gradients against the chain
+    rule on the masked score matrix."""
+    B, heads, d, grid, kk, L = case
+    q, k, v, do = _inputs(B, heads, d, grid, L, 94)
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    o, lse = ops.attn_forward_train(qg, kg, vg, grid, L, sparse_k=kk, mode=mode)
+    dq, dk, dv = ops.attn_backward(qg, kg, vg, o, dog, lse, grid, L, sparse_k=kk, mode=mode)
+    ops.check_status()
+    assert torch.equal(o, ops.skiparse_attn(qg, kg, vg, grid, kk, mode, text_len=L))
+    rq, rk, rv = O.skiparse_text_backward_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), L, kk, mode)
+    assert_grad_close(dq, rq, f"dq mode {mode}")
+    assert_grad_close(dk, rk, f"dk mode {mode}")
+    assert_grad_close(dv, rv, f"dv mode {mode}")
+    # lse: video rows [B*k][heads][n_pad] in set-slot order, then text rows [B][heads][L_pad]
+    nv = grid[0] * grid[1] * grid[2]
+    n = nv // kk
+    n_pad, l_pad = (n + 127) // 128 * 128, (L + 127) // 128 * 128
+    lv = lse[: B * kk * heads * n_pad].view(B * kk, heads, n_pad).double().cpu().numpy()
+    lt = lse[B * kk * heads * n_pad:].view(B, heads, l_pad).double().cpu().numpy()
+    scale = 1 / math.sqrt(d)
+    qd, kd = to_f64(q), to_f64(k)
+    sets = O.skiparse_sets(nv, kk, mode)
+    for b in range(B):
+        for h in range(heads):
+            ref = O.attention_head_lse_ref(qd[b, :L, h], kd[b, :, h], scale) / math.log(2.0)
+            np.testing.assert_allclose(lt[b, h, :L], ref, rtol=0, atol=2e-3)
+            for g, st in enumerate(sets):
+                rows = L + np.asarray(st)
+                keys = np.concatenate([np.arange(L), rows])
+                ref = O.attention_head_lse_ref(qd[b, rows, h], kd[b, keys, h], scale) / math.log(2.0)
+                np.testing.assert_allclose(lv[b * kk + g, h, :n], ref, rtol=0, atol=2e-3)
