@@ -528,14 +528,25 @@ def run_backward_op(args, rank, world, local_rank):
     dQ, dK)."""
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = syn.WORKLOADS[args.workload]
-    q, k, v = (t.to(dev) for t in syn.make_qkv(w, w.seed + 17 * rank))
-    do = syn.randn_bf16(tuple(q.shape), w.seed + 99 + 17 * rank).to(dev)
     attn = ATTN_MODE["value"]
+    if attn == "packed":
+        return run_packed_backward_op(args, rank, world, dev)
+    w = syn.WORKLOADS[args.workload]
+    if attn == "skiparse_text":
+        if not sparse(w):
+            raise SystemExit("--attn skiparse_text needs a Skiparse workload")
+        shape = (w.B, args.text_len + w.n_video, w.heads, w.head_dim)
+        q, k, v, do = (syn.randn_bf16(shape, w.seed + 17 * rank + i).to(dev) for i in range(4))
+    else:
+        q, k, v = (t.to(dev) for t in syn.make_qkv(w, w.seed + 17 * rank))
+        do = syn.randn_bf16(tuple(q.shape), w.seed + 99 + 17 * rank).to(dev)
     causal = attn == "frame_causal"
     factor = attn in ("spatial", "temporal", "temporal_causal")
     modes = [(w.skiparse_k, ops.OSP_SKIP_SINGLE), (w.skiparse_k, ops.OSP_SKIP_GROUP)] if sparse(w) else [(1, 0)]
     L = 0 if sparse(w) else w.text_len
+    text = attn == "skiparse_text"
+    if text:
+        L = args.text_len
     if factor:   # the factorized attention runs over the video tokens only
         q, k, v, do = (t[:, L:].contiguous() for t in (q, k, v, do))
         L = 0
@@ -588,6 +599,9 @@ def run_backward_op(args, rank, world, local_rank):
         pairs = w.B * T * HW * HW
     elif factor:
         pairs = w.B * HW * (T * (T + 1) // 2 if t_causal else T * T)
+    elif text:   # both modes: video queries see text + their set, text queries see everything
+        n_set, N = w.n_video // w.skiparse_k, L + w.n_video
+        pairs = 2 * w.B * (w.n_video * (L + n_set) + L * N)
     else:
         pairs = None
     flops = 2.5 * 4.0 * w.heads * w.head_dim * pairs if pairs is not None else 2.5 * step_flops(w)
@@ -599,16 +613,68 @@ def run_backward_op(args, rank, world, local_rank):
     per_set = attn in ("temporal", "temporal_causal") and T <= 64 and os.environ.get("OSP_TEMPORAL_BWD", "1") != "0"
     roof.update(traffic=None, bytes_per_step=nbytes,
                 kernel="attn_temporal_bwd_kernel" if per_set
-                else "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel")
+                else "attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel"
+                + (" (video and text query passes) + text_bwd_gather/combine" if text else ""))
     label = {"frame_causal": "frame-causal", "spatial": "spatial (per frame)", "temporal": "temporal (per position)",
-             "temporal_causal": "causal temporal (per position)"}.get(attn, "skiparse pair" if sparse(w) else "dense")
+             "temporal_causal": "causal temporal (per position)",
+             "skiparse_text": f"skiparse pair + {L} joined text tokens (unmasked pairs)"}.get(
+                 attn, "skiparse pair" if sparse(w) else "dense")
+    # launches per backward call: row sums, dK/dV, dQ (or its finalize); the joined-text form runs
+    # that for both query passes plus the gather and the combine
+    per_call = 1 if per_set else (8 if text else 3)
     return {"metric": "attention backward TFLOP/s (2.5x forward flops)", "value": round(world * tflops, 1),
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": dict(w.describe(), op="backward", attn=label, flops_per_step=flops,
                            l2="inputs > L2, no flush"),
-            "roofline": roof, "clocks": clocks, "gpu_launches": (1 if per_set else 3) * len(modes) * args.steps}
+            "roofline": roof, "clocks": clocks, "gpu_launches": per_call * len(modes) * args.steps}
+
+
+def run_packed_backward_op(args, rank, world, dev):
+    """Time the packed-batch backward (osp_attn_packed_backward: each sample's own chain rule on
+    the tcgen05 kernels through the segment table) after osp_attn_packed_train.  value = 2.5x
+    the block-diagonal forward flops / backward time."""
+    w = syn.PACKED_WORKLOADS[args.packed]
+    q, k, v = (t.to(dev) for t in syn.make_packed_qkv(w.heads, w.head_dim, w.total, w.seed + 17 * rank))
+    do = syn.randn_bf16(tuple(q.shape), w.seed + 99 + 17 * rank).to(dev)
+    o, lse = ops.attn_packed_train(q, k, v, w.bounds)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+
+    def step():
+        ops.attn_packed_backward(q, k, v, o, do, lse, w.bounds, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ops.check_status(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world, dev)
+    peaks, src = load_peaks()
+    flops = 2.5 * w.flops()
+    rows = w.total * w.heads
+    nbytes = 8 * 2 * rows * w.head_dim + 4 * rows
+    roof, tflops, _ = tensor_or_hbm_roofline(flops, nbytes, ms, peaks, src, clocks, ms * args.steps * 1e-3)
+    roof.update(traffic=None, bytes_per_step=nbytes,
+                kernel="attn_bwd_dkdv_kernel + attn_bwd_dq_kernel + attn_bwd_dvec_kernel (segment table)")
+    return {"metric": "packed-batch attention backward TFLOP/s (2.5x forward flops)", "value": round(world * tflops, 1),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(w.describe(), op="backward", attn="packed", flops_per_step=flops,
+                           l2="inputs > L2, no flush"),
+            "roofline": roof, "clocks": clocks, "gpu_launches": 3 * args.steps}
 
 
 # Every configuration of the measured workloads, each timed as its own step in the default run:
@@ -947,9 +1013,12 @@ def main():
     ap.add_argument("--workload", default="long_video", choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--attn", default="auto",
-                    choices=["auto", "dense", "skiparse", "frame_causal", "spatial", "temporal", "temporal_causal"],
+                    choices=["auto", "dense", "skiparse", "frame_causal", "spatial", "temporal", "temporal_causal",
+                             "skiparse_text", "packed"],
                     help="Skiparse workloads: time the Single+Group pair (auto/skiparse) or dense attention; "
-                         "frame_causal / spatial / temporal / temporal_causal: that backward (--op backward)")
+                         "frame_causal / spatial / temporal / temporal_causal / skiparse_text (the pair with "
+                         "--text-len text tokens joined) / packed (the --packed batch): that backward "
+                         "(--op backward)")
     ap.add_argument("--op", default="step",
                     choices=["step", "rope", "gather", "scatter", "cross", "packed", "spatial", "temporal",
                              "temporal_train", "frame_causal", "skiparse_text", "backward"],
@@ -965,7 +1034,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.attn in ("frame_causal", "spatial", "temporal", "temporal_causal") and args.op != "backward":
+    if args.attn in ("frame_causal", "spatial", "temporal", "temporal_causal", "skiparse_text",
+                     "packed") and args.op != "backward":
         ap.error(f"--attn {args.attn} applies to --op backward (use --op {args.attn.split('_')[0]} for the forward)")
     ATTN_MODE["value"] = args.attn
 
