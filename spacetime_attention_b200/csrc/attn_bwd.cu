@@ -39,6 +39,18 @@ constexpr int kProdWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kAccWarp = 10;
 constexpr int kRedWarp = 11;             // fused dQ: issues the bulk reduce-adds of dQ
+// dK/dV kernel: four compute warps per SM sub-partition, each turning 16 of a sub-tile's 64
+// query columns into P and dS (OSP_BWD_WIDE=0: two per sub-partition, 32 columns each).  More
+// warps per sub-partition keep its MUFU and issue slots busy while each warp waits on tensor
+// memory or on a barrier; a warp's chain (load, exponentials, pack, store) is half as long.
+#ifndef OSP_BWD_WIDE
+#define OSP_BWD_WIDE 1
+#endif
+constexpr int kDkCols = OSP_BWD_WIDE ? 16 : 32;          // query columns per compute warp and sub-tile
+constexpr int kDkComputeWarps = 4 * (64 / kDkCols);      // 16 or 8
+constexpr int kDkComputeThreads = 32 * kDkComputeWarps;
+constexpr int kDkProdWarp = kDkComputeWarps, kDkMmaWarp = kDkComputeWarps + 1, kDkAccWarp = kDkComputeWarps + 2,
+              kDkRedWarp = kDkComputeWarps + 3;
 #ifndef OSP_BWD_FUSE_DQ
 #define OSP_BWD_FUSE_DQ 1                // d = 64: dQ accumulated by the dK/dV kernel (no dQ kernel)
 #endif
@@ -65,7 +77,8 @@ struct BwdCfg {
   // shared memory by the compute warps, and adds it into an fp32 accumulator with one bulk
   // reduce-add per tile; the dQ kernel (which recomputes S, dP and P) is not launched.
   static constexpr bool kFuseDq = (D == 64) && OSP_BWD_FUSE_DQ;
-  static constexpr int kThreads = kFuseDq ? kBwdThreads + 32 : kBwdThreads;
+  // dK/dV kernel: compute warps, producer, two MMA issuers and (fused dQ) the reduce warp
+  static constexpr int kThreads = 32 * (kDkComputeWarps + (kFuseDq ? 4 : 3));
   static constexpr int kResOff = 0;                                 // two resident tiles
   static constexpr int kStageOff = 2 * kTileBytes;                  // stages of two tiles each
   static constexpr int kVecOff = kStageOff + kStages * 2 * kTileBytes;
@@ -203,6 +216,22 @@ __device__ __forceinline__ void bwd_load_tile(const CUtensorMap* tm, uint32_t ds
 // own consumed S / dP columns, so the two warps sharing a lane quarter never touch each other's
 // unread columns.  The tensor-memory A operand of K-step kk (16 rows of P / dS) starts at:
 __device__ __forceinline__ uint32_t packed_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
+// 32-lane x N-column tensor-memory loads (N = 16 or 32) and stores of N packed columns (8, 16)
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 16) tmem_ld16(taddr, r);
+  else tmem_ld32(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 8) tmem_st8(taddr, r);
+  else tmem_st16(taddr, r);
+}
+// The same for the dK/dV kernel's compute warps of kDkCols columns: K-step kk (queries 16kk ..
+// 16kk + 15) lies in warp column group 16kk / kDkCols, which packs its columns from its first.
+__device__ __forceinline__ uint32_t packed_col_dk(int kk) {
+  return (uint32_t)(kDkCols * ((16 * kk) / kDkCols) + ((16 * kk) % kDkCols) / 2);
+}
 
 __device__ __forceinline__ bool bwd_warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   const bool ok = mbar_wait(bar, parity, w);
@@ -266,43 +295,58 @@ __global__ void __launch_bounds__(256) attn_bwd_dvec_kernel(const __nv_bfloat16*
 // P and dS of one 32-column chunk for one TMEM lane (the thread's row).
 //   s, dp: raw scores / dP of the chunk; lse, dv: per-column (kCols) or per-row values.
 //   valid: columns [0, valid) of the chunk are real; vis: bit e clear masks column e out.
-template <bool kPerColumn>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
-                                          const float* lse_col, const float* dv_col, float lse_row, float dv_row,
-                                          int valid, uint32_t (&pk)[16], uint32_t (&dk)[16],
-                                          uint32_t vis = 0xffffffffu) {
-  if (valid >= 32 && vis == 0xffffffffu) {   // every column real and visible: no per-element mask
+// Per-column lse / Dv are read four columns at a time (16-byte shared loads, 16-byte aligned
+// pointers): every lane reads the same columns, and one broadcast load per four columns instead
+// of one per column keeps the shared-memory pipe, which the tensor core's operand reads also
+// use, free.
+template <bool kPerColumn, bool kMask, int kN>
+__device__ __forceinline__ void bwd_chunk_body(const uint32_t (&s)[kN], const uint32_t (&dp)[kN], float sl2,
+                                               const float* lse_col, const float* dv_col, float lse_row,
+                                               float dv_row, int valid, uint32_t (&pk)[kN / 2],
+                                               uint32_t (&dk)[kN / 2], uint32_t vis) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      float pv[2], dsv[2];
+  for (int e = 0; e < kN; e += 4) {
+    float l[4], dd[4];
+    if constexpr (kPerColumn) {
+      const float4 l4 = reinterpret_cast<const float4*>(lse_col)[e >> 2];
+      const float4 d4 = reinterpret_cast<const float4*>(dv_col)[e >> 2];
+      l[0] = l4.x; l[1] = l4.y; l[2] = l4.z; l[3] = l4.w;
+      dd[0] = d4.x; dd[1] = d4.y; dd[2] = d4.z; dd[3] = d4.w;
+    } else {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const float l = kPerColumn ? lse_col[e + u] : lse_row;
-        const float dd = kPerColumn ? dv_col[e + u] : dv_row;
-        pv[u] = ex2_approx(fmaf(__uint_as_float(s[e + u]), sl2, -l));
-        dsv[u] = pv[u] * (__uint_as_float(dp[e + u]) - dd);
+      for (int u = 0; u < 4; ++u) {
+        l[u] = lse_row;
+        dd[u] = dv_row;
       }
-      pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-      dk[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
     }
-    return;
-  }
+    float pv[4], dsv[4];
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
-    float pv[2], dsv[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const float l = kPerColumn ? lse_col[e + u] : lse_row;
-      const float dd = kPerColumn ? dv_col[e + u] : dv_row;
-      const float pe = ex2_approx(fmaf(__uint_as_float(s[e + u]), sl2, -l));
-      const float de = pe * (__uint_as_float(dp[e + u]) - dd);
-      const bool ok = e + u < valid && ((vis >> (e + u)) & 1u);
-      pv[u] = ok ? pe : 0.f;
-      dsv[u] = ok ? de : 0.f;
+    for (int u = 0; u < 4; ++u) {
+      pv[u] = ex2_approx(fmaf(__uint_as_float(s[e + u]), sl2, -l[u]));
+      dsv[u] = pv[u] * (__uint_as_float(dp[e + u]) - dd[u]);
+      if constexpr (kMask) {
+        const bool ok = e + u < valid && ((vis >> (e + u)) & 1u);
+        pv[u] = ok ? pv[u] : 0.f;
+        dsv[u] = ok ? dsv[u] : 0.f;
+      }
     }
     pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+    pk[(e >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
     dk[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+    dk[(e >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
   }
+}
+
+template <bool kPerColumn, int kN>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[kN], const uint32_t (&dp)[kN], float sl2,
+                                          const float* lse_col, const float* dv_col, float lse_row, float dv_row,
+                                          int valid, uint32_t (&pk)[kN / 2], uint32_t (&dk)[kN / 2],
+                                          uint32_t vis = 0xffffffffu) {
+  constexpr uint32_t kAll = kN >= 32 ? 0xffffffffu : ((1u << kN) - 1u);
+  if (valid >= kN && (vis & kAll) == kAll)   // every column real and visible: no per-element mask
+    bwd_chunk_body<kPerColumn, false, kN>(s, dp, sl2, lse_col, dv_col, lse_row, dv_row, valid, pk, dk, vis);
+  else
+    bwd_chunk_body<kPerColumn, true, kN>(s, dp, sl2, lse_col, dv_col, lse_row, dv_row, valid, pk, dk, vis);
 }
 
 // Writes one 128-row tile's fp32 accumulator row (TMEM columns [col, col + D)) as bf16, scaled.
@@ -329,9 +373,11 @@ __device__ __forceinline__ void bwd_store_row(uint32_t taddr, float scale, __nv_
 
 // fp32 variant: the row's D accumulator columns times scale, unrounded
 template <int D>
-__device__ __forceinline__ void bwd_store_row_f32(uint32_t taddr, float scale, float* dst, bool live) {
+__device__ __forceinline__ void bwd_store_row_f32(uint32_t taddr, float scale, float* dst, bool live,
+                                                  int part = -1) {
 #pragma unroll
   for (int cc = 0; cc < D / 32; ++cc) {
+    if (part >= 0 && (cc & 1) != part) continue;
     uint32_t r[32];
     tmem_ld32(taddr + 32 * cc, r);
     tmem_wait_ld();
@@ -392,7 +438,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(B_SFULL + u), 1);
-      mbar_init(bar(B_PREADY + u), kComputeThreads);
+      mbar_init(bar(B_PREADY + u), kDkComputeThreads);
     }
     mbar_init(bar(B_DONE), 1);
     mbar_init(bar(B_FIN), 1);
@@ -403,21 +449,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int u = 0; u < 2; ++u) {
         mbar_init(bar(B_DSFREE + u), 1);
         mbar_init(bar(B_DQFULL + u), 1);
-        mbar_init(bar(B_DQTFREE + u), kComputeThreads);
+        mbar_init(bar(B_DQTFREE + u), kDkComputeThreads);
       }
-      mbar_init(bar(B_STGFULL), kComputeThreads);
+      mbar_init(bar(B_STGFULL), kDkComputeThreads);
       mbar_init(bar(B_STGFREE), 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kProdWarp && lane == 0) {
+  if (warp == kDkProdWarp && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
   }
-  if (warp == kMmaWarp) {
+  if (warp == kDkMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -432,7 +478,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   auto sStr = [&](int s, int i) { return sbase + C::kStageOff + (uint32_t)((2 * s + i) * C::kTileBytes); };  // Q, dO
   auto sVec = [&](int s) { return sbase + C::kVecOff + (uint32_t)(s * C::kVecBytes); };
 
-  if (warp == kProdWarp) {
+  if (warp == kDkProdWarp) {
     // ------------------------------------------------------------------ TMA producer
     const bool leader = elect_one_sync();
     int issued = 0;
@@ -468,7 +514,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t)
       mbar_drain(bar(B_FULL + t % kStages), (t / kStages) & 1, p.timeout_ns);
     __syncwarp();
-  } else if (warp == kMmaWarp || warp == kAccWarp) {
+  } else if (warp == kDkMmaWarp || warp == kDkAccWarp) {
     // ------------------------------------------------------------------ MMA issuers
     const bool leader = elect_one_sync();
     constexpr uint32_t idesc_ss = idesc_bf16_f32(kBT, kSub, false);  // M = 128 keys, N = 64 queries, K-major
@@ -493,7 +539,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     auto issue_ts = [&](uint32_t d_col, uint32_t a_col, uint64_t b0, bool acc) {
 #pragma unroll
       for (int kk = 0; kk < kSub / 16; ++kk)
-        if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + packed_col_dk(kk), b0 + (uint64_t)(128 * kk), idesc_ts,
                            (acc || kk > 0) ? 1u : 0u);
     };
     // Sub-tile t = 2i + hh is rows 64hh .. 64hh+63 of query tile i, in score buffer t & 1.
@@ -501,7 +547,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // readers of buffer t & 1) have completed; warp 10 issues dV / dK of sub-tile t once the
     // compute warps have written P^T / dS^T.
     const int n_sub = 2 * nq;
-    if (warp == kMmaWarp) {
+    if (warp == kDkMmaWarp) {
       bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
       for (int t = 0; ok && t < n_sub; ++t) {
         const int i = t >> 1, hh = t & 1, s = i % kStages;
@@ -550,7 +596,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       mbar_drain(bar(B_FIN2), 0, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp == kRedWarp) {
+  } else if (warp == kDkRedWarp) {
     // ------------------------------------------------------------------ fused dQ: bulk reduce-add
     // of each query tile's fp32 dQ (staged in shared memory by the compute warps) into the
     // accumulator rows of this (sample*set, head); the staging tile is released once read
@@ -571,12 +617,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ compute warps 0-7
-    const int quarter = warp & 3, half = warp >> 2;
+    constexpr int kN = kDkCols;                              // query columns of this warp per sub-tile
+    constexpr int kGroups = kSub / kN;                       // column groups of a lane quarter
+    const int quarter = warp & 3, cg = warp >> 2;            // lane quarter, column group
     const int row = quarter * 32 + lane;                    // key row = tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
     const int kstart = p.frame_hw ? causal_block_start(kv0 + row, p.text_len, p.frame_hw) : 0;   // its block's start
-    // fused dQ: reads this warp's 32 x 32 block (query rows of its lane quarter, columns 32 half)
+    // fused dQ: reads this warp's 32 x kN block (query rows of its lane quarter, columns kN cg ..)
     // of dQ of local tile ix out of tensor memory and writes it into the staging tile: row-major
     // fp32, with the eight 16-byte chunks of each 32-float half row permuted by XOR (row & 7) so
     // that a warp's stores spread over all banks.  The accumulator rows keep that permutation
@@ -586,16 +634,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const int b = ix & 1;
       if (!bwd_warp_wait(bar(B_DQFULL + b), (ix >> 1) & 1, wc)) return false;
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + col_dq(b) + 32u * half, r);
+      uint32_t r[kN];
+      tmem_ldn<kN>(tmem + lane_base + col_dq(b) + (uint32_t)(kN * cg), r);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(B_DQTFREE + b));
       if (ix >= 1 && !bwd_warp_wait(bar(B_STGFREE), (ix - 1) & 1, wc)) return false;
-      const uint32_t rowb = sStg + (uint32_t)(row * D * 4 + half * 128);
+      // this warp's floats kN cg .. kN cg + kN - 1: half row (kN cg) / 32, its chunks from (kN cg % 32) / 4
+      const uint32_t rowb = sStg + (uint32_t)(row * D * 4 + ((kN * cg) / 32) * 128);
+      const int c0 = ((kN * cg) % 32) / 4;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t pc = (uint32_t)(c ^ (row & 7));
+      for (int c = 0; c < kN / 4; ++c) {
+        const uint32_t pc = (uint32_t)((c0 + c) ^ (row & 7));
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowb + 16u * pc), "r"(r[4 * c]),
                      "r"(r[4 * c + 1]), "r"(r[4 * c + 2]), "r"(r[4 * c + 3])
                      : "memory");
@@ -609,30 +659,32 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       const float* vec = reinterpret_cast<const float*>(smem + C::kVecOff + (il % kStages) * C::kVecBytes) +
-                         kSub * hh + 32 * half;
-      const int qa = i * kBT + kSub * hh + 32 * half;   // this warp's first query column
+                         kSub * hh + kN * cg;
+      const int qa = i * kBT + kSub * hh + kN * cg;   // this warp's first query column
       // a key row past the set's end (zero-fill, or in a packed batch the next sample's keys) gets
       // no valid column: its P and dS are zero, so the fused dQ product sums real keys only
       const int valid_q = (kv0 + row < n_rows) ? q_rows - qa : 0;
       const uint32_t vis = p.frame_hw ? causal_columns(qa, kstart) : 0xffffffffu;
-      const uint32_t tS = tmem + lane_base + col_s(bb) + 32 * half, tP = tmem + lane_base + col_dp(bb) + 32 * half;
-      uint32_t s[32], dp[32];
-      tmem_ld32(tS, s);
-      tmem_ld32(tP, dp);
+      const uint32_t tS = tmem + lane_base + col_s(bb) + (uint32_t)(kN * cg);
+      const uint32_t tP = tmem + lane_base + col_dp(bb) + (uint32_t)(kN * cg);
+      uint32_t s[kN], dp[kN];
+      tmem_ldn<kN>(tS, s);
+      tmem_ldn<kN>(tP, dp);
       tmem_wait_ld();
-      uint32_t pk[16], dk[16];
-      bwd_chunk<true>(s, dp, p.scale_log2, vec, vec + kBT, 0.f, 0.f, valid_q, pk, dk, vis);
-      tmem_st16(tS, pk);    // P^T over this warp's consumed S^T columns
-      tmem_st16(tP, dk);    // dS^T over this warp's consumed dP^T columns
+      uint32_t pk[kN / 2], dk[kN / 2];
+      bwd_chunk<true, kN>(s, dp, p.scale_log2, vec, vec + kBT, 0.f, 0.f, valid_q, pk, dk, vis);
+      // P^T and dS^T over this warp's consumed S^T / dP^T columns (its first kN / 2)
+      tmem_stn<kN / 2>(tS, pk);
+      tmem_stn<kN / 2>(tP, dk);
       if constexpr (C::kFuseDq) {
-        // dS^T row (this key) for queries 64hh + 32half .. +31 into the dS buffer of tile il:
-        // SW128 chunk hh, 16-byte column c = 4 half + v XOR (row & 7), 8-row groups 1 KB apart
+        // dS^T row (this key) for queries 64hh + kN cg .. into the dS buffer of tile il: SW128
+        // chunk hh, 16-byte column c = (kN / 8) cg + v XOR (row & 7), 8-row groups 1 KB apart
         const int b = il & 1;
         if (hh == 0 && il >= 2 && !bwd_warp_wait(bar(B_DSFREE + b), ((il >> 1) - 1) & 1, wc)) { ok = false; break; }
         const uint32_t base = sDs(b) + (uint32_t)(hh * kChunkBytes) + (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint32_t c = (uint32_t)((4 * half + v) ^ (row & 7));
+        for (int v = 0; v < kN / 8; ++v) {
+          const uint32_t c = (uint32_t)(((kN / 8) * cg + v) ^ (row & 7));
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + 16u * c), "r"(dk[4 * v]),
                        "r"(dk[4 * v + 1]), "r"(dk[4 * v + 2]), "r"(dk[4 * v + 3])
                        : "memory");
@@ -656,19 +708,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const int token = rb + bwd_slot_token(p.layout, live ? j : 0, g, p.k);
       const size_t off = (((size_t)b * p.N + token) * p.heads + h) * D;
       const bool store = live && index_ok(off + D - 1, p.elems, p.status);
+      // the first half of a quarter's column groups writes dV, the second dK; with two groups
+      // per half they split the 32-column chunks by parity
+      const bool is_dk = cg >= kGroups / 2;
+      const int part = kGroups > 2 ? (cg & 1) : -1;
       if (p.dk32) {
-        if (half == 0) bwd_store_row_f32<D>(tmem + lane_base + kColAcc0, 1.f, p.dv32 + off, store);
-        else bwd_store_row_f32<D>(tmem + lane_base + kColAcc1, p.scale, p.dk32 + off, store);
-      } else if (half == 0) {
-        bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store);
+        if (!is_dk) bwd_store_row_f32<D>(tmem + lane_base + kColAcc0, 1.f, p.dv32 + off, store, part);
+        else bwd_store_row_f32<D>(tmem + lane_base + kColAcc1, p.scale, p.dk32 + off, store, part);
+      } else if (!is_dk) {
+        bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store, part);
       } else {
-        bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, store);
+        bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, store, part);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kDkMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
