@@ -77,6 +77,13 @@ struct BwdCfg {
   // shared memory by the compute warps, and adds it into an fp32 accumulator with one bulk
   // reduce-add per tile; the dQ kernel (which recomputes S, dP and P) is not launched.
   static constexpr bool kFuseDq = (D == 64) && OSP_BWD_FUSE_DQ;
+  // Fused dQ: K and V also sit in tensor memory (32 columns each, packed bf16 pairs of channels,
+  // key = lane), so the score products S^T = K Q^T and dP^T = V dO^T read only their B operand
+  // from shared memory.  Both operands from shared memory cost an M = 128, N = 64, K = 16 product
+  // about 60 cycles of shared-memory reads (6 KB at 128 B per cycle) against 32 of math; with A in
+  // tensor memory it is bound by its math.  The dQ buffer is then single (its second copy's
+  // columns hold K and V).
+  static constexpr bool kKvTmem = kFuseDq;
   // dK/dV kernel: compute warps, producer, two MMA issuers and (fused dQ) the reduce warp
   static constexpr int kThreads = 32 * (kDkComputeWarps + (kFuseDq ? 4 : 3));
   static constexpr int kResOff = 0;                                 // two resident tiles
@@ -416,8 +423,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // fused dQ tensor-memory buffers (64 columns each, next to dV at 256 and dK at 384)
-  auto col_dq = [](int b) { return b ? 448u : 320u; };
+  // fused dQ: its tensor-memory buffer (64 columns next to dV at 256), and K, V (32 columns each
+  // after dK at 384)
+  constexpr uint32_t kColDq = 320, kColK = 448, kColV = 480;
+  const int B_KVT = B_STGFREE + 1;   // K and V are in tensor memory
 
   const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, false);
   const int tile = un.tile, h = un.h, bg = un.bg, b = un.b, g = un.g;
@@ -446,11 +455,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     mbar_init(bar(B_BUFFREE + 1), 1);
     mbar_init(bar(B_FIN2), 1);
     if constexpr (C::kFuseDq) {
-      for (int u = 0; u < 2; ++u) {
-        mbar_init(bar(B_DSFREE + u), 1);
-        mbar_init(bar(B_DQFULL + u), 1);
-        mbar_init(bar(B_DQTFREE + u), kDkComputeThreads);
-      }
+      for (int u = 0; u < 2; ++u) mbar_init(bar(B_DSFREE + u), 1);
+      mbar_init(bar(B_DQFULL), 1);
+      mbar_init(bar(B_DQTFREE), kDkComputeThreads);
+      mbar_init(bar(B_KVT), kDkComputeThreads);
       mbar_init(bar(B_STGFULL), kDkComputeThreads);
       mbar_init(bar(B_STGFREE), 1);
     }
@@ -547,16 +555,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // readers of buffer t & 1) have completed; warp 10 issues dV / dK of sub-tile t once the
     // compute warps have written P^T / dS^T.
     const int n_sub = 2 * nq;
+    // D_t = A (tensor memory: K or V, packed channel pairs, 8 columns per 16 channels) times B
+    // K-major (64 query rows x D)^T
+    auto issue_ts_kv = [&](uint32_t d_col, uint32_t a_col, uint64_t b0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+    };
     if (warp == kDkMmaWarp) {
       bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      if constexpr (C::kKvTmem) ok = ok && bwd_warp_wait(bar(B_KVT), 0, wc);
       for (int t = 0; ok && t < n_sub; ++t) {
         const int i = t >> 1, hh = t & 1, s = i % kStages;
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
         if (t >= 2 && !bwd_warp_wait(bar(B_BUFFREE + (t & 1)), ((t - 2) >> 1) & 1, wc)) break;
         tc_fence_after();
         const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
-        issue_ss(col_s(t & 1), dK, dQk + sub);    // S^T = K Q_sub^T
-        issue_ss(col_dp(t & 1), dV, dOk + sub);   // dP^T = V dO_sub^T
+        if constexpr (C::kKvTmem) {
+          issue_ts_kv(col_s(t & 1), kColK, dQk + sub);    // S^T = K Q_sub^T
+          issue_ts_kv(col_dp(t & 1), kColV, dOk + sub);   // dP^T = V dO_sub^T
+        } else {
+          issue_ss(col_s(t & 1), dK, dQk + sub);
+          issue_ss(col_dp(t & 1), dV, dOk + sub);
+        }
         if (leader) tc_commit(bar(B_SFULL + (t & 1)));
       }
       if (leader) tc_commit(bar(B_FIN));
@@ -578,15 +601,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if constexpr (C::kFuseDq) {
           if (hh == 1) {
             const int b = i & 1;
-            // the tensor-memory buffer's previous tile (i - 2) has been read out
-            if (i >= 2 && !bwd_warp_wait(bar(B_DQTFREE + b), ((i >> 1) - 1) & 1, wc)) break;
+            // the tensor-memory buffer's previous tile (i - 1) has been read out
+            if (i >= 1 && !bwd_warp_wait(bar(B_DQTFREE), (i - 1) & 1, wc)) break;
             tc_fence_after();
             const uint64_t da = sdesc_sw128(sDs(b), kChunkBytes, 1024);
 #pragma unroll
             for (int kk = 0; kk < kBT / 16; ++kk)   // 16 keys (two 8-row groups, 2 KB) per step
-              if (leader) mma_ss(tmem + col_dq(b), da + (uint64_t)(128 * kk), dKres_mn + (uint64_t)(128 * kk),
+              if (leader) mma_ss(tmem + kColDq, da + (uint64_t)(128 * kk), dKres_mn + (uint64_t)(128 * kk),
                                  idesc_dq, kk > 0 ? 1u : 0u);
-            if (leader) tc_commit(bar(B_DQFULL + b));
+            if (leader) tc_commit(bar(B_DQFULL));
             if (leader) tc_commit(bar(B_DSFREE + b));
           }
         }
@@ -631,14 +654,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     // (it depends on the row alone, so every key tile's contribution lands on the same element);
     // the finalize kernel undoes it.
     auto drain_dq = [&](int ix) -> bool {
-      const int b = ix & 1;
-      if (!bwd_warp_wait(bar(B_DQFULL + b), (ix >> 1) & 1, wc)) return false;
+      if (!bwd_warp_wait(bar(B_DQFULL), ix & 1, wc)) return false;
       tc_fence_after();
       uint32_t r[kN];
-      tmem_ldn<kN>(tmem + lane_base + col_dq(b) + (uint32_t)(kN * cg), r);
+      tmem_ldn<kN>(tmem + lane_base + kColDq + (uint32_t)(kN * cg), r);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(B_DQTFREE + b));
+      mbar_arrive(bar(B_DQTFREE));
       if (ix >= 1 && !bwd_warp_wait(bar(B_STGFREE), (ix - 1) & 1, wc)) return false;
       // this warp's floats kN cg .. kN cg + kN - 1: half row (kN cg) / 32, its chunks from (kN cg % 32) / 4
       const uint32_t rowb = sStg + (uint32_t)(row * D * 4 + ((kN * cg) / 32) * 128);
@@ -654,7 +676,28 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       mbar_arrive(bar(B_STGFULL));
       return true;
     };
-    for (int t = 0; t < 2 * nq; ++t) {
+    if constexpr (C::kKvTmem) {
+      // K (column groups 0, 1) or V (2, 3): this row's channels 32 (cg & 1) .. + 31, i.e. its
+      // 16-byte SW128 chunks 4 (cg & 1) .. + 3, as packed pairs into tensor-memory columns
+      // 16 (cg & 1) .. + 15 of the K or V block
+      ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      if (ok) {
+        const uint32_t src = sRes(cg >> 1) + (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
+        uint32_t r[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint32_t c = (uint32_t)((4 * (cg & 1) + v) ^ (row & 7));
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(r[4 * v]), "=r"(r[4 * v + 1]), "=r"(r[4 * v + 2]), "=r"(r[4 * v + 3])
+                       : "r"(src + 16u * c));
+        }
+        tmem_st16(tmem + lane_base + ((cg >> 1) ? kColV : kColK) + 16u * (uint32_t)(cg & 1), r);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_KVT));
+      }
+    }
+    for (int t = 0; ok && t < 2 * nq; ++t) {
       const int il = t >> 1, i = i0 + il, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
