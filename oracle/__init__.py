@@ -34,6 +34,7 @@ from .spacetime_oracle import (  # noqa: F401
     skiparse_sets,
     skiparse_text_attn_ref,
     skiparse_text_backward_ref,
+    skiparse_text_backward_rows_ref,
     softmax_rows,
     spatial_attn_ref,
     spatial_backward_ref,

@@ -733,3 +733,63 @@ def skiparse_text_backward_ref(q, k, v, do, text_len: int, k_ratio: int, mode: i
             out[1][b, :, h] = ds.T @ qh * scale
             out[2][b, :, h] = p.T @ dh
     return tuple(out)
+
+
+def skiparse_text_backward_rows_ref(q, k, v, do, text_len: int, k_ratio: int, mode: int, q_rows, k_rows,
+                                    heads=None, scale: float | None = None, chunk: int = 2048):
+    """Selected rows of the gradients of skiparse_text_attn_ref (text_len = 0: of
+    skiparse_attn_ref), without forming the N x N score matrix: dq for tokens ``q_rows``, dk and
+    dv for tokens ``k_rows``, for heads ``heads`` (all by default); each [B, rows, heads, d].
+    The same chain rule as skiparse_text_backward_ref on the masked score matrix: row r of a text
+    token sees every token, row r of a video token of set g the text tokens and set g.  The
+    row log-sum-exp and rowsum(dO * O) of every query come first, per group of rows that see the
+    same keys (the text rows; each set's rows), in chunks of ``chunk`` rows."""
+    B, N, nh, d = q.shape
+    L = int(text_len)
+    scale = default_scale(d) if scale is None else scale
+    sets = [L + np.asarray(st, dtype=np.int64) for st in skiparse_sets(N - L, k_ratio, mode)]
+    text = np.arange(L)
+    set_of = np.empty(N, dtype=np.int64)
+    set_of[:L] = -1
+    for g, st in enumerate(sets):
+        set_of[st] = g
+    # (rows, their keys) per group of rows that see the same keys
+    groups = ([(text, np.arange(N))] if L else []) + [(st, np.concatenate([text, st])) for st in sets]
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    qr, kr = np.asarray(q_rows, dtype=np.int64), np.asarray(k_rows, dtype=np.int64)
+    # only the groups whose rows are read: the text rows (they see every key), the sets of the
+    # selected video rows and keys, and every set if a text key is selected
+    need = {int(set_of[r]) for r in np.concatenate([qr, kr]) if r >= L}
+    if (kr < L).any():
+        need = set(range(len(sets)))
+    groups = ([groups[0]] if L else []) + [groups[(1 if L else 0) + g] for g in sorted(need)]
+    out = [np.empty((B, len(qr), len(heads_), d)), np.empty((B, len(kr), len(heads_), d)),
+           np.empty((B, len(kr), len(heads_), d))]
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            qh, kh, vh, dh = (np.asarray(a[b, :, h], np.float64) for a in (q, k, v, do))
+            lse = np.empty(N)
+            dsum = np.empty(N)
+            for rows, keys in groups:
+                for r0 in range(0, len(rows), chunk):
+                    rr = rows[r0:r0 + chunk]
+                    s = (qh[rr] @ kh[keys].T) * scale
+                    m = s.max(axis=1)
+                    e = np.exp(s - m[:, None])
+                    z = e.sum(axis=1)
+                    lse[rr] = m + np.log(z)
+                    dsum[rr] = (dh[rr] * ((e / z[:, None]) @ vh[keys])).sum(axis=1)
+            # dq of the selected query rows, over the keys each row sees
+            for i, r in enumerate(qr):
+                keys = np.arange(N) if r < L else np.concatenate([text, sets[set_of[r]]])
+                p = np.exp((kh[keys] @ qh[r]) * scale - lse[r])
+                ds = p * (vh[keys] @ dh[r] - dsum[r])
+                out[0][b, i, hi] = ds @ kh[keys] * scale
+            # dk, dv of the selected key rows, over the query rows that see each key
+            for i, j in enumerate(kr):
+                rows = np.arange(N) if j < L else np.concatenate([text, sets[set_of[j]]])
+                p = np.exp((qh[rows] @ kh[j]) * scale - lse[rows])
+                ds = p * (dh[rows] @ vh[j] - dsum[rows])
+                out[1][b, i, hi] = ds @ qh[rows] * scale
+                out[2][b, i, hi] = p @ dh[rows]
+    return tuple(out)

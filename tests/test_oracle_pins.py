@@ -741,3 +741,26 @@ def test_skiparse_text_backward_reduces_to_skiparse_and_dense():
     # one set: every token sees every token, the dense backward
     for a, b in zip(O.skiparse_text_backward_ref(q, k, v, G, 4, 1, O.SKIP_GROUP), O.attn_backward_ref(q, k, v, G)):
         np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("text_len", [0, 3])
+def test_skiparse_text_backward_rows_match_finite_differences(text_len):
+    # 3 (or no) text tokens + 12 video tokens in k = 2 Group Skip sets (groups of 2), B = 2; the
+    # selected rows include text and video tokens of both sets
+    rng = np.random.default_rng(87 + text_len)
+    N = text_len + 12
+    q, k, v = (rng.standard_normal((2, N, 3, 4)) for _ in range(3))
+    G = rng.standard_normal((2, N, 3, 4))
+    rows = sorted({0, 1, N - 1, text_len, text_len + 3})
+    heads = [0, 2]
+    loss = lambda q_, k_, v_: float((O.skiparse_text_attn_ref(q_, k_, v_, text_len, 2, O.SKIP_GROUP, scale=0.7)
+                                     * G).sum())
+    dq, dk, dv = O.skiparse_text_backward_rows_ref(q, k, v, G, text_len, 2, O.SKIP_GROUP, rows, rows, heads=heads,
+                                                   scale=0.7, chunk=5)
+    fq = _fd_grad(lambda x: loss(x, k, v), q)
+    fk = _fd_grad(lambda x: loss(q, x, v), k)
+    fv = _fd_grad(lambda x: loss(q, k, x), v)
+    sel = np.ix_(range(2), rows, heads, range(4))
+    np.testing.assert_allclose(dq, fq[sel], rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, fk[sel], rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, fv[sel], rtol=1e-6, atol=1e-8)
