@@ -743,15 +743,17 @@ def test_skiparse_text_backward_reduces_to_skiparse_and_dense():
         np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
 
 
-@pytest.mark.parametrize("text_len", [0, 3])
-def test_skiparse_text_backward_rows_match_finite_differences(text_len):
+@pytest.mark.parametrize("text_len,text_rows", [(0, False), (3, True), (3, False)])
+def test_skiparse_text_backward_rows_match_finite_differences(text_len, text_rows):
     # 3 (or no) text tokens + 12 video tokens in k = 2 Group Skip sets (groups of 2), B = 2; the
-    # selected rows include text and video tokens of both sets
+    # selected rows are text and video tokens of both sets, or video tokens of one set only (the
+    # other set's row statistics are then not computed)
     rng = np.random.default_rng(87 + text_len)
     N = text_len + 12
     q, k, v = (rng.standard_normal((2, N, 3, 4)) for _ in range(3))
     G = rng.standard_normal((2, N, 3, 4))
-    rows = sorted({0, 1, N - 1, text_len, text_len + 3})
+    rows = sorted({0, 1, N - 1, text_len, text_len + 3}) if text_rows or not text_len else \
+        [text_len, text_len + 1, text_len + 4, text_len + 9]
     heads = [0, 2]
     loss = lambda q_, k_, v_: float((O.skiparse_text_attn_ref(q_, k_, v_, text_len, 2, O.SKIP_GROUP, scale=0.7)
                                      * G).sum())
