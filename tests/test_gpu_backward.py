@@ -199,3 +199,34 @@ def test_skiparse_text_backward_matches_oracle(gpu, case, mode):
                 keys = np.concatenate([np.arange(L), rows])
                 ref = O.attention_head_lse_ref(qd[b, rows, h], kd[b, keys, h], scale) / math.log(2.0)
                 np.testing.assert_allclose(lv[b * kk + g, h, :n], ref, rtol=0, atol=2e-3)
+
+
+FULL_SKIP = [("open_sora_plan", 0), ("open_sora_plan", 226), ("long_video", 0)]
+
+
+@pytest.mark.parametrize("wl,L", FULL_SKIP, ids=[f"{w}_L{L}" for w, L in FULL_SKIP])
+def test_full_size_skiparse_backward_sampled(gpu, wl, L):
+    """Skiparse training at full size (Open-Sora Plan d = 96, 24 heads, 28,800 video tokens, k = 4;
+    long video d = 128, 32 heads, 36,864 tokens, k = 4), Single then Group Skip on the same
+    buffers, with and without 226 joined text tokens: sampled dQ rows and dK / dV rows of one head
+    (video rows from the first and last set, and text rows) against the oracle's row form."""
+    w = syn.WORKLOADS[wl]
+    kk, nv = w.skiparse_k, w.n_video
+    shape = (w.B, L + nv, w.heads, w.head_dim)
+    q, k, v, do = (syn.randn_bf16(shape, w.seed + 40 + i) for i in range(4))
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    h = w.heads - 1
+    q1, k1, v1, do1 = (to_f64(t[:, :, h:h + 1]) for t in (q, k, v, do))
+    rng = np.random.default_rng(12)
+    for mode in (0, 1):
+        o, lse = ops.attn_forward_train(qg, kg, vg, w.grid, L, sparse_k=kk, mode=mode)
+        dq, dk, dv = ops.attn_backward(qg, kg, vg, o, dog, lse, w.grid, L, sparse_k=kk, mode=mode)
+        ops.check_status()
+        sets = O.skiparse_sets(nv, kk, mode)
+        vid = [sets[0][0], sets[0][-1], sets[-1][0], sets[-1][-1],
+               *rng.choice(sets[0], 2).tolist(), *rng.choice(sets[-1], 2).tolist()]
+        rows = sorted({L + int(x) for x in vid} | ({0, L - 1} if L else set()))
+        rq, rk, rv = O.skiparse_text_backward_rows_ref(q1, k1, v1, do1, L, kk, mode, rows, rows)
+        assert_grad_close(dq[0, rows, h], rq[0, :, 0], f"dq mode {mode}")
+        assert_grad_close(dk[0, rows, h], rk[0, :, 0], f"dk mode {mode}")
+        assert_grad_close(dv[0, rows, h], rv[0, :, 0], f"dv mode {mode}")
