@@ -81,6 +81,22 @@ def tensor_peak(peaks: dict, src: str, clocks: dict | None, region_s: float):
     return burst, f"{src} burst bf16 GEMM: timed region {region_s:.2f} s, {clk}"
 
 
+MUFU_EX2_PER_CLK_SM = 16   # ex2.approx.f32 per clock per SM (four per SM sub-partition per clock)
+
+
+def exp_rate(flops: float, head_dim: int, attn_ms: float, sms: int, clocks: dict | None) -> dict:
+    """The secondary bound of the attention kernel at small head_dim: one exponential per unmasked
+    (query, key) score, flops / (4 d) of them, against the MUFU rate at the sampled median SM
+    clock (its maximum if not sampled)."""
+    mhz = (clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz") or 1965.0
+    exps = flops / (4.0 * head_dim)
+    achieved = exps / (attn_ms * 1e-3) / 1e12
+    peak = MUFU_EX2_PER_CLK_SM * sms * float(mhz) * 1e6 / 1e12
+    return {"achieved": round(achieved, 3), "peak": round(peak, 3), "unit": "Texp/s", "frac": round(achieved / peak, 4),
+            "exps_per_step": exps, "peak_source": f"{MUFU_EX2_PER_CLK_SM} ex2 per clock per SM x {sms} SMs at "
+                                                  f"{float(mhz):.0f} MHz"}
+
+
 def tensor_or_hbm_roofline(flops: float, nbytes: float, ms: float, peaks: dict, src: str, clocks, region_s: float):
     """Roofline of a launch that may be bound by either unit: the bound is the unit whose time at
     its peak is the longer one; frac = achieved / that unit's peak."""
@@ -755,7 +771,8 @@ def per_config_entry(w, kind, t: dict, steps: int, sms: int, flushed: bool) -> d
          "frac": round(attn_tf / peak, 4), "peak": peak, "peak_source": peak_src,
          "l2": "L2 flushed (256 MiB write) before every step, outside its events" if flushed
                else "inputs larger than L2, no flush",
-         "clocks": t["clocks"], "gpu_launches": launches_per_step(w, sms, kind) * steps}
+         "clocks": t["clocks"], "gpu_launches": launches_per_step(w, sms, kind) * steps,
+         "exp_rate": exp_rate(flops, w.head_dim, t["attn_ms"], sms, t["clocks"])}
     if w.seq_len < 4096:
         e["us_per_step"] = round(ms * 1e3, 2)
         e["note"] = "launch-latency bound; its roofline fraction is not meaningful"
@@ -863,7 +880,9 @@ def run_ours(args, rank, world, local_rank):
                      "frac_of_sustained_peak": round(achieved / float(peaks.get("bf16_tflops_sustained",
                                                                                  peaks["bf16_tflops"])), 4),
                      "avg_launch_ms": round(attn_ms, 4),
-                     "flops_per_launch": flops},
+                     "flops_per_launch": flops,
+                     "secondary": dict(exp_rate(flops, w.head_dim, attn_ms, sms, clocks),
+                                       bound="mufu (one exponential per score)")},
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes, "ms_per_step": round(e2e_ms, 4),
                 "steps": e2e_steps, "copies": "pinned host <-> device on two copy streams, double-buffered, "
