@@ -38,7 +38,6 @@ constexpr int kComputeThreads = 256;
 constexpr int kProdWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kAccWarp = 10;
-constexpr int kRedWarp = 11;             // fused dQ: issues the bulk reduce-adds of dQ
 // dK/dV kernel: four compute warps per SM sub-partition, each turning 16 of a sub-tile's 64
 // query columns into P and dS (OSP_BWD_WIDE=0: two per sub-partition, 32 columns each).  More
 // warps per sub-partition keep its MUFU and issue slots busy while each warp waits on tensor
@@ -443,7 +442,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
   const int B_KVT = B_STGFREE + 1;   // K and V are in tensor memory
 
   const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, false);
-  const int tile = un.tile, h = un.h, bg = un.bg, b = un.b, g = un.g;
+  const int tile = un.tile, h = un.h, b = un.b, g = un.g;
   const int n_rows = un.n, rb = un.row_base;   // the set's rows; its first packed row (packed batches)
   const int kv0 = tile * kBT;
   // query tiles i0 .. n_tiles-1 (frame-causal: the first query that may see key kv0 opens the range)
@@ -810,7 +809,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   // frame-causal: a head's query tiles in reverse, so that those seeing the most keys start first
   const BwdUnit un = bwd_unit<kPk>(p, seg, (int)blockIdx.x, p.frame_hw != 0, kPk ? 0 : p.q_tiles);
-  const int tile = un.tile, h = un.h, bg = un.bg, b = un.b, g = un.g;
+  const int tile = un.tile, h = un.h, b = un.b, g = un.g;
   const int n_rows = un.n, rb = un.row_base;   // the set's rows; its first packed row (packed batches)
   const int q_rows = kPk ? n_rows : p.q_rows;  // its query rows
   const int q0 = tile * kBT;
