@@ -803,6 +803,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_RES = 0, B_FULL = 1, B_EMPTY = 1 + kStages, B_SFULL = 1 + 2 * kStages, B_PREADY = B_SFULL + 2,
             B_DONE = B_PREADY + 2, B_FIN = B_DONE + 1, B_BUFFREE = B_FIN + 1, B_FIN2 = B_BUFFREE + 2;
+  const int B_QT = B_FIN2 + 1;   // Q and dO are in tensor memory
+  // Q and dO also sit in tensor memory (packed channel pairs, query = lane) after the dQ
+  // accumulator, so the score products S = Q K^T and dP = dO V^T read only K / V from shared memory
+  constexpr uint32_t kColQ = 384, kColDo = 448;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -834,6 +838,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(B_BUFFREE + 0), 1);
     mbar_init(bar(B_BUFFREE + 1), 1);
     mbar_init(bar(B_FIN2), 1);
+    mbar_init(bar(B_QT), kComputeThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -908,17 +913,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     // sub-tile t = 2j + hh: keys 64hh .. 64hh+63 of key tile j, score buffer t & 1; the two
     // issuing warps split as in the dK/dV kernel
+    // D_t = A (tensor memory: Q or dO, 8 columns per 16 channels) times B K-major (64 keys x D)^T
+    auto issue_ts_q = [&](uint32_t d_col, uint32_t a_col, uint64_t b0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+        if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + off, idesc_ss, kk > 0 ? 1u : 0u);
+      }
+    };
+    (void)dQ;
+    (void)dO;
     const int n_sub = 2 * nk;
     if (warp == kMmaWarp) {
-      bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      bool ok = bwd_warp_wait(bar(B_RES), 0, wc) && bwd_warp_wait(bar(B_QT), 0, wc);
       for (int t = 0; ok && t < n_sub; ++t) {
         const int j = t >> 1, hh = t & 1, s = j % kStages;
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (j / kStages) & 1, wc)) break;
         if (t >= 2 && !bwd_warp_wait(bar(B_BUFFREE + (t & 1)), ((t - 2) >> 1) & 1, wc)) break;
         tc_fence_after();
         const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
-        issue_ss(col_s(t & 1), dQ, dKk + sub);    // S = Q K_sub^T
-        issue_ss(col_dp(t & 1), dO, dVk + sub);   // dP = dO V_sub^T
+        issue_ts_q(col_s(t & 1), kColQ, dKk + sub);     // S = Q K_sub^T
+        issue_ts_q(col_dp(t & 1), kColDo, dVk + sub);   // dP = dO V_sub^T
         if (leader) tc_commit(bar(B_SFULL + (t & 1)));
       }
       if (leader) tc_commit(bar(B_FIN));
@@ -947,9 +962,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool vin = live && index_ok(vec_row + qs, p.vec_elems, p.status);
     const float lse_r = vin ? p.lse[vec_row + qs] : 0.f;
     const float dv_r = vin ? p.dvec[vec_row + qs] : 0.f;
-    bool ok = true;
+    // Q (half 0) or dO (half 1): this row's D channels, SW128 chunks of 64 channels, as packed
+    // pairs into the tensor-memory block
+    bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+    if (ok) {
+      uint32_t r[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {   // 16-byte chunk c: channels 8c .. 8c + 7
+        const uint32_t src = sRes(half) + (uint32_t)((c >> 3) * kChunkBytes + (row >> 3) * 1024 + (row & 7) * 128) +
+                             16u * (uint32_t)((c & 7) ^ (row & 7));
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(r[4 * c]), "=r"(r[4 * c + 1]), "=r"(r[4 * c + 2]), "=r"(r[4 * c + 3])
+                     : "r"(src));
+      }
+      const uint32_t dst = tmem + lane_base + (half ? kColDo : kColQ);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tmem_st32(dst + 32u * c, *reinterpret_cast<const uint32_t(*)[32]>(&r[32 * c]));
+      if constexpr (D % 64) tmem_st16(dst + 32u * (D / 64), *reinterpret_cast<const uint32_t(*)[16]>(&r[32 * (D / 64)]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_QT));
+    }
     const int klim = p.frame_hw ? min(n_rows, causal_limit(qs, p.text_len, p.frame_hw)) : n_rows;   // keys it sees
-    for (int t = 0; t < 2 * nk; ++t) {
+    for (int t = 0; ok && t < 2 * nk; ++t) {
       const int j = t >> 1, hh = t & 1, bb = t & 1;
       if (!bwd_warp_wait(bar(B_SFULL + bb), (t >> 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
