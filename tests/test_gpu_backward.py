@@ -160,6 +160,7 @@ SKIP_TEXT = [
     (2, 1, 64, (2, 16, 16), 4, 140),     # text over a tile boundary; B = 2
     (1, 2, 96, (4, 10, 15), 2, 17),      # sets of 300: ragged tiles
     (1, 1, 128, (4, 16, 18), 4, 33),
+    (2, 2, 64, (2, 4, 8), 2, 10),        # sets of 32 rows (one partial tile) and 10 text rows
 ]
 
 
