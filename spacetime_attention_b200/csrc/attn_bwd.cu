@@ -60,7 +60,7 @@ constexpr uint32_t kTmemCols = 512;
 // while the compute warps turn sub-tile t into P / dS.  Tensor-memory columns: buffer b holds S
 // (or S^T) at 128b .. 128b+63 and dP (dP^T) at 128b+64 .. 128b+127; accumulators at 256 and 384.
 constexpr int kSub = 64;
-constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
+constexpr uint32_t kColAcc0 = 256;   // dV (dK kernel) or dQ (dQ kernel); dK at BwdCfg::kColDk
 __device__ __forceinline__ uint32_t col_s(int buf) { return 128u * buf; }
 __device__ __forceinline__ uint32_t col_dp(int buf) { return 128u * buf + 64u; }
 // descriptor offset (16-byte units) of the second 64-row sub-tile of a 128-row SW128 tile
@@ -83,6 +83,11 @@ struct BwdCfg {
   // tensor memory it is bound by its math.  The dQ buffer is then single (its second copy's
   // columns hold K and V).
   static constexpr bool kKvTmem = kFuseDq;
+  // d = 96: dK's accumulator moves up to columns 352 .. 447 (next to dV at 256), which leaves
+  // 448 .. 495 for K, so S^T = K Q^T also takes A from tensor memory (V does not fit; dP^T keeps
+  // both operands in shared memory)
+  static constexpr bool kKTmem = (D == 96);
+  static constexpr uint32_t kColDk = (D == 96) ? 352u : 384u;
   // dK/dV kernel: compute warps, producer, two MMA issuers and (fused dQ) the reduce warp
   static constexpr int kThreads = 32 * (kDkComputeWarps + (kFuseDq ? 4 : 3));
   static constexpr int kResOff = 0;                                 // two resident tiles
@@ -471,10 +476,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       for (int u = 0; u < 2; ++u) mbar_init(bar(B_DSFREE + u), 1);
       mbar_init(bar(B_DQFULL), 1);
       mbar_init(bar(B_DQTFREE), kDkComputeThreads);
-      mbar_init(bar(B_KVT), kDkComputeThreads);
       mbar_init(bar(B_STGFULL), kDkComputeThreads);
       mbar_init(bar(B_STGFREE), 1);
     }
+    if constexpr (C::kKvTmem || C::kKTmem) mbar_init(bar(B_KVT), kDkComputeThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -579,7 +584,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     };
     if (warp == kDkMmaWarp) {
       bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
-      if constexpr (C::kKvTmem) ok = ok && bwd_warp_wait(bar(B_KVT), 0, wc);
+      if constexpr (C::kKvTmem || C::kKTmem) ok = ok && bwd_warp_wait(bar(B_KVT), 0, wc);
       for (int t = 0; ok && t < n_sub; ++t) {
         const int i = t >> 1, hh = t & 1, s = i % kStages;
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
@@ -589,6 +594,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if constexpr (C::kKvTmem) {
           issue_ts_kv(col_s(t & 1), kColK, dQk + sub);    // S^T = K Q_sub^T
           issue_ts_kv(col_dp(t & 1), kColV, dOk + sub);   // dP^T = V dO_sub^T
+        } else if constexpr (C::kKTmem) {
+          issue_ts_kv(col_s(t & 1), kColK, dQk + sub);
+          issue_ss(col_dp(t & 1), dV, dOk + sub);
         } else {
           issue_ss(col_s(t & 1), dK, dQk + sub);
           issue_ss(col_dp(t & 1), dV, dOk + sub);
@@ -608,7 +616,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tc_fence_after();
         const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
         issue_ts(kColAcc0, col_s(t & 1), dOmn + sub, t > 0);    // dV += P^T dO_sub
-        issue_ts(kColAcc1, col_dp(t & 1), dQmn + sub, t > 0);   // dK += dS^T Q_sub
+        issue_ts(C::kColDk, col_dp(t & 1), dQmn + sub, t > 0);   // dK += dS^T Q_sub
         if (leader) tc_commit(bar(B_BUFFREE + (t & 1)));      // buffer t & 1 may be overwritten
         if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));   // both halves of tile i consumed
         if constexpr (C::kFuseDq) {
@@ -709,6 +717,28 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(B_KVT));
       }
+    } else if constexpr (C::kKTmem) {
+      // K only (d = 96): column groups 0 .. 2 take this row's 16-byte chunks 4 cg .. 4 cg + 3
+      // (channels 32 cg ..; chunk c lies in SW128 block c / 8) into columns 16 cg .. + 15
+      ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      if (ok) {
+        if (cg < 3) {
+          uint32_t r[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int c = 4 * cg + v;
+            const uint32_t src = sRes(0) + (uint32_t)((c >> 3) * kChunkBytes + (row >> 3) * 1024 + (row & 7) * 128) +
+                                 16u * (uint32_t)((c & 7) ^ (row & 7));
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(r[4 * v]), "=r"(r[4 * v + 1]), "=r"(r[4 * v + 2]), "=r"(r[4 * v + 3])
+                         : "r"(src));
+          }
+          tmem_st16(tmem + lane_base + kColK + 16u * (uint32_t)cg, r);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(B_KVT));
+      }
     }
     for (int t = 0; ok && t < 2 * nq; ++t) {
       const int il = t >> 1, i = i0 + il, hh = t & 1, bb = t & 1;
@@ -770,11 +800,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       const int part = kGroups > 2 ? (cg & 1) : -1;
       if (p.dk32) {
         if (!is_dk) bwd_store_row_f32<D>(tmem + lane_base + kColAcc0, 1.f, p.dv32 + off, store, part);
-        else bwd_store_row_f32<D>(tmem + lane_base + kColAcc1, p.scale, p.dk32 + off, store, part);
+        else bwd_store_row_f32<D>(tmem + lane_base + C::kColDk, p.scale, p.dk32 + off, store, part);
       } else if (!is_dk) {
         bwd_store_row<D>(tmem + lane_base + kColAcc0, 1.f, p.dv + off, store, part);
       } else {
-        bwd_store_row<D>(tmem + lane_base + kColAcc1, p.scale, p.dk + off, store, part);
+        bwd_store_row<D>(tmem + lane_base + C::kColDk, p.scale, p.dk + off, store, part);
       }
     }
   }
