@@ -50,6 +50,13 @@ constexpr int kDkComputeWarps = 4 * (64 / kDkCols);      // 16 or 8
 constexpr int kDkComputeThreads = 32 * kDkComputeWarps;
 constexpr int kDkProdWarp = kDkComputeWarps, kDkMmaWarp = kDkComputeWarps + 1, kDkAccWarp = kDkComputeWarps + 2,
               kDkRedWarp = kDkComputeWarps + 3;
+// One thread issues every product of the dK/dV kernel (1), or the score products and the
+// accumulating products come from two warps with a buffer-free barrier between them (0); -1
+// (default): one issuer at d = 64 and 128, two at d = 96 (same-box A/B with one issuer: d = 128
+// +4 %, d = 64 +1 %, d = 96 -2 %).
+#ifndef OSP_BWD_ONE_ISSUER
+#define OSP_BWD_ONE_ISSUER -1
+#endif
 #ifndef OSP_BWD_FUSE_DQ
 #define OSP_BWD_FUSE_DQ 1                // d = 64: dQ accumulated by the dK/dV kernel (no dQ kernel)
 #endif
@@ -88,6 +95,7 @@ struct BwdCfg {
   // both operands in shared memory)
   static constexpr bool kKTmem = (D == 96);
   static constexpr uint32_t kColDk = (D == 96) ? 352u : 384u;
+  static constexpr bool kOneIssuer = OSP_BWD_ONE_ISSUER < 0 ? (D != 96) : (OSP_BWD_ONE_ISSUER != 0);
   // dK/dV kernel: compute warps, producer, two MMA issuers and (fused dQ) the reduce warp
   static constexpr int kThreads = 32 * (kDkComputeWarps + (kFuseDq ? 4 : 3));
   static constexpr int kResOff = 0;                                 // two resident tiles
@@ -582,7 +590,79 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (leader) mma_ts(tmem + d_col, tmem + a_col + 8u * kk, b0 + off, idesc_ss, kk > 0 ? 1u : 0u);
       }
     };
-    if (warp == kDkMmaWarp) {
+    // fused dQ: dQ_i = dS_i K, A = dS_i^T from shared memory (MN-major: rows = keys, queries
+    // contiguous in two 64-query SW128 chunks 16 KB apart), B = the resident K (MN-major, N = D)
+    constexpr uint32_t idesc_dq = idesc_bf16_f32(kBT, D, true, true);
+    const uint64_t dKres_mn = sdesc_sw128(sRes(0), kChunkBytes, 1024);
+    auto issue_scores = [&](int t) {   // S^T and dP^T of sub-tile t into score buffer t & 1
+      const int hh = t & 1, s = (t >> 1) % kStages;
+      const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
+      if constexpr (C::kKvTmem) {
+        issue_ts_kv(col_s(t & 1), kColK, dQk + sub);    // S^T = K Q_sub^T
+        issue_ts_kv(col_dp(t & 1), kColV, dOk + sub);   // dP^T = V dO_sub^T
+      } else if constexpr (C::kKTmem) {
+        issue_ts_kv(col_s(t & 1), kColK, dQk + sub);
+        issue_ss(col_dp(t & 1), dV, dOk + sub);
+      } else {
+        issue_ss(col_s(t & 1), dK, dQk + sub);
+        issue_ss(col_dp(t & 1), dV, dOk + sub);
+      }
+      if (leader) tc_commit(bar(B_SFULL + (t & 1)));
+    };
+    auto issue_accum = [&](int t) {   // dV, dK of sub-tile t from score buffer t & 1
+      const int hh = t & 1, s = (t >> 1) % kStages;
+      const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
+      issue_ts(kColAcc0, col_s(t & 1), dOmn + sub, t > 0);    // dV += P^T dO_sub
+      issue_ts(C::kColDk, col_dp(t & 1), dQmn + sub, t > 0);   // dK += dS^T Q_sub
+    };
+    auto issue_dq = [&](int i) -> bool {   // dQ of local tile i, after its second sub-tile
+      const int b = i & 1;
+      // the tensor-memory buffer's previous tile (i - 1) has been read out
+      if (i >= 1 && !bwd_warp_wait(bar(B_DQTFREE), (i - 1) & 1, wc)) return false;
+      tc_fence_after();
+      const uint64_t da = sdesc_sw128(sDs(b), kChunkBytes, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kBT / 16; ++kk)   // 16 keys (two 8-row groups, 2 KB) per step
+        if (leader) mma_ss(tmem + kColDq, da + (uint64_t)(128 * kk), dKres_mn + (uint64_t)(128 * kk), idesc_dq,
+                           kk > 0 ? 1u : 0u);
+      if (leader) tc_commit(bar(B_DQFULL));
+      if (leader) tc_commit(bar(B_DSFREE + b));
+      return true;
+    };
+    if (C::kOneIssuer && warp == kDkMmaWarp) {
+      // one thread issues every product: the first two sub-tiles' scores, then per sub-tile t its
+      // dV and dK, the scores of t + 2 into the buffer those just read (the tensor pipe runs one
+      // thread's products in order), and after a tile's second sub-tile its dQ
+      bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
+      if constexpr (C::kKvTmem || C::kKTmem) ok = ok && bwd_warp_wait(bar(B_KVT), 0, wc);
+      if (ok && n_sub > 0) ok = bwd_warp_wait(bar(B_FULL + 0), 0, wc);
+      for (int t = 0; ok && t < n_sub && t < 2; ++t) {
+        tc_fence_after();
+        issue_scores(t);
+      }
+      for (int t = 0; ok && t < n_sub; ++t) {
+        const int i = t >> 1, hh = t & 1, s = i % kStages;
+        if (!bwd_warp_wait(bar(B_PREADY + (t & 1)), (t >> 1) & 1, wc)) break;
+        tc_fence_after();
+        issue_accum(t);
+        if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));   // tile i's Q and dO are consumed
+        const int tn = t + 2;
+        if (tn < n_sub) {
+          const int in = tn >> 1;
+          if ((tn & 1) == 0 && !bwd_warp_wait(bar(B_FULL + in % kStages), (in / kStages) & 1, wc)) break;
+          tc_fence_after();
+          issue_scores(tn);
+        }
+        if constexpr (C::kFuseDq) {
+          if (hh == 1 && !issue_dq(i)) break;
+        }
+        if (t == n_sub - 1 && leader) tc_commit(bar(B_DONE));
+      }
+      if (leader) tc_commit(bar(B_FIN));
+      mbar_drain(bar(B_FIN), 0, p.timeout_ns);
+    } else if (C::kOneIssuer) {
+      // (the accumulating-product warp has nothing to issue when one thread issues everything)
+    } else if (warp == kDkMmaWarp) {
       bool ok = bwd_warp_wait(bar(B_RES), 0, wc);
       if constexpr (C::kKvTmem || C::kKTmem) ok = ok && bwd_warp_wait(bar(B_KVT), 0, wc);
       for (int t = 0; ok && t < n_sub; ++t) {
@@ -590,49 +670,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (i / kStages) & 1, wc)) break;
         if (t >= 2 && !bwd_warp_wait(bar(B_BUFFREE + (t & 1)), ((t - 2) >> 1) & 1, wc)) break;
         tc_fence_after();
-        const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
-        if constexpr (C::kKvTmem) {
-          issue_ts_kv(col_s(t & 1), kColK, dQk + sub);    // S^T = K Q_sub^T
-          issue_ts_kv(col_dp(t & 1), kColV, dOk + sub);   // dP^T = V dO_sub^T
-        } else if constexpr (C::kKTmem) {
-          issue_ts_kv(col_s(t & 1), kColK, dQk + sub);
-          issue_ss(col_dp(t & 1), dV, dOk + sub);
-        } else {
-          issue_ss(col_s(t & 1), dK, dQk + sub);
-          issue_ss(col_dp(t & 1), dV, dOk + sub);
-        }
-        if (leader) tc_commit(bar(B_SFULL + (t & 1)));
+        issue_scores(t);
       }
       if (leader) tc_commit(bar(B_FIN));
       mbar_drain(bar(B_FIN), 0, p.timeout_ns);
     } else {
-      // fused dQ: dQ_i = dS_i K, A = dS_i^T from shared memory (MN-major: rows = keys, queries
-      // contiguous in two 64-query SW128 chunks 16 KB apart), B = the resident K (MN-major, N = D)
-      constexpr uint32_t idesc_dq = idesc_bf16_f32(kBT, D, true, true);
-      const uint64_t dKres_mn = sdesc_sw128(sRes(0), kChunkBytes, 1024);
       for (int t = 0; t < n_sub; ++t) {
         const int i = t >> 1, hh = t & 1, s = i % kStages;
         if (!bwd_warp_wait(bar(B_PREADY + (t & 1)), (t >> 1) & 1, wc)) break;
         tc_fence_after();
-        const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
-        issue_ts(kColAcc0, col_s(t & 1), dOmn + sub, t > 0);    // dV += P^T dO_sub
-        issue_ts(C::kColDk, col_dp(t & 1), dQmn + sub, t > 0);   // dK += dS^T Q_sub
+        issue_accum(t);
         if (leader) tc_commit(bar(B_BUFFREE + (t & 1)));      // buffer t & 1 may be overwritten
         if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));   // both halves of tile i consumed
         if constexpr (C::kFuseDq) {
-          if (hh == 1) {
-            const int b = i & 1;
-            // the tensor-memory buffer's previous tile (i - 1) has been read out
-            if (i >= 1 && !bwd_warp_wait(bar(B_DQTFREE), (i - 1) & 1, wc)) break;
-            tc_fence_after();
-            const uint64_t da = sdesc_sw128(sDs(b), kChunkBytes, 1024);
-#pragma unroll
-            for (int kk = 0; kk < kBT / 16; ++kk)   // 16 keys (two 8-row groups, 2 KB) per step
-              if (leader) mma_ss(tmem + kColDq, da + (uint64_t)(128 * kk), dKres_mn + (uint64_t)(128 * kk),
-                                 idesc_dq, kk > 0 ? 1u : 0u);
-            if (leader) tc_commit(bar(B_DQFULL));
-            if (leader) tc_commit(bar(B_DSFREE + b));
-          }
+          if (hh == 1 && !issue_dq(i)) break;
         }
         if (t == n_sub - 1 && leader) tc_commit(bar(B_DONE));
       }
