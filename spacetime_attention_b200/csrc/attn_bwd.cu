@@ -1005,6 +1005,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     (void)dQ;
     (void)dO;
     const int n_sub = 2 * nk;
+    auto issue_scores = [&](int t) {   // S and dP of sub-tile t into score buffer t & 1
+      const int hh = t & 1, s = (t >> 1) % kStages;
+      const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
+      issue_ts_q(col_s(t & 1), kColQ, dKk + sub);     // S = Q K_sub^T
+      issue_ts_q(col_dp(t & 1), kColDo, dVk + sub);   // dP = dO V_sub^T
+      if (leader) tc_commit(bar(B_SFULL + (t & 1)));
+    };
+    auto issue_accum = [&](int t) {   // dQ += dS K_sub, dS from score buffer t & 1
+      const int hh = t & 1, s = (t >> 1) % kStages;
+      issue_ts(kColAcc0, col_dp(t & 1), dKmn + stage_off(s) + (hh ? kSubDescOff : 0), t > 0);
+    };
+    // (one thread issuing both, as in the dK/dV kernel, measured -5 % at d = 96 and -0.6 % at
+    // d = 128 here)
     if (warp == kMmaWarp) {
       bool ok = bwd_warp_wait(bar(B_RES), 0, wc) && bwd_warp_wait(bar(B_QT), 0, wc);
       for (int t = 0; ok && t < n_sub; ++t) {
@@ -1012,10 +1025,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (hh == 0 && !bwd_warp_wait(bar(B_FULL + s), (j / kStages) & 1, wc)) break;
         if (t >= 2 && !bwd_warp_wait(bar(B_BUFFREE + (t & 1)), ((t - 2) >> 1) & 1, wc)) break;
         tc_fence_after();
-        const uint64_t sub = stage_off(s) + (hh ? kSubDescOff : 0);
-        issue_ts_q(col_s(t & 1), kColQ, dKk + sub);     // S = Q K_sub^T
-        issue_ts_q(col_dp(t & 1), kColDo, dVk + sub);   // dP = dO V_sub^T
-        if (leader) tc_commit(bar(B_SFULL + (t & 1)));
+        issue_scores(t);
       }
       if (leader) tc_commit(bar(B_FIN));
       mbar_drain(bar(B_FIN), 0, p.timeout_ns);
@@ -1024,7 +1034,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int j = t >> 1, hh = t & 1, s = j % kStages;
         if (!bwd_warp_wait(bar(B_PREADY + (t & 1)), (t >> 1) & 1, wc)) break;
         tc_fence_after();
-        issue_ts(kColAcc0, col_dp(t & 1), dKmn + stage_off(s) + (hh ? kSubDescOff : 0), t > 0);   // dQ += dS K_sub
+        issue_accum(t);
         if (leader) tc_commit(bar(B_BUFFREE + (t & 1)));
         if (hh == 1 && leader) tc_commit(bar(B_EMPTY + s));
         if (t == n_sub - 1 && leader) tc_commit(bar(B_DONE));
