@@ -793,3 +793,50 @@ def skiparse_text_backward_rows_ref(q, k, v, do, text_len: int, k_ratio: int, mo
                 out[1][b, i, hi] = ds @ qh[rows] * scale
                 out[2][b, i, hi] = p @ dh[rows]
     return tuple(out)
+
+
+def frame_causal_backward_rows_ref(q, k, v, do, grid: Sequence[int], text_len: int, q_rows, k_rows, heads=None,
+                                   scale: float | None = None, chunk: int = 2048):
+    """Selected rows of the gradients of frame_causal_attn_ref without forming the N x N score
+    matrix: dq for tokens ``q_rows``, dk and dv for tokens ``k_rows``, for heads ``heads`` (all by
+    default); each [B, rows, heads, d].  Row r sees the first frame_causal_limit(r) tokens; the
+    row log-sum-exp and rowsum(dO * O) of every row come first, per group of rows with the same
+    limit (the text block; each frame), in chunks of ``chunk`` rows."""
+    T, H, W = (int(a) for a in grid)
+    B, N, nh, d = q.shape
+    L = int(text_len)
+    HW = H * W
+    scale = default_scale(d) if scale is None else scale
+    lim = np.array([frame_causal_limit(r, L, HW) for r in range(N)])
+    groups = ([np.arange(L)] if L else []) + [L + t * HW + np.arange(HW) for t in range(T)]
+    heads_ = np.arange(nh) if heads is None else np.asarray(heads)
+    qr, kr = np.asarray(q_rows, dtype=np.int64), np.asarray(k_rows, dtype=np.int64)
+    out = [np.empty((B, len(qr), len(heads_), d)), np.empty((B, len(kr), len(heads_), d)),
+           np.empty((B, len(kr), len(heads_), d))]
+    for b in range(B):
+        for hi, h in enumerate(heads_):
+            qh, kh, vh, dh = (np.asarray(a[b, :, h], np.float64) for a in (q, k, v, do))
+            lse = np.empty(N)
+            dsum = np.empty(N)
+            for rows in groups:
+                n_keys = lim[rows[0]]
+                for r0 in range(0, len(rows), chunk):
+                    rr = rows[r0:r0 + chunk]
+                    s = (qh[rr] @ kh[:n_keys].T) * scale
+                    m = s.max(axis=1)
+                    e = np.exp(s - m[:, None])
+                    z = e.sum(axis=1)
+                    lse[rr] = m + np.log(z)
+                    dsum[rr] = (dh[rr] * ((e / z[:, None]) @ vh[:n_keys])).sum(axis=1)
+            for i, r in enumerate(qr):
+                keys = np.arange(lim[r])
+                p = np.exp((kh[keys] @ qh[r]) * scale - lse[r])
+                ds = p * (vh[keys] @ dh[r] - dsum[r])
+                out[0][b, i, hi] = ds @ kh[keys] * scale
+            for i, j in enumerate(kr):
+                rows = np.nonzero(lim > j)[0]          # the rows whose limit covers key j
+                p = np.exp((qh[rows] @ kh[j]) * scale - lse[rows])
+                ds = p * (dh[rows] @ vh[j] - dsum[rows])
+                out[1][b, i, hi] = ds @ qh[rows] * scale
+                out[2][b, i, hi] = p @ dh[rows]
+    return tuple(out)

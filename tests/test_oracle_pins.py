@@ -766,3 +766,20 @@ def test_skiparse_text_backward_rows_match_finite_differences(text_len, text_row
     np.testing.assert_allclose(dq, fq[sel], rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(dk, fk[sel], rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(dv, fv[sel], rtol=1e-6, atol=1e-8)
+
+
+def test_frame_causal_backward_rows_match_finite_differences():
+    # 2 text tokens + 3 frames of 2 x 2, B = 2; selected rows: text, first and last frame
+    rng = np.random.default_rng(91)
+    grid, L = (3, 2, 2), 2
+    N = L + 12
+    q, k, v = (rng.standard_normal((2, N, 3, 4)) for _ in range(3))
+    G = rng.standard_normal((2, N, 3, 4))
+    rows = [0, 1, 2, 5, 9, 13]
+    heads = [1, 2]
+    loss = lambda q_, k_, v_: float((O.frame_causal_attn_ref(q_, k_, v_, grid, L, scale=0.6) * G).sum())
+    dq, dk, dv = O.frame_causal_backward_rows_ref(q, k, v, G, grid, L, rows, rows, heads=heads, scale=0.6, chunk=3)
+    sel = np.ix_(range(2), rows, heads, range(4))
+    np.testing.assert_allclose(dq, _fd_grad(lambda x: loss(x, k, v), q)[sel], rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dk, _fd_grad(lambda x: loss(q, x, v), k)[sel], rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dv, _fd_grad(lambda x: loss(q, k, x), v)[sel], rtol=1e-6, atol=1e-8)
