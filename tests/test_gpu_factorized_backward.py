@@ -129,3 +129,54 @@ def test_per_set_temporal_training_forward_equals_inference(gpu, monkeypatch, ca
     o_inf = ops.attn_temporal(qg, kg, vg, grid, causal=causal)
     ops.check_status()
     assert torch.equal(o_train, o_inf)
+
+
+def test_full_size_factorized_and_frame_causal_backward_sampled(gpu):
+    """CogVideoX-2B grid at full size (13x30x45, 30 heads, d = 64): spatial, temporal (both in
+    time directions) and frame-causal (with the 226 text tokens) training, sampled rows of one
+    head against the oracle: spatial on whole frames through the dense row form, temporal on a
+    subset of positions through temporal_backward_ref, frame-causal through its row form."""
+    w = syn.WORKLOADS["cogvideox_2b"]
+    T, H, W = w.grid
+    HW, L = H * W, w.text_len
+    h = 7
+    q, k, v, do = (syn.randn_bf16((1, L + T * HW, w.heads, w.head_dim), w.seed + 60 + i) for i in range(4))
+    qg, kg, vg, dog = (t.to(gpu) for t in (q, k, v, do))
+    vid = [t[:, L:].contiguous() for t in (qg, kg, vg, dog)]
+    qv, kv, vv, dov = (to_f64(t[:, L:, h:h + 1]) for t in (q, k, v, do))
+    scale = 1 / math.sqrt(w.head_dim)
+    rng = np.random.default_rng(21)
+    # spatial: frames 0, 6 and 12, sampled rows of each
+    o, lse = ops.attn_spatial_train(*vid[:3], w.grid)
+    dq, dk, dv = ops.attn_spatial_backward(vid[0], vid[1], vid[2], o, vid[3], lse, w.grid)
+    ops.check_status()
+    for t in (0, 6, T - 1):
+        f = slice(t * HW, (t + 1) * HW)
+        rows = sorted({0, HW - 1, *rng.integers(0, HW, size=4).tolist()})
+        rq, rk, rv = O.attention_head_backward_rows_ref(qv[0, f, 0], kv[0, f, 0], vv[0, f, 0], dov[0, f, 0], scale,
+                                                        rows, rows)
+        sel = [t * HW + r for r in rows]
+        assert_grad_close(dq[0, sel, h], rq, f"spatial dq frame {t}")
+        assert_grad_close(dk[0, sel, h], rk, f"spatial dk frame {t}")
+        assert_grad_close(dv[0, sel, h], rv, f"spatial dv frame {t}")
+    # temporal: 64 positions (their T tokens each) against temporal_backward_ref on that subset
+    pos = np.sort(rng.choice(HW, size=64, replace=False))
+    idx = (pos[None, :] + HW * np.arange(T)[:, None]).reshape(-1)          # frame-major, as a (T, 1, 64) grid
+    for causal in (False, True):
+        o, lse = ops.attn_temporal_train(*vid[:3], w.grid, causal=causal)
+        dq, dk, dv = ops.attn_temporal_backward(vid[0], vid[1], vid[2], o, vid[3], lse, w.grid, causal=causal)
+        ops.check_status()
+        ref = O.temporal_backward_ref(qv[:, idx], kv[:, idx], vv[:, idx], dov[:, idx], (T, 1, len(pos)), causal=causal)
+        for got, r, name in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
+            assert_grad_close(got[0, idx, h], r[0, :, 0], f"temporal {name} causal={causal}")
+    # frame-causal over text + video: text rows, rows of the first and last frames
+    o, lse = ops.attn_frame_causal_train(qg, kg, vg, w.grid, L)
+    dq, dk, dv = ops.attn_frame_causal_backward(qg, kg, vg, o, dog, lse, w.grid, L)
+    ops.check_status()
+    rows = sorted({0, L - 1, L, L + HW - 1, L + (T - 1) * HW, L + T * HW - 1,
+                   *(L + rng.integers(0, T * HW, size=4)).tolist()})
+    q1, k1, v1, d1 = (to_f64(t[:, :, h:h + 1]) for t in (q, k, v, do))
+    rq, rk, rv = O.frame_causal_backward_rows_ref(q1, k1, v1, d1, w.grid, L, rows, rows)
+    assert_grad_close(dq[0, rows, h], rq[0, :, 0], "frame-causal dq")
+    assert_grad_close(dk[0, rows, h], rk[0, :, 0], "frame-causal dk")
+    assert_grad_close(dv[0, rows, h], rv[0, :, 0], "frame-causal dv")
