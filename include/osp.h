@@ -194,7 +194,11 @@ int osp_attn_forward_train(const void* q, const void* k, const void* v, void* o,
  *   inputs.  Arithmetic: tcgen05 tensor cores, bf16 operands (P and dS rounded to bf16), fp32
  *   accumulation in tensor memory, outputs rounded to bf16.  Scratch: rowsum(dO * O) in a
  *   stream-ordered block (B * G * heads * n_pad floats) from the library's memory pool.
- *   Three kernel launches (row sums, dK/dV, dQ).
+ *   Three kernel launches: row sums, dK/dV, and dQ (head_dim 96, 128), or at head_dim 64 the
+ *   row sums, dK/dV with dQ accumulated into an fp32 scratch block (B * G * heads * n_pad * 64
+ *   floats, same pool) by bulk reduce-adds, and a finalize that rounds dQ to bf16; the order of
+ *   those fp32 additions follows the CTAs' timing, so dQ at head_dim 64 can differ from run to
+ *   run in its last bits (dK, dV and the other head dims are reproducible).
  *   Skiparse with text_len > 0: the video queries' part runs over B*k gathered samples of
  *   [set g's n rows; the text rows] (queries: the first n), the text queries' part over the
  *   natural samples (queries: the first text_len rows); dK and dV of a row sum their fp32
