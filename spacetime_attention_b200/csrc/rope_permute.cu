@@ -24,6 +24,19 @@ namespace osp {
 namespace {
 
 constexpr int kThreads = 256;
+// Heads per step of the one-, two- and three-tensor kernels: 12, 12 and 12 independent 16-byte
+// loads in flight per thread (as many as fit the 128 registers of two CTAs per SM without spills;
+// same-box A/B against 8, 8, 9: RoPE +5 % on the CogVideoX-2B and Open-Sora Plan grids, gather
+// +4 %, scatter +3 %).
+#ifndef OSP_ROPE_HS1
+#define OSP_ROPE_HS1 12
+#endif
+#ifndef OSP_ROPE_HS2
+#define OSP_ROPE_HS2 6
+#endif
+#ifndef OSP_ROPE_HS3
+#define OSP_ROPE_HS3 4
+#endif
 constexpr int kMaxPairs = 128;   // head_dim <= 256
 constexpr int kMaxTensors = 3;   // q, k, v
 
@@ -161,8 +174,8 @@ __device__ __forceinline__ bool rope_pair_f32(uint32_t w, const RotRegs& t, uint
 template <int MAP, int NT>
 __global__ void __launch_bounds__(kThreads, 2) permute_rope_kernel(const PermuteParams p,
                                                                    const __grid_constant__ PackParam<MAP> tab) {
-  // heads per step: about 8 independent 16-byte loads in flight per thread over the NT tensors
-  constexpr int HS = NT == 1 ? 8 : (NT == 2 ? 4 : 3);
+  // heads per step: about 12 independent 16-byte loads in flight per thread over the NT tensors
+  constexpr int HS = NT == 1 ? OSP_ROPE_HS1 : (NT == 2 ? OSP_ROPE_HS2 : OSP_ROPE_HS3);
   __shared__ double omega[kMaxPairs];
   const int npairs = p.head_dim >> 1;
   // Frequencies of every channel pair: pair j of a chunk of size d_a -> theta^(-2j/d_a).
